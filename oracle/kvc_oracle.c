@@ -1,0 +1,312 @@
+/*
+ * kvc_oracle.c -- plain fp64 CPU oracle for attention-saliency KV-cache compaction.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may call, link or load this
+ * file or the library built from it.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg use it.  It shares no code, header, table or helper with
+ * the CUDA library; the two meet only in the seeded input generator.
+ *
+ * What it computes, step by step, in the order the method is described:
+ *
+ *   score   The saliency of a cached token is the softmaxed attention it receives from the
+ *           last `w` queries (the observation window).  SnapKV is the decoding-time
+ *           compressor that scores this way (FastKV page, sec. 1 "Problemstellung", and
+ *           StructKV page, "Probleemstelling"); FastKV's TSP layer selects tokens by such
+ *           a saliency score (FastKV page, sec. 2A "Token-Selective Propagation").
+ *           Window query i of head g sits at position t_i = N - w + i and sees keys
+ *           j <= t_i (causal).  x_j = q.k_j / sqrt(D); p_j = exp(x_j - m) / l with
+ *           m = max_j x_j and l = sum_j exp(x_j - m) over the visible keys.
+ *   aggregate
+ *           The per-KV-head score sums p over the window queries and over the G query
+ *           heads that share the KV head (q head g reads KV head g / G).  For TSP and for
+ *           StructKV the sum also runs over all heads; StructKV further sums over all
+ *           layers up to the pivot (StructKV page, sec. 1 "Global In-Degree Centrality").
+ *   pool    1-D max-pool of odd width P over the candidate range C = [S, N - w), edges
+ *           clipped to C.
+ *   select  The k_sel = budget - S - w largest pooled scores on C, ties to the lower
+ *           index; kept = sinks [0, S)  U  selected  U  recent window [N - w, N), in
+ *           ascending order.  Sinks and recent tokens are always kept (CentroidKV page,
+ *           "Inferentie Pipeline", Preservation; FastKV page, sec. 2A: the selected
+ *           tokens plus a window of the newest tokens are propagated).
+ *   gather  Row r of the compact cache is the source row idx[r], byte for byte.
+ *
+ * Everything is done in double precision with plain loops; inputs arrive as raw fp32 or
+ * bf16 bytes and are widened exactly.  Parallelism, where present, is only over
+ * independent (layer, batch, KV head) units, and partial results are combined in a fixed
+ * order so that the output does not depend on the thread count.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+enum { OR_F32 = 0, OR_BF16 = 1, OR_F64 = 2 };
+enum { OR_SCOPE_PER_KV_HEAD = 0, OR_SCOPE_ALL_HEADS = 1 };
+
+/* Exact widening of one element to double. */
+static double widen(const void *base, int dtype, size_t i)
+{
+    if (dtype == OR_F32) return (double)((const float *)base)[i];
+    if (dtype == OR_F64) return ((const double *)base)[i];
+    /* bf16: the upper half of an IEEE binary32 */
+    uint32_t bits = ((uint32_t)((const uint16_t *)base)[i]) << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* score: one (layer, batch, KV head) unit                                               */
+/* ------------------------------------------------------------------------------------ */
+
+typedef struct {
+    int B, Hq, Hkv, N, D, w, L, dtype;
+    const void *q, *k;
+    double *unit_scores; /* [L*B*Hkv][N] */
+    int next_unit, n_units;
+    pthread_mutex_t lock;
+} score_job;
+
+/* s[j] = sum over the G heads of KV head h and the w window queries of p_{g,i,j}. */
+static void score_unit(const score_job *J, int unit, double *row)
+{
+    const int N = J->N, D = J->D, w = J->w, G = J->Hq / J->Hkv;
+    const int h = unit % J->Hkv;
+    const int b = (unit / J->Hkv) % J->B;
+    const int layer = unit / (J->Hkv * J->B);
+    const double inv_sqrt_d = 1.0 / sqrt((double)D);
+    double *s = J->unit_scores + (size_t)unit * N;
+    for (int j = 0; j < N; ++j) s[j] = 0.0;
+
+    /* K rows of this unit start here (layout [L][B][Hkv][N][D]) */
+    const size_t k_base = (((size_t)layer * J->B + b) * J->Hkv + h) * (size_t)N * D;
+    for (int gg = 0; gg < G; ++gg) {
+        const int g = h * G + gg;
+        for (int i = 0; i < w; ++i) {
+            /* query row (layout [L][B][Hq][w][D]) */
+            const size_t q_base = ((((size_t)layer * J->B + b) * J->Hq + g) * w + i) * (size_t)D;
+            const int t = N - w + i; /* position of this window query */
+            double m = -INFINITY;
+            for (int j = 0; j <= t; ++j) {
+                double x = 0.0;
+                for (int d = 0; d < D; ++d)
+                    x += widen(J->q, J->dtype, q_base + d) * widen(J->k, J->dtype, k_base + (size_t)j * D + d);
+                row[j] = x * inv_sqrt_d;
+                if (row[j] > m) m = row[j];
+            }
+            double l = 0.0;
+            for (int j = 0; j <= t; ++j) l += exp(row[j] - m);
+            for (int j = 0; j <= t; ++j) s[j] += exp(row[j] - m) / l;
+            /* keys j > t are masked: they receive nothing from this query */
+        }
+    }
+}
+
+static void *score_worker(void *arg)
+{
+    score_job *J = (score_job *)arg;
+    double *row = (double *)malloc(sizeof(double) * (size_t)J->N);
+    if (!row) return (void *)1;
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        int u = J->next_unit++;
+        pthread_mutex_unlock(&J->lock);
+        if (u >= J->n_units) break;
+        score_unit(J, u, row);
+    }
+    free(row);
+    return NULL;
+}
+
+/*
+ * oracle_score -- per-token saliency scores, summed over window queries and heads, and
+ * over layers.
+ *   q       [L, B, Hq, w, D]      fp32 / bf16 / fp64 (dtype)
+ *   k       [L, B, Hkv, N, D]     same dtype
+ *   scores  scope PER_KV_HEAD: [B, Hkv, N];  scope ALL_HEADS: [B, 1, N]   (fp64, written)
+ * Returns 0, or -1 on bad arguments / allocation failure.
+ */
+int oracle_score(int B, int Hq, int Hkv, int N, int D, int w, int L, int scope,
+                 const void *q, const void *k, int dtype, double *scores, int n_threads)
+{
+    if (B < 1 || Hkv < 1 || Hq < Hkv || Hq % Hkv || N < 1 || D < 1 || w < 1 || w > N || L < 1) return -1;
+    if (scope != OR_SCOPE_PER_KV_HEAD && scope != OR_SCOPE_ALL_HEADS) return -1;
+    score_job J;
+    J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.N = N; J.D = D; J.w = w; J.L = L; J.dtype = dtype;
+    J.q = q; J.k = k;
+    J.n_units = L * B * Hkv;
+    J.next_unit = 0;
+    J.unit_scores = (double *)malloc(sizeof(double) * (size_t)J.n_units * N);
+    if (!J.unit_scores) return -1;
+    pthread_mutex_init(&J.lock, NULL);
+    if (n_threads < 1) n_threads = 1;
+    if (n_threads > J.n_units) n_threads = J.n_units;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)n_threads);
+    int rc = 0;
+    for (int t = 1; t < n_threads; ++t) pthread_create(&th[t], NULL, score_worker, &J);
+    if (score_worker(&J)) rc = -1;
+    for (int t = 1; t < n_threads; ++t) {
+        void *r;
+        pthread_join(th[t], &r);
+        if (r) rc = -1;
+    }
+    free(th);
+    pthread_mutex_destroy(&J.lock);
+
+    /* fixed-order reduction: over layers, then (for ALL_HEADS) over KV heads */
+    const int Hs = scope == OR_SCOPE_PER_KV_HEAD ? Hkv : 1;
+    memset(scores, 0, sizeof(double) * (size_t)B * Hs * N);
+    for (int layer = 0; layer < L; ++layer)
+        for (int b = 0; b < B; ++b)
+            for (int h = 0; h < Hkv; ++h) {
+                const double *src = J.unit_scores + (((size_t)layer * B + b) * Hkv + h) * N;
+                double *dst = scores + ((size_t)b * Hs + (Hs == 1 ? 0 : h)) * N;
+                for (int j = 0; j < N; ++j) dst[j] += src[j];
+            }
+    free(J.unit_scores);
+    return rc;
+}
+
+/*
+ * oracle_accumulate -- acc[b, o, j] += sum over the Hi/Ho source heads i of group o of
+ * src[b, i, j].  Group o holds source heads o*(Hi/Ho) ... (o+1)*(Hi/Ho)-1.
+ */
+int oracle_accumulate(double *acc, const double *src, int B, int Hi, int Ho, int N)
+{
+    if (B < 1 || Hi < 1 || Ho < 1 || Hi % Ho || N < 0) return -1;
+    const int R = Hi / Ho;
+    for (int b = 0; b < B; ++b)
+        for (int o = 0; o < Ho; ++o)
+            for (int r = 0; r < R; ++r) {
+                const double *s = src + ((size_t)b * Hi + o * R + r) * N;
+                double *a = acc + ((size_t)b * Ho + o) * N;
+                for (int j = 0; j < N; ++j) a[j] += s[j];
+            }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* pool                                                                                  */
+/* ------------------------------------------------------------------------------------ */
+
+/*
+ * oracle_pool -- out[j] = max{ in[t] : lo <= t < hi, |t - j| <= (P-1)/2 } for lo <= j < hi;
+ * out[j] = in[j] outside [lo, hi).  Rows of length N, B*H rows.  P must be odd and >= 1.
+ */
+int oracle_pool(const double *in, double *out, int B, int H, int N, int lo, int hi, int P)
+{
+    if (B < 1 || H < 1 || N < 0 || lo < 0 || hi > N || lo > hi || P < 1 || P % 2 == 0) return -1;
+    const int r = (P - 1) / 2;
+    for (size_t row = 0; row < (size_t)B * H; ++row) {
+        const double *a = in + row * N;
+        double *o = out + row * N;
+        for (int j = 0; j < N; ++j) {
+            if (j < lo || j >= hi) { o[j] = a[j]; continue; }
+            int t0 = j - r < lo ? lo : j - r;
+            int t1 = j + r > hi - 1 ? hi - 1 : j + r;
+            double m = a[t0];
+            for (int t = t0 + 1; t <= t1; ++t)
+                if (a[t] > m) m = a[t];
+            o[j] = m;
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* select                                                                                */
+/* ------------------------------------------------------------------------------------ */
+
+typedef struct { double v; int j; } cand;
+
+/* larger score first; equal scores: lower index first */
+static int cand_cmp(const void *pa, const void *pb)
+{
+    const cand *a = (const cand *)pa, *b = (const cand *)pb;
+    if (a->v > b->v) return -1;
+    if (a->v < b->v) return 1;
+    return (a->j > b->j) - (a->j < b->j);
+}
+
+static int int_cmp(const void *pa, const void *pb)
+{
+    int a = *(const int *)pa, b = *(const int *)pb;
+    return (a > b) - (a < b);
+}
+
+/*
+ * oracle_select -- per row: sort the candidates C = [S, N - w) by (score desc, index asc),
+ * keep the first budget - S - w, add the sinks [0, S) and the window [N - w, N), and write
+ * the `budget` kept positions in ascending order to idx[row][0..budget).
+ * Requires S >= 0, w >= 0, budget >= S + w + 1 and budget <= N.
+ */
+int oracle_select(const double *pooled, int B, int H, int N, int S, int w, int budget, int32_t *idx)
+{
+    if (B < 1 || H < 1 || S < 0 || w < 0 || budget < S + w + 1 || budget > N) return -1;
+    const int n_c = N - w - S;
+    const int k_sel = budget - S - w;
+    cand *c = (cand *)malloc(sizeof(cand) * (size_t)(n_c > 0 ? n_c : 1));
+    int *kept = (int *)malloc(sizeof(int) * (size_t)budget);
+    if (!c || !kept) { free(c); free(kept); return -1; }
+    for (size_t row = 0; row < (size_t)B * H; ++row) {
+        const double *s = pooled + row * N;
+        for (int t = 0; t < n_c; ++t) { c[t].v = s[S + t]; c[t].j = S + t; }
+        qsort(c, (size_t)n_c, sizeof(cand), cand_cmp);
+        int n = 0;
+        for (int j = 0; j < S; ++j) kept[n++] = j;
+        for (int t = 0; t < k_sel; ++t) kept[n++] = c[t].j;
+        for (int j = N - w; j < N; ++j) kept[n++] = j;
+        qsort(kept, (size_t)n, sizeof(int), int_cmp);
+        for (int t = 0; t < budget; ++t) idx[row * budget + t] = kept[t];
+    }
+    free(c);
+    free(kept);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* gather                                                                                */
+/* ------------------------------------------------------------------------------------ */
+
+/*
+ * oracle_gather -- dst[b, h, r, :] = src[b, h, idx[b, h', r], :] with h' = h when
+ * Hidx == Hsrc and h' = 0 when Hidx == 1.  Rows are `row_bytes` raw bytes.
+ */
+int oracle_gather(const void *src, int B, int Hsrc, int N, size_t row_bytes,
+                  const int32_t *idx, int Hidx, int K, void *dst)
+{
+    if (B < 1 || Hsrc < 1 || N < 1 || K < 0 || (Hidx != 1 && Hidx != Hsrc)) return -1;
+    const unsigned char *s = (const unsigned char *)src;
+    unsigned char *d = (unsigned char *)dst;
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < Hsrc; ++h)
+            for (int r = 0; r < K; ++r) {
+                int j = idx[((size_t)b * Hidx + (Hidx == 1 ? 0 : h)) * K + r];
+                if (j < 0 || j >= N) return -1;
+                memcpy(d + (((size_t)b * Hsrc + h) * K + r) * row_bytes,
+                       s + (((size_t)b * Hsrc + h) * N + j) * row_bytes, row_bytes);
+            }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* TSP row count                                                                         */
+/* ------------------------------------------------------------------------------------ */
+
+/*
+ * oracle_tsp_count -- rows propagated by Token-Selective Propagation: floor(rate * N)
+ * selected tokens (at most the N - S - w candidates) plus the S sinks and the w recent
+ * tokens.  The TSP rate is its own knob, separate from the KV-retention budget (FastKV
+ * page, sec. 2B "Entkoppelte KV-Cache-Reduktion").  Returns 0 when rate <= 0 or when
+ * floor(rate * N) < 1 (no token would be selected).
+ */
+int oracle_tsp_count(int N, int w, int S, double rate)
+{
+    if (rate <= 0.0) return 0;
+    long sel = (long)floor(rate * (double)N);
+    long n_c = (long)N - w - S;
+    if (sel > n_c) sel = n_c;
+    if (sel < 1) return 0; /* nothing to select: not a valid TSP configuration */
+    return (int)(sel + S + w);
+}

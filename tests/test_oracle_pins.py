@@ -1,0 +1,308 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle itself.
+
+No page prints a worked numerical example of the saliency path, so every pin here is a
+closed form, an invariant, a special case that reduces to a textbook/library routine, or
+brute force on a tiny input.  Each is chosen so that a plausible slip in the oracle (a
+wrong logit scale, an off-by-one in the causal mask, a wrong GQA head mapping, a missing
+max-shift, a reversed tie-break, a wrong pool radius or edge clipping) fails at least one.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+from oracle import oracle as O
+
+
+def _zeros_case(B, Hq, Hkv, N, D, w, L=1):
+    q = torch.randn(L, B, Hq, w, D, dtype=torch.float64, generator=torch.Generator().manual_seed(1))
+    k = torch.zeros(L, B, Hkv, N, D, dtype=torch.float64)
+    return q, k
+
+
+def _uniform_closed_form(N, w, G):
+    """All logits equal: query i (position N-w+i) spreads 1/(t_i+1) over keys 0..t_i."""
+    s = np.zeros(N)
+    for i in range(w):
+        t = N - w + i
+        s[: t + 1] += 1.0 / (t + 1)
+    return G * s
+
+
+@pytest.mark.parametrize("N,w,G", [(17, 3, 2), (40, 8, 4), (5, 5, 1)])
+def test_all_equal_logits_closed_form(N, w, G):
+    # K == 0 makes every logit 0; the softmax is then uniform over the visible keys.
+    q, k = _zeros_case(1, 2 * G, 2, N, 16, w)
+    s = O.score(q, k, window=w)
+    ref = _uniform_closed_form(N, w, G)
+    for h in range(2):
+        np.testing.assert_allclose(s[0, h], ref, rtol=0, atol=1e-14)
+
+
+def test_two_key_logistic_pins_scale():
+    # One query at position 1 sees keys 0 and 1; with q = a e0 and k_j = b_j e0 the logits
+    # are a b_j / sqrt(D), and the softmax of two logits is the logistic function.
+    D = 16
+    for a, b0, b1 in [(2.0, 3.0, -1.0), (0.5, -4.0, 6.0), (8.0, 1.0, 1.25)]:
+        q = torch.zeros(1, 1, 1, 1, D, dtype=torch.float64)
+        k = torch.zeros(1, 1, 1, 2, D, dtype=torch.float64)
+        q[..., 0] = a
+        k[0, 0, 0, 0, 0] = b0
+        k[0, 0, 0, 1, 0] = b1
+        s = O.score(q, k, window=1)
+        x0, x1 = a * b0 / math.sqrt(D), a * b1 / math.sqrt(D)
+        assert s[0, 0, 0] == pytest.approx(scipy.special.expit(x0 - x1), abs=1e-15)
+        assert s[0, 0, 1] == pytest.approx(scipy.special.expit(x1 - x0), abs=1e-15)
+
+
+def test_causal_mask_boundary():
+    # The last key is visible to the last window query only: with equal logits it gets
+    # exactly G / N, and the key before it gets G (1/(N-1) + 1/N) for w = 2.
+    N, w, G = 9, 2, 3
+    q, k = _zeros_case(1, G, 1, N, 8, w)
+    s = O.score(q, k, window=w)[0, 0]
+    assert s[N - 1] == pytest.approx(G / N, abs=1e-15)
+    assert s[N - 2] == pytest.approx(G * (1 / (N - 1) + 1 / N), abs=1e-15)
+
+
+def test_dominant_key_and_no_overflow():
+    # One key with a logit gap >= 50 over all others takes all of the mass of every window
+    # query that sees it.  Logits near 1000 also check that the max is subtracted
+    # (exp(1000) overflows double).
+    B, Hq, Hkv, N, D, w = 1, 4, 2, 64, 32, 4
+    G = Hq // Hkv
+    g = torch.Generator().manual_seed(3)
+    k = torch.randn(1, B, Hkv, N, D, dtype=torch.float64, generator=g) * 0.01
+    q = torch.zeros(1, B, Hq, w, D, dtype=torch.float64)
+    q[..., 0] = 100.0
+    k[..., 0] += 50.0  # all logits ~ 100*50/sqrt(32) ~ 884
+    k[0, 0, :, 10, 0] = 60.0  # key 10 wins by ~177
+    s = O.score(q, k, window=w)
+    assert np.all(np.isfinite(s))
+    np.testing.assert_allclose(s[0, :, 10], G * w, rtol=1e-12)
+    assert s[0, :, np.arange(N) != 10].max() < 1e-60
+
+
+def test_gqa_mapping_contiguous_groups():
+    # q head g reads KV head g // G.  Heads 0,1 (group of KV head 0) have q = 0, so their
+    # attention is uniform; heads 2,3 point at key 7 of KV head 1 with a huge gap.
+    B, Hq, Hkv, N, D, w = 1, 4, 2, 30, 16, 3
+    G = Hq // Hkv
+    g = torch.Generator().manual_seed(5)
+    k = torch.randn(1, B, Hkv, N, D, dtype=torch.float64, generator=g)
+    q = torch.zeros(1, B, Hq, w, D, dtype=torch.float64)
+    direction = k[0, 0, 1, 7] / k[0, 0, 1, 7].norm()
+    q[0, 0, 2:] = 400.0 * direction
+    s = O.score(q, k, window=w)
+    np.testing.assert_allclose(s[0, 0], _uniform_closed_form(N, w, G), atol=1e-13)
+    assert s[0, 1, 7] == pytest.approx(G * w, rel=1e-9)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_mass_invariant(dtype):
+    # Every window query distributes probability 1, so the scores of a KV head sum to G*w.
+    B, Hq, Hkv, N, D, w = 2, 8, 2, 300, 128, 6
+    g = torch.Generator().manual_seed(11)
+    q = torch.randn(1, B, Hq, w, D, generator=g).to(dtype)
+    k = torch.randn(1, B, Hkv, N, D, generator=g).to(dtype)
+    s = O.score(q, k, window=w)
+    np.testing.assert_allclose(s.sum(axis=-1), (Hq // Hkv) * w, rtol=1e-12)
+    assert np.all(s >= 0)
+
+
+def test_matches_library_softmax():
+    # Cross-check against torch's float64 softmax (a library routine) with a causal mask.
+    B, Hq, Hkv, N, D, w = 1, 6, 3, 50, 24, 5
+    G = Hq // Hkv
+    g = torch.Generator().manual_seed(7)
+    q = torch.randn(1, B, Hq, w, D, dtype=torch.float64, generator=g) * 2
+    k = torch.randn(1, B, Hkv, N, D, dtype=torch.float64, generator=g)
+    s = O.score(q, k, window=w)
+    pos = torch.arange(N - w, N)[:, None]
+    mask = torch.arange(N)[None, :] > pos
+    for h in range(Hkv):
+        tot = torch.zeros(N, dtype=torch.float64)
+        for gg in range(G):
+            logits = q[0, 0, h * G + gg] @ k[0, 0, h].T / math.sqrt(D)
+            tot += torch.softmax(logits.masked_fill(mask, -math.inf), dim=-1).sum(0)
+        np.testing.assert_allclose(s[0, h], tot.numpy(), rtol=1e-12, atol=1e-15)
+
+
+def test_layers_and_heads_are_sums():
+    # StructKV's cumulative score is a plain sum over layers; ALL_HEADS sums KV heads.
+    L, B, Hq, Hkv, N, D, w = 3, 2, 4, 2, 40, 16, 4
+    g = torch.Generator().manual_seed(9)
+    q = torch.randn(L, B, Hq, w, D, dtype=torch.float64, generator=g)
+    k = torch.randn(L, B, Hkv, N, D, dtype=torch.float64, generator=g)
+    s_all = O.score(q, k, window=w)
+    s_sum = sum(O.score(q[l:l + 1], k[l:l + 1], window=w) for l in range(L))
+    np.testing.assert_allclose(s_all, s_sum, rtol=1e-13)
+    g_all = O.score(q, k, window=w, scope=O.SCOPE_ALL_HEADS)
+    np.testing.assert_allclose(g_all[:, 0], s_all.sum(axis=1), rtol=1e-13)
+    np.testing.assert_allclose(g_all.sum(axis=-1), L * Hq * w, rtol=1e-12)
+
+
+def test_thread_count_does_not_change_result():
+    g = torch.Generator().manual_seed(13)
+    q = torch.randn(2, 2, 4, 4, 32, generator=g)
+    k = torch.randn(2, 2, 2, 100, 32, generator=g)
+    a = O.score(q, k, window=4, threads=1)
+    b = O.score(q, k, window=4, threads=7)
+    assert np.array_equal(a, b)
+
+
+# ------------------------------------------------------------------------------ accumulate
+
+def test_accumulate_group_sums():
+    src = np.arange(2 * 6 * 5, dtype=np.float64).reshape(2, 6, 5)
+    acc = np.ones((2, 3, 5))
+    out = O.accumulate(acc.copy(), src)
+    np.testing.assert_array_equal(out, 1 + src.reshape(2, 3, 2, 5).sum(axis=2))
+
+
+# ------------------------------------------------------------------------------------ pool
+
+@pytest.mark.parametrize("P", [1, 3, 7])
+def test_pool_delta_gives_clipped_plateau(P):
+    N, lo, hi = 30, 2, 25
+    r = (P - 1) // 2
+    for j0 in [lo, lo + 1, 12, hi - 2, hi - 1]:
+        x = np.zeros((1, 1, N))
+        x[0, 0, j0] = 1.0
+        out = O.pool(x, lo, hi, P)[0, 0]
+        want = np.zeros(N)
+        want[max(lo, j0 - r): min(hi - 1, j0 + r) + 1] = 1.0
+        np.testing.assert_array_equal(out, want)
+
+
+def test_pool_ramp_and_no_leak_from_outside():
+    N, lo, hi, P = 20, 3, 15, 5
+    x = np.arange(N, dtype=np.float64)[None, None].copy()
+    x[0, 0, lo - 1] = 1e9  # outside C: must not leak into pooled values
+    x[0, 0, hi] = 1e9
+    out = O.pool(x, lo, hi, P)[0, 0]
+    for j in range(lo, hi):
+        assert out[j] == min(hi - 1, j + 2)
+    assert out[lo - 1] == 1e9 and out[hi] == 1e9  # pass-through outside C
+
+
+def test_pool_matches_sliding_window_library():
+    g = np.random.default_rng(0)
+    x = g.random((2, 3, 57))
+    lo, hi, P = 4, 50, 7
+    r = P // 2
+    out = O.pool(x, lo, hi, P)
+    seg = np.pad(x[..., lo:hi], ((0, 0), (0, 0), (r, r)), constant_values=-np.inf)
+    want = np.lib.stride_tricks.sliding_window_view(seg, P, axis=-1).max(axis=-1)
+    np.testing.assert_array_equal(out[..., lo:hi], want)
+    np.testing.assert_array_equal(out[..., :lo], x[..., :lo])
+    np.testing.assert_array_equal(out[..., hi:], x[..., hi:])
+
+
+# ---------------------------------------------------------------------------------- select
+
+def _brute_force_selected(vals, k_sel):
+    """Among all k_sel-subsets of candidate positions, the one with the largest multiset
+    of values and, among those, the lexicographically smallest positions."""
+    n = len(vals)
+    best = None
+    for comb in itertools.combinations(range(n), k_sel):
+        key = (sorted((-vals[c] for c in comb)), comb)
+        if best is None or key < best:
+            best = key
+    return list(best[1])
+
+
+def test_select_brute_force_with_ties():
+    g = np.random.default_rng(1)
+    for trial in range(25):
+        N, S, w = 14, 1, 2
+        budget = S + w + int(g.integers(1, 6))
+        vals = g.integers(0, 4, size=N).astype(np.float64)  # many ties
+        idx = O.select(vals[None, None], S, w, budget)[0, 0]
+        k_sel = budget - S - w
+        sel = [S + c for c in _brute_force_selected(vals[S:N - w], k_sel)]
+        want = sorted(list(range(S)) + sel + list(range(N - w, N)))
+        assert list(idx) == want
+
+
+def test_select_matches_library_sort_and_invariants():
+    g = np.random.default_rng(2)
+    B, H, N, S, w = 2, 3, 500, 4, 16
+    vals = np.round(g.random((B, H, N)), 2)  # ties are common
+    for budget in [S + w + 1, 60, 200, N]:
+        idx = O.select(vals, S, w, budget)
+        assert idx.shape == (B, H, budget)
+        for b in range(B):
+            for h in range(H):
+                row = idx[b, h]
+                assert np.all(np.diff(row) > 0)
+                assert set(range(S)) <= set(row) and set(range(N - w, N)) <= set(row)
+                ranked = sorted(range(S, N - w), key=lambda j: (-vals[b, h, j], j))
+                sel = set(ranked[: budget - S - w])
+                assert set(row) == sel | set(range(S)) | set(range(N - w, N))
+
+
+def test_select_nested_in_budget_and_rejects_bad_budgets():
+    g = np.random.default_rng(3)
+    vals = g.random((1, 1, 200))
+    prev = set()
+    for budget in range(10, 200, 17):
+        cur = set(O.select(vals, 2, 5, budget)[0, 0])
+        assert prev <= cur
+        prev = cur
+    with pytest.raises(ValueError):
+        O.select(vals, 2, 5, 7)  # budget < S + w + 1
+    with pytest.raises(ValueError):
+        O.select(vals, 2, 5, 201)  # budget > N
+
+
+def test_select_all_equal_takes_lowest_indices():
+    idx = O.select(np.ones((1, 1, 20)), 1, 3, 8)[0, 0]
+    assert list(idx) == [0, 1, 2, 3, 4, 17, 18, 19]
+
+
+# ---------------------------------------------------------------------------------- gather
+
+def test_gather_is_a_row_copy():
+    g = torch.Generator().manual_seed(4)
+    src = torch.randn(2, 3, 40, 16, generator=g).to(torch.bfloat16)
+    idx = np.stack([np.stack([np.sort(np.random.default_rng(b * 3 + h).choice(40, 7, replace=False))
+                              for h in range(3)]) for b in range(2)]).astype(np.int32)
+    out = O.gather(src, idx)
+    for b in range(2):
+        for h in range(3):
+            assert torch.equal(out[b, h].view(torch.int16), src[b, h, idx[b, h]].view(torch.int16))
+    shared = idx[:, :1]
+    out1 = O.gather(src, shared)
+    for h in range(3):
+        assert torch.equal(out1[:, h], src[torch.arange(2)[:, None], h, torch.from_numpy(shared[:, 0]).long()])
+
+
+# ------------------------------------------------------------------------------------- TSP
+
+def test_tsp_count():
+    assert O.tsp_count(65536, 32, 1, 0.2) == 13107 + 1 + 32
+    assert O.tsp_count(100, 10, 1, 0.0) == 0
+    assert O.tsp_count(100, 10, 1, 0.001) == 0  # floor(0.1) = 0 tokens
+    assert O.tsp_count(100, 10, 1, 1.0) == 100  # capped at the 89 candidates
+
+
+def test_compress_composition_invariants():
+    g = torch.Generator().manual_seed(21)
+    q = torch.randn(1, 2, 4, 4, 32, generator=g)
+    k = torch.randn(1, 2, 2, 120, 32, generator=g)
+    v = torch.randn(2, 2, 120, 32, generator=g)
+    hidden = torch.randn(2, 120, 48, generator=g)
+    out = O.compress(q, k, v, window=4, n_sink=1, pool_kernel=3, kv_budget=20, tsp_rate=0.25,
+                     hidden=hidden)
+    assert out["idx"].shape == (2, 2, 20)
+    assert out["tsp_idx"].shape == (2, 1, 30 + 5)
+    np.testing.assert_allclose(out["tsp_scores"][:, 0], out["scores"].sum(axis=1), rtol=1e-14)
+    for b in range(2):
+        assert torch.equal(out["hidden_out"][b], hidden[b, torch.from_numpy(out["tsp_idx"][b, 0]).long()])
+        for h in range(2):
+            assert torch.equal(out["k_out"][b, h], k[0, b, h, torch.from_numpy(out["idx"][b, h]).long()])
