@@ -1,0 +1,386 @@
+"""Throughput of attention-saliency KV-cache compaction on B200.
+
+One step = one kvc_compress call over one batch of the workload (default: the Llama-3.1-8B
+head layout at 128K context, batch 4): window-softmax scoring, group sums, max-pool,
+top-k with sinks and recent window, and the K/V gather.  Inputs are seeded synthetic
+tensors resident in HBM before timing starts.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvc|reference] [--workload NAME]
+
+With N > 1 it runs under torchrun, one rank per GPU; every rank compacts its own batch of
+independent sequences (weak scaling, no collective on the data path) and the time is the
+max over ranks.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from long_context_kv_kvc_b200 import synth  # noqa: E402
+
+METRIC = "KV tokens compressed/sec and achieved HBM GB/s (% of peak) at 128K ctx"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ----------------------------------------------------------------------------- host logic
+
+def rank_seeds(wl: synth.Workload, rank: int) -> tuple:
+    """Seeds of the sequences that rank `rank` compacts: rank 0 uses the workload's own
+    seeds, rank r the next B seeds after rank r-1's (independent sequences)."""
+    return tuple(int(s) + rank * wl.B for s in wl.seeds)
+
+
+def algorithmic_bytes(wl: synth.Workload) -> dict:
+    """Compulsory HBM bytes of one compaction call, by stage.
+
+    score:  every key row of every layer once, the window queries once, and the fp32 score
+            rows written once (B * Hs * N * 4);
+    select: the score rows read and pooled rows written/read (kept in L2 in practice but
+            counted), the kept index lists written;
+    gather: the kept K and V rows read and written (and the TSP hidden rows).
+    """
+    e = 4 if wl.dtype == "f32" else 2
+    L, B, Hq, Hkv, N, D, w = wl.n_layers, wl.B, wl.Hq, wl.Hkv, wl.N, wl.D, wl.window
+    Hs = Hkv if wl.scope == synth.SCOPE_PER_KV_HEAD else 1
+    k_read = L * B * Hkv * N * D * e
+    q_read = L * B * Hq * w * D * e
+    score_write = B * Hs * N * 4
+    score = k_read + q_read + score_write
+    kb = wl.kv_budget
+    gather = 2 * (2 * B * Hkv * kb * D * e)  # K and V, read + write
+    idx = B * Hs * kb * 4
+    if wl.tsp_rate > 0:
+        n_tsp = tsp_count(wl)
+        gather += 2 * B * n_tsp * wl.hidden_dim * e
+        idx += B * n_tsp * 4
+    return {"score": score, "k_read": k_read, "q_read": q_read, "score_write": score_write,
+            "gather": gather, "idx": idx, "total": k_read + q_read + gather + idx}
+
+
+def tsp_count(wl) -> int:
+    if wl.tsp_rate <= 0:
+        return 0
+    sel = int(np.floor(float(np.float32(wl.tsp_rate)) * wl.N))
+    sel = min(sel, wl.N - wl.window - wl.n_sink)
+    return sel + wl.n_sink + wl.window if sel >= 1 else 0
+
+
+def measured_peaks() -> tuple:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_digest(*names) -> str:
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "long_context_kv_kvc_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str, digest: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current
+    kernel source; otherwise None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        rec = d[kernel][workload]
+        return rec["dram_bytes_per_launch"] if rec.get("source_digest") == digest else None
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        return summarize_clocks(rows)
+
+
+def summarize_clocks(rows) -> dict:
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def num(x):
+        try:
+            return float(x)
+        except ValueError:
+            return None
+
+    sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+    mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+    reasons = set()
+    for r in rows:
+        for i, n in enumerate(names):
+            if r[5 + i].lower().startswith("active"):
+                reasons.add(n)
+    loaded = [s for s, r in zip(sm, rows) if (num(r[3]) or 0) > 300] or sm
+    return {"sm_mhz": statistics.median(loaded) if loaded else None,
+            "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- CPU legs
+
+def oracle_sample(wl: synth.Workload, inputs: dict, heads: int, threads: int) -> tuple:
+    """Runs the fp64 oracle on sequence 0, KV heads [0, heads) (the sample) and returns
+    (seconds, equivalent context tokens = N * heads / Hkv)."""
+    from oracle import oracle as O
+    G = wl.G
+    q = inputs["q"][:, :1, :heads * G]
+    k = inputs["k"][:, :1, :heads]
+    v = inputs["v"][:1, :heads]
+    wsub = wl.replace(B=1, Hq=heads * G, Hkv=heads)
+    t0 = time.perf_counter()
+    O.compress(q, k, v, window=wl.window, n_sink=wl.n_sink, pool_kernel=wl.pool_kernel,
+               kv_budget=wl.kv_budget, scope=wl.scope, threads=threads)
+    dt = time.perf_counter() - t0
+    del wsub
+    return dt, wl.N * heads / wl.Hkv
+
+
+def run_reference(args, wl, rank, world):
+    """The oracle as the reference arm: each step is one bounded sample of the workload."""
+    if rank != 0:
+        return 0
+    inputs = synth.make_inputs(wl, seeds=rank_seeds(wl, 0), with_hidden=False)
+    cores = os.cpu_count() or 1
+    heads = 1
+    for _ in range(max(args.warmup, 0)):
+        oracle_sample(wl, inputs, heads, 1)
+    total_t, total_tok = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, tok = oracle_sample(wl, inputs, heads, 1)
+        total_t += dt
+        total_tok += tok
+    value = total_tok / total_t
+    sample = f"sequence 0, KV head 0 of {wl.Hkv} ({wl.N} tokens x 1/{wl.Hkv} of the heads) per step"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_of(wl, world),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": sample, "host_cores": cores},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(wl, world) -> dict:
+    return {"workload": wl.name, "B_per_gpu": wl.B, "global_batch": wl.B * world, "Hq": wl.Hq,
+            "Hkv": wl.Hkv, "N": wl.N, "D": wl.D, "window": wl.window, "n_layers": wl.n_layers,
+            "kv_budget": wl.kv_budget, "pool_kernel": wl.pool_kernel, "n_sink": wl.n_sink,
+            "tsp_rate": wl.tsp_rate, "parallelism": f"batch-sharded replicas x{world} (no collective)",
+            "l2": "inputs larger than L2 (1 GiB of K per GPU), no flush"}
+
+
+# ----------------------------------------------------------------------------- GPU leg
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="kvc", choices=["kvc", "reference"])
+    ap.add_argument("--workload", default=synth.LLAMA8B_128K_B4.name, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--flags", type=int, default=0, help="kvc_params.flags (1 = CUDA-core scoring)")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    wl = synth.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        return run_reference(args, wl, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    from long_context_kv_kvc_b200 import kvc
+
+    inputs = synth.make_inputs(wl, seeds=rank_seeds(wl, rank))
+    dev = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inputs.items()}
+    p = kvc.params_for(wl, flags=args.flags)
+    comp = kvc.Compressor(p)
+    stream = torch.cuda.current_stream()
+
+    # one set of stage events per timed step (score stage = the dominant kernel)
+    n_ev = kvc.KVC_STAGE_COUNT + 1
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    for evs in events:
+        for e in evs:
+            e.record(stream)  # materialise the underlying cudaEvent_t
+    handles = [(ctypes.c_void_p * n_ev)(*[e.cuda_event for e in evs]) for evs in events]
+
+    def step(i=None):
+        p.stage_events = ctypes.cast(handles[i], ctypes.POINTER(ctypes.c_void_p)) if i is not None else None
+        comp.run_device(dev["q"], dev["k"], dev["v"], dev.get("hidden"))
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    if kvc.kvc_poll_error() != kvc.KVC_OK:
+        raise RuntimeError("device-side error during warm-up")
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    # keep the GPU busy ~1 s under the sampler before the timed region
+    t_end = time.time() + 1.0
+    while time.time() < t_end:
+        step()
+        torch.cuda.synchronize()
+
+    n_before = kvc.kvc_launch_count()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    launches = (kvc.kvc_launch_count() - n_before) // 1
+    clocks = sampler.stop()
+    ms = t0.elapsed_time(t1)
+    if kvc.kvc_poll_error() != kvc.KVC_OK:
+        raise RuntimeError("device-side error during the timed region")
+
+    stage_ms = [[evs[s].elapsed_time(evs[s + 1]) for s in range(n_ev - 1)] for evs in events]
+    score_ms = sum(x[kvc.KVC_STAGE_SCORE] for x in stage_ms) / args.steps
+    select_ms = sum(x[kvc.KVC_STAGE_SELECT] for x in stage_ms) / args.steps
+    gather_ms = sum(x[kvc.KVC_STAGE_GATHER] for x in stage_ms) / args.steps
+
+    t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    ms_step = ms_max / args.steps
+    tokens = wl.B * wl.N * world
+    value = tokens / (ms_step / 1e3)
+
+    ab = algorithmic_bytes(wl)
+    peak, peak_kind = measured_peaks()
+    achieved = ab["score"] / (score_ms / 1e3) / 1e9
+    digest = source_digest("score_tc.cu" if not (args.flags & 1) and wl.dtype == "bf16" else "score_simt.cu")
+    kernel_name = "score_tc" if not (args.flags & 1) and wl.dtype == "bf16" else "score_simt"
+    traffic = recorded_traffic(kernel_name, wl.name, digest)
+
+    # end to end through the public API: pinned host inputs -> device -> compact cache -> host
+    e2e = None
+    if args.e2e_steps > 0:
+        host = {k: v.pin_memory() for k, v in inputs.items() if isinstance(v, torch.Tensor)}
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        d2h = sum(v.numel() * v.element_size() for v in comp.out.values())
+        comp(host["q"], host["k"], host["v"], host.get("hidden"))  # warm-up
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            comp(host["q"], host["k"], host["v"], host.get("hidden"))
+        e1.record(stream)
+        torch.cuda.synchronize()
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device="cuda")
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": tokens / (float(te.item()) / args.e2e_steps / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = min(wl.Hkv, os.cpu_count() or 1)
+        dt, tok = oracle_sample(wl, inputs, wl.Hkv, threads)
+        cpu = {"value": tok / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": f"sequence 0 of {wl.B}, all {wl.Hkv} KV heads ({wl.N} tokens), fp64 oracle, "
+                         f"one thread per KV head", "seconds": dt}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic", "config": config_of(wl, world),
+            "hbm_gbs": ab["total"] * world / (ms_step / 1e3) / 1e9,
+            "hbm_frac_of_peak": ab["total"] / (ms_step / 1e3) / 1e9 / peak,
+            "stages_ms": {"score": score_ms, "select": select_ms, "gather": gather_ms},
+            "roofline": {"kernel": kernel_name, "bound": "hbm", "achieved": achieved, "peak": peak,
+                         "peak_source": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": traffic, "algorithmic_bytes_per_launch": ab["score"]},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

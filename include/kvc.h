@@ -1,0 +1,246 @@
+/*
+ * kvc.h -- C ABI of libkvc.so: attention-saliency KV-cache compaction on NVIDIA B200
+ * (sm_100a).
+ *
+ * The library scores every cached token by the softmaxed attention of the last `window`
+ * queries, sums the scores over the window, the GQA group and optionally over all heads
+ * and layers, max-pools them, keeps a top-k budget per KV head plus the attention sinks
+ * and the recent window, and gathers the kept K/V rows (or, for Token-Selective
+ * Propagation, the kept hidden-state rows) into a compact cache.
+ *
+ * Sources of the operation (web summaries of the papers):
+ *   - FastKV, sec. 1 "Problemstellung": SnapKV / StreamingLLM compress the KV cache after
+ *     prefill (decoding-only eviction);
+ *   - FastKV, sec. 2A "Token-Selective Propagation": a saliency score selects the tokens
+ *     that are propagated, plus a window of the most recent tokens;
+ *   - FastKV, sec. 2B "Entkoppelte KV-Cache-Reduktion": the TSP rate and the KV retention
+ *     rate are separate knobs;
+ *   - StructKV, sec. 1 "Global In-Degree Centrality": the cumulative score of a token is
+ *     the sum of its attention scores over all layers up to the pivot;
+ *   - CentroidKV, "Inferentie Pipeline" (Preservation): attention sinks and recent tokens
+ *     are always kept;
+ *   - CentroidKV, "Probleemstelling" (Eviction): tokens are evicted by attention score.
+ * The pages do not write the score formula down; the definition used here is the
+ * standard window-softmax one:
+ *     x[g,i,j] = q[g,i] . k[j] / sqrt(D)                (query i of head g, key j)
+ *     window query i sits at position N - window + i and sees keys j <= N - window + i
+ *     p[g,i,j] = exp(x[g,i,j] - m[g,i]) / l[g,i]        (softmax over the visible keys)
+ *     s[h,j]   = sum over heads g with g / G == h, and over i, of p[g,i,j]
+ * with G = Hq / Hkv (contiguous head groups).  Candidates are C = [n_sink, N - window);
+ * the pooled score of j in C is the max of s over {t in C : |t - j| <= (pool_kernel-1)/2};
+ * k_sel = budget - n_sink - window candidates with the largest pooled score are kept,
+ * equal scores going to the lower index; the kept list is sinks + selected + window in
+ * ascending position order.
+ *
+ * Conventions for every entry point:
+ *   Ownership  The caller owns every buffer.  The library allocates no device memory;
+ *              scratch comes from the caller's workspace `ws` (size from
+ *              kvc_workspace_size).  Pointers named "device" must be device (or managed)
+ *              memory of the current device.
+ *   Layout     All tensors are dense, row-major (C order), with the shapes given below.
+ *   Asynchrony All work is enqueued on `stream` (a cudaStream_t; 0 = legacy default
+ *              stream).  No call synchronises the host except kvc_poll_error.  Outputs are
+ *              valid in stream order.
+ *   Errors     Arguments are validated on the host before anything is enqueued; a call
+ *              that returns anything but KVC_OK has enqueued nothing, except KVC_ERR_CUDA
+ *              (a CUDA launch failed part way).  Device-side problems (a bounded wait that
+ *              gave up, an index out of range in kvc_gather) never fault or hang the GPU:
+ *              the kernel skips the work, records a flag, and kvc_poll_error reports it.
+ *   Threading  Calls are thread-safe; concurrent calls need distinct workspaces.
+ *   Alignment  q, k, v, hidden and all outputs must be 16-byte aligned; ws 256-byte.
+ */
+#ifndef KVC_H
+#define KVC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KVC_API __attribute__((visibility("default")))
+#else
+#define KVC_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *kvc_stream_t; /* identical to cudaStream_t */
+
+typedef enum kvc_status {
+    KVC_OK = 0,
+    KVC_ERR_ARG = 1,         /* null pointer, non-positive or inconsistent shape          */
+    KVC_ERR_UNSUPPORTED = 2, /* D != 128, unknown dtype/scope, G*window > 256             */
+    KVC_ERR_BUDGET = 3,      /* budget < n_sink + window + 1, budget > N, empty TSP        */
+    KVC_ERR_ALIGN = 4,       /* pointer or row size not 16-byte aligned (ws: 256-byte)     */
+    KVC_ERR_WORKSPACE = 5,   /* ws_bytes smaller than kvc_workspace_size                  */
+    KVC_ERR_CUDA = 6,        /* a CUDA runtime call failed                                */
+    KVC_ERR_TIMEOUT = 7,     /* a device-side bounded wait gave up (reported by poll)      */
+    KVC_ERR_INDEX = 8        /* kvc_gather met an index outside [0, N) (reported by poll)  */
+} kvc_status;
+
+enum { KVC_F32 = 0, KVC_BF16 = 1 };
+
+enum {
+    KVC_SCOPE_PER_KV_HEAD = 0, /* one score row per (batch, KV head)                    */
+    KVC_SCOPE_ALL_HEADS = 1    /* one score row per batch element: summed over KV heads */
+};
+
+/* kvc_params.flags */
+enum {
+    KVC_FLAG_SIMT_SCORE = 1u << 0 /* score with the CUDA-core (FFMA) kernels even for bf16 */
+};
+
+/* Entries of kvc_params.stage_events: events recorded on the stream between the stages
+ * of kvc_compress (index i is recorded before stage i; the last after the last stage). */
+enum {
+    KVC_STAGE_SCORE = 0,  /* window softmax + group/layer sums          */
+    KVC_STAGE_SELECT = 1, /* head sums for TSP, pooling, top-k          */
+    KVC_STAGE_GATHER = 2, /* compact K/V (and hidden-row) copies        */
+    KVC_STAGE_COUNT = 3
+};
+
+typedef struct kvc_params {
+    int32_t B;           /* batch (independent sequences)                                  */
+    int32_t Hq;          /* query heads                                                    */
+    int32_t Hkv;         /* KV heads; Hq % Hkv == 0, q head g reads KV head g / (Hq/Hkv)    */
+    int32_t N;           /* cached tokens per sequence                                     */
+    int32_t D;           /* head dimension; must be 128                                    */
+    int32_t window;      /* observation-window queries w; 1 <= w < N                       */
+    int32_t dtype;       /* KVC_F32 or KVC_BF16: q, K, V and hidden rows                    */
+    int32_t n_sink;      /* attention sinks kept at positions [0, n_sink); >= 0             */
+    int32_t pool_kernel; /* odd width of the 1-D max-pool; 1 disables pooling               */
+    int32_t kv_budget;   /* kept KV rows per row of scores, INCLUDING sinks and window      */
+    int32_t scope;       /* KVC_SCOPE_PER_KV_HEAD or KVC_SCOPE_ALL_HEADS                    */
+    int32_t n_layers;    /* >= 1: q and k hold this many layers; scores are summed over them */
+    float tsp_rate;      /* > 0: Token-Selective Propagation of floor(rate*N) tokens       */
+    int32_t hidden_dim;  /* elements per hidden-state row (TSP only)                       */
+    int64_t spin_limit;  /* iterations a device-side wait may spin; 0 = library default    */
+    uint32_t flags;      /* KVC_FLAG_*                                                      */
+    uint32_t reserved;   /* must be 0                                                      */
+    void *const *stage_events; /* optional: KVC_STAGE_COUNT+1 cudaEvent_t (kvc_compress)  */
+} kvc_params;
+
+/*
+ * kvc_workspace_size -- bytes of device workspace that kvc_score / kvc_compress need for
+ * these parameters.  Host only; enqueues nothing.
+ */
+KVC_API kvc_status kvc_workspace_size(const kvc_params *p, size_t *bytes);
+
+/*
+ * kvc_score -- saliency scores (the definition above), summed over window queries, the
+ * GQA group and the n_layers layers; for KVC_SCOPE_ALL_HEADS also over all KV heads.
+ *   q       device, [n_layers, B, Hq, window, D]   dtype   (post-RoPE window queries)
+ *   k       device, [n_layers, B, Hkv, N, D]       dtype   (post-RoPE keys)
+ *   scores  device, [B, Hs, N] fp32, written; Hs = Hkv (PER_KV_HEAD) or 1 (ALL_HEADS).
+ *           Every position gets its score, window keys included.
+ *   ws      device workspace of >= kvc_workspace_size(p) bytes.
+ * Sources: FastKV sec. 2A (saliency), StructKV sec. 1 (sum over layers).
+ */
+KVC_API kvc_status kvc_score(const kvc_params *p, const void *q, const void *k, float *scores,
+                     void *ws, size_t ws_bytes, kvc_stream_t stream);
+
+/*
+ * kvc_accumulate -- acc[b, o, j] += sum_{r < Hi/Ho} src[b, o*(Hi/Ho) + r, j].
+ *   acc  device [B, Ho, N] fp32, read and written;  src  device [B, Hi, N] fp32.
+ *   Hi % Ho == 0.  The sum runs in a fixed order (deterministic).
+ * Source: StructKV sec. 1 (cumulative sums over heads/layers); FastKV sec. 2A (TSP uses
+ * one head-summed score per token).
+ */
+KVC_API kvc_status kvc_accumulate(float *acc, const float *src, int32_t B, int32_t Hi, int32_t Ho,
+                          int32_t N, kvc_stream_t stream);
+
+/*
+ * kvc_pool -- 1-D max-pool over [lo, hi) with odd width `kernel`, edges clipped:
+ *   out[r, j] = max{ in[r, t] : lo <= t < hi, |t - j| <= (kernel-1)/2 }  for lo <= j < hi,
+ *   out[r, j] = in[r, j]                                                  otherwise.
+ *   in, out  device [B, H, N] fp32 (distinct buffers).  0 <= lo <= hi <= N.
+ */
+KVC_API kvc_status kvc_pool(const float *in, float *out, int32_t B, int32_t H, int32_t N, int32_t lo,
+                    int32_t hi, int32_t kernel, kvc_stream_t stream);
+
+/*
+ * kvc_topk_workspace_size -- device workspace of kvc_topk for B*H rows of length N.
+ */
+KVC_API kvc_status kvc_topk_workspace_size(int32_t B, int32_t H, int32_t N, size_t *bytes);
+
+/*
+ * kvc_topk -- per row of `pooled`: keep the k_sel = budget - n_sink - window largest values
+ * among positions [n_sink, N - window) (equal values: lower position first), add the
+ * positions [0, n_sink) and [N - window, N), and write the `budget` kept positions in
+ * ascending order.  Values must not be NaN; -0.0 ranks equal to +0.0.
+ *   pooled  device [B, H, N] fp32;   idx  device [B, H, budget] int32, written.
+ *   Requires n_sink >= 0, window >= 0, n_sink + window + 1 <= budget <= N (else
+ *   KVC_ERR_BUDGET).
+ * Source: CentroidKV "Probleemstelling" (eviction by attention score) and "Inferentie
+ * Pipeline" (sinks and recent tokens preserved); FastKV sec. 2A (recent window).
+ */
+KVC_API kvc_status kvc_topk(const float *pooled, int32_t B, int32_t H, int32_t N, int32_t n_sink,
+                    int32_t window, int32_t budget, int32_t *idx, void *ws, size_t ws_bytes,
+                    kvc_stream_t stream);
+
+/*
+ * kvc_gather -- dst[b, h, r, :] = src[b, h, idx[b, h', r], :] as raw bytes, with h' = h
+ * when Hidx == Hsrc and h' = 0 when Hidx == 1 (one index list shared by all heads).
+ *   src  device [B, Hsrc, N, row_bytes];  idx  device [B, Hidx, K] int32;
+ *   dst  device [B, Hsrc, K, row_bytes], written.  row_bytes % 16 == 0.
+ * An index outside [0, N) leaves its destination row zero-filled and makes the next
+ * kvc_poll_error return KVC_ERR_INDEX.
+ * Source: FastKV sec. 2B (KV entries kept per layer), sec. 2A (propagated rows).
+ */
+KVC_API kvc_status kvc_gather(const void *src, int32_t B, int32_t Hsrc, int32_t N, size_t row_bytes,
+                      const int32_t *idx, int32_t Hidx, int32_t K, void *dst,
+                      kvc_stream_t stream);
+
+/*
+ * kvc_compress -- the whole path: score -> (head/layer sums) -> pool -> top-k -> gather.
+ *   q, k      as in kvc_score (all n_layers layers are scored).
+ *   v         device [B, Hkv, N, D] dtype: the values of the LAST layer in k.
+ *   k_out     device [B, Hkv, kv_budget, D], v_out likewise: rows of the last layer's K
+ *             and of v at the kept positions.
+ *   idx_out   device [B, Hs, kv_budget] int32 kept positions (Hs as in kvc_score; with
+ *             KVC_SCOPE_ALL_HEADS one list is shared by all KV heads).
+ *   TSP (tsp_rate > 0; otherwise hidden, hidden_out and tsp_idx_out must be NULL):
+ *   hidden    device [B, N, hidden_dim] dtype;
+ *   tsp_idx_out device [B, 1, kvc_tsp_count(N, window, n_sink, tsp_rate)] int32: kept
+ *             positions of the head-summed (all KV heads) pooled scores;
+ *   hidden_out device [B, kvc_tsp_count(...), hidden_dim]: the propagated rows.
+ *   ws        device workspace of >= kvc_workspace_size(p) bytes.
+ * Sources: all of the above.
+ */
+KVC_API kvc_status kvc_compress(const kvc_params *p, const void *q, const void *k, const void *v,
+                        void *k_out, void *v_out, int32_t *idx_out, const void *hidden,
+                        void *hidden_out, int32_t *tsp_idx_out, void *ws, size_t ws_bytes,
+                        kvc_stream_t stream);
+
+/*
+ * kvc_tsp_count -- rows propagated by TSP: min(floor(tsp_rate * N), N - window - n_sink)
+ * selected tokens plus n_sink + window; 0 when tsp_rate <= 0 or floor(tsp_rate*N) < 1.
+ * Source: FastKV sec. 2B (the TSP rate sets how many tokens continue past the TSP layer).
+ */
+KVC_API int32_t kvc_tsp_count(int32_t N, int32_t window, int32_t n_sink, float tsp_rate);
+
+/*
+ * kvc_poll_error -- synchronises `stream`, then returns (and clears) the first device-side
+ * problem recorded since the last poll on this device: KVC_ERR_TIMEOUT, KVC_ERR_INDEX, or
+ * KVC_OK.  KVC_ERR_CUDA if the synchronisation itself failed.
+ */
+KVC_API kvc_status kvc_poll_error(kvc_stream_t stream);
+
+/*
+ * kvc_launch_count -- number of CUDA kernels this library has launched in this process
+ * (all devices, all threads), for diagnostics and benchmarks.  Host only.
+ */
+KVC_API uint64_t kvc_launch_count(void);
+
+/* kvc_status_string -- static description of a status code (never NULL). */
+KVC_API const char *kvc_status_string(kvc_status status);
+
+/* kvc_version -- library version string, e.g. "kvc 0.1.0 sm_100a". */
+KVC_API const char *kvc_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVC_H */

@@ -1,0 +1,350 @@
+// api.cu -- the C ABI of libkvc.so: argument validation, workspace layout and the
+// launch sequence of each entry point.  See include/kvc.h for the contracts.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <atomic>
+
+#include "kvc_internal.cuh"
+
+namespace kvc {
+
+static __device__ unsigned int g_error_word;
+static std::atomic<unsigned long long> g_launches{0};
+
+void count_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+
+unsigned int* device_error_word() {
+    // one address per device; cudaGetSymbolAddress is cheap but not free
+    static unsigned int* cache[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return nullptr;
+    if (dev < 64 && cache[dev]) return cache[dev];
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
+    if (dev < 64) cache[dev] = (unsigned int*)p;
+    return (unsigned int*)p;
+}
+
+}  // namespace kvc
+
+using namespace kvc;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+size_t esize(int dtype) { return dtype == KVC_F32 ? 4 : 2; }
+
+// Workspace layout of one call.
+struct Plan {
+    int U = 0, nq = 0, Hs = 0, n_tsp = 0;
+    bool units = false;  // unit scores need a reduction (several layers or all heads)
+    bool use_tc = false;
+    int n_chunks = 0, chunk = 0;
+    size_t off_partial = 0, off_lse = 0, off_units = 0, off_scores = 0, off_pooled = 0;
+    size_t off_tsp_scores = 0, off_tsp_pooled = 0, off_tc = 0, tc_bytes = 0, total = 0;
+};
+
+kvc_status check_params(const kvc_params* p) {
+    if (!p) return KVC_ERR_ARG;
+    if (p->reserved != 0) return KVC_ERR_ARG;
+    if (p->B < 1 || p->Hq < 1 || p->Hkv < 1 || p->N < 1 || p->window < 1 || p->n_layers < 1)
+        return KVC_ERR_ARG;
+    if (p->Hq % p->Hkv) return KVC_ERR_ARG;
+    if (p->D != kHeadDim) return KVC_ERR_UNSUPPORTED;
+    if (p->dtype != KVC_F32 && p->dtype != KVC_BF16) return KVC_ERR_UNSUPPORTED;
+    if (p->scope != KVC_SCOPE_PER_KV_HEAD && p->scope != KVC_SCOPE_ALL_HEADS) return KVC_ERR_UNSUPPORTED;
+    if ((long long)(p->Hq / p->Hkv) * p->window > 256) return KVC_ERR_UNSUPPORTED;
+    if (p->n_sink < 0 || p->window >= p->N) return KVC_ERR_ARG;
+    if (p->pool_kernel < 1 || p->pool_kernel % 2 == 0) return KVC_ERR_ARG;
+    if (!(p->tsp_rate >= 0.f) || p->spin_limit < 0) return KVC_ERR_ARG;
+    // every unit's K block must be addressable with 64-bit offsets and N fits int32
+    if ((long long)p->n_layers * p->B * p->Hkv > (1LL << 30)) return KVC_ERR_ARG;
+    return KVC_OK;
+}
+
+kvc_status check_budget(int N, int S, int w, int budget) {
+    if ((long long)S + w + 1 > budget || budget > N) return KVC_ERR_BUDGET;
+    return KVC_OK;
+}
+
+ScoreJob make_job(const kvc_params* p, const void* q, const void* k) {
+    ScoreJob j{};
+    j.q = q;
+    j.k = k;
+    j.dtype = p->dtype;
+    j.U = p->n_layers * p->B * p->Hkv;
+    j.N = p->N;
+    j.window = p->window;
+    j.G = p->Hq / p->Hkv;
+    j.nq = j.G * p->window;
+    j.spin_limit = p->spin_limit > 0 ? p->spin_limit : (1LL << 26);
+    return j;
+}
+
+// Fills `pl` for kvc_score (compress = false) or kvc_compress (compress = true).
+void make_plan(const kvc_params* p, bool compress, Plan* pl) {
+    Plan P;
+    const ScoreJob job = make_job(p, nullptr, nullptr);
+    P.U = job.U;
+    P.nq = job.nq;
+    P.Hs = p->scope == KVC_SCOPE_PER_KV_HEAD ? p->Hkv : 1;
+    P.units = p->n_layers > 1 || p->scope == KVC_SCOPE_ALL_HEADS;
+    P.use_tc = !(p->flags & KVC_FLAG_SIMT_SCORE) && tc_score_supported(job);
+    P.n_tsp = kvc_tsp_count(p->N, p->window, p->n_sink, p->tsp_rate);
+    size_t off = 0;
+    if (P.use_tc) {
+        P.tc_bytes = tc_score_workspace(P.U, p->N, P.nq);
+        P.off_tc = off;
+        off = align_up(off + P.tc_bytes);
+    } else {
+        const size_t pb = simt_score_workspace(P.U, p->N, P.nq, &P.n_chunks, &P.chunk);
+        P.off_partial = off;
+        off = align_up(off + pb);
+    }
+    P.off_lse = off;
+    off = align_up(off + (size_t)P.U * P.nq * sizeof(float));
+    const size_t row = (size_t)p->N * sizeof(float);
+    if (P.units) {
+        P.off_units = off;
+        off = align_up(off + (size_t)P.U * row);
+    }
+    if (compress) {
+        P.off_scores = off;
+        off = align_up(off + (size_t)p->B * P.Hs * row);
+        P.off_pooled = off;
+        off = align_up(off + (size_t)p->B * P.Hs * row);
+        if (p->tsp_rate > 0.f) {
+            P.off_tsp_scores = off;
+            off = align_up(off + (size_t)p->B * row);
+            P.off_tsp_pooled = off;
+            off = align_up(off + (size_t)p->B * row);
+        }
+    }
+    P.total = off;
+    *pl = P;
+}
+
+// Runs the scoring stage: unit scores (and their reduction) into `scores` [B, Hs, N].
+kvc_status run_score(const kvc_params* p, const Plan& P, const void* q, const void* k, float* scores,
+                     char* ws, cudaStream_t s) {
+    ScoreJob job = make_job(p, q, k);
+    job.unit_scores = P.units ? (float*)(ws + P.off_units) : scores;
+    job.lse = (float*)(ws + P.off_lse);
+    job.err = device_error_word();
+    if (!job.err) return KVC_ERR_CUDA;
+    cudaError_t e;
+    if (P.use_tc) {
+        job.tc_ws = ws + P.off_tc;
+        job.tc_ws_bytes = P.tc_bytes;
+        e = tc_score(job, s);
+    } else {
+        job.partial = (float2*)(ws + P.off_partial);
+        job.n_chunks = P.n_chunks;
+        job.chunk = P.chunk;
+        e = simt_score(job, s);
+    }
+    if (e != cudaSuccess) return KVC_ERR_CUDA;
+    if (P.units) {
+        e = reduce_units(job.unit_scores, p->n_layers, p->B, p->Hkv, p->N,
+                         p->scope == KVC_SCOPE_ALL_HEADS, scores, s);
+        if (e != cudaSuccess) return KVC_ERR_CUDA;
+    }
+    return KVC_OK;
+}
+
+kvc_status record_stage(const kvc_params* p, int i, cudaStream_t s) {
+    if (!p->stage_events || !p->stage_events[i]) return KVC_OK;
+    return cudaEventRecord((cudaEvent_t)p->stage_events[i], s) == cudaSuccess ? KVC_OK : KVC_ERR_CUDA;
+}
+
+#define KVC_TRY(x)                         \
+    do {                                   \
+        kvc_status st_ = (x);              \
+        if (st_ != KVC_OK) return st_;     \
+    } while (0)
+#define KVC_CUDA(x)                                      \
+    do {                                                 \
+        if ((x) != cudaSuccess) return KVC_ERR_CUDA;     \
+    } while (0)
+
+}  // namespace
+
+extern "C" {
+
+kvc_status kvc_workspace_size(const kvc_params* p, size_t* bytes) {
+    if (!bytes) return KVC_ERR_ARG;
+    KVC_TRY(check_params(p));
+    Plan P;
+    make_plan(p, true, &P);
+    *bytes = P.total;
+    return KVC_OK;
+}
+
+kvc_status kvc_score(const kvc_params* p, const void* q, const void* k, float* scores, void* ws,
+                     size_t ws_bytes, kvc_stream_t stream) {
+    KVC_TRY(check_params(p));
+    if (!q || !k || !scores || !ws) return KVC_ERR_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(scores) || ((uintptr_t)ws & (kAlign - 1)))
+        return KVC_ERR_ALIGN;
+    Plan P;
+    make_plan(p, false, &P);
+    if (ws_bytes < P.total) return KVC_ERR_WORKSPACE;
+    return run_score(p, P, q, k, scores, (char*)ws, (cudaStream_t)stream);
+}
+
+kvc_status kvc_accumulate(float* acc, const float* src, int32_t B, int32_t Hi, int32_t Ho, int32_t N,
+                          kvc_stream_t stream) {
+    if (!acc || !src || B < 1 || Hi < 1 || Ho < 1 || N < 0 || Hi % Ho) return KVC_ERR_ARG;
+    KVC_CUDA(kvc::accumulate(acc, src, B, Hi, Ho, N, (cudaStream_t)stream));
+    return KVC_OK;
+}
+
+kvc_status kvc_pool(const float* in, float* out, int32_t B, int32_t H, int32_t N, int32_t lo,
+                    int32_t hi, int32_t kernel, kvc_stream_t stream) {
+    if (!in || !out || in == out || B < 1 || H < 1 || N < 0) return KVC_ERR_ARG;
+    if (lo < 0 || hi > N || lo > hi || kernel < 1 || kernel % 2 == 0) return KVC_ERR_ARG;
+    KVC_CUDA(kvc::pool(in, out, B * H, N, lo, hi, kernel, (cudaStream_t)stream));
+    return KVC_OK;
+}
+
+kvc_status kvc_topk_workspace_size(int32_t B, int32_t H, int32_t N, size_t* bytes) {
+    if (!bytes || B < 1 || H < 1 || N < 1) return KVC_ERR_ARG;
+    *bytes = 0;
+    return KVC_OK;
+}
+
+kvc_status kvc_topk(const float* pooled, int32_t B, int32_t H, int32_t N, int32_t n_sink,
+                    int32_t window, int32_t budget, int32_t* idx, void* ws, size_t ws_bytes,
+                    kvc_stream_t stream) {
+    (void)ws;
+    (void)ws_bytes;
+    if (!pooled || !idx || B < 1 || H < 1 || N < 1 || n_sink < 0 || window < 0) return KVC_ERR_ARG;
+    KVC_TRY(check_budget(N, n_sink, window, budget));
+    KVC_CUDA(kvc::topk(pooled, B * H, N, n_sink, window, budget, idx, (cudaStream_t)stream));
+    return KVC_OK;
+}
+
+kvc_status kvc_gather(const void* src, int32_t B, int32_t Hsrc, int32_t N, size_t row_bytes,
+                      const int32_t* idx, int32_t Hidx, int32_t K, void* dst, kvc_stream_t stream) {
+    if (!src || !idx || !dst || B < 1 || Hsrc < 1 || N < 1 || K < 0 || row_bytes == 0) return KVC_ERR_ARG;
+    if (Hidx != 1 && Hidx != Hsrc) return KVC_ERR_ARG;
+    if (row_bytes % 16 || !aligned16(src) || !aligned16(dst)) return KVC_ERR_ALIGN;
+    unsigned* err = device_error_word();
+    if (!err) return KVC_ERR_CUDA;
+    KVC_CUDA(kvc::gather(src, dst, nullptr, nullptr, B, Hsrc, N, row_bytes, idx, Hidx, K, err,
+                         (cudaStream_t)stream));
+    return KVC_OK;
+}
+
+kvc_status kvc_compress(const kvc_params* p, const void* q, const void* k, const void* v, void* k_out,
+                        void* v_out, int32_t* idx_out, const void* hidden, void* hidden_out,
+                        int32_t* tsp_idx_out, void* ws, size_t ws_bytes, kvc_stream_t stream) {
+    KVC_TRY(check_params(p));
+    if (!q || !k || !v || !k_out || !v_out || !idx_out || !ws) return KVC_ERR_ARG;
+    const bool tsp = p->tsp_rate > 0.f;
+    if (tsp) {
+        if (!hidden || !hidden_out || !tsp_idx_out || p->hidden_dim < 1) return KVC_ERR_ARG;
+    } else if (hidden || hidden_out || tsp_idx_out) {
+        return KVC_ERR_ARG;
+    }
+    KVC_TRY(check_budget(p->N, p->n_sink, p->window, p->kv_budget));
+    Plan P;
+    make_plan(p, true, &P);
+    if (tsp && P.n_tsp == 0) return KVC_ERR_BUDGET;
+    const void* ptrs[] = {q, k, v, k_out, v_out, idx_out, hidden, hidden_out, tsp_idx_out};
+    for (const void* ptr : ptrs)
+        if (ptr && !aligned16(ptr)) return KVC_ERR_ALIGN;
+    if ((uintptr_t)ws & (kAlign - 1)) return KVC_ERR_ALIGN;
+    if (tsp && ((size_t)p->hidden_dim * esize(p->dtype)) % 16) return KVC_ERR_ALIGN;
+    if (ws_bytes < P.total) return KVC_ERR_WORKSPACE;
+    unsigned* err = device_error_word();
+    if (!err) return KVC_ERR_CUDA;
+
+    cudaStream_t s = (cudaStream_t)stream;
+    char* w = (char*)ws;
+    const int N = p->N, S = p->n_sink, win = p->window, B = p->B, Hkv = p->Hkv;
+    float* scores = (float*)(w + P.off_scores);
+    float* pooled = (float*)(w + P.off_pooled);
+
+    KVC_TRY(record_stage(p, KVC_STAGE_SCORE, s));
+    KVC_TRY(run_score(p, P, q, k, scores, w, s));
+
+    KVC_TRY(record_stage(p, KVC_STAGE_SELECT, s));
+    KVC_CUDA(kvc::pool(scores, pooled, B * P.Hs, N, S, N - win, p->pool_kernel, s));
+    KVC_CUDA(kvc::topk(pooled, B * P.Hs, N, S, win, p->kv_budget, idx_out, s));
+    float* tsp_pooled = nullptr;
+    if (tsp) {
+        float* tsp_scores = (float*)(w + P.off_tsp_scores);
+        tsp_pooled = (float*)(w + P.off_tsp_pooled);
+        const float* src = scores;
+        if (P.Hs > 1) {
+            KVC_CUDA(cudaMemsetAsync(tsp_scores, 0, (size_t)B * N * sizeof(float), s));
+            KVC_CUDA(kvc::accumulate(tsp_scores, scores, B, P.Hs, 1, N, s));
+            src = tsp_scores;
+        }
+        KVC_CUDA(kvc::pool(src, tsp_pooled, B, N, S, N - win, p->pool_kernel, s));
+        KVC_CUDA(kvc::topk(tsp_pooled, B, N, S, win, P.n_tsp, tsp_idx_out, s));
+    }
+
+    KVC_TRY(record_stage(p, KVC_STAGE_GATHER, s));
+    const size_t row = (size_t)p->D * esize(p->dtype);
+    const char* k_last = (const char*)k + (size_t)(p->n_layers - 1) * B * Hkv * N * row;
+    KVC_CUDA(kvc::gather(k_last, k_out, v, v_out, B, Hkv, N, row, idx_out, P.Hs, p->kv_budget, err, s));
+    if (tsp) {
+        KVC_CUDA(kvc::gather(hidden, hidden_out, nullptr, nullptr, B, 1, N,
+                             (size_t)p->hidden_dim * esize(p->dtype), tsp_idx_out, 1, P.n_tsp, err, s));
+    }
+    KVC_TRY(record_stage(p, KVC_STAGE_COUNT, s));
+    return KVC_OK;
+}
+
+int32_t kvc_tsp_count(int32_t N, int32_t window, int32_t n_sink, float tsp_rate) {
+    if (!(tsp_rate > 0.f) || N < 1) return 0;
+    long long sel = (long long)floor((double)tsp_rate * (double)N);
+    const long long n_c = (long long)N - window - n_sink;
+    if (sel > n_c) sel = n_c;
+    if (sel < 1) return 0;
+    return (int32_t)(sel + n_sink + window);
+}
+
+kvc_status kvc_poll_error(kvc_stream_t stream) {
+    unsigned* err = device_error_word();
+    if (!err) return KVC_ERR_CUDA;
+    unsigned h = 0;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return KVC_ERR_CUDA;
+    if (cudaMemcpy(&h, err, sizeof h, cudaMemcpyDeviceToHost) != cudaSuccess) return KVC_ERR_CUDA;
+    if (h) {
+        const unsigned zero = 0;
+        if (cudaMemcpy(err, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess) return KVC_ERR_CUDA;
+    }
+    if (h & kErrTimeout) return KVC_ERR_TIMEOUT;
+    if (h & kErrIndex) return KVC_ERR_INDEX;
+    return KVC_OK;
+}
+
+const char* kvc_status_string(kvc_status st) {
+    switch (st) {
+        case KVC_OK: return "ok";
+        case KVC_ERR_ARG: return "invalid argument (null pointer or bad shape)";
+        case KVC_ERR_UNSUPPORTED: return "unsupported configuration (head dim, dtype, scope or window size)";
+        case KVC_ERR_BUDGET: return "budget out of range (needs n_sink + window + 1 <= budget <= N)";
+        case KVC_ERR_ALIGN: return "misaligned pointer or row size (16 bytes; workspace 256 bytes)";
+        case KVC_ERR_WORKSPACE: return "workspace too small";
+        case KVC_ERR_CUDA: return "CUDA runtime error";
+        case KVC_ERR_TIMEOUT: return "a device-side bounded wait gave up";
+        case KVC_ERR_INDEX: return "gather index out of range";
+    }
+    return "unknown status";
+}
+
+uint64_t kvc_launch_count(void) { return (uint64_t)g_launches.load(std::memory_order_relaxed); }
+
+const char* kvc_version(void) { return "kvc 0.1.0 sm_100a"; }
+
+}  // extern "C"

@@ -1,0 +1,74 @@
+// kvc_internal.cuh -- declarations shared by the translation units of libkvc.so.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kvc.h"
+
+namespace kvc {
+
+constexpr int kHeadDim = 128;  // D: the only head dimension the kernels are built for
+
+// bits of the per-device error word (see kvc_poll_error)
+constexpr unsigned kErrTimeout = 1u;
+constexpr unsigned kErrIndex = 2u;
+
+// counts kernel launches issued by the library (kvc_launch_count)
+void count_launches(int n);
+
+// per-device error word, set by kernels with atomicOr, read and cleared by kvc_poll_error
+unsigned int* device_error_word();
+
+// log2(e) / sqrt(128): logits are taken to base 2 so that exp becomes exp2
+constexpr float kLog2eOverSqrtD = 0.12751743082459868f;
+
+// One scoring job: every (layer, batch, KV head) "unit" u = (layer*B + b)*Hkv + h.
+// Unit u reads the G*window query rows starting at q + u*G*window*D (heads h*G..h*G+G-1
+// are adjacent) and the N key rows starting at k + u*N*D.
+struct ScoreJob {
+    const void* q;
+    const void* k;
+    int dtype;
+    int U;        // units = n_layers * B * Hkv
+    int N;
+    int window;
+    int G;
+    int nq;       // G * window query rows per unit
+    float* unit_scores;  // [U][N] fp32 output (sum over the unit's query rows)
+    // workspace
+    float2* partial;     // SIMT: [U][n_chunks][nq] (m, l) partial softmax stats
+    float* lse;          // [U][nq] log2-sum-exp per query row
+    int n_chunks;
+    int chunk;
+    // tensor-core path
+    void* tc_ws;
+    size_t tc_ws_bytes;
+    unsigned* err;
+    long long spin_limit;
+};
+
+// CUDA-core (FFMA) scoring, fp32 or bf16 inputs
+size_t simt_score_workspace(int U, int N, int nq, int* n_chunks, int* chunk);
+cudaError_t simt_score(const ScoreJob& job, cudaStream_t s);
+
+// tensor-core scoring (bf16, tcgen05 + TMA); returns false if the shape is not supported
+bool tc_score_supported(const ScoreJob& job);
+size_t tc_score_workspace(int U, int N, int nq);
+cudaError_t tc_score(const ScoreJob& job, cudaStream_t s);
+
+// sums of unit scores over layers (and KV heads for the all-heads scope)
+cudaError_t reduce_units(const float* unit_scores, int L, int B, int Hkv, int N, int all_heads,
+                         float* out, cudaStream_t s);
+cudaError_t accumulate(float* acc, const float* src, int B, int Hi, int Ho, int N, cudaStream_t s);
+cudaError_t pool(const float* in, float* out, int rows, int N, int lo, int hi, int kernel,
+                 cudaStream_t s);
+cudaError_t topk(const float* pooled, int rows, int N, int n_sink, int window, int budget,
+                 int32_t* idx, cudaStream_t s);
+// two gathers of the same shape in one launch (src1/dst1 may be null)
+cudaError_t gather(const void* src0, void* dst0, const void* src1, void* dst1, int B, int Hsrc,
+                   int N, size_t row_bytes, const int32_t* idx, int Hidx, int K, unsigned* err,
+                   cudaStream_t s);
+
+}  // namespace kvc

@@ -1,0 +1,242 @@
+// select.cu -- score sums, 1-D max-pool and top-k selection of kept positions.
+//
+// Top-k is a radix select on order-preserving 32-bit keys of the pooled fp32 scores
+// (four 8-bit digits, most significant first), followed by a stable compaction that
+// writes the kept candidate positions in ascending order: every candidate above the
+// threshold value T, and the lowest-indexed candidates equal to T up to the budget.
+// Sinks [0, S) and the recent window [N - w, N) are written around them (CentroidKV page,
+// "Inferentie Pipeline": sinks and recent tokens are preserved; FastKV page, sec. 2A: the
+// selected tokens plus a window of the newest tokens).  One CTA of 1024 threads owns a
+// row; each warp owns a contiguous segment of it, so all loads are coalesced and the only
+// block-wide steps are the digit search and one scan of per-warp counts.
+#include "kvc_internal.cuh"
+
+namespace kvc {
+namespace {
+
+// ------------------------------------------------------------------------------- sums
+
+__global__ void reduce_units_kernel(const float* __restrict__ units, int L, int B, int Hkv, int N,
+                                    int all_heads, float* __restrict__ out) {
+    const int Hs = all_heads ? 1 : Hkv;
+    const long long total = (long long)B * Hs * N;
+    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
+         e += (long long)gridDim.x * blockDim.x) {
+        const int j = (int)(e % N);
+        const long long bh = e / N;
+        const int hs = (int)(bh % Hs);
+        const int b = (int)(bh / Hs);
+        const int h0 = all_heads ? 0 : hs, h1 = all_heads ? Hkv : hs + 1;
+        float s = 0.f;
+        for (int l = 0; l < L; ++l)
+            for (int h = h0; h < h1; ++h) s += units[(((size_t)l * B + b) * Hkv + h) * N + j];
+        out[e] = s;
+    }
+}
+
+__global__ void accumulate_kernel(float* __restrict__ acc, const float* __restrict__ src, int B,
+                                  int Hi, int Ho, int N) {
+    const int R = Hi / Ho;
+    const long long total = (long long)B * Ho * N;
+    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
+         e += (long long)gridDim.x * blockDim.x) {
+        const int j = (int)(e % N);
+        const long long bo = e / N;
+        const int o = (int)(bo % Ho);
+        const int b = (int)(bo / Ho);
+        float s = acc[e];
+        for (int r = 0; r < R; ++r) s += src[((size_t)b * Hi + o * R + r) * N + j];
+        acc[e] = s;
+    }
+}
+
+// ------------------------------------------------------------------------------- pool
+
+__global__ void pool_kernel(const float* __restrict__ in, float* __restrict__ out, int rows, int N,
+                            int lo, int hi, int radius) {
+    const long long total = (long long)rows * N;
+    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
+         e += (long long)gridDim.x * blockDim.x) {
+        const int j = (int)(e % N);
+        const float* r = in + (e - j);
+        float m;
+        if (j < lo || j >= hi) {
+            m = r[j];
+        } else {
+            const int t0 = max(lo, j - radius), t1 = min(hi - 1, j + radius);
+            m = r[t0];
+            for (int t = t0 + 1; t <= t1; ++t) m = fmaxf(m, r[t]);
+        }
+        out[e] = m;
+    }
+}
+
+// ------------------------------------------------------------------------------- top-k
+
+constexpr int kTopkThreads = 1024;
+constexpr int kWarps = kTopkThreads / 32;
+
+// Monotone map from fp32 to uint32 (larger value -> larger key); -0.0 maps like +0.0.
+__device__ __forceinline__ uint32_t order_key(float v) {
+    uint32_t b = __float_as_uint(v);
+    if (b == 0x80000000u) b = 0u;
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+    unsigned m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+__global__ void __launch_bounds__(kTopkThreads)
+topk_kernel(const float* __restrict__ pooled, int N, int S, int w, int budget,
+            int32_t* __restrict__ idx) {
+    __shared__ unsigned hist[kWarps][256];
+    __shared__ unsigned wsum[8];
+    __shared__ uint32_t s_prefix;
+    __shared__ int s_krem;
+    __shared__ int wcnt_gt[kWarps], wcnt_eq[kWarps];
+
+    const int row = blockIdx.x;
+    const float* v = pooled + (size_t)row * N;
+    int32_t* out = idx + (size_t)row * budget;
+    const int lo = S, hi = N - w, k_sel = budget - S - w;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // warp `warp` owns candidates [seg0, seg1)
+    const int n_c = hi - lo;
+    const int seg = (n_c + kWarps - 1) / kWarps;
+    const int seg0 = lo + min(n_c, warp * seg), seg1 = lo + min(n_c, (warp + 1) * seg);
+
+    for (int i = tid; i < S; i += kTopkThreads) out[i] = i;
+    for (int i = tid; i < w; i += kTopkThreads) out[budget - w + i] = N - w + i;
+
+    if (tid == 0) {
+        s_prefix = 0u;
+        s_krem = k_sel;
+    }
+    uint32_t prefix = 0, mask = 0;
+    int krem = k_sel;
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        for (int i = tid; i < kWarps * 256; i += kTopkThreads) (&hist[0][0])[i] = 0u;
+        __syncthreads();
+        for (int j = seg0 + lane; j < seg1; j += 32) {
+            const uint32_t key = order_key(v[j]);
+            if ((key & mask) == prefix) {
+                const unsigned digit = (key >> shift) & 255u;
+                const unsigned peers = __match_any_sync(__activemask(), digit);
+                if (lane == __ffs(peers) - 1) atomicAdd(&hist[warp][digit], (unsigned)__popc(peers));
+            }
+        }
+        __syncthreads();
+        // bins are scanned from the top: incl(d) = #keys with digit >= d
+        unsigned incl = 0, tot = 0;
+        if (tid < 256) {
+            for (int wi = 0; wi < kWarps; ++wi) tot += hist[wi][tid];
+            incl = tot;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const unsigned y = __shfl_down_sync(0xffffffffu, incl, off);
+                if (lane + off < 32) incl += y;
+            }
+            if (lane == 0) wsum[warp] = incl;
+        }
+        __syncthreads();
+        if (tid < 256) {
+            for (int wi = warp + 1; wi < 8; ++wi) incl += wsum[wi];
+            const unsigned excl = incl - tot;
+            if (excl < (unsigned)krem && (unsigned)krem <= incl) {
+                s_prefix = prefix | ((uint32_t)tid << shift);
+                s_krem = krem - (int)excl;
+            }
+        }
+        __syncthreads();
+        prefix = s_prefix;
+        krem = s_krem;
+        mask |= 255u << shift;
+    }
+    const uint32_t T = prefix;  // the k_sel-th largest key; take krem of the keys equal to T
+
+    // counts per warp segment
+    int n_gt = 0, n_eq = 0;
+    for (int j = seg0 + lane; j < seg1; j += 32) {
+        const uint32_t key = order_key(v[j]);
+        n_gt += key > T;
+        n_eq += key == T;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        n_gt += __shfl_xor_sync(0xffffffffu, n_gt, off);
+        n_eq += __shfl_xor_sync(0xffffffffu, n_eq, off);
+    }
+    if (lane == 0) {
+        wcnt_gt[warp] = n_gt;
+        wcnt_eq[warp] = n_eq;
+    }
+    __syncthreads();
+    int gt_before = 0, eq_before = 0;
+    for (int wi = 0; wi < warp; ++wi) {
+        gt_before += wcnt_gt[wi];
+        eq_before += wcnt_eq[wi];
+    }
+    // stable compaction in position order
+    int taken = gt_before + min(eq_before, krem);
+    int eq_seen = eq_before;
+    for (int base = seg0; base < seg1; base += 32) {
+        const int j = base + lane;
+        const uint32_t key = j < seg1 ? order_key(v[j]) : 0u;
+        const bool gt = j < seg1 && key > T;
+        const bool eq = j < seg1 && key == T;
+        const unsigned eq_mask = __ballot_sync(0xffffffffu, eq);
+        const bool take = gt || (eq && eq_seen + __popc(eq_mask & lanemask_lt()) < krem);
+        const unsigned take_mask = __ballot_sync(0xffffffffu, take);
+        const int pos = taken + __popc(take_mask & lanemask_lt());
+        if (take && pos < k_sel) out[S + pos] = j;  // pos < k_sel always holds; kept as a guard
+        taken += __popc(take_mask);
+        eq_seen += __popc(eq_mask);
+    }
+}
+
+int grid_for(long long total, int threads) {
+    long long g = (total + threads - 1) / threads;
+    if (g > 148LL * 32) g = 148LL * 32;
+    return (int)(g < 1 ? 1 : g);
+}
+
+}  // namespace
+
+cudaError_t reduce_units(const float* units, int L, int B, int Hkv, int N, int all_heads, float* out,
+                         cudaStream_t s) {
+    const long long total = (long long)B * (all_heads ? 1 : Hkv) * N;
+    reduce_units_kernel<<<grid_for(total, 256), 256, 0, s>>>(units, L, B, Hkv, N, all_heads, out);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t accumulate(float* acc, const float* src, int B, int Hi, int Ho, int N, cudaStream_t s) {
+    const long long total = (long long)B * Ho * N;
+    if (total == 0) return cudaSuccess;
+    accumulate_kernel<<<grid_for(total, 256), 256, 0, s>>>(acc, src, B, Hi, Ho, N);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t pool(const float* in, float* out, int rows, int N, int lo, int hi, int kernel,
+                 cudaStream_t s) {
+    const long long total = (long long)rows * N;
+    if (total == 0) return cudaSuccess;
+    pool_kernel<<<grid_for(total, 256), 256, 0, s>>>(in, out, rows, N, lo, hi, (kernel - 1) / 2);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t topk(const float* pooled, int rows, int N, int n_sink, int window, int budget,
+                 int32_t* idx, cudaStream_t s) {
+    if (rows == 0) return cudaSuccess;
+    topk_kernel<<<rows, kTopkThreads, 0, s>>>(pooled, N, n_sink, window, budget, idx);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace kvc

@@ -1,0 +1,241 @@
+"""ctypes binding of libkvc.so (include/kvc.h).
+
+Argument marshalling only: every step of the compaction runs in the library's CUDA
+kernels.  PyTorch supplies device memory and the current stream.  Importing this module
+loads the in-tree libkvc.so and raises if it is missing; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkvc.so")
+
+KVC_OK, KVC_ERR_ARG, KVC_ERR_UNSUPPORTED, KVC_ERR_BUDGET, KVC_ERR_ALIGN = 0, 1, 2, 3, 4
+KVC_ERR_WORKSPACE, KVC_ERR_CUDA, KVC_ERR_TIMEOUT, KVC_ERR_INDEX = 5, 6, 7, 8
+KVC_F32, KVC_BF16 = 0, 1
+KVC_SCOPE_PER_KV_HEAD, KVC_SCOPE_ALL_HEADS = 0, 1
+KVC_FLAG_SIMT_SCORE = 1
+KVC_STAGE_SCORE, KVC_STAGE_SELECT, KVC_STAGE_GATHER, KVC_STAGE_COUNT = 0, 1, 2, 3
+
+EXPORTED = ("kvc_workspace_size", "kvc_score", "kvc_accumulate", "kvc_pool", "kvc_topk_workspace_size",
+            "kvc_topk", "kvc_gather", "kvc_compress", "kvc_tsp_count", "kvc_poll_error",
+            "kvc_status_string", "kvc_version", "kvc_launch_count")
+
+
+class KvcError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {kvc_status_string(status)} (status {status})")
+
+
+class Params(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("N", ctypes.c_int32),
+        ("D", ctypes.c_int32), ("window", ctypes.c_int32), ("dtype", ctypes.c_int32),
+        ("n_sink", ctypes.c_int32), ("pool_kernel", ctypes.c_int32), ("kv_budget", ctypes.c_int32),
+        ("scope", ctypes.c_int32), ("n_layers", ctypes.c_int32), ("tsp_rate", ctypes.c_float),
+        ("hidden_dim", ctypes.c_int32), ("spin_limit", ctypes.c_int64), ("flags", ctypes.c_uint32),
+        ("reserved", ctypes.c_uint32), ("stage_events", ctypes.POINTER(ctypes.c_void_p)),
+    ]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python -m long_context_kv_kvc_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, vp, i32, sz, st = ctypes.POINTER(Params), ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.c_int
+    sig = {
+        "kvc_workspace_size": (st, [P, ctypes.POINTER(sz)]),
+        "kvc_score": (st, [P, vp, vp, vp, vp, sz, vp]),
+        "kvc_accumulate": (st, [vp, vp, i32, i32, i32, i32, vp]),
+        "kvc_pool": (st, [vp, vp, i32, i32, i32, i32, i32, i32, vp]),
+        "kvc_topk_workspace_size": (st, [i32, i32, i32, ctypes.POINTER(sz)]),
+        "kvc_topk": (st, [vp, i32, i32, i32, i32, i32, i32, vp, vp, sz, vp]),
+        "kvc_gather": (st, [vp, i32, i32, i32, sz, vp, i32, i32, vp, vp]),
+        "kvc_compress": (st, [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "kvc_tsp_count": (i32, [i32, i32, i32, ctypes.c_float]),
+        "kvc_poll_error": (st, [vp]),
+        "kvc_status_string": (ctypes.c_char_p, [st]),
+        "kvc_version": (ctypes.c_char_p, []),
+        "kvc_launch_count": (ctypes.c_uint64, []),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype, f.argtypes = res, args
+    return L
+
+
+lib = _load()
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(st: int, what: str):
+    if st != KVC_OK:
+        raise KvcError(st, what)
+
+
+def dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.float32:
+        return KVC_F32
+    if dt == torch.bfloat16:
+        return KVC_BF16
+    raise ValueError(f"unsupported dtype {dt}")
+
+
+def make_params(*, B, Hq, Hkv, N, window, dtype, n_sink=1, pool_kernel=7, kv_budget, D=128,
+                scope=KVC_SCOPE_PER_KV_HEAD, n_layers=1, tsp_rate=0.0, hidden_dim=0, spin_limit=0,
+                flags=0) -> Params:
+    p = Params()
+    p.B, p.Hq, p.Hkv, p.N, p.D, p.window = B, Hq, Hkv, N, D, window
+    p.dtype = dtype if isinstance(dtype, int) else dtype_code(dtype)
+    p.n_sink, p.pool_kernel, p.kv_budget, p.scope, p.n_layers = n_sink, pool_kernel, kv_budget, scope, n_layers
+    p.tsp_rate, p.hidden_dim, p.spin_limit, p.flags, p.reserved = tsp_rate, hidden_dim, spin_limit, flags, 0
+    p.stage_events = None
+    return p
+
+
+def params_for(wl, **overrides) -> Params:
+    """Parameters of a synth.Workload (same field names)."""
+    kw = dict(B=wl.B, Hq=wl.Hq, Hkv=wl.Hkv, N=wl.N, D=wl.D, window=wl.window,
+              dtype=KVC_F32 if wl.dtype == "f32" else KVC_BF16, n_sink=wl.n_sink,
+              pool_kernel=wl.pool_kernel, kv_budget=wl.kv_budget, scope=wl.scope,
+              n_layers=wl.n_layers, tsp_rate=wl.tsp_rate, hidden_dim=wl.hidden_dim)
+    kw.update(overrides)
+    return make_params(**kw)
+
+
+# ------------------------------------------------------------------------ entry points
+
+def kvc_workspace_size(p: Params) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib.kvc_workspace_size(ctypes.byref(p), ctypes.byref(n)), "kvc_workspace_size")
+    return n.value
+
+
+def kvc_score(p: Params, q, k, scores, ws, stream=None):
+    _check(lib.kvc_score(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(scores), _ptr(ws),
+                         ws.numel() * ws.element_size(), _stream(stream)), "kvc_score")
+
+
+def kvc_accumulate(acc, src, stream=None):
+    B, Ho, N = acc.shape
+    Hi = src.shape[1]
+    _check(lib.kvc_accumulate(_ptr(acc), _ptr(src), B, Hi, Ho, N, _stream(stream)), "kvc_accumulate")
+
+
+def kvc_pool(inp, out, lo, hi, kernel, stream=None):
+    B, H, N = inp.shape
+    _check(lib.kvc_pool(_ptr(inp), _ptr(out), B, H, N, lo, hi, kernel, _stream(stream)), "kvc_pool")
+
+
+def kvc_topk_workspace_size(B, H, N) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib.kvc_topk_workspace_size(B, H, N, ctypes.byref(n)), "kvc_topk_workspace_size")
+    return n.value
+
+
+def kvc_topk(pooled, n_sink, window, budget, idx, ws=None, stream=None):
+    B, H, N = pooled.shape
+    nb = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(lib.kvc_topk(_ptr(pooled), B, H, N, n_sink, window, budget, _ptr(idx), _ptr(ws), nb,
+                        _stream(stream)), "kvc_topk")
+
+
+def kvc_gather(src, idx, dst, stream=None):
+    """src [B, Hsrc, N, ...] -> dst [B, Hsrc, K, ...] via idx [B, Hidx, K]."""
+    B, Hsrc, N = src.shape[:3]
+    row_bytes = src[0, 0, 0].numel() * src.element_size() if src.dim() > 3 else src.element_size()
+    Hidx, K = idx.shape[1], idx.shape[2]
+    _check(lib.kvc_gather(_ptr(src), B, Hsrc, N, row_bytes, _ptr(idx), Hidx, K, _ptr(dst),
+                          _stream(stream)), "kvc_gather")
+
+
+def kvc_compress(p: Params, q, k, v, k_out, v_out, idx_out, hidden=None, hidden_out=None,
+                 tsp_idx_out=None, ws=None, stream=None):
+    _check(lib.kvc_compress(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(k_out), _ptr(v_out),
+                            _ptr(idx_out), _ptr(hidden), _ptr(hidden_out), _ptr(tsp_idx_out), _ptr(ws),
+                            ws.numel() * ws.element_size(), _stream(stream)), "kvc_compress")
+
+
+def kvc_tsp_count(N, window, n_sink, rate) -> int:
+    return int(lib.kvc_tsp_count(N, window, n_sink, float(rate)))
+
+
+def kvc_poll_error(stream=None) -> int:
+    return int(lib.kvc_poll_error(_stream(stream)))
+
+
+def kvc_status_string(st: int) -> str:
+    return lib.kvc_status_string(st).decode()
+
+
+def kvc_launch_count() -> int:
+    return int(lib.kvc_launch_count())
+
+
+def kvc_version() -> str:
+    return lib.kvc_version().decode()
+
+
+# ------------------------------------------------------------------ convenience front
+
+def output_shapes(p: Params) -> dict:
+    Hs = p.Hkv if p.scope == KVC_SCOPE_PER_KV_HEAD else 1
+    shapes = {"k_out": (p.B, p.Hkv, p.kv_budget, p.D), "v_out": (p.B, p.Hkv, p.kv_budget, p.D),
+              "idx_out": (p.B, Hs, p.kv_budget)}
+    if p.tsp_rate > 0:
+        n = kvc_tsp_count(p.N, p.window, p.n_sink, p.tsp_rate)
+        shapes.update(tsp_idx_out=(p.B, 1, n), hidden_out=(p.B, n, p.hidden_dim))
+    return shapes
+
+
+class Compressor:
+    """Holds the workspace and output buffers of one parameter set; `__call__` runs the
+    whole path through kvc_compress.  Inputs on the host are copied to the device and the
+    outputs copied back (the end-to-end form); device inputs are used in place."""
+
+    def __init__(self, p: Params, device="cuda"):
+        self.p = p
+        self.device = torch.device(device)
+        td = torch.float32 if p.dtype == KVC_F32 else torch.bfloat16
+        self.ws = torch.empty(max(kvc_workspace_size(p), 256), dtype=torch.uint8, device=self.device)
+        self.out = {}
+        for name, shape in output_shapes(p).items():
+            dt = torch.int32 if name.endswith("idx_out") else td
+            self.out[name] = torch.empty(shape, dtype=dt, device=self.device)
+
+    def run_device(self, q, k, v, hidden=None, stream=None):
+        o = self.out
+        kvc_compress(self.p, q, k, v, o["k_out"], o["v_out"], o["idx_out"], hidden, o.get("hidden_out"),
+                     o.get("tsp_idx_out"), self.ws, stream)
+        return o
+
+    def __call__(self, q, k, v, hidden=None, stream=None):
+        if q.is_cuda:
+            return self.run_device(q, k, v, hidden, stream)
+        dev = [t.to(self.device, non_blocking=True) if t is not None else None for t in (q, k, v, hidden)]
+        o = self.run_device(*dev, stream=stream)
+        host = {name: t.to("cpu", non_blocking=True) for name, t in o.items()}
+        (stream or torch.cuda.current_stream()).synchronize()
+        return host

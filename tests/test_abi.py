@@ -1,0 +1,142 @@
+"""The C ABI without a GPU: the library loads, exports every symbol the header declares,
+its struct layout matches the C compiler's, and argument validation returns the
+documented status codes before anything touches the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kvc.h")
+
+
+@pytest.fixture(scope="module")
+def K():
+    from long_context_kv_kvc_b200 import build
+    build.build()
+    from long_context_kv_kvc_b200 import kvc
+    return kvc
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return re.findall(r"KVC_API\s+[\w\s\*]+?\b(kvc_\w+)\s*\(", text)
+
+
+def test_exports_every_declared_symbol(K):
+    names = declared_symbols()
+    assert len(names) >= 12
+    out = subprocess.check_output(["nm", "-D", "--defined-only", K.LIB_PATH], text=True)
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    for n in names:
+        assert n in exported, n
+        assert hasattr(K.lib, n)
+    assert set(names) == set(K.EXPORTED)
+
+
+def test_params_layout_matches_c(K, tmp_path):
+    fields = [f[0] for f in K.Params._fields_]
+    src = tmp_path / "layout.c"
+    body = "".join(f'printf("%zu ", offsetof(kvc_params, {f}));' for f in fields)
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "kvc.h"\n'
+                   f'int main(void){{ printf("%zu ", sizeof(kvc_params)); {body} return 0; }}\n')
+    exe = tmp_path / "layout"
+    subprocess.check_call(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
+    got = list(map(int, subprocess.check_output([str(exe)], text=True).split()))
+    want = [ctypes.sizeof(K.Params)] + [getattr(K.Params, f).offset for f in fields]
+    assert got == want
+
+
+def test_header_compiles_as_c_and_cxx(tmp_path):
+    for comp, ext in (("gcc", "c"), ("g++", "cpp")):
+        src = tmp_path / f"inc.{ext}"
+        src.write_text('#include "kvc.h"\nint main(void){ return (int)KVC_OK; }\n')
+        subprocess.check_call([comp, "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src),
+                               "-o", str(tmp_path / f"inc_{ext}")])
+
+
+def _p(K, **kw):
+    base = dict(B=1, Hq=32, Hkv=8, N=4096, window=32, dtype=K.KVC_BF16, kv_budget=512)
+    base.update(kw)
+    return K.make_params(**base)
+
+
+FAKE = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first
+
+
+def _compress_status(K, p, ws_bytes=1 << 40, **ptrs):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, k_out=FAKE, v_out=FAKE, idx=FAKE, hidden=None, hidden_out=None,
+                tsp_idx=None, ws=FAKE)
+    args.update(ptrs)
+    return K.lib.kvc_compress(ctypes.byref(p), args["q"], args["k"], args["v"], args["k_out"],
+                              args["v_out"], args["idx"], args["hidden"], args["hidden_out"],
+                              args["tsp_idx"], args["ws"], ws_bytes, None)
+
+
+def test_validation_codes(K):
+    assert _compress_status(K, _p(K, D=64)) == K.KVC_ERR_UNSUPPORTED
+    assert _compress_status(K, _p(K, dtype=7)) == K.KVC_ERR_UNSUPPORTED
+    assert _compress_status(K, _p(K, scope=5)) == K.KVC_ERR_UNSUPPORTED
+    assert _compress_status(K, _p(K, window=64, Hq=32, Hkv=4)) == K.KVC_ERR_UNSUPPORTED  # G*w > 256
+    assert _compress_status(K, _p(K, Hq=30)) == K.KVC_ERR_ARG  # Hq % Hkv
+    assert _compress_status(K, _p(K, B=0)) == K.KVC_ERR_ARG
+    assert _compress_status(K, _p(K, pool_kernel=4)) == K.KVC_ERR_ARG
+    assert _compress_status(K, _p(K, N=20, window=20, Hq=8, kv_budget=10)) == K.KVC_ERR_ARG  # window >= N
+    assert _compress_status(K, _p(K), q=None) == K.KVC_ERR_ARG
+    assert _compress_status(K, _p(K, kv_budget=33)) == K.KVC_ERR_BUDGET  # < S + w + 1
+    assert _compress_status(K, _p(K, kv_budget=4097)) == K.KVC_ERR_BUDGET  # > N
+    assert _compress_status(K, _p(K), k=ctypes.c_void_p((1 << 20) + 8)) == K.KVC_ERR_ALIGN
+    assert _compress_status(K, _p(K), ws=ctypes.c_void_p((1 << 20) + 16)) == K.KVC_ERR_ALIGN
+    assert _compress_status(K, _p(K), ws_bytes=100) == K.KVC_ERR_WORKSPACE
+    # TSP: buffers required when the rate is set, forbidden otherwise
+    assert _compress_status(K, _p(K, tsp_rate=0.2, hidden_dim=4096)) == K.KVC_ERR_ARG
+    assert _compress_status(K, _p(K), hidden=FAKE) == K.KVC_ERR_ARG
+    assert _compress_status(K, _p(K, tsp_rate=1e-5, hidden_dim=4096), hidden=FAKE, hidden_out=FAKE,
+                            tsp_idx=FAKE) == K.KVC_ERR_BUDGET  # floor(rate * N) == 0
+    assert _compress_status(K, _p(K, tsp_rate=0.2, hidden_dim=4100), hidden=FAKE, hidden_out=FAKE,
+                            tsp_idx=FAKE) == K.KVC_ERR_ALIGN  # 8200-byte rows
+    p = _p(K)
+    p.reserved = 1
+    assert _compress_status(K, p) == K.KVC_ERR_ARG
+
+
+def test_other_entry_points_validate(K):
+    L = K.lib
+    assert L.kvc_topk(FAKE, 1, 1, 100, 1, 8, 9, FAKE, None, 0, None) == K.KVC_ERR_BUDGET
+    assert L.kvc_topk(FAKE, 1, 1, 100, 1, 8, 101, FAKE, None, 0, None) == K.KVC_ERR_BUDGET
+    assert L.kvc_topk(None, 1, 1, 100, 1, 8, 20, FAKE, None, 0, None) == K.KVC_ERR_ARG
+    assert L.kvc_pool(FAKE, FAKE, 1, 1, 100, 0, 100, 7, None) == K.KVC_ERR_ARG  # in == out
+    assert L.kvc_pool(FAKE, ctypes.c_void_p(1 << 21), 1, 1, 100, 0, 100, 6, None) == K.KVC_ERR_ARG
+    assert L.kvc_pool(FAKE, ctypes.c_void_p(1 << 21), 1, 1, 100, 50, 40, 7, None) == K.KVC_ERR_ARG
+    assert L.kvc_accumulate(FAKE, FAKE, 1, 6, 4, 10, None) == K.KVC_ERR_ARG
+    assert L.kvc_gather(FAKE, 1, 8, 100, 24, FAKE, 1, 10, FAKE, None) == K.KVC_ERR_ALIGN
+    assert L.kvc_gather(FAKE, 1, 8, 100, 256, FAKE, 3, 10, FAKE, None) == K.KVC_ERR_ARG
+    p = _p(K)
+    assert L.kvc_score(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, 10, None) == K.KVC_ERR_WORKSPACE
+    n = ctypes.c_size_t()
+    assert L.kvc_workspace_size(None, ctypes.byref(n)) == K.KVC_ERR_ARG
+
+
+def test_workspace_size_scales(K):
+    small = K.kvc_workspace_size(_p(K))
+    big = K.kvc_workspace_size(_p(K, N=131072, B=4, kv_budget=4096))
+    assert 0 < small < big
+    # compress needs the score rows and their pooled copy at least
+    assert big >= 2 * 4 * 8 * 131072 * 4
+
+
+def test_tsp_count_matches_oracle(K, oracle_lib):
+    import numpy as np
+    for N, w, S, rate in [(65536, 32, 1, 0.2), (100, 10, 1, 0.0), (100, 10, 1, 0.001), (100, 10, 1, 1.0),
+                          (1000, 8, 4, 0.37), (131072, 32, 0, 0.05)]:
+        r32 = float(np.float32(rate))
+        assert K.kvc_tsp_count(N, w, S, r32) == oracle_lib.tsp_count(N, w, S, r32)
+
+
+def test_status_strings(K):
+    for st in range(0, 9):
+        assert len(K.kvc_status_string(st)) >= 2
+    assert "unknown" in K.kvc_status_string(99)
+    assert K.kvc_version().startswith("kvc ")

@@ -1,0 +1,222 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle, on seeded inputs.
+
+Sizes span several key tiles and end in ragged tails; the full 128K / batch-4 workload is
+checked on sampled (batch, KV head) rows plus invariants that hold at any size.
+"""
+import numpy as np
+import pytest
+import torch
+
+from long_context_kv_kvc_b200 import synth
+from oracle import oracle as O
+from parity_util import check_gather, check_index_sets, check_scores
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def K():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from long_context_kv_kvc_b200 import build
+    build.build()
+    from long_context_kv_kvc_b200 import kvc
+    torch.cuda.set_device(0)
+    return kvc
+
+
+def _dev(inp):
+    return {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+
+
+def run_case(K, wl, flags=0, check_exact=True):
+    inp = synth.make_inputs(wl)
+    dev = _dev(inp)
+    p = K.params_for(wl, flags=flags)
+    comp = K.Compressor(p)
+    out = comp(dev["q"], dev["k"], dev["v"], dev.get("hidden"))
+    Hs = wl.Hkv if wl.scope == K.KVC_SCOPE_PER_KV_HEAD else 1
+    scores = torch.empty((wl.B, Hs, wl.N), dtype=torch.float32, device="cuda")
+    K.kvc_score(p, dev["q"], dev["k"], scores, comp.ws)
+    assert K.kvc_poll_error() == K.KVC_OK
+    ref = O.compress(inp["q"], inp["k"], inp["v"], window=wl.window, n_sink=wl.n_sink,
+                     pool_kernel=wl.pool_kernel, kv_budget=wl.kv_budget, scope=wl.scope,
+                     tsp_rate=float(np.float32(wl.tsp_rate)), hidden=inp["hidden"])
+    check_scores(scores.cpu().numpy(), ref["scores"])
+    exact = check_index_sets(out["idx_out"].cpu().numpy(), ref["pooled"], wl.N, wl.n_sink, wl.window,
+                             wl.kv_budget)
+    if check_exact:
+        assert exact == 1.0, f"exact index-set match rate {exact}"
+    check_gather(out["k_out"], dev["k"][-1], out["idx_out"].cpu().numpy())
+    check_gather(out["v_out"], dev["v"], out["idx_out"].cpu().numpy())
+    if wl.tsp_rate > 0:
+        n_tsp = K.kvc_tsp_count(wl.N, wl.window, wl.n_sink, wl.tsp_rate)
+        tsp_exact = check_index_sets(out["tsp_idx_out"].cpu().numpy(), ref["tsp_pooled"], wl.N, wl.n_sink,
+                                     wl.window, n_tsp)
+        if check_exact:
+            assert tsp_exact == 1.0
+        check_gather(out["hidden_out"].unsqueeze(1), dev["hidden"].unsqueeze(1),
+                     out["tsp_idx_out"].cpu().numpy())
+    return out, ref, scores
+
+
+def test_tiny_f32(K):
+    run_case(K, synth.TINY)
+
+
+BF16_CASES = [
+    # several 128-key tiles with a ragged tail, full GQA group (G*w = 128)
+    dict(B=1, Hq=8, Hkv=2, N=1000, window=32, kv_budget=200, n_hubs=16),
+    # G*w = 32, two sequences, longer
+    dict(B=2, Hq=4, Hkv=1, N=4133, window=8, kv_budget=500, n_hubs=64),
+    # the 8B head layout on a short context, odd N
+    dict(B=1, Hq=32, Hkv=8, N=2053, window=32, kv_budget=1024, n_hubs=32),
+    # no sinks, four sinks, pooling off and P = 3
+    dict(B=1, Hq=8, Hkv=2, N=777, window=16, kv_budget=100, n_sink=0, n_hubs=8),
+    dict(B=1, Hq=8, Hkv=2, N=1531, window=32, kv_budget=300, n_sink=4, pool_kernel=1, n_hubs=8),
+    dict(B=1, Hq=8, Hkv=2, N=1200, window=24, kv_budget=400, pool_kernel=3, n_hubs=8),
+    # budget at its extremes: S + w + 1 and N
+    dict(B=1, Hq=4, Hkv=1, N=600, window=32, kv_budget=34, n_hubs=4),
+    dict(B=1, Hq=4, Hkv=1, N=600, window=32, kv_budget=600, n_hubs=4),
+]
+
+
+@pytest.mark.parametrize("flags", [0, 1], ids=["default", "simt"])
+@pytest.mark.parametrize("case", range(len(BF16_CASES)))
+def test_bf16_cases(K, case, flags):
+    wl = synth.scaled(synth.LLAMA8B_32K, **BF16_CASES[case])
+    run_case(K, wl, flags=flags)
+
+
+def test_structkv_layers_all_heads(K):
+    wl = synth.scaled(synth.STRUCTKV_8L_32K, N=1500, n_layers=3, kv_budget=300, n_hubs=20)
+    run_case(K, wl)
+
+
+def test_fastkv_tsp(K):
+    wl = synth.scaled(synth.FASTKV_TSP_64K, N=3000, kv_budget=256, hidden_dim=512, n_hubs=30)
+    run_case(K, wl)
+
+
+def test_f32_wider(K):
+    wl = synth.scaled(synth.TINY, B=2, Hq=8, Hkv=2, N=3001, window=16, kv_budget=333, n_hubs=40)
+    run_case(K, wl)
+
+
+# --------------------------------------------------------------------- stand-alone kernels
+
+def test_topk_edges(K):
+    g = np.random.default_rng(0)
+    cases = []
+    cases.append((np.ones((1, 1, 50), np.float32), 1, 3, 10))            # all ties
+    cases.append((np.zeros((2, 3, 64), np.float32), 0, 0, 5))             # no sinks, no window
+    v = g.standard_normal((1, 2, 300)).astype(np.float32)                 # negative values
+    cases.append((v, 2, 5, 120))
+    z = np.zeros((1, 1, 40), np.float32)
+    z[0, 0, ::2] = -0.0                                                   # -0.0 ties with +0.0
+    cases.append((z, 1, 1, 12))
+    r = np.round(g.random((3, 2, 200_003)), 3).astype(np.float32)        # long rows, many ties
+    cases.append((r, 1, 32, 4096))
+    cases.append((g.random((1, 1, 100)).astype(np.float32), 1, 8, 100))  # budget = N
+    for vals, S, w, budget in cases:
+        B, H, N = vals.shape
+        idx = torch.empty((B, H, budget), dtype=torch.int32, device="cuda")
+        K.kvc_topk(torch.from_numpy(vals).cuda(), S, w, budget, idx)
+        ref = O.select(vals.astype(np.float64), S, w, budget)
+        assert np.array_equal(idx.cpu().numpy(), ref), (S, w, budget, N)
+
+
+def test_pool_edges(K):
+    g = np.random.default_rng(1)
+    x = g.random((2, 3, 257)).astype(np.float32)
+    for lo, hi, P in [(0, 257, 1), (0, 257, 7), (5, 200, 9), (40, 40, 7), (1, 225, 3), (256, 257, 7)]:
+        out = torch.empty((2, 3, 257), dtype=torch.float32, device="cuda")
+        K.kvc_pool(torch.from_numpy(x).cuda(), out, lo, hi, P)
+        ref = O.pool(x.astype(np.float64), lo, hi, P)
+        assert np.array_equal(out.cpu().numpy().astype(np.float64), ref)
+
+
+def test_accumulate(K):
+    g = np.random.default_rng(2)
+    src = g.random((2, 8, 1000)).astype(np.float32)
+    acc = g.random((2, 2, 1000)).astype(np.float32)
+    a = torch.from_numpy(acc).cuda()
+    K.kvc_accumulate(a, torch.from_numpy(src).cuda())
+    ref = O.accumulate(acc.astype(np.float64), src.astype(np.float64))
+    np.testing.assert_allclose(a.cpu().numpy(), ref, rtol=1e-6)
+
+
+def test_gather_rows_and_bad_index(K):
+    g = torch.Generator().manual_seed(3)
+    src = torch.randn(2, 4, 300, 128, generator=g).to(torch.bfloat16).cuda()
+    idx = torch.sort(torch.randperm(300, generator=g)[:37]).values.int().repeat(2, 4, 1).cuda()
+    dst = torch.empty(2, 4, 37, 128, dtype=torch.bfloat16, device="cuda")
+    K.kvc_gather(src, idx, dst)
+    assert K.kvc_poll_error() == K.KVC_OK
+    check_gather(dst, src, idx.cpu().numpy())
+    shared = idx[:, :1].contiguous()
+    K.kvc_gather(src, shared, dst)
+    check_gather(dst, src, shared.cpu().numpy())
+    bad = idx.clone()
+    bad[1, 2, 5] = 300
+    bad[0, 0, 0] = -1
+    K.kvc_gather(src, bad, dst)
+    assert K.kvc_poll_error() == K.KVC_ERR_INDEX
+    assert K.kvc_poll_error() == K.KVC_OK  # cleared
+    assert torch.count_nonzero(dst[1, 2, 5].float()) == 0 and torch.count_nonzero(dst[0, 0, 0].float()) == 0
+    assert torch.equal(dst[1, 2, 4], src[1, 2, int(bad[1, 2, 4])])
+
+
+def test_deterministic(K):
+    wl = synth.scaled(synth.LLAMA8B_32K, N=3000, n_hubs=16)
+    inp = _dev(synth.make_inputs(wl))
+    p = K.params_for(wl)
+    comp = K.Compressor(p)
+    a = {k: v.clone() for k, v in comp(inp["q"], inp["k"], inp["v"]).items()}
+    b = comp(inp["q"], inp["k"], inp["v"])
+    for name in a:
+        assert torch.equal(a[name], b[name]), name
+
+
+def test_tensor_core_matches_simt_path(K):
+    """The bf16 tensor-core scores agree with the CUDA-core (FFMA) scores on the GPU."""
+    wl = synth.scaled(synth.LLAMA8B_32K, B=2, N=9000, n_hubs=64)
+    inp = _dev(synth.make_inputs(wl))
+    out = {}
+    for flags in (0, K.KVC_FLAG_SIMT_SCORE):
+        p = K.params_for(wl, flags=flags)
+        ws = torch.empty(K.kvc_workspace_size(p), dtype=torch.uint8, device="cuda")
+        s = torch.empty((wl.B, wl.Hkv, wl.N), dtype=torch.float32, device="cuda")
+        K.kvc_score(p, inp["q"], inp["k"], s, ws)
+        out[flags] = s.double().cpu().numpy()
+    check_scores(out[0], out[K.KVC_FLAG_SIMT_SCORE], rtol=2e-5)
+
+
+# ------------------------------------------------------------------- full-size workload
+
+def test_full_size_128k_batch4_sampled(K):
+    """The benchmarked workload in the benchmarked launch configuration: scores and index
+    sets of sampled (sequence, KV head) rows against the oracle, gathers of every row,
+    and the probability-mass invariant on every row."""
+    wl = synth.LLAMA8B_128K_B4
+    inp = synth.make_inputs(wl)
+    dev = _dev(inp)
+    p = K.params_for(wl)
+    comp = K.Compressor(p)
+    out = comp(dev["q"], dev["k"], dev["v"])
+    scores = torch.empty((wl.B, wl.Hkv, wl.N), dtype=torch.float32, device="cuda")
+    K.kvc_score(p, dev["q"], dev["k"], scores, comp.ws)
+    assert K.kvc_poll_error() == K.KVC_OK
+    s = scores.double().cpu().numpy()
+    np.testing.assert_allclose(s.sum(axis=-1), wl.G * wl.window, rtol=1e-4)
+    idx = out["idx_out"].cpu().numpy()
+    check_gather(out["k_out"], dev["k"][0], idx)
+    check_gather(out["v_out"], dev["v"], idx)
+    G = wl.G
+    for b, h in [(0, 0), (3, 7), (1, 4)]:
+        q = inp["q"][:, b:b + 1, h * G:(h + 1) * G]
+        k = inp["k"][:, b:b + 1, h:h + 1]
+        ref_s = O.score(q, k, window=wl.window)[0, 0]
+        check_scores(s[b, h], ref_s)
+        ref_p = O.pool(ref_s[None, None], wl.n_sink, wl.N - wl.window, wl.pool_kernel)[0, 0]
+        check_index_sets(idx[b, h][None], ref_p[None], wl.N, wl.n_sink, wl.window, wl.kv_budget)
