@@ -214,6 +214,26 @@ KVC_API kvc_status kvc_compress(const kvc_params *p, const void *q, const void *
                         kvc_stream_t stream);
 
 /*
+ * kvc_score_noalloc -- kvc_score for callers that cannot allocate device memory.  The
+ * pages have no counterpart: it exists for engines that have already given all device
+ * memory to their own pool, or plugin interfaces that forbid cudaMalloc/cudaFree during a
+ * step, and so cannot pass a workspace.  Same arguments and results as kvc_score without
+ * ws/ws_bytes; it always scores with the CUDA-core kernels and keeps their scratch in a
+ * 4 MiB array compiled into the library, which every GPU that loads the library holds
+ * until the process exits.
+ *   Returns KVC_ERR_WORKSPACE when the scratch these parameters need exceeds 4 MiB (about
+ *   n_layers * B * Hkv * ceil(N / 2048) * G * window * 8 bytes, plus n_layers * B * Hkv * N
+ *   * 4 bytes when several layers or all heads are summed).
+ *   The first call on each device looks up the array's address (with that device
+ *   current); make it before any stream capture begins.  All calls on a device share the
+ *   array: calls whose kernels may overlap on the GPU race and must be ordered by the
+ *   caller.  It allocates nothing and clears nothing between calls (every scratch byte it
+ *   reads is written earlier in the same call).
+ */
+KVC_API kvc_status kvc_score_noalloc(const kvc_params *p, const void *q, const void *k, float *scores,
+                                     kvc_stream_t stream);
+
+/*
  * kvc_tsp_count -- rows propagated by TSP: min(floor(tsp_rate * N), N - window - n_sink)
  * selected tokens plus n_sink + window; 0 when tsp_rate <= 0 or floor(tsp_rate*N) < 1.
  * Source: FastKV sec. 2B (the TSP rate sets how many tokens continue past the TSP layer).

@@ -23,7 +23,7 @@ KVC_STAGE_SCORE, KVC_STAGE_SELECT, KVC_STAGE_GATHER, KVC_STAGE_COUNT = 0, 1, 2, 
 
 EXPORTED = ("kvc_workspace_size", "kvc_score", "kvc_accumulate", "kvc_pool", "kvc_topk_workspace_size",
             "kvc_topk", "kvc_gather", "kvc_compress", "kvc_tsp_count", "kvc_poll_error",
-            "kvc_status_string", "kvc_version", "kvc_launch_count")
+            "kvc_status_string", "kvc_version", "kvc_launch_count", "kvc_score_noalloc")
 
 
 class KvcError(RuntimeError):
@@ -62,6 +62,7 @@ def _load():
         "kvc_status_string": (ctypes.c_char_p, [st]),
         "kvc_version": (ctypes.c_char_p, []),
         "kvc_launch_count": (ctypes.c_uint64, []),
+        "kvc_score_noalloc": (st, [P, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -136,6 +137,13 @@ def kvc_workspace_size(p: Params) -> int:
 def kvc_score(p: Params, q, k, scores, ws, stream=None):
     _check(lib.kvc_score(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(scores), _ptr(ws),
                          ws.numel() * ws.element_size(), _stream(stream)), "kvc_score")
+
+
+def kvc_score_noalloc(p: Params, q, k, scores, stream=None):
+    """kvc_score without a workspace, for callers that cannot allocate device memory; the
+    library's fixed 4 MiB per-device scratch array stands in for it (see include/kvc.h)."""
+    _check(lib.kvc_score_noalloc(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(scores), _stream(stream)),
+           "kvc_score_noalloc")
 
 
 def kvc_accumulate(acc, src, stream=None):
