@@ -88,7 +88,12 @@ enum {
 
 /* kvc_params.flags */
 enum {
-    KVC_FLAG_SIMT_SCORE = 1u << 0 /* score with the CUDA-core (FFMA) kernels even for bf16 */
+    KVC_FLAG_SIMT_SCORE = 1u << 0, /* score with the CUDA-core (FFMA) kernels even for bf16  */
+    /* Test hook for failure detection: the tensor-core scoring kernel's cross-CTA wait
+     * watches a flag that nothing sets, so it gives up after spin_limit polls; the scores
+     * of the units involved come out as zeros and kvc_poll_error returns KVC_ERR_TIMEOUT.
+     * Nothing faults or hangs.  Ignored by the CUDA-core path (it has no such wait). */
+    KVC_FLAG_INJECT_WAIT_TIMEOUT = 1u << 1
 };
 
 /* Entries of kvc_params.stage_events: events recorded on the stream between the stages

@@ -83,7 +83,8 @@ ScoreJob make_job(const kvc_params* p, const void* q, const void* k) {
     j.window = p->window;
     j.G = p->Hq / p->Hkv;
     j.nq = j.G * p->window;
-    j.spin_limit = p->spin_limit > 0 ? p->spin_limit : (1LL << 26);
+    j.spin_limit = p->spin_limit > 0 ? p->spin_limit : (1LL << 22);
+    j.inject_timeout = (p->flags & KVC_FLAG_INJECT_WAIT_TIMEOUT) ? 1 : 0;
     return j;
 }
 

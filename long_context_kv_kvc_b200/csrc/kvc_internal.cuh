@@ -47,6 +47,7 @@ struct ScoreJob {
     size_t tc_ws_bytes;
     unsigned* err;
     long long spin_limit;
+    int inject_timeout;  // test hook: the cross-CTA wait watches a flag nothing sets
 };
 
 // CUDA-core (FFMA) scoring, fp32 or bf16 inputs

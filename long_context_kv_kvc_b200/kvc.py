@@ -19,6 +19,7 @@ KVC_ERR_WORKSPACE, KVC_ERR_CUDA, KVC_ERR_TIMEOUT, KVC_ERR_INDEX = 5, 6, 7, 8
 KVC_F32, KVC_BF16 = 0, 1
 KVC_SCOPE_PER_KV_HEAD, KVC_SCOPE_ALL_HEADS = 0, 1
 KVC_FLAG_SIMT_SCORE = 1
+KVC_FLAG_INJECT_WAIT_TIMEOUT = 2
 KVC_STAGE_SCORE, KVC_STAGE_SELECT, KVC_STAGE_GATHER, KVC_STAGE_COUNT = 0, 1, 2, 3
 
 EXPORTED = ("kvc_workspace_size", "kvc_score", "kvc_accumulate", "kvc_pool", "kvc_topk_workspace_size",

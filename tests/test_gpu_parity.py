@@ -78,6 +78,13 @@ BF16_CASES = [
     # budget at its extremes: S + w + 1 and N
     dict(B=1, Hq=4, Hkv=1, N=600, window=32, kv_budget=34, n_hubs=4),
     dict(B=1, Hq=4, Hkv=1, N=600, window=32, kv_budget=600, n_hubs=4),
+    # one partial key tile; an exact multiple of the tile
+    dict(B=1, Hq=4, Hkv=1, N=100, window=8, kv_budget=20, n_hubs=4),
+    dict(B=1, Hq=8, Hkv=2, N=1024, window=32, kv_budget=256, n_hubs=8),
+    # many short units: a unit has fewer tiles than there are CTAs (each CTA spans units)
+    dict(B=4, Hq=32, Hkv=8, N=1000, window=32, kv_budget=128, n_hubs=8),
+    # few long units: a unit has more tiles than there are CTAs
+    dict(B=1, Hq=4, Hkv=1, N=40000, window=32, kv_budget=2000, n_hubs=64),
 ]
 
 
@@ -190,6 +197,26 @@ def test_tensor_core_matches_simt_path(K):
         K.kvc_score(p, inp["q"], inp["k"], s, ws)
         out[flags] = s.double().cpu().numpy()
     check_scores(out[0], out[K.KVC_FLAG_SIMT_SCORE], rtol=2e-5)
+
+
+def test_injected_wait_timeout_is_reported_and_recovers(K):
+    """Failure detection without a GPU fault: the cross-CTA wait of the tensor-core kernel
+    is pointed at a flag nothing sets; it gives up after a few polls, the call completes,
+    kvc_poll_error reports KVC_ERR_TIMEOUT, and the next normal call is correct."""
+    wl = synth.scaled(synth.LLAMA8B_32K, N=3000, n_hubs=16)
+    inp = _dev(synth.make_inputs(wl, with_v=False))
+    bad = K.params_for(wl, flags=K.KVC_FLAG_INJECT_WAIT_TIMEOUT, spin_limit=200)
+    ws = torch.empty(K.kvc_workspace_size(bad), dtype=torch.uint8, device="cuda")
+    s = torch.empty((wl.B, wl.Hkv, wl.N), dtype=torch.float32, device="cuda")
+    K.kvc_score(bad, inp["q"], inp["k"], s, ws)
+    assert K.kvc_poll_error() == K.KVC_ERR_TIMEOUT
+    assert K.kvc_poll_error() == K.KVC_OK
+    good = K.params_for(wl)
+    K.kvc_score(good, inp["q"], inp["k"], s, ws)
+    assert K.kvc_poll_error() == K.KVC_OK
+    ref = O.score(synth.make_inputs(wl, with_v=False)["q"], synth.make_inputs(wl, with_v=False)["k"],
+                  window=wl.window)
+    check_scores(s.cpu().numpy(), ref)
 
 
 # ------------------------------------------------------------------- full-size workload
