@@ -239,6 +239,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--flags", type=int, default=0, help="kvc_params.flags (1 = CUDA-core scoring)")
+    ap.add_argument("--no-clocks", action="store_true",
+                    help="skip nvidia-smi clock sampling and its 1 s warm loop (for profiler runs)")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -284,13 +286,15 @@ def main():
     if kvc.kvc_poll_error() != kvc.KVC_OK:
         raise RuntimeError("device-side error during warm-up")
 
-    sampler = ClockSampler(local)
-    sampler.start()
-    # keep the GPU busy ~1 s under the sampler before the timed region
-    t_end = time.time() + 1.0
-    while time.time() < t_end:
-        step()
-        torch.cuda.synchronize()
+    sampler = None
+    if not args.no_clocks:
+        sampler = ClockSampler(local)
+        sampler.start()
+        # keep the GPU busy ~1 s under the sampler before the timed region
+        t_end = time.time() + 1.0
+        while time.time() < t_end:
+            step()
+            torch.cuda.synchronize()
 
     n_before = kvc.kvc_launch_count()
     if world > 1:
@@ -306,7 +310,7 @@ def main():
     if world > 1:
         dist.barrier()
     launches = (kvc.kvc_launch_count() - n_before) // 1
-    clocks = sampler.stop()
+    clocks = sampler.stop() if sampler else None
     ms = t0.elapsed_time(t1)
     if kvc.kvc_poll_error() != kvc.KVC_OK:
         raise RuntimeError("device-side error during the timed region")

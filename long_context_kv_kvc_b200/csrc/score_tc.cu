@@ -11,28 +11,28 @@
 //
 // Design for B200.  The softmax normaliser lse_r is global over all N keys, so every
 // logit is needed twice: once for lse_r (phase 1) and once for its probability (phase 2).
-// Storing logits would cost more HBM traffic than K itself, so K tiles are read twice and
-// the schedule makes the second read hit L2:
-//   * one persistent CTA per SM (cooperative launch, so all CTAs are resident), 128-key
-//     tiles dealt round-robin over the CTAs in global order (unit-major);
-//   * each CTA runs phase 1 on its tile i while running phase 2 on its tile i - lag, with
-//     lag about one unit's worth of tiles, so the tile is re-read from L2 (~1 unit of K,
-//     32 MiB at 128K, is in flight across the GPU);
-//   * phase 1:  D1[128 q x 128 keys] = Q K^T (tcgen05.mma kind::f16, M = N = 128, fp32
-//     accumulator in TMEM); one thread per query row keeps an online (max, sum) over the
-//     CTA's tiles of the unit; the CTA's partial goes to global memory and the last CTA
-//     of the unit (atomic counter) merges the partials in a fixed order into lse and
-//     raises the unit's ready flag;
-//   * phase 2:  D2[128 keys x 128 q] = K Q^T (the transposed product, so a thread owns a
-//     key and sums over queries in registers); waits (bounded) for the unit's ready flag.
-// Warp roles: warp 0 issues TMA loads (K tiles through a 4-stage ring, Q of the current
-// unit for each phase), warp 1 owns TMEM and issues the MMAs from one thread, warps 4-7
-// run phase-1 statistics, warps 8-11 run phase-2 sums.  TMEM holds two phase-1 and two
-// phase-2 accumulators (4 x 128 columns).  Every wait is bounded: a wait that runs out
-// sets the per-device error word and the kernel finishes without blocking.
+// Storing logits would cost more HBM traffic than K itself, so K is read twice and the
+// second read is scheduled to hit L2:
+//   * one persistent CTA per SM (cooperative launch: all CTAs resident), 128-key tiles
+//     dealt round-robin over the CTAs in global (unit-major) order;
+//   * phase 1 streams K from HBM: D1[128 q x 128 keys] = Q K^T (tcgen05.mma kind::f16,
+//     M = N = 128, fp32 accumulator in TMEM); one thread per query row keeps an online
+//     (max, sum) over the CTA's tiles of a unit and hands it to the publisher warp;
+//   * the publisher warp writes the CTA's partial, and the last CTA of each 16-CTA group
+//     and then the last group of the unit merge the partials (fixed order) into lse and
+//     raise the unit's ready flag -- off the consumers' path;
+//   * phase 2 re-reads each tile a bounded number of tiles behind phase 1 (so it comes
+//     from L2, loaded evict-first): D2[128 keys x 128 q] = K Q^T, a thread owns a key and
+//     sums 2^(y - lse) over the query rows once the unit's ready flag is up.
+// The two phases have separate TMA producers, shared-memory rings (16 KiB half-tiles of
+// 64 columns, the 128-byte swizzle atom) and MMA issuers, so a phase-2 wait never stalls
+// the HBM stream.  Warps: 0 phase-1 TMA, 1 TMEM owner + phase-1 MMA, 2 phase-2 TMA,
+// 3 phase-2 MMA, 4-7 phase-1 statistics, 8-11 phase-2 sums, 12 publisher.  Every wait is
+// bounded: a wait that runs out sets the per-device error word and the kernel still ends.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 
 #include "kvc_internal.cuh"
@@ -42,11 +42,14 @@ namespace {
 
 constexpr int kTileKeys = 128;                         // keys per tile (MMA N / M)
 constexpr int kQRows = 128;                            // query rows per unit (padded)
-constexpr int kStages = 4;                             // K-tile ring depth
-constexpr int kTileBytes = kTileKeys * kHeadDim * 2;   // 32 KiB of bf16
-constexpr int kHalfBytes = kTileBytes / 2;             // one 64-column (128-byte) TMA box
-constexpr int kThreads = 384;
-constexpr int kMaxCtas = 160;                          // partial slots per row (>= #SMs)
+constexpr int kBoxBytes = kTileKeys * 64 * 2;          // a 128-row x 64-column bf16 box: 16 KiB
+constexpr int kStagesA = 6;                            // phase-1 ring (HBM stream)
+constexpr int kStagesB = 3;                            // phase-2 ring (L2 re-read)
+constexpr int kWarps = 13;
+constexpr int kThreads = kWarps * 32;
+constexpr int kMaxCtas = 160;                          // partial slots per unit (>= #SMs)
+constexpr int kGroup = 16;                             // CTAs per first-level merge group
+constexpr int kMaxGroups = kMaxCtas / kGroup;
 constexpr uint32_t kTmemCols = 512;
 constexpr long long kBarrierTimeoutNs = 4000000000LL;  // hang guard for intra-CTA waits
 
@@ -58,26 +61,33 @@ struct TcArgs {
     CUtensorMap tmap_k;  // K as [U][N][128] bf16, box 64 x 128 x 1, 128-byte swizzle
     CUtensorMap tmap_q;  // padded Q as [U*128][128] bf16, box 64 x 128, 128-byte swizzle
     float* unit_scores;  // [U][N]
-    float2* partial;     // [U][128][kMaxCtas] (max, sum) per CTA
+    float2* partial;     // [U][kMaxCtas][128] (max, sum) per CTA
+    float2* gpartial;    // [U][kMaxGroups][128] (max, sum) per merge group
     float* lse;          // [U][128]
-    unsigned* count;     // [U] CTAs that have published their partial
+    unsigned* gcount;    // [U][kMaxGroups] partials published per group
+    unsigned* count;     // [U] groups merged
     unsigned* ready;     // [U] lse published
     unsigned* never;     // a flag nothing sets (wait-timeout injection)
     unsigned* err;
     long long spin_limit;
-    int U, N, w, nq, T_u, total_tiles, P, lag, inject;
+    int U, N, w, nq, T_u, total_tiles, P, max_lead, inject;
 };
 
 struct __align__(1024) Smem {
-    uint8_t ktile[kStages][kTileBytes];
-    uint8_t q[2][kTileBytes];
+    uint8_t ringA[kStagesA][kBoxBytes];
+    uint8_t ringB[kStagesB][kBoxBytes];
+    uint8_t q[2][2 * kBoxBytes];  // Q of the current unit of phase 1 / phase 2 (two boxes)
     float lse[kQRows];
-    uint64_t full[kStages], empty[kStages];
+    float2 pub[2][kQRows];
+    int pub_unit[2];
+    uint64_t fullA[kStagesA], emptyA[kStagesA], fullB[kStagesB], emptyB[kStagesB];
     uint64_t qfull[2], qempty[2];
     uint64_t d1full[2], d1empty[2], d2full[2], d2empty[2];
+    uint64_t pub_full[2], pub_empty[2];
     uint32_t tmem_base;
     int abort;
-    int flag1, flag2;
+    int flag2;
+    int p1_issued, p2_issued;  // tiles whose loads each producer has issued (L2 lead control)
 };
 
 // ------------------------------------------------------------------------ PTX wrappers
@@ -120,14 +130,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Bounded wait for the phase of `bar` with the given parity.  On time-out (a broken
 // pipeline, never a normal run) it records the error, puts the CTA in fail-fast mode and
 // returns, so that the kernel always terminates.
-__device__ __forceinline__ void mbar_wait(uint64_t* bar, uint32_t parity, Smem& sm, unsigned* err) {
+__device__ __forceinline__ void mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, unsigned* err) {
     if (mbar_try_wait(bar, parity)) return;
     const long long t0 = globaltimer();
     while (!mbar_try_wait(bar, parity)) {
-        if (*(volatile int*)&sm.abort) return;
+        if (*abort) return;
         if (globaltimer() - t0 > kBarrierTimeoutNs) {
             atomicOr(err, kErrTimeout);
-            *(volatile int*)&sm.abort = 1;
+            *abort = 1;
             return;
         }
     }
@@ -139,6 +149,23 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
         ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
         : "memory");
+}
+
+// Same, with an L2 eviction-policy hint (a createpolicy value).
+__device__ __forceinline__ void tma_load_3d_hint(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
+                                                 int z, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5}], [%2], %6;"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z),
+          "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
 }
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
@@ -162,10 +189,10 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
     return d;
 }
 
-// Descriptor of K-slice kk (16 columns = 32 bytes) of a 128 x 128 bf16 tile stored as two
-// 64-column boxes.
-__device__ __forceinline__ uint64_t tile_desc(const uint8_t* tile, int kk) {
-    return sw128_desc(smem_u32(tile) + (kk >> 2) * kHalfBytes + (kk & 3) * 32);
+// Descriptor of K-slice kk (16 columns = 32 bytes, kk < 4) of a 128-row x 64-column bf16
+// box.
+__device__ __forceinline__ uint64_t box_desc(const uint8_t* box, int kk) {
+    return sw128_desc(smem_u32(box) + kk * 32);
 }
 
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t accumulate) {
@@ -181,27 +208,39 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                  : "memory");
 }
 
-// 32 consecutive fp32 columns of this thread's TMEM lane; the values are only valid after
-// tmem_wait, which takes them as in/out operands so no use can be scheduled before it.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+// 64 consecutive fp32 columns of this thread's TMEM lane (one tcgen05.ld).  The values are
+// only valid after tmem_wait64, which takes them as in/out operands so that no use can be
+// scheduled before the wait.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {"
+        "%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+        "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63"
+        "}, [%64];"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
           "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+          "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+          "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+          "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+          "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
         : "r"(taddr)
         : "memory");
 }
 
-__device__ __forceinline__ void tmem_wait(uint32_t (&r)[32]) {
+__device__ __forceinline__ void tmem_wait64(uint32_t (&r)[64]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;"
                  : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
-                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
-                   "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
-                   "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
-                   "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+                   "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                   "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]),
+                   "+r"(r[32]), "+r"(r[33]), "+r"(r[34]), "+r"(r[35]), "+r"(r[36]), "+r"(r[37]), "+r"(r[38]), "+r"(r[39]),
+                   "+r"(r[40]), "+r"(r[41]), "+r"(r[42]), "+r"(r[43]), "+r"(r[44]), "+r"(r[45]), "+r"(r[46]), "+r"(r[47]),
+                   "+r"(r[48]), "+r"(r[49]), "+r"(r[50]), "+r"(r[51]), "+r"(r[52]), "+r"(r[53]), "+r"(r[54]), "+r"(r[55]),
+                   "+r"(r[56]), "+r"(r[57]), "+r"(r[58]), "+r"(r[59]), "+r"(r[60]), "+r"(r[61]), "+r"(r[62]), "+r"(r[63])
                  :
                  : "memory");
 }
@@ -210,6 +249,32 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^y on the FMA pipe, for y <= ~0 (the kernel's arguments are logits minus a running
+// max or minus the log-sum-exp).  Cody-Waite range reduction y = n + f with n = round(y)
+// and f in [-1/2, 1/2]; 2^f from a degree-5 polynomial with equioscillating relative error
+// (Remez exchange, fitted by exp2_poly_fit.py next to this library, binary32 coefficients);
+// 2^n is added to the exponent field.  Arguments below -125 are clamped, which returns about
+// 2^-125 instead of 0 (absolute error below 3e-38).  Relative error about 2.3e-7 on [-125, 0].
+__device__ __forceinline__ float exp2_poly(float y) {
+    y = fmaxf(y, -125.0f);
+    const float t = y + 12582912.0f;  // 1.5 * 2^23: y rounded to an integer lands in t's low bits
+    const float n = t - 12582912.0f;
+    const float f = y - n;
+    float p = fmaf(f, 0.0013276472454890609f, 0.009675540961325169f);
+    p = fmaf(p, f, 0.05550713092088699f);
+    p = fmaf(p, f, 0.24022120237350464f);
+    p = fmaf(p, f, 0.6931469440460205f);
+    p = fmaf(p, f, 1.0000001192092896f);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Exponentials of the fully visible tiles: two of every eight go to the FMA pipe so that
+// the MUFU and the FMA pipes finish together.
+template <int E>
+__device__ __forceinline__ float exp2_mixed(float y) {
+    return (E & 7) >= 6 ? exp2_poly(y) : ex2(y);
 }
 
 __device__ __forceinline__ void named_sync(int id, int n) {
@@ -222,24 +287,124 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
     return v;
 }
 
-// Order of jobs of one CTA: phase 1 runs `lag` tiles ahead of phase 2.
-struct JobIter {
-    int n, lag, i1 = 0, i2 = 0;
-    __device__ JobIter(int n_, int lag_) : n(n_), lag(lag_) {}
-    __device__ bool next(int& phase, int& i) {
-        if (i1 < n && i1 - i2 < lag) {
-            phase = 0;
-            i = i1++;
-            return true;
-        }
-        if (i2 < n) {
-            phase = 1;
-            i = i2++;
-            return true;
-        }
-        return false;
+// The CTAs that hold tiles of unit u form the cyclic range [first, first + n) mod P with
+// first = u*T_u mod P and n = min(T_u, P) (tiles are dealt round-robin).
+struct Contributors {
+    int first, n, P;
+    __device__ Contributors(const TcArgs& a, int u)
+        : first((int)(((long long)u * a.T_u) % a.P)), n(min(a.T_u, a.P)), P(a.P) {}
+    __device__ bool has(int c) const {
+        int rel = c - first;
+        if (rel < 0) rel += P;
+        return rel < n;
     }
+    // how many of the CTAs [lo, hi) contribute
+    __device__ int count(int lo, int hi) const {
+        const int a_hi = min(first + n, P);                          // [first, a_hi)
+        const int b_hi = first + n > P ? first + n - P : 0;          // [0, b_hi)
+        return max(0, min(hi, a_hi) - max(lo, first)) + max(0, min(hi, b_hi) - lo);
+    }
+    __device__ int group_size(int g) const { return count(g * kGroup, min(P, (g + 1) * kGroup)); }
 };
+
+// Merges (max, sum) pairs of one row: src[i * stride] for the i in [0, n) with use(i).
+template <typename Use>
+__device__ __forceinline__ float2 merge_row(const float2* src, int n, size_t stride, Use use) {
+    float M = -INFINITY, S = 0.f;
+    for (int i0 = 0; i0 < n; i0 += kGroup) {
+        float2 v[kGroup];
+#pragma unroll
+        for (int i = 0; i < kGroup; ++i)
+            v[i] = (i0 + i < n && use(i0 + i)) ? __ldcg(src + (size_t)(i0 + i) * stride) : make_float2(-INFINITY, 0.f);
+        float cm = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < kGroup; ++i) cm = fmaxf(cm, v[i].x);
+        if (cm == -INFINITY) continue;
+        float cs = 0.f;
+#pragma unroll
+        for (int i = 0; i < kGroup; ++i)
+            if (v[i].x != -INFINITY) cs += v[i].y * ex2(v[i].x - cm);
+        if (cm > M) {
+            S = (M == -INFINITY ? 0.f : S * ex2(M - cm)) + cs;
+            M = cm;
+        } else {
+            S += cs * ex2(cm - M);
+        }
+    }
+    return make_float2(M, S);
+}
+
+// Online (max, sum) update of one query row with 64 logits (keys j0 .. j0+63); keys after
+// t_r are masked unless the whole tile is visible.
+__device__ __forceinline__ void stats_update(const uint32_t (&x)[64], bool full_tile, int j0, int t_r, float& m,
+                                             float& l) {
+    float cm = -INFINITY;
+    if (full_tile) {
+        float mx[8];
+#pragma unroll
+        for (int g = 0; g < 8; ++g) mx[g] = __uint_as_float(x[g]);
+#pragma unroll
+        for (int e = 8; e < 64; ++e) mx[e & 7] = fmaxf(mx[e & 7], __uint_as_float(x[e]));
+        cm = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+    } else {
+#pragma unroll
+        for (int e = 0; e < 64; ++e)
+            if (j0 + e <= t_r) cm = fmaxf(cm, __uint_as_float(x[e]));
+    }
+    if (cm == -INFINITY) return;
+    const float mn = fmaxf(m, cm * kLog2eOverSqrtD);
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (full_tile) {
+#pragma unroll
+        for (int e = 0; e < 64; e += 8) {
+            acc[0] += exp2_mixed<0>(fmaf(__uint_as_float(x[e + 0]), kLog2eOverSqrtD, -mn));
+            acc[1] += exp2_mixed<1>(fmaf(__uint_as_float(x[e + 1]), kLog2eOverSqrtD, -mn));
+            acc[2] += exp2_mixed<2>(fmaf(__uint_as_float(x[e + 2]), kLog2eOverSqrtD, -mn));
+            acc[3] += exp2_mixed<3>(fmaf(__uint_as_float(x[e + 3]), kLog2eOverSqrtD, -mn));
+            acc[4] += exp2_mixed<4>(fmaf(__uint_as_float(x[e + 4]), kLog2eOverSqrtD, -mn));
+            acc[5] += exp2_mixed<5>(fmaf(__uint_as_float(x[e + 5]), kLog2eOverSqrtD, -mn));
+            acc[6] += exp2_mixed<6>(fmaf(__uint_as_float(x[e + 6]), kLog2eOverSqrtD, -mn));
+            acc[7] += exp2_mixed<7>(fmaf(__uint_as_float(x[e + 7]), kLog2eOverSqrtD, -mn));
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 64; ++e)
+            if (j0 + e <= t_r) acc[e & 7] += ex2(fmaf(__uint_as_float(x[e]), kLog2eOverSqrtD, -mn));
+    }
+    const float sum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+    l = (m == -INFINITY ? 0.f : l * ex2(m - mn)) + sum;
+    m = mn;
+}
+
+// Sum over 64 query rows (columns q0 .. q0+63) of 2^(y - lse) for key j.
+__device__ __forceinline__ float prob_sum(const uint32_t (&x)[64], const float* lse, bool full_tile, int q0, int j,
+                                          const TcArgs& a) {
+    if (full_tile) {
+        const float4* L4 = reinterpret_cast<const float4*>(lse + q0);
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int e8 = 0; e8 < 8; ++e8) {
+            const float4 La = L4[2 * e8], Lb = L4[2 * e8 + 1];
+            const int e = 8 * e8;
+            acc[0] += exp2_mixed<0>(fmaf(__uint_as_float(x[e + 0]), kLog2eOverSqrtD, -La.x));
+            acc[1] += exp2_mixed<1>(fmaf(__uint_as_float(x[e + 1]), kLog2eOverSqrtD, -La.y));
+            acc[2] += exp2_mixed<2>(fmaf(__uint_as_float(x[e + 2]), kLog2eOverSqrtD, -La.z));
+            acc[3] += exp2_mixed<3>(fmaf(__uint_as_float(x[e + 3]), kLog2eOverSqrtD, -La.w));
+            acc[4] += exp2_mixed<4>(fmaf(__uint_as_float(x[e + 4]), kLog2eOverSqrtD, -Lb.x));
+            acc[5] += exp2_mixed<5>(fmaf(__uint_as_float(x[e + 5]), kLog2eOverSqrtD, -Lb.y));
+            acc[6] += exp2_mixed<6>(fmaf(__uint_as_float(x[e + 6]), kLog2eOverSqrtD, -Lb.z));
+            acc[7] += exp2_mixed<7>(fmaf(__uint_as_float(x[e + 7]), kLog2eOverSqrtD, -Lb.w));
+        }
+        return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+    }
+    float s = 0.f;
+#pragma unroll
+    for (int e = 0; e < 64; ++e) {
+        const int qr = q0 + e;
+        if (qr < a.nq && j <= a.N - a.w + (qr % a.w)) s += ex2(fmaf(__uint_as_float(x[e]), kLog2eOverSqrtD, -lse[qr]));
+    }
+    return s;
+}
 
 // ------------------------------------------------------------------------ the kernel
 
@@ -249,11 +414,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cta = blockIdx.x, P = a.P;
     const int n_local = cta < a.total_tiles ? (a.total_tiles - cta + P - 1) / P : 0;
+    volatile int* abort = &sm.abort;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&sm.full[s], 1);
-            mbar_init(&sm.empty[s], 1);
+        for (int s = 0; s < kStagesA; ++s) {
+            mbar_init(&sm.fullA[s], 1);
+            mbar_init(&sm.emptyA[s], 1);
+        }
+        for (int s = 0; s < kStagesB; ++s) {
+            mbar_init(&sm.fullB[s], 1);
+            mbar_init(&sm.emptyB[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.qfull[b], 1);
@@ -262,8 +432,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             mbar_init(&sm.d1empty[b], 4);
             mbar_init(&sm.d2full[b], 1);
             mbar_init(&sm.d2empty[b], 4);
+            mbar_init(&sm.pub_full[b], kQRows);
+            mbar_init(&sm.pub_empty[b], 1);
         }
         sm.abort = 0;
+        sm.p1_issued = 0;
+        sm.p2_issued = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
@@ -278,114 +452,114 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------------ producer
+    if (warp == 0 || warp == 2) {
+        // ------------------------------------------------------------ TMA producers
         if (lane == 0) {
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&a.tmap_k)) : "memory");
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&a.tmap_q)) : "memory");
-            JobIter it(n_local, a.lag);
-            int ph, i, k = 0;
-            int qunit[2] = {-1, -1}, qloads[2] = {0, 0};
-            while (it.next(ph, i)) {
+            const int ph = warp == 0 ? 0 : 1;
+            const CUtensorMap* mk = &a.tmap_k;
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(mk)) : "memory");
+            const uint64_t evict_first = policy_evict_first();
+            uint8_t(*ring)[kBoxBytes] = ph == 0 ? sm.ringA : sm.ringB;
+            uint64_t* full = ph == 0 ? sm.fullA : sm.fullB;
+            uint64_t* empty = ph == 0 ? sm.emptyA : sm.emptyB;
+            const int stages = ph == 0 ? kStagesA : kStagesB;
+            volatile int* mine = ph == 0 ? &sm.p1_issued : &sm.p2_issued;
+            volatile int* other = ph == 0 ? &sm.p2_issued : &sm.p1_issued;
+            int k = 0, qunit = -1, qloads = 0;
+            for (int i = 0; i < n_local && !*abort; ++i) {
                 const int t = cta + i * P, u = t / a.T_u, ti = t - u * a.T_u;
-                if (u != qunit[ph]) {
-                    if (qloads[ph] > 0) mbar_wait(&sm.qempty[ph], (qloads[ph] - 1) & 1, sm, a.err);
-                    mbar_expect_tx(&sm.qfull[ph], kTileBytes);
-                    tma_load_2d(sm.q[ph], &a.tmap_q, &sm.qfull[ph], 0, u * kQRows);
-                    tma_load_2d(sm.q[ph] + kHalfBytes, &a.tmap_q, &sm.qfull[ph], 64, u * kQRows);
-                    qunit[ph] = u;
-                    ++qloads[ph];
+                // phase 1 stays at most max_lead tiles ahead of phase 2 (L2 footprint);
+                // phase 2 never loads a tile before phase 1 has (so its read hits L2)
+                const long long t0 = globaltimer();
+                while (ph == 0 ? (i - *other >= a.max_lead) : (i >= *other)) {
+                    if (*abort) break;
+                    if (globaltimer() - t0 > kBarrierTimeoutNs) {
+                        atomicOr(a.err, kErrTimeout);
+                        *abort = 1;
+                        break;
+                    }
+                    __nanosleep(128);
                 }
-                const int s = k % kStages;
-                mbar_wait(&sm.empty[s], ((k / kStages) & 1) ^ 1, sm, a.err);
-                mbar_expect_tx(&sm.full[s], kTileBytes);
-                tma_load_3d(sm.ktile[s], &a.tmap_k, &sm.full[s], 0, ti * kTileKeys, u);
-                tma_load_3d(sm.ktile[s] + kHalfBytes, &a.tmap_k, &sm.full[s], 64, ti * kTileKeys, u);
-                ++k;
+                if (u != qunit) {
+                    if (qloads > 0) mbar_wait(&sm.qempty[ph], (qloads - 1) & 1, abort, a.err);
+                    mbar_expect_tx(&sm.qfull[ph], 2 * kBoxBytes);
+                    tma_load_2d(sm.q[ph], &a.tmap_q, &sm.qfull[ph], 0, u * kQRows);
+                    tma_load_2d(sm.q[ph] + kBoxBytes, &a.tmap_q, &sm.qfull[ph], 64, u * kQRows);
+                    qunit = u;
+                    ++qloads;
+                }
+                for (int h = 0; h < 2; ++h, ++k) {
+                    const int s = k % stages;
+                    mbar_wait(&empty[s], ((k / stages) & 1) ^ 1, abort, a.err);
+                    mbar_expect_tx(&full[s], kBoxBytes);
+                    if (ph == 0)
+                        tma_load_3d(ring[s], mk, &full[s], 64 * h, ti * kTileKeys, u);
+                    else
+                        tma_load_3d_hint(ring[s], mk, &full[s], 64 * h, ti * kTileKeys, u, evict_first);
+                }
+                *mine = i + 1;
             }
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------------ MMA issuer
+    } else if (warp == 1 || warp == 3) {
+        // ------------------------------------------------------------ MMA issuers
         if (lane == 0) {
-            JobIter it(n_local, a.lag);
-            int ph, i, k = 0, n1 = 0, n2 = 0;
-            int qunit[2] = {-1, -1}, qloads[2] = {0, 0};
-            while (it.next(ph, i)) {
+            const int ph = warp == 1 ? 0 : 1;
+            uint8_t(*ring)[kBoxBytes] = ph == 0 ? sm.ringA : sm.ringB;
+            uint64_t* full = ph == 0 ? sm.fullA : sm.fullB;
+            uint64_t* empty = ph == 0 ? sm.emptyA : sm.emptyB;
+            uint64_t* dfull = ph == 0 ? sm.d1full : sm.d2full;
+            uint64_t* dempty = ph == 0 ? sm.d1empty : sm.d2empty;
+            const int stages = ph == 0 ? kStagesA : kStagesB;
+            const uint32_t dbase = tmem + (ph == 0 ? 0u : 256u);
+            int k = 0, qunit = -1, qloads = 0;
+            for (int i = 0; i < n_local && !*abort; ++i) {
                 const int t = cta + i * P, u = t / a.T_u;
-                if (u != qunit[ph]) {
+                if (u != qunit) {
                     // the previous Q of this phase is free once every MMA issued so far is done
-                    if (qunit[ph] >= 0) umma_commit(&sm.qempty[ph]);
-                    mbar_wait(&sm.qfull[ph], qloads[ph] & 1, sm, a.err);
-                    qunit[ph] = u;
-                    ++qloads[ph];
+                    if (qunit >= 0) umma_commit(&sm.qempty[ph]);
+                    mbar_wait(&sm.qfull[ph], qloads & 1, abort, a.err);
+                    qunit = u;
+                    ++qloads;
                 }
-                const int s = k % kStages;
-                mbar_wait(&sm.full[s], (k / kStages) & 1, sm, a.err);
-                uint32_t d;
-                const uint8_t *A, *B;
-                uint64_t* done;
-                if (ph == 0) {
-                    const int b = n1 & 1;
-                    mbar_wait(&sm.d1empty[b], ((n1 >> 1) & 1) ^ 1, sm, a.err);
-                    d = tmem + b * 128;
-                    A = sm.q[0];
-                    B = sm.ktile[s];
-                    done = &sm.d1full[b];
-                    ++n1;
-                } else {
-                    const int b = n2 & 1;
-                    mbar_wait(&sm.d2empty[b], ((n2 >> 1) & 1) ^ 1, sm, a.err);
-                    d = tmem + 256 + b * 128;
-                    A = sm.ktile[s];
-                    B = sm.q[1];
-                    done = &sm.d2full[b];
-                    ++n2;
-                }
+                const int b = i & 1;
+                mbar_wait(&dempty[b], ((i >> 1) & 1) ^ 1, abort, a.err);
                 tc_fence_after();
+                const uint32_t d = dbase + b * 128;
+                for (int h = 0; h < 2; ++h, ++k) {
+                    const int s = k % stages;
+                    mbar_wait(&full[s], (k / stages) & 1, abort, a.err);
+                    tc_fence_after();
+                    const uint8_t* qbox = sm.q[ph] + h * kBoxBytes;
 #pragma unroll
-                for (int kk = 0; kk < kHeadDim / 16; ++kk) umma_bf16(d, tile_desc(A, kk), tile_desc(B, kk), kk > 0);
-                umma_commit(&sm.empty[s]);
-                umma_commit(done);
-                ++k;
+                    for (int kk = 0; kk < 4; ++kk) {
+                        if (ph == 0)
+                            umma_bf16(d, box_desc(qbox, kk), box_desc(ring[s], kk), (h | kk) != 0);
+                        else
+                            umma_bf16(d, box_desc(ring[s], kk), box_desc(qbox, kk), (h | kk) != 0);
+                    }
+                    umma_commit(&empty[s]);
+                }
+                umma_commit(&dfull[b]);
             }
         }
     } else if (warp >= 4 && warp < 8) {
-        // ------------------------------------------------------------------ phase 1: statistics
+        // ------------------------------------------------------------ phase 1: statistics
         const int r = threadIdx.x - 128;  // query row == TMEM lane
-        const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+        const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
         const int t_r = a.N - a.w + (r % a.w);  // last key this row sees
-        int cur = -1;
+        int cur = -1, npub = 0;
         float m = -INFINITY, l = 0.f;
         for (int i = 0; i <= n_local; ++i) {
             const int t = cta + i * P;
             const int u = i < n_local ? t / a.T_u : -2;
             if (u != cur && cur >= 0) {
-                // publish this CTA's (max, sum) of unit `cur`; the last CTA merges them
-                a.partial[((size_t)cur * kQRows + r) * kMaxCtas + cta] = make_float2(m, l);
-                named_sync(1, 128);
-                if (r == 0) {
-                    __threadfence();
-                    const int n_contrib = min(a.T_u, P);
-                    const unsigned old = atomicAdd(&a.count[cur], 1u);
-                    sm.flag1 = (old == (unsigned)(n_contrib - 1));
-                }
-                named_sync(1, 128);
-                if (sm.flag1) {
-                    __threadfence();
-                    const int n_contrib = min(a.T_u, P);
-                    const float2* pr = a.partial + ((size_t)cur * kQRows + r) * kMaxCtas;
-                    float M = -INFINITY;
-                    for (int c = 0; c < n_contrib; ++c) M = fmaxf(M, __ldcg(pr + (cur * a.T_u + c) % P).x);
-                    float S = 0.f;
-                    for (int c = 0; c < n_contrib; ++c) {
-                        const float2 v = __ldcg(pr + (cur * a.T_u + c) % P);
-                        if (v.x != -INFINITY) S += v.y * exp2f(v.x - M);
-                    }
-                    a.lse[(size_t)cur * kQRows + r] = M + log2f(S);
-                    __threadfence();
-                    named_sync(1, 128);
-                    if (r == 0) atomicExch(&a.ready[cur], 1u);
-                }
+                // hand this CTA's (max, sum) of unit `cur` to the publisher warp
+                const int slot = npub & 1;
+                mbar_wait(&sm.pub_empty[slot], ((npub >> 1) & 1) ^ 1, abort, a.err);
+                sm.pub[slot][r] = make_float2(m, l);
+                if (r == 0) sm.pub_unit[slot] = cur;
+                mbar_arrive(&sm.pub_full[slot]);
+                ++npub;
             }
             if (i == n_local) break;
             if (u != cur) {
@@ -395,51 +569,32 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             }
             const int ti = t - u * a.T_u;
             const int b = i & 1;
-            mbar_wait(&sm.d1full[b], (i >> 1) & 1, sm, a.err);
+            mbar_wait(&sm.d1full[b], (i >> 1) & 1, abort, a.err);
             tc_fence_after();
             const bool full_tile = (ti + 1) * kTileKeys <= a.N - a.w + 1;
             const int j0 = ti * kTileKeys;
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                uint32_t x[32];
+            {
+                uint32_t x[64];
                 __syncwarp();
-                tmem_ld32(tmem + lane_base + b * 128 + c * 32, x);
-                tmem_wait(x);
-                if (c == 3) {
-                    // the accumulator is free for the next MMA once all four chunks are loaded
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm.d1empty[b]);
-                }
-                float cm = -INFINITY;
-                if (full_tile) {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) cm = fmaxf(cm, __uint_as_float(x[e]));
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (j0 + c * 32 + e <= t_r) cm = fmaxf(cm, __uint_as_float(x[e]));
-                }
-                if (cm != -INFINITY) {
-                    const float mn = fmaxf(m, cm * kLog2eOverSqrtD);
-                    float sum = 0.f;
-                    if (full_tile) {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) sum += ex2(fmaf(__uint_as_float(x[e]), kLog2eOverSqrtD, -mn));
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (j0 + c * 32 + e <= t_r) sum += ex2(fmaf(__uint_as_float(x[e]), kLog2eOverSqrtD, -mn));
-                    }
-                    l = (m == -INFINITY ? 0.f : l * ex2(m - mn)) + sum;
-                    m = mn;
-                }
+                tmem_ld64(tl + b * 128, x);
+                tmem_wait64(x);
+                stats_update(x, full_tile, j0, t_r, m, l);
+            }
+            {
+                uint32_t x[64];
+                __syncwarp();
+                tmem_ld64(tl + b * 128 + 64, x);
+                tmem_wait64(x);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.d1empty[b]);
+                stats_update(x, full_tile, j0 + 64, t_r, m, l);
             }
         }
-    } else if (warp >= 8) {
-        // ------------------------------------------------------------------ phase 2: scores
+    } else if (warp >= 8 && warp < 12) {
+        // ------------------------------------------------------------ phase 2: scores
         const int r = threadIdx.x - 256;  // key within the tile == TMEM lane
-        const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+        const uint32_t tl = tmem + 256 + ((uint32_t)(32 * (warp & 3)) << 16);
         int cur = -1;
         bool gave_up = false;
         for (int i = 0; i < n_local; ++i) {
@@ -466,42 +621,84 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                 cur = u;
             }
             const int b = i & 1;
-            mbar_wait(&sm.d2full[b], (i >> 1) & 1, sm, a.err);
+            mbar_wait(&sm.d2full[b], (i >> 1) & 1, abort, a.err);
             tc_fence_after();
             const int j = ti * kTileKeys + r;
             const bool full_tile = (ti + 1) * kTileKeys <= a.N - a.w + 1;
-            float s = 0.f;
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                uint32_t x[32];
+            float s;
+            {
+                uint32_t x[64];
                 __syncwarp();
-                tmem_ld32(tmem + lane_base + 256 + b * 128 + c * 32, x);
-                tmem_wait(x);
-                if (c == 3) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm.d2empty[b]);
-                }
-                const float4* L4 = reinterpret_cast<const float4*>(sm.lse + c * 32);
-                if (full_tile) {
-#pragma unroll
-                    for (int e4 = 0; e4 < 8; ++e4) {
-                        const float4 L = L4[e4];
-                        s += ex2(fmaf(__uint_as_float(x[4 * e4 + 0]), kLog2eOverSqrtD, -L.x));
-                        s += ex2(fmaf(__uint_as_float(x[4 * e4 + 1]), kLog2eOverSqrtD, -L.y));
-                        s += ex2(fmaf(__uint_as_float(x[4 * e4 + 2]), kLog2eOverSqrtD, -L.z));
-                        s += ex2(fmaf(__uint_as_float(x[4 * e4 + 3]), kLog2eOverSqrtD, -L.w));
-                    }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int qr = c * 32 + e;
-                        if (qr < a.nq && j <= a.N - a.w + (qr % a.w))
-                            s += ex2(fmaf(__uint_as_float(x[e]), kLog2eOverSqrtD, -sm.lse[qr]));
-                    }
-                }
+                tmem_ld64(tl + b * 128, x);
+                tmem_wait64(x);
+                s = prob_sum(x, sm.lse, full_tile, 0, j, a);
+            }
+            {
+                uint32_t x[64];
+                __syncwarp();
+                tmem_ld64(tl + b * 128 + 64, x);
+                tmem_wait64(x);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.d2empty[b]);
+                s += prob_sum(x, sm.lse, full_tile, 64, j, a);
             }
             if (j < a.N) a.unit_scores[(size_t)u * a.N + j] = s;
+        }
+    } else if (warp == 12) {
+        // ------------------------------------------------------------ publisher / merger
+        int cur = -1, npub = 0;
+        for (int i = 0; i < n_local; ++i) {
+            const int u = (cta + i * P) / a.T_u;
+            const bool last_tile_of_unit = (i + 1 == n_local) || ((cta + (i + 1) * P) / a.T_u != u);
+            cur = u;
+            if (!last_tile_of_unit) continue;
+            const int slot = npub & 1;
+            mbar_wait(&sm.pub_full[slot], (npub >> 1) & 1, abort, a.err);
+            float2* dst = a.partial + ((size_t)cur * kMaxCtas + cta) * kQRows;
+#pragma unroll
+            for (int k4 = 0; k4 < kQRows / 32; ++k4) dst[lane + 32 * k4] = sm.pub[slot][lane + 32 * k4];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.pub_empty[slot]);
+            ++npub;
+            __threadfence();
+            __syncwarp();
+            // first level: the last CTA of this 16-CTA group merges the group's partials
+            const Contributors con(a, cur);
+            const int g = cta / kGroup;
+            unsigned old = 0;
+            if (lane == 0) old = atomicAdd(&a.gcount[cur * kMaxGroups + g], 1u);
+            old = __shfl_sync(0xffffffffu, old, 0);
+            if (old + 1 != (unsigned)con.group_size(g)) continue;
+            __threadfence();
+            const float2* gsrc = a.partial + ((size_t)cur * kMaxCtas + g * kGroup) * kQRows;
+            const int gn = min(kGroup, P - g * kGroup);
+            float2* gdst = a.gpartial + ((size_t)cur * kMaxGroups + g) * kQRows;
+#pragma unroll 1
+            for (int k4 = 0; k4 < kQRows / 32; ++k4) {
+                const int row = lane + 32 * k4;
+                gdst[row] = merge_row(gsrc + row, gn, kQRows, [&](int c) { return con.has(g * kGroup + c); });
+            }
+            __threadfence();
+            __syncwarp();
+            // second level: the last group of the unit merges the groups into lse
+            int n_groups = 0;
+            for (int gg = 0; gg * kGroup < P; ++gg) n_groups += con.group_size(gg) > 0;
+            if (lane == 0) old = atomicAdd(&a.count[cur], 1u);
+            old = __shfl_sync(0xffffffffu, old, 0);
+            if (old + 1 != (unsigned)n_groups) continue;
+            __threadfence();
+            const float2* usrc = a.gpartial + (size_t)cur * kMaxGroups * kQRows;
+            const int ng_all = (P + kGroup - 1) / kGroup;
+#pragma unroll 1
+            for (int k4 = 0; k4 < kQRows / 32; ++k4) {
+                const int row = lane + 32 * k4;
+                const float2 ms = merge_row(usrc + row, ng_all, kQRows, [&](int gg) { return con.group_size(gg) > 0; });
+                a.lse[(size_t)cur * kQRows + row] = ms.x + log2f(ms.y);
+            }
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) atomicExch(&a.ready[cur], 1u);
         }
     }
 
@@ -534,12 +731,16 @@ __global__ void tc_prep_kernel(const __nv_bfloat16* __restrict__ q, __nv_bfloat1
         flags[e] = 0u;
 }
 
+__global__ void exp2_poly_kernel(const float* __restrict__ y, float* __restrict__ out, int n) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) out[i] = exp2_poly(y[i]);
+}
+
 // ------------------------------------------------------------------------ host side
 
 size_t a256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct TcLayout {
-    size_t qpad, partial, lse, flags, total;
+    size_t qpad, partial, gpartial, lse, flags, n_flags, total;
 };
 
 TcLayout tc_layout(int U) {
@@ -548,11 +749,14 @@ TcLayout tc_layout(int U) {
     L.qpad = off;
     off = a256(off + (size_t)U * kQRows * kHeadDim * 2);
     L.partial = off;
-    off = a256(off + (size_t)U * kQRows * kMaxCtas * sizeof(float2));
+    off = a256(off + (size_t)U * kMaxCtas * kQRows * sizeof(float2));
+    L.gpartial = off;
+    off = a256(off + (size_t)U * kMaxGroups * kQRows * sizeof(float2));
     L.lse = off;
     off = a256(off + (size_t)U * kQRows * sizeof(float));
-    L.flags = off;  // count[U], ready[U], never
-    off = a256(off + (size_t)(2 * U + 1) * sizeof(unsigned));
+    L.flags = off;  // gcount[U][kMaxGroups], count[U], ready[U], never
+    L.n_flags = (size_t)U * kMaxGroups + 2 * (size_t)U + 1;
+    off = a256(off + L.n_flags * sizeof(unsigned));
     L.total = off;
     return L;
 }
@@ -571,17 +775,24 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 int sm_count() {
-    static int cache[64] = {0};
+    static std::atomic<int> cache[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-    if (dev < 64 && cache[dev]) return cache[dev];
+    if (dev < 64 && cache[dev].load()) return cache[dev].load();
     int n = 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    if (dev < 64) cache[dev] = n;
+    if (dev < 64) cache[dev].store(n);
     return n;
 }
 
 }  // namespace
+
+cudaError_t debug_exp2(const float* y, float* out, int n, cudaStream_t s) {
+    if (n <= 0) return cudaSuccess;
+    exp2_poly_kernel<<<std::min((n + 255) / 256, 148 * 4), 256, 0, s>>>(y, out, n);
+    count_launches(1);
+    return cudaGetLastError();
+}
 
 bool tc_score_supported(const ScoreJob& j) {
     return j.dtype == KVC_BF16 && j.nq >= 1 && j.nq <= kQRows && j.N >= 1 && j.U >= 1 &&
@@ -600,10 +811,12 @@ cudaError_t tc_score(const ScoreJob& j, cudaStream_t s) {
     TcArgs a{};
     a.unit_scores = j.unit_scores;
     a.partial = (float2*)(ws + L.partial);
+    a.gpartial = (float2*)(ws + L.gpartial);
     a.lse = (float*)(ws + L.lse);
-    a.count = flags;
-    a.ready = flags + j.U;
-    a.never = flags + 2 * j.U;
+    a.gcount = flags;
+    a.count = flags + (size_t)j.U * kMaxGroups;
+    a.ready = a.count + j.U;
+    a.never = a.ready + j.U;
     a.err = j.err;
     a.spin_limit = j.spin_limit;
     a.U = j.U;
@@ -614,8 +827,10 @@ cudaError_t tc_score(const ScoreJob& j, cudaStream_t s) {
     a.total_tiles = a.U * a.T_u;
     const int n_sm = sm_count();
     if (n_sm <= 0) return cudaErrorNoDevice;
-    a.P = min(min(n_sm, kMaxCtas), a.total_tiles);
-    a.lag = (a.T_u + a.P - 1) / a.P + 1;
+    a.P = std::min(std::min(n_sm, kMaxCtas), a.total_tiles);
+    // phase 1 may run this many tiles ahead of phase 2: a unit's worth plus slack for the
+    // merge, while keeping the tiles between the two reads (max_lead x P x 32 KiB) in L2
+    a.max_lead = (a.T_u + a.P - 1) / a.P + 8;
     a.inject = j.inject_timeout;
 
     auto encode = encode_fn();
@@ -643,7 +858,7 @@ cudaError_t tc_score(const ScoreJob& j, cudaStream_t s) {
 
     const long long pieces = (long long)j.U * kQRows * (kHeadDim / 8);
     const int prep_grid = (int)std::min<long long>((pieces + 255) / 256, 148LL * 8);
-    tc_prep_kernel<<<prep_grid, 256, 0, s>>>((const __nv_bfloat16*)j.q, qpad, j.U, j.nq, flags, 2 * j.U + 1);
+    tc_prep_kernel<<<prep_grid, 256, 0, s>>>((const __nv_bfloat16*)j.q, qpad, j.U, j.nq, flags, (int)L.n_flags);
     count_launches(1);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

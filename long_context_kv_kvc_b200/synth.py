@@ -80,13 +80,16 @@ LLAMA8B_32K = Workload("llama8b-32k", B=1, Hq=32, Hkv=8, N=32768, D=128, window=
                        pool_kernel=7, kv_budget=2048)
 LLAMA8B_128K_B4 = Workload("llama8b-128k-b4", B=4, Hq=32, Hkv=8, N=131072, D=128, window=32,
                            dtype="bf16", pool_kernel=7, kv_budget=4096, seeds=(0, 1, 2, 3))
+LLAMA8B_128K_B1 = Workload("llama8b-128k-b1", B=1, Hq=32, Hkv=8, N=131072, D=128, window=32,
+                           dtype="bf16", pool_kernel=7, kv_budget=4096)
 STRUCTKV_8L_32K = Workload("structkv-8layer-32k", B=1, Hq=32, Hkv=8, N=32768, D=128, window=32,
                            dtype="bf16", pool_kernel=7, kv_budget=2048, n_layers=8,
                            scope=SCOPE_ALL_HEADS, hub_shared_frac=0.6)
 FASTKV_TSP_64K = Workload("fastkv-tsp20-64k", B=1, Hq=32, Hkv=8, N=65536, D=128, window=32,
                           dtype="bf16", pool_kernel=7, kv_budget=1024, tsp_rate=0.2, hidden_dim=4096)
 
-WORKLOADS = {w.name: w for w in (TINY, LLAMA8B_32K, LLAMA8B_128K_B4, STRUCTKV_8L_32K, FASTKV_TSP_64K)}
+WORKLOADS = {w.name: w for w in (TINY, LLAMA8B_32K, LLAMA8B_128K_B4, LLAMA8B_128K_B1, STRUCTKV_8L_32K,
+                                 FASTKV_TSP_64K)}
 
 
 def _stream(seed: int, *key: int) -> np.random.Generator:
