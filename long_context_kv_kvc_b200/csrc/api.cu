@@ -227,7 +227,11 @@ kvc_status kvc_topk(const float* pooled, int32_t B, int32_t H, int32_t N, int32_
     (void)ws_bytes;
     if (!pooled || !idx || B < 1 || H < 1 || N < 1 || n_sink < 0 || window < 0) return KVC_ERR_ARG;
     KVC_TRY(check_budget(N, n_sink, window, budget));
-    KVC_CUDA(kvc::topk(pooled, B * H, N, n_sink, window, budget, idx, (cudaStream_t)stream));
+    if (kvc::topk_fused_fits(N, n_sink, window)) {
+        KVC_CUDA(kvc::topk_fused(pooled, B * H, N, n_sink, window, budget, 1, idx, (cudaStream_t)stream));
+    } else {
+        KVC_CUDA(kvc::topk(pooled, B * H, N, n_sink, window, budget, idx, (cudaStream_t)stream));
+    }
     return KVC_OK;
 }
 
@@ -277,20 +281,28 @@ kvc_status kvc_compress(const kvc_params* p, const void* q, const void* k, const
     KVC_TRY(run_score(p, P, q, k, scores, w, s));
 
     KVC_TRY(record_stage(p, KVC_STAGE_SELECT, s));
-    KVC_CUDA(kvc::pool(scores, pooled, B * P.Hs, N, S, N - win, p->pool_kernel, s));
-    KVC_CUDA(kvc::topk(pooled, B * P.Hs, N, S, win, p->kv_budget, idx_out, s));
-    float* tsp_pooled = nullptr;
+    const bool fused = kvc::topk_fused_fits(N, S, win);
+    if (fused) {
+        KVC_CUDA(kvc::topk_fused(scores, B * P.Hs, N, S, win, p->kv_budget, p->pool_kernel, idx_out, s));
+    } else {
+        KVC_CUDA(kvc::pool(scores, pooled, B * P.Hs, N, S, N - win, p->pool_kernel, s));
+        KVC_CUDA(kvc::topk(pooled, B * P.Hs, N, S, win, p->kv_budget, idx_out, s));
+    }
     if (tsp) {
         float* tsp_scores = (float*)(w + P.off_tsp_scores);
-        tsp_pooled = (float*)(w + P.off_tsp_pooled);
+        float* tsp_pooled = (float*)(w + P.off_tsp_pooled);
         const float* src = scores;
         if (P.Hs > 1) {
             KVC_CUDA(cudaMemsetAsync(tsp_scores, 0, (size_t)B * N * sizeof(float), s));
             KVC_CUDA(kvc::accumulate(tsp_scores, scores, B, P.Hs, 1, N, s));
             src = tsp_scores;
         }
-        KVC_CUDA(kvc::pool(src, tsp_pooled, B, N, S, N - win, p->pool_kernel, s));
-        KVC_CUDA(kvc::topk(tsp_pooled, B, N, S, win, P.n_tsp, tsp_idx_out, s));
+        if (fused) {
+            KVC_CUDA(kvc::topk_fused(src, B, N, S, win, P.n_tsp, p->pool_kernel, tsp_idx_out, s));
+        } else {
+            KVC_CUDA(kvc::pool(src, tsp_pooled, B, N, S, N - win, p->pool_kernel, s));
+            KVC_CUDA(kvc::topk(tsp_pooled, B, N, S, win, P.n_tsp, tsp_idx_out, s));
+        }
     }
 
     KVC_TRY(record_stage(p, KVC_STAGE_GATHER, s));

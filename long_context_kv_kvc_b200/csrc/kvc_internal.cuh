@@ -70,6 +70,11 @@ cudaError_t pool(const float* in, float* out, int rows, int N, int lo, int hi, i
                  cudaStream_t s);
 cudaError_t topk(const float* pooled, int rows, int N, int n_sink, int window, int budget,
                  int32_t* idx, cudaStream_t s);
+// pool (odd width `kernel` over [n_sink, N - window)) and top-k in one launch, one 8-CTA
+// cluster per row; for rows whose candidates fit the clusters' shared memory
+bool topk_fused_fits(int N, int n_sink, int window);
+cudaError_t topk_fused(const float* scores, int rows, int N, int n_sink, int window, int budget, int kernel,
+                       int32_t* idx, cudaStream_t s);
 // two gathers of the same shape in one launch (src1/dst1 may be null)
 cudaError_t gather(const void* src0, void* dst0, const void* src1, void* dst1, int B, int Hsrc,
                    int N, size_t row_bytes, const int32_t* idx, int Hidx, int K, unsigned* err,

@@ -27,7 +27,8 @@
 // The two phases have separate TMA producers, shared-memory rings (16 KiB half-tiles of
 // 64 columns, the 128-byte swizzle atom) and MMA issuers, so a phase-2 wait never stalls
 // the HBM stream.  Warps: 0 phase-1 TMA, 1 TMEM owner + phase-1 MMA, 2 phase-2 TMA,
-// 3 phase-2 MMA, 4-7 phase-1 statistics, 8-11 phase-2 sums, 12 publisher.  Every wait is
+// 3 phase-2 MMA, 4-11 phase-1 statistics (two warpgroups, one per TMEM accumulator),
+// 12-19 phase-2 sums (likewise), 20-23 publisher (one thread per query row).  Every wait is
 // bounded: a wait that runs out sets the per-device error word and the kernel still ends.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -45,7 +46,7 @@ constexpr int kQRows = 128;                            // query rows per unit (p
 constexpr int kBoxBytes = kTileKeys * 64 * 2;          // a 128-row x 64-column bf16 box: 16 KiB
 constexpr int kStagesA = 6;                            // phase-1 ring (HBM stream)
 constexpr int kStagesB = 3;                            // phase-2 ring (L2 re-read)
-constexpr int kWarps = 13;
+constexpr int kWarps = 24;  // 4 producer/MMA, 2 x 4 phase-1, 2 x 4 phase-2, 4 publisher
 constexpr int kThreads = kWarps * 32;
 constexpr int kMaxCtas = 160;                          // partial slots per unit (>= #SMs)
 constexpr int kGroup = 16;                             // CTAs per first-level merge group
@@ -77,8 +78,8 @@ struct __align__(1024) Smem {
     uint8_t ringA[kStagesA][kBoxBytes];
     uint8_t ringB[kStagesB][kBoxBytes];
     uint8_t q[2][2 * kBoxBytes];  // Q of the current unit of phase 1 / phase 2 (two boxes)
-    float lse[kQRows];
-    float2 pub[2][kQRows];
+    float lse[2][kQRows];         // per phase-2 warpgroup
+    float2 pub[2][2][kQRows];     // [slot][phase-1 warpgroup][row]
     int pub_unit[2];
     uint64_t fullA[kStagesA], emptyA[kStagesA], fullB[kStagesB], emptyB[kStagesB];
     uint64_t qfull[2], qempty[2];
@@ -86,7 +87,8 @@ struct __align__(1024) Smem {
     uint64_t pub_full[2], pub_empty[2];
     uint32_t tmem_base;
     int abort;
-    int flag2;
+    int flag2[2];
+    int pub_flag;
     int p1_issued, p2_issued;  // tiles whose loads each producer has issued (L2 lead control)
 };
 
@@ -208,39 +210,29 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                  : "memory");
 }
 
-// 64 consecutive fp32 columns of this thread's TMEM lane (one tcgen05.ld).  The values are
-// only valid after tmem_wait64, which takes them as in/out operands so that no use can be
+// 32 consecutive fp32 columns of this thread's TMEM lane (one tcgen05.ld).  The values are
+// only valid after tmem_wait32, which takes them as in/out operands so that no use can be
 // scheduled before the wait.
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {"
         "%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
-        "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
-        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63"
-        "}, [%64];"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31"
+        "}, [%32];"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
           "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
-          "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
-          "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
-          "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
-          "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr)
         : "memory");
 }
 
-__device__ __forceinline__ void tmem_wait64(uint32_t (&r)[64]) {
+__device__ __forceinline__ void tmem_wait32(uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;"
                  : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
                    "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
                    "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
-                   "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]),
-                   "+r"(r[32]), "+r"(r[33]), "+r"(r[34]), "+r"(r[35]), "+r"(r[36]), "+r"(r[37]), "+r"(r[38]), "+r"(r[39]),
-                   "+r"(r[40]), "+r"(r[41]), "+r"(r[42]), "+r"(r[43]), "+r"(r[44]), "+r"(r[45]), "+r"(r[46]), "+r"(r[47]),
-                   "+r"(r[48]), "+r"(r[49]), "+r"(r[50]), "+r"(r[51]), "+r"(r[52]), "+r"(r[53]), "+r"(r[54]), "+r"(r[55]),
-                   "+r"(r[56]), "+r"(r[57]), "+r"(r[58]), "+r"(r[59]), "+r"(r[60]), "+r"(r[61]), "+r"(r[62]), "+r"(r[63])
+                   "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
                  :
                  : "memory");
 }
@@ -334,76 +326,54 @@ __device__ __forceinline__ float2 merge_row(const float2* src, int n, size_t str
     return make_float2(M, S);
 }
 
-// Online (max, sum) update of one query row with 64 logits (keys j0 .. j0+63); keys after
-// t_r are masked unless the whole tile is visible.
-__device__ __forceinline__ void stats_update(const uint32_t (&x)[64], bool full_tile, int j0, int t_r, float& m,
-                                             float& l) {
-    float cm = -INFINITY;
-    if (full_tile) {
-        float mx[8];
+// Online (max, sum) update of one query row with 32 logits (invisible keys already set
+// to -inf).
+__device__ __forceinline__ void stats_update(const uint32_t (&x)[32], float& m, float& l) {
+    float mx[8];
 #pragma unroll
-        for (int g = 0; g < 8; ++g) mx[g] = __uint_as_float(x[g]);
+    for (int g = 0; g < 8; ++g) mx[g] = __uint_as_float(x[g]);
 #pragma unroll
-        for (int e = 8; e < 64; ++e) mx[e & 7] = fmaxf(mx[e & 7], __uint_as_float(x[e]));
-        cm = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-    } else {
-#pragma unroll
-        for (int e = 0; e < 64; ++e)
-            if (j0 + e <= t_r) cm = fmaxf(cm, __uint_as_float(x[e]));
-    }
+    for (int e = 8; e < 32; ++e) mx[e & 7] = fmaxf(mx[e & 7], __uint_as_float(x[e]));
+    const float cm =
+        fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
     if (cm == -INFINITY) return;
     const float mn = fmaxf(m, cm * kLog2eOverSqrtD);
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    if (full_tile) {
 #pragma unroll
-        for (int e = 0; e < 64; e += 8) {
-            acc[0] += exp2_mixed<0>(fmaf(__uint_as_float(x[e + 0]), kLog2eOverSqrtD, -mn));
-            acc[1] += exp2_mixed<1>(fmaf(__uint_as_float(x[e + 1]), kLog2eOverSqrtD, -mn));
-            acc[2] += exp2_mixed<2>(fmaf(__uint_as_float(x[e + 2]), kLog2eOverSqrtD, -mn));
-            acc[3] += exp2_mixed<3>(fmaf(__uint_as_float(x[e + 3]), kLog2eOverSqrtD, -mn));
-            acc[4] += exp2_mixed<4>(fmaf(__uint_as_float(x[e + 4]), kLog2eOverSqrtD, -mn));
-            acc[5] += exp2_mixed<5>(fmaf(__uint_as_float(x[e + 5]), kLog2eOverSqrtD, -mn));
-            acc[6] += exp2_mixed<6>(fmaf(__uint_as_float(x[e + 6]), kLog2eOverSqrtD, -mn));
-            acc[7] += exp2_mixed<7>(fmaf(__uint_as_float(x[e + 7]), kLog2eOverSqrtD, -mn));
-        }
-    } else {
-#pragma unroll
-        for (int e = 0; e < 64; ++e)
-            if (j0 + e <= t_r) acc[e & 7] += ex2(fmaf(__uint_as_float(x[e]), kLog2eOverSqrtD, -mn));
+    for (int e = 0; e < 32; e += 8) {
+        acc[0] += exp2_mixed<0>(fmaf(__uint_as_float(x[e + 0]), kLog2eOverSqrtD, -mn));
+        acc[1] += exp2_mixed<1>(fmaf(__uint_as_float(x[e + 1]), kLog2eOverSqrtD, -mn));
+        acc[2] += exp2_mixed<2>(fmaf(__uint_as_float(x[e + 2]), kLog2eOverSqrtD, -mn));
+        acc[3] += exp2_mixed<3>(fmaf(__uint_as_float(x[e + 3]), kLog2eOverSqrtD, -mn));
+        acc[4] += exp2_mixed<4>(fmaf(__uint_as_float(x[e + 4]), kLog2eOverSqrtD, -mn));
+        acc[5] += exp2_mixed<5>(fmaf(__uint_as_float(x[e + 5]), kLog2eOverSqrtD, -mn));
+        acc[6] += exp2_mixed<6>(fmaf(__uint_as_float(x[e + 6]), kLog2eOverSqrtD, -mn));
+        acc[7] += exp2_mixed<7>(fmaf(__uint_as_float(x[e + 7]), kLog2eOverSqrtD, -mn));
     }
     const float sum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
     l = (m == -INFINITY ? 0.f : l * ex2(m - mn)) + sum;
     m = mn;
 }
 
-// Sum over 64 query rows (columns q0 .. q0+63) of 2^(y - lse) for key j.
-__device__ __forceinline__ float prob_sum(const uint32_t (&x)[64], const float* lse, bool full_tile, int q0, int j,
-                                          const TcArgs& a) {
-    if (full_tile) {
-        const float4* L4 = reinterpret_cast<const float4*>(lse + q0);
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+// Sum over 32 query rows (invisible ones already set to -inf) of 2^(y - lse) for this
+// thread's key.
+__device__ __forceinline__ float prob_sum(const uint32_t (&x)[32], const float* lse) {
+    const float4* L4 = reinterpret_cast<const float4*>(lse);
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int e8 = 0; e8 < 8; ++e8) {
-            const float4 La = L4[2 * e8], Lb = L4[2 * e8 + 1];
-            const int e = 8 * e8;
-            acc[0] += exp2_mixed<0>(fmaf(__uint_as_float(x[e + 0]), kLog2eOverSqrtD, -La.x));
-            acc[1] += exp2_mixed<1>(fmaf(__uint_as_float(x[e + 1]), kLog2eOverSqrtD, -La.y));
-            acc[2] += exp2_mixed<2>(fmaf(__uint_as_float(x[e + 2]), kLog2eOverSqrtD, -La.z));
-            acc[3] += exp2_mixed<3>(fmaf(__uint_as_float(x[e + 3]), kLog2eOverSqrtD, -La.w));
-            acc[4] += exp2_mixed<4>(fmaf(__uint_as_float(x[e + 4]), kLog2eOverSqrtD, -Lb.x));
-            acc[5] += exp2_mixed<5>(fmaf(__uint_as_float(x[e + 5]), kLog2eOverSqrtD, -Lb.y));
-            acc[6] += exp2_mixed<6>(fmaf(__uint_as_float(x[e + 6]), kLog2eOverSqrtD, -Lb.z));
-            acc[7] += exp2_mixed<7>(fmaf(__uint_as_float(x[e + 7]), kLog2eOverSqrtD, -Lb.w));
-        }
-        return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+    for (int e8 = 0; e8 < 4; ++e8) {
+        const float4 La = L4[2 * e8], Lb = L4[2 * e8 + 1];
+        const int e = 8 * e8;
+        acc[0] += exp2_mixed<0>(fmaf(__uint_as_float(x[e + 0]), kLog2eOverSqrtD, -La.x));
+        acc[1] += exp2_mixed<1>(fmaf(__uint_as_float(x[e + 1]), kLog2eOverSqrtD, -La.y));
+        acc[2] += exp2_mixed<2>(fmaf(__uint_as_float(x[e + 2]), kLog2eOverSqrtD, -La.z));
+        acc[3] += exp2_mixed<3>(fmaf(__uint_as_float(x[e + 3]), kLog2eOverSqrtD, -La.w));
+        acc[4] += exp2_mixed<4>(fmaf(__uint_as_float(x[e + 4]), kLog2eOverSqrtD, -Lb.x));
+        acc[5] += exp2_mixed<5>(fmaf(__uint_as_float(x[e + 5]), kLog2eOverSqrtD, -Lb.y));
+        acc[6] += exp2_mixed<6>(fmaf(__uint_as_float(x[e + 6]), kLog2eOverSqrtD, -Lb.z));
+        acc[7] += exp2_mixed<7>(fmaf(__uint_as_float(x[e + 7]), kLog2eOverSqrtD, -Lb.w));
     }
-    float s = 0.f;
-#pragma unroll
-    for (int e = 0; e < 64; ++e) {
-        const int qr = q0 + e;
-        if (qr < a.nq && j <= a.N - a.w + (qr % a.w)) s += ex2(fmaf(__uint_as_float(x[e]), kLog2eOverSqrtD, -lse[qr]));
-    }
-    return s;
+    return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
 }
 
 // ------------------------------------------------------------------------ the kernel
@@ -432,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             mbar_init(&sm.d1empty[b], 4);
             mbar_init(&sm.d2full[b], 1);
             mbar_init(&sm.d2empty[b], 4);
-            mbar_init(&sm.pub_full[b], kQRows);
+            mbar_init(&sm.pub_full[b], 2 * kQRows);
             mbar_init(&sm.pub_empty[b], 1);
         }
         sm.abort = 0;
@@ -542,10 +512,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                 umma_commit(&dfull[b]);
             }
         }
-    } else if (warp >= 4 && warp < 8) {
+    } else if (warp >= 4 && warp < 12) {
         // ------------------------------------------------------------ phase 1: statistics
-        const int r = threadIdx.x - 128;  // query row == TMEM lane
-        const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+        // warpgroup w takes the local tiles i with i % 2 == w (accumulator buffer w)
+        const int w = (warp - 4) >> 2;
+        const int r = threadIdx.x - 128 - 128 * w;  // query row == TMEM lane
+        const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + w * 128;
         const int t_r = a.N - a.w + (r % a.w);  // last key this row sees
         int cur = -1, npub = 0;
         float m = -INFINITY, l = 0.f;
@@ -553,11 +525,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             const int t = cta + i * P;
             const int u = i < n_local ? t / a.T_u : -2;
             if (u != cur && cur >= 0) {
-                // hand this CTA's (max, sum) of unit `cur` to the publisher warp
+                // hand this warpgroup's (max, sum) of unit `cur` to the publisher warp
                 const int slot = npub & 1;
                 mbar_wait(&sm.pub_empty[slot], ((npub >> 1) & 1) ^ 1, abort, a.err);
-                sm.pub[slot][r] = make_float2(m, l);
-                if (r == 0) sm.pub_unit[slot] = cur;
+                sm.pub[slot][w][r] = make_float2(m, l);
+                if (r == 0 && w == 0) sm.pub_unit[slot] = cur;
                 mbar_arrive(&sm.pub_full[slot]);
                 ++npub;
             }
@@ -567,40 +539,45 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                 m = -INFINITY;
                 l = 0.f;
             }
+            if ((i & 1) != w) continue;
             const int ti = t - u * a.T_u;
-            const int b = i & 1;
-            mbar_wait(&sm.d1full[b], (i >> 1) & 1, abort, a.err);
+            mbar_wait(&sm.d1full[w], (i >> 1) & 1, abort, a.err);
             tc_fence_after();
             const bool full_tile = (ti + 1) * kTileKeys <= a.N - a.w + 1;
-            const int j0 = ti * kTileKeys;
-            {
-                uint32_t x[64];
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t x[32];
                 __syncwarp();
-                tmem_ld64(tl + b * 128, x);
-                tmem_wait64(x);
-                stats_update(x, full_tile, j0, t_r, m, l);
-            }
-            {
-                uint32_t x[64];
-                __syncwarp();
-                tmem_ld64(tl + b * 128 + 64, x);
-                tmem_wait64(x);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.d1empty[b]);
-                stats_update(x, full_tile, j0 + 64, t_r, m, l);
+                tmem_ld32(tl + c * 32, x);
+                tmem_wait32(x);
+                if (c == 3) {
+                    // the accumulator can take the next tile once it is in registers
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sm.d1empty[w]);
+                }
+                if (!full_tile) {
+                    // causal mask: this row sees keys j <= t_r
+                    const int j0 = ti * kTileKeys + c * 32;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (j0 + e > t_r) x[e] = __float_as_uint(-INFINITY);
+                }
+                stats_update(x, m, l);
             }
         }
-    } else if (warp >= 8 && warp < 12) {
+    } else if (warp >= 12 && warp < 20) {
         // ------------------------------------------------------------ phase 2: scores
-        const int r = threadIdx.x - 256;  // key within the tile == TMEM lane
-        const uint32_t tl = tmem + 256 + ((uint32_t)(32 * (warp & 3)) << 16);
+        const int w = (warp - 12) >> 2;
+        const int r = threadIdx.x - 384 - 128 * w;  // key within the tile == TMEM lane
+        const uint32_t tl = tmem + 256 + ((uint32_t)(32 * (warp & 3)) << 16) + w * 128;
+        float* lse = sm.lse[w];
         int cur = -1;
         bool gave_up = false;
-        for (int i = 0; i < n_local; ++i) {
+        for (int i = w; i < n_local; i += 2) {
             const int t = cta + i * P, u = t / a.T_u, ti = t - u * a.T_u;
             if (u != cur) {
-                named_sync(2, 128);  // all threads are done with the previous unit's lse
+                named_sync(2 + w, 128);  // all threads are done with the previous unit's lse
                 if (r == 0) {
                     const unsigned* flag = a.inject ? a.never : a.ready + u;
                     bool ok = ld_acquire(flag) != 0;
@@ -612,93 +589,94 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                         atomicOr(a.err, kErrTimeout);
                         gave_up = true;  // later units do not wait again
                     }
-                    sm.flag2 = ok;
+                    sm.flag2[w] = ok;
                 }
-                named_sync(2, 128);
-                const bool ok = sm.flag2;
-                sm.lse[r] = (ok && r < a.nq) ? __ldcg(a.lse + (size_t)u * kQRows + r) : INFINITY;
-                named_sync(2, 128);
+                named_sync(2 + w, 128);
+                const bool ok = sm.flag2[w];
+                lse[r] = (ok && r < a.nq) ? __ldcg(a.lse + (size_t)u * kQRows + r) : INFINITY;
+                named_sync(2 + w, 128);
                 cur = u;
             }
-            const int b = i & 1;
-            mbar_wait(&sm.d2full[b], (i >> 1) & 1, abort, a.err);
+            mbar_wait(&sm.d2full[w], (i >> 1) & 1, abort, a.err);
             tc_fence_after();
             const int j = ti * kTileKeys + r;
             const bool full_tile = (ti + 1) * kTileKeys <= a.N - a.w + 1;
-            float s;
-            {
-                uint32_t x[64];
+            float s = 0.f;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t x[32];
                 __syncwarp();
-                tmem_ld64(tl + b * 128, x);
-                tmem_wait64(x);
-                s = prob_sum(x, sm.lse, full_tile, 0, j, a);
-            }
-            {
-                uint32_t x[64];
-                __syncwarp();
-                tmem_ld64(tl + b * 128 + 64, x);
-                tmem_wait64(x);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.d2empty[b]);
-                s += prob_sum(x, sm.lse, full_tile, 64, j, a);
+                tmem_ld32(tl + c * 32, x);
+                tmem_wait32(x);
+                if (c == 3) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sm.d2empty[w]);
+                }
+                if (!full_tile) {
+                    // causal mask: query row q (position N - w + q % w) sees this key iff j <= that
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (j > a.N - a.w + (c * 32 + e) % a.w) x[e] = __float_as_uint(-INFINITY);
+                }
+                s += prob_sum(x, lse + c * 32);
             }
             if (j < a.N) a.unit_scores[(size_t)u * a.N + j] = s;
         }
-    } else if (warp == 12) {
+    } else if (warp >= 20) {
         // ------------------------------------------------------------ publisher / merger
-        int cur = -1, npub = 0;
+        // one thread per query row; named barrier 4 spans these four warps
+        const int r = threadIdx.x - 640;
+        int npub = 0;
         for (int i = 0; i < n_local; ++i) {
-            const int u = (cta + i * P) / a.T_u;
-            const bool last_tile_of_unit = (i + 1 == n_local) || ((cta + (i + 1) * P) / a.T_u != u);
-            cur = u;
+            const int cur = (cta + i * P) / a.T_u;
+            const bool last_tile_of_unit = (i + 1 == n_local) || ((cta + (i + 1) * P) / a.T_u != cur);
             if (!last_tile_of_unit) continue;
             const int slot = npub & 1;
             mbar_wait(&sm.pub_full[slot], (npub >> 1) & 1, abort, a.err);
-            float2* dst = a.partial + ((size_t)cur * kMaxCtas + cta) * kQRows;
-#pragma unroll
-            for (int k4 = 0; k4 < kQRows / 32; ++k4) dst[lane + 32 * k4] = sm.pub[slot][lane + 32 * k4];
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.pub_empty[slot]);
-            ++npub;
+            {
+                // merge the two phase-1 warpgroups' (max, sum) of the row; publish the CTA's
+                const float2 p0 = sm.pub[slot][0][r], p1 = sm.pub[slot][1][r];
+                const float M = fmaxf(p0.x, p1.x);
+                float S = 0.f;
+                if (p0.x != -INFINITY) S += p0.y * ex2(p0.x - M);
+                if (p1.x != -INFINITY) S += p1.y * ex2(p1.x - M);
+                a.partial[((size_t)cur * kMaxCtas + cta) * kQRows + r] = make_float2(M, S);
+            }
             __threadfence();
-            __syncwarp();
+            named_sync(4, 128);
+            if (r == 0) mbar_arrive(&sm.pub_empty[slot]);
+            ++npub;
             // first level: the last CTA of this 16-CTA group merges the group's partials
             const Contributors con(a, cur);
             const int g = cta / kGroup;
-            unsigned old = 0;
-            if (lane == 0) old = atomicAdd(&a.gcount[cur * kMaxGroups + g], 1u);
-            old = __shfl_sync(0xffffffffu, old, 0);
-            if (old + 1 != (unsigned)con.group_size(g)) continue;
+            if (r == 0) sm.pub_flag = atomicAdd(&a.gcount[cur * kMaxGroups + g], 1u) + 1 == (unsigned)con.group_size(g);
+            named_sync(4, 128);
+            const bool group_last = sm.pub_flag;
+            named_sync(4, 128);
+            if (!group_last) continue;
             __threadfence();
-            const float2* gsrc = a.partial + ((size_t)cur * kMaxCtas + g * kGroup) * kQRows;
             const int gn = min(kGroup, P - g * kGroup);
-            float2* gdst = a.gpartial + ((size_t)cur * kMaxGroups + g) * kQRows;
-#pragma unroll 1
-            for (int k4 = 0; k4 < kQRows / 32; ++k4) {
-                const int row = lane + 32 * k4;
-                gdst[row] = merge_row(gsrc + row, gn, kQRows, [&](int c) { return con.has(g * kGroup + c); });
-            }
+            a.gpartial[((size_t)cur * kMaxGroups + g) * kQRows + r] =
+                merge_row(a.partial + ((size_t)cur * kMaxCtas + g * kGroup) * kQRows + r, gn, kQRows,
+                          [&](int c) { return con.has(g * kGroup + c); });
             __threadfence();
-            __syncwarp();
+            named_sync(4, 128);
             // second level: the last group of the unit merges the groups into lse
             int n_groups = 0;
             for (int gg = 0; gg * kGroup < P; ++gg) n_groups += con.group_size(gg) > 0;
-            if (lane == 0) old = atomicAdd(&a.count[cur], 1u);
-            old = __shfl_sync(0xffffffffu, old, 0);
-            if (old + 1 != (unsigned)n_groups) continue;
+            if (r == 0) sm.pub_flag = atomicAdd(&a.count[cur], 1u) + 1 == (unsigned)n_groups;
+            named_sync(4, 128);
+            const bool unit_last = sm.pub_flag;
+            named_sync(4, 128);
+            if (!unit_last) continue;
             __threadfence();
-            const float2* usrc = a.gpartial + (size_t)cur * kMaxGroups * kQRows;
-            const int ng_all = (P + kGroup - 1) / kGroup;
-#pragma unroll 1
-            for (int k4 = 0; k4 < kQRows / 32; ++k4) {
-                const int row = lane + 32 * k4;
-                const float2 ms = merge_row(usrc + row, ng_all, kQRows, [&](int gg) { return con.group_size(gg) > 0; });
-                a.lse[(size_t)cur * kQRows + row] = ms.x + log2f(ms.y);
-            }
+            const float2 ms = merge_row(a.gpartial + (size_t)cur * kMaxGroups * kQRows + r, (P + kGroup - 1) / kGroup,
+                                        kQRows, [&](int gg) { return con.group_size(gg) > 0; });
+            a.lse[(size_t)cur * kQRows + r] = ms.x + log2f(ms.y);
             __threadfence();
-            __syncwarp();
-            if (lane == 0) atomicExch(&a.ready[cur], 1u);
+            named_sync(4, 128);
+            if (r == 0) atomicExch(&a.ready[cur], 1u);
         }
     }
 

@@ -9,7 +9,11 @@
 // selected tokens plus a window of the newest tokens).  One CTA of 1024 threads owns a
 // row; each warp owns a contiguous segment of it, so all loads are coalesced and the only
 // block-wide steps are the digit search and one scan of per-warp counts.
+#include <cooperative_groups.h>
+
 #include "kvc_internal.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace kvc {
 namespace {
@@ -198,6 +202,198 @@ topk_kernel(const float* __restrict__ pooled, int N, int S, int w, int budget,
     }
 }
 
+// --------------------------------------------------------------- cluster top-k (fused pool)
+//
+// One 8-CTA thread-block cluster owns a row.  CTA k of the cluster pools the candidates
+// [lo + k*seg, lo + (k+1)*seg) (reading the raw scores with their pool halo) into
+// order-preserving keys in its shared memory; the radix select then runs three digit
+// passes (11, 11 and 10 bits) over shared memory, combining the CTAs' histograms through
+// distributed shared memory, and every CTA takes the same digit decision.  The stable
+// compaction writes the kept positions in ascending order: CTA k starts after the
+// candidates its lower-ranked siblings keep.
+
+constexpr int kClusterCtas = 8;
+constexpr int kCtThreads = 512;
+constexpr int kCtWarps = kCtThreads / 32;
+constexpr int kBins = 2048;
+constexpr int kSegMax = 24576;  // keys per CTA: 96 KiB of shared memory (two CTAs per SM)
+
+struct TopkSmem {
+    uint32_t hist[kBins];
+    uint32_t slice_tot[kBins / kClusterCtas];  // this CTA's slice of the cluster-wide totals
+    uint32_t slice_sum;
+    int gt, eq;
+    int wcnt_gt[kCtWarps], wcnt_eq[kCtWarps];
+    uint32_t keys[kSegMax];
+};
+
+__global__ void __launch_bounds__(kCtThreads, 2) __cluster_dims__(kClusterCtas, 1, 1)
+topk_cluster_kernel(const float* __restrict__ scores, int N, int S, int w, int budget, int radius, int seg,
+                    int32_t* __restrict__ idx) {
+    extern __shared__ uint8_t smem_raw[];
+    TopkSmem& sm = *reinterpret_cast<TopkSmem*>(smem_raw);
+    cg::cluster_group cluster = cg::this_cluster();
+    const int rank = (int)cluster.block_rank();
+    const int row = blockIdx.x / kClusterCtas;
+    const float* v = scores + (size_t)row * N;
+    int32_t* out = idx + (size_t)row * budget;
+    const int lo = S, hi = N - w, k_sel = budget - S - w;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int s0 = lo + min(hi - lo, rank * seg), s1 = lo + min(hi - lo, (rank + 1) * seg);
+    const int n_mine = s1 - s0;
+
+    if (rank == 0) {
+        for (int i = tid; i < S; i += kCtThreads) out[i] = i;
+        for (int i = tid; i < w; i += kCtThreads) out[budget - w + i] = N - w + i;
+    }
+    // pooled keys of this CTA's candidates (max over the clipped window of raw scores)
+    for (int e = tid; e < n_mine; e += kCtThreads) {
+        const int j = s0 + e;
+        const int t0 = max(lo, j - radius), t1 = min(hi - 1, j + radius);
+        float m = __ldg(v + t0);
+        for (int t = t0 + 1; t <= t1; ++t) m = fmaxf(m, __ldg(v + t));
+        sm.keys[e] = order_key(m);
+    }
+
+    uint32_t prefix = 0, mask = 0;
+    int krem = k_sel;
+    const int shifts[3] = {21, 10, 0};
+    const int widths[3] = {11, 11, 10};
+    for (int pass = 0; pass < 3; ++pass) {
+        const int shift = shifts[pass];
+        const uint32_t dmask = (1u << widths[pass]) - 1u;
+        for (int i = tid; i < kBins; i += kCtThreads) sm.hist[i] = 0u;
+        __syncthreads();
+        for (int e = tid; e < n_mine; e += kCtThreads) {
+            const uint32_t key = sm.keys[e];
+            if ((key & mask) == prefix) {
+                const unsigned digit = (key >> shift) & dmask;
+                const unsigned peers = __match_any_sync(__activemask(), digit);
+                if (lane == __ffs(peers) - 1) atomicAdd(&sm.hist[digit], (unsigned)__popc(peers));
+            }
+        }
+        cluster.sync();  // every CTA's histogram is complete
+        // this CTA totals the bins [rank*256, rank*256 + 256) over the cluster
+        constexpr int kSlice = kBins / kClusterCtas;
+        if (tid < kSlice) {
+            const int bin = rank * kSlice + tid;
+            uint32_t t = 0;
+#pragma unroll
+            for (int c = 0; c < kClusterCtas; ++c) t += cluster.map_shared_rank(sm.hist, c)[bin];
+            sm.slice_tot[tid] = t;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            uint32_t t = 0;
+            for (int i = lane; i < kSlice; i += 32) t += sm.slice_tot[i];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+            if (lane == 0) sm.slice_sum = t;
+        }
+        cluster.sync();  // slice totals are visible cluster-wide
+        // every CTA finds the same digit: the slice holding the krem-th largest, then the bin
+        if (warp == 0) {
+            uint32_t above = 0;
+            int s_star = 0;
+            for (int c = kClusterCtas - 1; c >= 0; --c) {
+                const uint32_t t = *cluster.map_shared_rank(&sm.slice_sum, c);
+                if (above + t >= (uint32_t)krem) {
+                    s_star = c;
+                    break;
+                }
+                above += t;
+            }
+            const uint32_t* tot = cluster.map_shared_rank(sm.slice_tot, s_star);
+            // scan the slice's 256 bins from the top, 32 at a time
+            int digit = -1;
+            for (int base = kSlice - 32; base >= 0 && digit < 0; base -= 32) {
+                const uint32_t t = tot[base + lane];
+                // inclusive suffix sum within this group of 32 (lane 31 is the top bin)
+                uint32_t incl = t;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const uint32_t y = __shfl_down_sync(0xffffffffu, incl, off);
+                    if (lane + off < 32) incl += y;
+                }
+                const uint32_t excl = incl - t;
+                const bool hit = above + excl < (uint32_t)krem && (uint32_t)krem <= above + incl;
+                const unsigned b = __ballot_sync(0xffffffffu, hit);
+                if (b) {
+                    const int l = __ffs(b) - 1;
+                    const uint32_t ex = __shfl_sync(0xffffffffu, excl, l);
+                    digit = s_star * kSlice + base + l;
+                    if (lane == 0) {
+                        sm.gt = digit;
+                        sm.eq = krem - (int)(above + ex);
+                    }
+                }
+                above += __shfl_sync(0xffffffffu, incl, 0);
+            }
+        }
+        __syncthreads();
+        prefix |= (uint32_t)sm.gt << shift;
+        mask |= dmask << shift;
+        krem = sm.eq;
+        cluster.sync();  // nobody reads this pass's histograms any more
+    }
+    const uint32_t T = prefix;  // the k_sel-th largest key; keep krem of the keys equal to T
+
+    // per-warp counts over contiguous warp segments of this CTA's keys
+    const int wseg = (n_mine + kCtWarps - 1) / kCtWarps;
+    const int w0 = min(n_mine, warp * wseg), w1 = min(n_mine, (warp + 1) * wseg);
+    int n_gt = 0, n_eq = 0;
+    for (int e = w0 + lane; e < w1; e += 32) {
+        const uint32_t key = sm.keys[e];
+        n_gt += key > T;
+        n_eq += key == T;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        n_gt += __shfl_xor_sync(0xffffffffu, n_gt, off);
+        n_eq += __shfl_xor_sync(0xffffffffu, n_eq, off);
+    }
+    if (lane == 0) {
+        sm.wcnt_gt[warp] = n_gt;
+        sm.wcnt_eq[warp] = n_eq;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int g = 0, q = 0;
+        for (int i = 0; i < kCtWarps; ++i) {
+            g += sm.wcnt_gt[i];
+            q += sm.wcnt_eq[i];
+        }
+        sm.gt = g;
+        sm.eq = q;
+    }
+    cluster.sync();  // CTA totals visible
+    int gt_before = 0, eq_before = 0;
+    for (int c = 0; c < rank; ++c) {
+        gt_before += *cluster.map_shared_rank(&sm.gt, c);
+        eq_before += *cluster.map_shared_rank(&sm.eq, c);
+    }
+    for (int i = 0; i < warp; ++i) {
+        gt_before += sm.wcnt_gt[i];
+        eq_before += sm.wcnt_eq[i];
+    }
+    int taken = gt_before + min(eq_before, krem);
+    int eq_seen = eq_before;
+    for (int base = w0; base < w1; base += 32) {
+        const int e = base + lane;
+        const uint32_t key = e < w1 ? sm.keys[e] : 0u;
+        const bool gt = e < w1 && key > T;
+        const bool eq = e < w1 && key == T;
+        const unsigned eq_mask = __ballot_sync(0xffffffffu, eq);
+        const bool take = gt || (eq && eq_seen + __popc(eq_mask & lanemask_lt()) < krem);
+        const unsigned take_mask = __ballot_sync(0xffffffffu, take);
+        const int pos = taken + __popc(take_mask & lanemask_lt());
+        if (take && pos < k_sel) out[S + pos] = s0 + e;  // pos < k_sel always holds; kept as a guard
+        taken += __popc(take_mask);
+        eq_seen += __popc(eq_mask);
+    }
+    cluster.sync();  // siblings may still read this CTA's counts until here
+}
+
 int grid_for(long long total, int threads) {
     long long g = (total + threads - 1) / threads;
     if (g > 148LL * 32) g = 148LL * 32;
@@ -227,6 +423,33 @@ cudaError_t pool(const float* in, float* out, int rows, int N, int lo, int hi, i
     const long long total = (long long)rows * N;
     if (total == 0) return cudaSuccess;
     pool_kernel<<<grid_for(total, 256), 256, 0, s>>>(in, out, rows, N, lo, hi, (kernel - 1) / 2);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+bool topk_fused_fits(int N, int n_sink, int window) {
+    const int n_c = N - n_sink - window;
+    return (n_c + kClusterCtas - 1) / kClusterCtas <= kSegMax;
+}
+
+cudaError_t topk_fused(const float* scores, int rows, int N, int n_sink, int window, int budget, int kernel,
+                       int32_t* idx, cudaStream_t s) {
+    if (rows == 0) return cudaSuccess;
+    const int n_c = N - n_sink - window;
+    const int seg = (n_c + kClusterCtas - 1) / kClusterCtas;
+    if (seg > kSegMax) return cudaErrorInvalidValue;
+    const size_t smem = sizeof(TopkSmem) - sizeof(uint32_t) * (size_t)(kSegMax - seg);
+    static bool attr_done[64] = {false};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 64 || !attr_done[dev]) {
+        e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(TopkSmem));
+        if (e != cudaSuccess) return e;
+        if (dev < 64) attr_done[dev] = true;
+    }
+    topk_cluster_kernel<<<rows * kClusterCtas, kCtThreads, smem, s>>>(scores, N, n_sink, window, budget,
+                                                                     (kernel - 1) / 2, seg, idx);
     count_launches(1);
     return cudaGetLastError();
 }
