@@ -17,13 +17,16 @@
 //     dealt round-robin over the CTAs in global (unit-major) order;
 //   * phase 1 streams K from HBM: D1[128 q x 128 keys] = Q K^T (tcgen05.mma kind::f16,
 //     M = N = 128, fp32 accumulator in TMEM); one thread per query row keeps an online
-//     (max, sum) over the CTA's tiles of a unit and hands it to the publisher warp;
-//   * the publisher warp writes the CTA's partial, and the last CTA of each 16-CTA group
-//     and then the last group of the unit merge the partials (fixed order) into lse and
-//     raise the unit's ready flag -- off the consumers' path;
+//     (max, sum) over the CTA's tiles of a unit and hands it to the publisher warps;
+//   * the publisher rescales the CTA's sum to a fixed per-row reference (the logit of the
+//     row with the key at its own position, computed before the kernel) and adds it to the
+//     unit's fp64 total with a fire-and-forget atomic, then bumps the unit's arrival count
+//     -- no merge step, so phase 2 can start a few microseconds after the last CTA of the
+//     unit (fp64 addition order only moves the total by ~1e-16, far below fp32);
 //   * phase 2 re-reads each tile a bounded number of tiles behind phase 1 (so it comes
 //     from L2, loaded evict-first): D2[128 keys x 128 q] = K Q^T, a thread owns a key and
-//     sums 2^(y - lse) over the query rows once the unit's ready flag is up.
+//     sums 2^(y - lse) over the query rows once every CTA of the unit has arrived,
+//     lse = ref + log2(total).
 // The two phases have separate TMA producers, shared-memory rings (16 KiB half-tiles of
 // 64 columns, the 128-byte swizzle atom) and MMA issuers, so a phase-2 wait never stalls
 // the HBM stream.  Warps: 0 phase-1 TMA, 1 TMEM owner + phase-1 MMA, 2 phase-2 TMA,
@@ -44,13 +47,25 @@ namespace {
 constexpr int kTileKeys = 128;                         // keys per tile (MMA N / M)
 constexpr int kQRows = 128;                            // query rows per unit (padded)
 constexpr int kBoxBytes = kTileKeys * 64 * 2;          // a 128-row x 64-column bf16 box: 16 KiB
-constexpr int kStagesA = 6;                            // phase-1 ring (HBM stream)
-constexpr int kStagesB = 3;                            // phase-2 ring (L2 re-read)
+#ifndef KVC_TC_STAGES_A
+#define KVC_TC_STAGES_A 4
+#endif
+#ifndef KVC_TC_STAGES_B
+#define KVC_TC_STAGES_B 3
+#endif
+#ifndef KVC_TC_Q_SLOTS
+#define KVC_TC_Q_SLOTS 3
+#endif
+#ifndef KVC_TC_LEAD_SLACK
+#define KVC_TC_LEAD_SLACK 8
+#endif
+constexpr int kStagesA = KVC_TC_STAGES_A;              // phase-1 ring (HBM stream)
+constexpr int kStagesB = KVC_TC_STAGES_B;              // phase-2 ring (L2 re-read)
+constexpr int kQSlots = KVC_TC_Q_SLOTS;                // Q of the CTA's last units, by unit ordinal
+constexpr int kLeadSlack = KVC_TC_LEAD_SLACK;          // phase-1 lead beyond one unit, in tiles
 constexpr int kWarps = 24;  // 4 producer/MMA, 2 x 4 phase-1, 2 x 4 phase-2, 4 publisher
 constexpr int kThreads = kWarps * 32;
-constexpr int kMaxCtas = 160;                          // partial slots per unit (>= #SMs)
-constexpr int kGroup = 16;                             // CTAs per first-level merge group
-constexpr int kMaxGroups = kMaxCtas / kGroup;
+constexpr int kMaxCtas = 160;                          // upper bound on the persistent grid
 constexpr uint32_t kTmemCols = 512;
 constexpr long long kBarrierTimeoutNs = 4000000000LL;  // hang guard for intra-CTA waits
 
@@ -62,13 +77,10 @@ struct TcArgs {
     CUtensorMap tmap_k;  // K as [U][N][128] bf16, box 64 x 128 x 1, 128-byte swizzle
     CUtensorMap tmap_q;  // padded Q as [U*128][128] bf16, box 64 x 128, 128-byte swizzle
     float* unit_scores;  // [U][N]
-    float2* partial;     // [U][kMaxCtas][128] (max, sum) per CTA
-    float2* gpartial;    // [U][kMaxGroups][128] (max, sum) per merge group
-    float* lse;          // [U][128]
-    unsigned* gcount;    // [U][kMaxGroups] partials published per group
-    unsigned* count;     // [U] groups merged
-    unsigned* ready;     // [U] lse published
-    unsigned* never;     // a flag nothing sets (wait-timeout injection)
+    const float* ref;    // [U][128] per-row reference logit (base 2): the row's own-position key
+    double* sum;         // [U][128] sum over keys of 2^(y - ref), accumulated by all CTAs
+    unsigned* count;     // [U] CTAs that have added their part of unit u
+    unsigned* never;     // a counter nothing increments (wait-timeout injection)
     unsigned* err;
     long long spin_limit;
     int U, N, w, nq, T_u, total_tiles, P, max_lead, inject;
@@ -77,18 +89,17 @@ struct TcArgs {
 struct __align__(1024) Smem {
     uint8_t ringA[kStagesA][kBoxBytes];
     uint8_t ringB[kStagesB][kBoxBytes];
-    uint8_t q[2][2 * kBoxBytes];  // Q of the current unit of phase 1 / phase 2 (two boxes)
+    uint8_t q[kQSlots][2 * kBoxBytes];  // Q of the CTA's k-th unit in slot k % kQSlots (two boxes)
     float lse[2][kQRows];         // per phase-2 warpgroup
     float2 pub[2][2][kQRows];     // [slot][phase-1 warpgroup][row]
     int pub_unit[2];
     uint64_t fullA[kStagesA], emptyA[kStagesA], fullB[kStagesB], emptyB[kStagesB];
-    uint64_t qfull[2], qempty[2];
+    uint64_t qfull[kQSlots], qempty[kQSlots];
     uint64_t d1full[2], d1empty[2], d2full[2], d2empty[2];
     uint64_t pub_full[2], pub_empty[2];
     uint32_t tmem_base;
     int abort;
     int flag2[2];
-    int pub_flag;
     int p1_issued, p2_issued;  // tiles whose loads each producer has issued (L2 lead control)
 };
 
@@ -262,11 +273,16 @@ __device__ __forceinline__ float exp2_poly(float y) {
     return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
-// Exponentials of the fully visible tiles: two of every eight go to the FMA pipe so that
-// the MUFU and the FMA pipes finish together.
+// Exponentials of the fully visible tiles.  KVC_TC_POLY_EVERY = n > 0 sends one of every n
+// to the FMA-pipe polynomial; in this kernel all-MUFU measured fastest on B200 (the
+// polynomial costs about 13 issue slots, and the consumers are issue- and latency-bound
+// rather than MUFU-bound), so the default is 0.
+#ifndef KVC_TC_POLY_EVERY
+#define KVC_TC_POLY_EVERY 0
+#endif
 template <int E>
 __device__ __forceinline__ float exp2_mixed(float y) {
-    return (E & 7) >= 6 ? exp2_poly(y) : ex2(y);
+    return (KVC_TC_POLY_EVERY > 0 && (E % KVC_TC_POLY_EVERY) == KVC_TC_POLY_EVERY - 1) ? exp2_poly(y) : ex2(y);
 }
 
 __device__ __forceinline__ void named_sync(int id, int n) {
@@ -277,53 +293,6 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
     unsigned v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
-}
-
-// The CTAs that hold tiles of unit u form the cyclic range [first, first + n) mod P with
-// first = u*T_u mod P and n = min(T_u, P) (tiles are dealt round-robin).
-struct Contributors {
-    int first, n, P;
-    __device__ Contributors(const TcArgs& a, int u)
-        : first((int)(((long long)u * a.T_u) % a.P)), n(min(a.T_u, a.P)), P(a.P) {}
-    __device__ bool has(int c) const {
-        int rel = c - first;
-        if (rel < 0) rel += P;
-        return rel < n;
-    }
-    // how many of the CTAs [lo, hi) contribute
-    __device__ int count(int lo, int hi) const {
-        const int a_hi = min(first + n, P);                          // [first, a_hi)
-        const int b_hi = first + n > P ? first + n - P : 0;          // [0, b_hi)
-        return max(0, min(hi, a_hi) - max(lo, first)) + max(0, min(hi, b_hi) - lo);
-    }
-    __device__ int group_size(int g) const { return count(g * kGroup, min(P, (g + 1) * kGroup)); }
-};
-
-// Merges (max, sum) pairs of one row: src[i * stride] for the i in [0, n) with use(i).
-template <typename Use>
-__device__ __forceinline__ float2 merge_row(const float2* src, int n, size_t stride, Use use) {
-    float M = -INFINITY, S = 0.f;
-    for (int i0 = 0; i0 < n; i0 += kGroup) {
-        float2 v[kGroup];
-#pragma unroll
-        for (int i = 0; i < kGroup; ++i)
-            v[i] = (i0 + i < n && use(i0 + i)) ? __ldcg(src + (size_t)(i0 + i) * stride) : make_float2(-INFINITY, 0.f);
-        float cm = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < kGroup; ++i) cm = fmaxf(cm, v[i].x);
-        if (cm == -INFINITY) continue;
-        float cs = 0.f;
-#pragma unroll
-        for (int i = 0; i < kGroup; ++i)
-            if (v[i].x != -INFINITY) cs += v[i].y * ex2(v[i].x - cm);
-        if (cm > M) {
-            S = (M == -INFINITY ? 0.f : S * ex2(M - cm)) + cs;
-            M = cm;
-        } else {
-            S += cs * ex2(cm - M);
-        }
-    }
-    return make_float2(M, S);
 }
 
 // Online (max, sum) update of one query row with 32 logits (invisible keys already set
@@ -395,9 +364,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             mbar_init(&sm.fullB[s], 1);
             mbar_init(&sm.emptyB[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < kQSlots; ++b) {
             mbar_init(&sm.qfull[b], 1);
-            mbar_init(&sm.qempty[b], 1);
+            mbar_init(&sm.qempty[b], 2);  // released by both MMA issuers
+        }
+        for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.d1full[b], 1);
             mbar_init(&sm.d1empty[b], 4);
             mbar_init(&sm.d2full[b], 1);
@@ -435,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             const int stages = ph == 0 ? kStagesA : kStagesB;
             volatile int* mine = ph == 0 ? &sm.p1_issued : &sm.p2_issued;
             volatile int* other = ph == 0 ? &sm.p2_issued : &sm.p1_issued;
-            int k = 0, qunit = -1, qloads = 0;
+            int k = 0, qunit = -1, ord = -1;
             for (int i = 0; i < n_local && !*abort; ++i) {
                 const int t = cta + i * P, u = t / a.T_u, ti = t - u * a.T_u;
                 // phase 1 stays at most max_lead tiles ahead of phase 2 (L2 footprint);
@@ -451,12 +422,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                     __nanosleep(128);
                 }
                 if (u != qunit) {
-                    if (qloads > 0) mbar_wait(&sm.qempty[ph], (qloads - 1) & 1, abort, a.err);
-                    mbar_expect_tx(&sm.qfull[ph], 2 * kBoxBytes);
-                    tma_load_2d(sm.q[ph], &a.tmap_q, &sm.qfull[ph], 0, u * kQRows);
-                    tma_load_2d(sm.q[ph] + kBoxBytes, &a.tmap_q, &sm.qfull[ph], 64, u * kQRows);
+                    // the CTA's ord-th unit: phase 1 loads its Q into slot ord % kQSlots once both
+                    // phases are done with the unit that used the slot kQSlots units ago
                     qunit = u;
-                    ++qloads;
+                    ++ord;
+                    if (ph == 0) {
+                        const int slot = ord % kQSlots;
+                        if (ord >= kQSlots) mbar_wait(&sm.qempty[slot], ((ord / kQSlots) - 1) & 1, abort, a.err);
+                        mbar_expect_tx(&sm.qfull[slot], 2 * kBoxBytes);
+                        tma_load_2d(sm.q[slot], &a.tmap_q, &sm.qfull[slot], 0, u * kQRows);
+                        tma_load_2d(sm.q[slot] + kBoxBytes, &a.tmap_q, &sm.qfull[slot], 64, u * kQRows);
+                    }
                 }
                 for (int h = 0; h < 2; ++h, ++k) {
                     const int s = k % stages;
@@ -481,15 +457,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             uint64_t* dempty = ph == 0 ? sm.d1empty : sm.d2empty;
             const int stages = ph == 0 ? kStagesA : kStagesB;
             const uint32_t dbase = tmem + (ph == 0 ? 0u : 256u);
-            int k = 0, qunit = -1, qloads = 0;
+            int k = 0, qunit = -1, ord = -1;
+            const uint8_t* qtile = sm.q[0];
             for (int i = 0; i < n_local && !*abort; ++i) {
                 const int t = cta + i * P, u = t / a.T_u;
                 if (u != qunit) {
-                    // the previous Q of this phase is free once every MMA issued so far is done
-                    if (qunit >= 0) umma_commit(&sm.qempty[ph]);
-                    mbar_wait(&sm.qfull[ph], qloads & 1, abort, a.err);
+                    // this phase is done with the previous unit's Q slot once its MMAs finish
+                    if (ord >= 0) umma_commit(&sm.qempty[ord % kQSlots]);
+                    ++ord;
+                    mbar_wait(&sm.qfull[ord % kQSlots], (ord / kQSlots) & 1, abort, a.err);
+                    qtile = sm.q[ord % kQSlots];
                     qunit = u;
-                    ++qloads;
                 }
                 const int b = i & 1;
                 mbar_wait(&dempty[b], ((i >> 1) & 1) ^ 1, abort, a.err);
@@ -499,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                     const int s = k % stages;
                     mbar_wait(&full[s], (k / stages) & 1, abort, a.err);
                     tc_fence_after();
-                    const uint8_t* qbox = sm.q[ph] + h * kBoxBytes;
+                    const uint8_t* qbox = qtile + h * kBoxBytes;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         if (ph == 0)
@@ -579,11 +557,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             if (u != cur) {
                 named_sync(2 + w, 128);  // all threads are done with the previous unit's lse
                 if (r == 0) {
-                    const unsigned* flag = a.inject ? a.never : a.ready + u;
-                    bool ok = ld_acquire(flag) != 0;
+                    // unit u is complete once every CTA holding tiles of it has added its part
+                    const unsigned* cnt = a.inject ? a.never : a.count + u;
+                    const unsigned n_contrib = (unsigned)min(a.T_u, a.P);
+                    bool ok = ld_acquire(cnt) >= n_contrib;
                     for (long long spins = 0; !ok && !gave_up && spins < a.spin_limit; ++spins) {
                         __nanosleep(64);
-                        ok = ld_acquire(flag) != 0;
+                        ok = ld_acquire(cnt) >= n_contrib;
                     }
                     if (!ok) {
                         atomicOr(a.err, kErrTimeout);
@@ -593,7 +573,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                 }
                 named_sync(2 + w, 128);
                 const bool ok = sm.flag2[w];
-                lse[r] = (ok && r < a.nq) ? __ldcg(a.lse + (size_t)u * kQRows + r) : INFINITY;
+                lse[r] = (ok && r < a.nq)
+                             ? (float)((double)__ldg(a.ref + (size_t)u * kQRows + r) + log2(__ldcg(a.sum + (size_t)u * kQRows + r)))
+                             : INFINITY;
                 named_sync(2 + w, 128);
                 cur = u;
             }
@@ -624,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             if (j < a.N) a.unit_scores[(size_t)u * a.N + j] = s;
         }
     } else if (warp >= 20) {
-        // ------------------------------------------------------------ publisher / merger
+        // ------------------------------------------------------------ publisher
         // one thread per query row; named barrier 4 spans these four warps
         const int r = threadIdx.x - 640;
         int npub = 0;
@@ -634,49 +616,22 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             if (!last_tile_of_unit) continue;
             const int slot = npub & 1;
             mbar_wait(&sm.pub_full[slot], (npub >> 1) & 1, abort, a.err);
-            {
-                // merge the two phase-1 warpgroups' (max, sum) of the row; publish the CTA's
-                const float2 p0 = sm.pub[slot][0][r], p1 = sm.pub[slot][1][r];
-                const float M = fmaxf(p0.x, p1.x);
-                float S = 0.f;
-                if (p0.x != -INFINITY) S += p0.y * ex2(p0.x - M);
-                if (p1.x != -INFINITY) S += p1.y * ex2(p1.x - M);
-                a.partial[((size_t)cur * kMaxCtas + cta) * kQRows + r] = make_float2(M, S);
-            }
-            __threadfence();
+            const float2 p0 = sm.pub[slot][0][r], p1 = sm.pub[slot][1][r];
             named_sync(4, 128);
             if (r == 0) mbar_arrive(&sm.pub_empty[slot]);
             ++npub;
-            // first level: the last CTA of this 16-CTA group merges the group's partials
-            const Contributors con(a, cur);
-            const int g = cta / kGroup;
-            if (r == 0) sm.pub_flag = atomicAdd(&a.gcount[cur * kMaxGroups + g], 1u) + 1 == (unsigned)con.group_size(g);
-            named_sync(4, 128);
-            const bool group_last = sm.pub_flag;
-            named_sync(4, 128);
-            if (!group_last) continue;
-            __threadfence();
-            const int gn = min(kGroup, P - g * kGroup);
-            a.gpartial[((size_t)cur * kMaxGroups + g) * kQRows + r] =
-                merge_row(a.partial + ((size_t)cur * kMaxCtas + g * kGroup) * kQRows + r, gn, kQRows,
-                          [&](int c) { return con.has(g * kGroup + c); });
+            // this CTA's sum over its keys of 2^(y - ref), added into the unit's fp64 total
+            const float M = fmaxf(p0.x, p1.x);
+            if (M != -INFINITY) {
+                float S = 0.f;
+                if (p0.x != -INFINITY) S += p0.y * ex2(p0.x - M);
+                if (p1.x != -INFINITY) S += p1.y * ex2(p1.x - M);
+                const double ref = (double)__ldg(a.ref + (size_t)cur * kQRows + r);
+                atomicAdd(a.sum + (size_t)cur * kQRows + r, (double)S * exp2((double)M - ref));
+            }
             __threadfence();
             named_sync(4, 128);
-            // second level: the last group of the unit merges the groups into lse
-            int n_groups = 0;
-            for (int gg = 0; gg * kGroup < P; ++gg) n_groups += con.group_size(gg) > 0;
-            if (r == 0) sm.pub_flag = atomicAdd(&a.count[cur], 1u) + 1 == (unsigned)n_groups;
-            named_sync(4, 128);
-            const bool unit_last = sm.pub_flag;
-            named_sync(4, 128);
-            if (!unit_last) continue;
-            __threadfence();
-            const float2 ms = merge_row(a.gpartial + (size_t)cur * kMaxGroups * kQRows + r, (P + kGroup - 1) / kGroup,
-                                        kQRows, [&](int gg) { return con.group_size(gg) > 0; });
-            a.lse[(size_t)cur * kQRows + r] = ms.x + log2f(ms.y);
-            __threadfence();
-            named_sync(4, 128);
-            if (r == 0) atomicExch(&a.ready[cur], 1u);
+            if (r == 0) atomicAdd(a.count + cur, 1u);
         }
     }
 
@@ -689,10 +644,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
     }
 }
 
-// Copies the unit's query rows into a zero-padded [U][128][128] block (rows >= nq are 0)
-// and clears the per-unit counters and flags of this call.
-__global__ void tc_prep_kernel(const __nv_bfloat16* __restrict__ q, __nv_bfloat16* __restrict__ qpad, int U, int nq,
-                               unsigned* __restrict__ flags, int n_flags) {
+// Copies the unit's query rows into a zero-padded [U][128][128] block (rows >= nq are 0),
+// computes each row's reference logit (base 2) with the key at the row's own position, and
+// clears the per-unit sums and counters of this call.
+__global__ void tc_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                               __nv_bfloat16* __restrict__ qpad, float* __restrict__ ref, double* __restrict__ sum,
+                               unsigned* __restrict__ flags, int n_flags, int U, int N, int w, int nq) {
     const long long total = (long long)U * kQRows * (kHeadDim / 8);  // 16-byte pieces
     for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
          e += (long long)gridDim.x * blockDim.x) {
@@ -703,6 +660,19 @@ __global__ void tc_prep_kernel(const __nv_bfloat16* __restrict__ q, __nv_bfloat1
         uint4 v = make_uint4(0, 0, 0, 0);
         if (r < nq) v = *reinterpret_cast<const uint4*>(q + ((u * nq + r) * kHeadDim + piece * 8));
         *reinterpret_cast<uint4*>(qpad + (row * kHeadDim + piece * 8)) = v;
+    }
+    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < (long long)U * kQRows;
+         e += (long long)gridDim.x * blockDim.x) {
+        const int r = (int)(e % kQRows);
+        const long long u = e / kQRows;
+        float x = 0.f;
+        if (r < nq) {
+            const __nv_bfloat16* qr = q + (u * nq + r) * kHeadDim;
+            const __nv_bfloat16* kr = k + (u * N + (N - w + r % w)) * kHeadDim;
+            for (int d = 0; d < kHeadDim; ++d) x = fmaf(__bfloat162float(qr[d]), __bfloat162float(kr[d]), x);
+        }
+        ref[e] = x * kLog2eOverSqrtD;
+        sum[e] = 0.0;
     }
     for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n_flags;
          e += (long long)gridDim.x * blockDim.x)
@@ -718,7 +688,7 @@ __global__ void exp2_poly_kernel(const float* __restrict__ y, float* __restrict_
 size_t a256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct TcLayout {
-    size_t qpad, partial, gpartial, lse, flags, n_flags, total;
+    size_t qpad, ref, sum, flags, n_flags, total;
 };
 
 TcLayout tc_layout(int U) {
@@ -726,14 +696,12 @@ TcLayout tc_layout(int U) {
     size_t off = 0;
     L.qpad = off;
     off = a256(off + (size_t)U * kQRows * kHeadDim * 2);
-    L.partial = off;
-    off = a256(off + (size_t)U * kMaxCtas * kQRows * sizeof(float2));
-    L.gpartial = off;
-    off = a256(off + (size_t)U * kMaxGroups * kQRows * sizeof(float2));
-    L.lse = off;
+    L.ref = off;
     off = a256(off + (size_t)U * kQRows * sizeof(float));
-    L.flags = off;  // gcount[U][kMaxGroups], count[U], ready[U], never
-    L.n_flags = (size_t)U * kMaxGroups + 2 * (size_t)U + 1;
+    L.sum = off;
+    off = a256(off + (size_t)U * kQRows * sizeof(double));
+    L.flags = off;  // count[U], never
+    L.n_flags = (size_t)U + 1;
     off = a256(off + L.n_flags * sizeof(unsigned));
     L.total = off;
     return L;
@@ -788,13 +756,10 @@ cudaError_t tc_score(const ScoreJob& j, cudaStream_t s) {
 
     TcArgs a{};
     a.unit_scores = j.unit_scores;
-    a.partial = (float2*)(ws + L.partial);
-    a.gpartial = (float2*)(ws + L.gpartial);
-    a.lse = (float*)(ws + L.lse);
-    a.gcount = flags;
-    a.count = flags + (size_t)j.U * kMaxGroups;
-    a.ready = a.count + j.U;
-    a.never = a.ready + j.U;
+    a.ref = (const float*)(ws + L.ref);
+    a.sum = (double*)(ws + L.sum);
+    a.count = flags;
+    a.never = flags + j.U;
     a.err = j.err;
     a.spin_limit = j.spin_limit;
     a.U = j.U;
@@ -808,7 +773,7 @@ cudaError_t tc_score(const ScoreJob& j, cudaStream_t s) {
     a.P = std::min(std::min(n_sm, kMaxCtas), a.total_tiles);
     // phase 1 may run this many tiles ahead of phase 2: a unit's worth plus slack for the
     // merge, while keeping the tiles between the two reads (max_lead x P x 32 KiB) in L2
-    a.max_lead = (a.T_u + a.P - 1) / a.P + 8;
+    a.max_lead = (a.T_u + a.P - 1) / a.P + kLeadSlack;
     a.inject = j.inject_timeout;
 
     auto encode = encode_fn();
@@ -836,7 +801,9 @@ cudaError_t tc_score(const ScoreJob& j, cudaStream_t s) {
 
     const long long pieces = (long long)j.U * kQRows * (kHeadDim / 8);
     const int prep_grid = (int)std::min<long long>((pieces + 255) / 256, 148LL * 8);
-    tc_prep_kernel<<<prep_grid, 256, 0, s>>>((const __nv_bfloat16*)j.q, qpad, j.U, j.nq, flags, (int)L.n_flags);
+    tc_prep_kernel<<<prep_grid, 256, 0, s>>>((const __nv_bfloat16*)j.q, (const __nv_bfloat16*)j.k, qpad,
+                                             (float*)(ws + L.ref), (double*)(ws + L.sum), flags, (int)L.n_flags,
+                                             j.U, j.N, j.window, j.nq);
     count_launches(1);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
