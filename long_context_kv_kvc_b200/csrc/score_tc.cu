@@ -12,27 +12,35 @@
 // Design for B200.  The softmax normaliser lse_r is global over all N keys, so every
 // logit is needed twice: once for lse_r (phase 1) and once for its probability (phase 2).
 // Storing logits would cost more HBM traffic than K itself, so K is read twice and the
-// second read is scheduled to hit L2:
+// second read is scheduled to hit L2.  With 128 query rows per unit the work is two
+// exponentials per byte of K, which makes the special-function unit, not HBM, the
+// tightest resource; the kernel is therefore organised to keep every consumer warp fed:
 //   * one persistent CTA per SM (cooperative launch: all CTAs resident), 128-key tiles
 //     dealt round-robin over the CTAs in global (unit-major) order;
-//   * phase 1 streams K from HBM: D1[128 q x 128 keys] = Q K^T (tcgen05.mma kind::f16,
-//     M = N = 128, fp32 accumulator in TMEM); one thread per query row keeps an online
-//     (max, sum) over the CTA's tiles of a unit and hands it to the publisher warps;
-//   * the publisher rescales the CTA's sum to a fixed per-row reference (the logit of the
-//     row with the key at its own position, computed before the kernel) and adds it to the
-//     unit's fp64 total with a fire-and-forget atomic, then bumps the unit's arrival count
-//     -- no merge step, so phase 2 can start a few microseconds after the last CTA of the
-//     unit (fp64 addition order only moves the total by ~1e-16, far below fp32);
-//   * phase 2 re-reads each tile a bounded number of tiles behind phase 1 (so it comes
-//     from L2, loaded evict-first): D2[128 keys x 128 q] = K Q^T, a thread owns a key and
-//     sums 2^(y - lse) over the query rows once every CTA of the unit has arrived,
-//     lse = ref + log2(total).
-// The two phases have separate TMA producers, shared-memory rings (16 KiB half-tiles of
-// 64 columns, the 128-byte swizzle atom) and MMA issuers, so a phase-2 wait never stalls
-// the HBM stream.  Warps: 0 phase-1 TMA, 1 TMEM owner + phase-1 MMA, 2 phase-2 TMA,
-// 3 phase-2 MMA, 4-11 phase-1 statistics (two warpgroups, one per TMEM accumulator),
-// 12-19 phase-2 sums (likewise), 20-23 publisher (one thread per query row).  Every wait is
-// bounded: a wait that runs out sets the per-device error word and the kernel still ends.
+//   * phase 1 streams K from HBM: D[128 q x 128 keys] = Q K^T (tcgen05.mma kind::f16,
+//     M = N = 128, fp32 accumulator in TMEM); phase 2 re-reads each tile a bounded number
+//     of tiles later (so it comes from L2, loaded evict-first): D[128 keys x 128 q] = K Q^T;
+//   * two MMA issuers (one per phase) claim job numbers from a shared counter when their
+//     next job is ready -- a phase-2 tile once its unit's lse is known -- and job n fills
+//     TMEM accumulator n % 4; four consumer warpgroups each drain one accumulator and handle
+//     either kind of job, so the exponentials do not wait on the cross-CTA dependency while
+//     phase-1 work exists.  Accumulators are taken in job order and the phase-1 record ring
+//     is released through a monotonic counter: a parity wait on an mbarrier that may lag two
+//     phases behind its waiter would pass early;
+//   * a phase-1 job yields per query row the tile's (max, sum of 2^(y - max)); a publisher
+//     warp merges them in tile order, rescales the CTA's sum to a fixed per-row reference
+//     (the row's logit with the key at its own position, computed before the kernel), adds
+//     it to the unit's fp64 total with a fire-and-forget atomic and bumps the unit's arrival
+//     count (fp64 addition order moves the total by ~1e-16, far below fp32);
+//   * an lse warp waits for each unit's count, turns the totals into lse = ref + log2(total)
+//     in shared memory and releases the unit's phase-2 jobs; a phase-2 job gives each key
+//     of the tile its sum over the query rows of 2^(y - lse).
+// Two TMA producers with their own shared-memory rings (16 KiB half-tiles of 64 columns,
+// the 128-byte swizzle atom) keep the HBM stream independent of phase-2 waits.  Warps:
+// 0 phase-1 TMA, 1 TMEM owner + phase-1 MMA, 2 phase-2 TMA, 3 phase-2 MMA, 4 lse,
+// 5 publisher, 6-7 idle, 8-23 consumers (four warpgroups, one per accumulator).  Every
+// wait is bounded: a wait that runs out sets the per-device error word and the kernel
+// still ends.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -63,8 +71,11 @@ constexpr int kStagesA = KVC_TC_STAGES_A;              // phase-1 ring (HBM stre
 constexpr int kStagesB = KVC_TC_STAGES_B;              // phase-2 ring (L2 re-read)
 constexpr int kQSlots = KVC_TC_Q_SLOTS;                // Q of the CTA's last units, by unit ordinal
 constexpr int kLeadSlack = KVC_TC_LEAD_SLACK;          // phase-1 lead beyond one unit, in tiles
-constexpr int kWarps = 24;  // 4 producer/MMA, 2 x 4 phase-1, 2 x 4 phase-2, 4 publisher
+constexpr int kAcc = 4;                // TMEM accumulators (128 columns each) = consumer warpgroups
+constexpr int kRec = 8;                // phase-1 tile records between consumers and publisher
+constexpr int kWarps = 24;
 constexpr int kThreads = kWarps * 32;
+constexpr int kConsumer0 = 8;          // first consumer warp
 constexpr int kMaxCtas = 160;                          // upper bound on the persistent grid
 constexpr uint32_t kTmemCols = 512;
 constexpr long long kBarrierTimeoutNs = 4000000000LL;  // hang guard for intra-CTA waits
@@ -90,16 +101,20 @@ struct __align__(1024) Smem {
     uint8_t ringA[kStagesA][kBoxBytes];
     uint8_t ringB[kStagesB][kBoxBytes];
     uint8_t q[kQSlots][2 * kBoxBytes];  // Q of the CTA's k-th unit in slot k % kQSlots (two boxes)
-    float lse[2][kQRows];         // per phase-2 warpgroup
-    float2 pub[2][2][kQRows];     // [slot][phase-1 warpgroup][row]
-    int pub_unit[2];
+    float2 rec[kRec][kQRows];           // phase-1 tile i: per row (tile max, sum of 2^(y - max))
+    float lse[2][kQRows];               // lse of the CTA's k-th unit in slot k % 2
+    int4 job[kAcc];                     // {kind, unit, tile within unit, record or lse slot}
     uint64_t fullA[kStagesA], emptyA[kStagesA], fullB[kStagesB], emptyB[kStagesB];
     uint64_t qfull[kQSlots], qempty[kQSlots];
-    uint64_t d1full[2], d1empty[2], d2full[2], d2empty[2];
-    uint64_t pub_full[2], pub_empty[2];
+    uint64_t accfull[kAcc], accempty[kAcc];
+    uint64_t recfull[kRec];
+    uint64_t lsefull[2];
+    unsigned lse_done[2];  // consumer warps done with the lse slot (monotonic)
+    int next_job;          // job numbers claimed by the two MMA issuers
+    int jobs_started;      // jobs that own their accumulator (taken in job order)
+    int rec_consumed;      // phase-1 records the publisher has read (monotonic)
     uint32_t tmem_base;
     int abort;
-    int flag2[2];
     int p1_issued, p2_issued;  // tiles whose loads each producer has issued (L2 lead control)
 };
 
@@ -156,6 +171,22 @@ __device__ __forceinline__ void mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+// Bounded wait until the shared counter *c (written by other warps of the CTA) reaches v.
+__device__ __forceinline__ void spin_until_at_least(int* c, int v, volatile int* abort, unsigned* err) {
+    volatile int* vc = c;
+    if (*vc >= v) return;
+    const long long t0 = globaltimer();
+    while (*vc < v) {
+        if (*abort) return;
+        if (globaltimer() - t0 > kBarrierTimeoutNs) {
+            atomicOr(err, kErrTimeout);
+            *abort = 1;
+            return;
+        }
+    }
+    __threadfence_block();
+}
+
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
                                             int z) {
     asm volatile(
@@ -202,18 +233,23 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
     return d;
 }
 
-// Descriptor of K-slice kk (16 columns = 32 bytes, kk < 4) of a 128-row x 64-column bf16
-// box.
-__device__ __forceinline__ uint64_t box_desc(const uint8_t* box, int kk) {
-    return sw128_desc(smem_u32(box) + kk * 32);
-}
-
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t accumulate) {
+template <int ACC>
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b) {
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate)
+        ::"r"(d_tmem), "l"(a), "l"(b), "r"(kIdesc), "n"(ACC)
         : "memory");
+}
+
+// The 8 MMAs (K = 128 in slices of 16) of one 128 x 128 x 128 product; the operands are the
+// two 64-column halves (h) of A and B, given as descriptors of half 0 and the half stride.
+__device__ __forceinline__ void umma_half(uint32_t d, uint64_t a, uint64_t b, int h) {
+    if (h == 0) umma_bf16<0>(d, a, b);
+    else umma_bf16<1>(d, a, b);
+    umma_bf16<1>(d, a + 2, b + 2);
+    umma_bf16<1>(d, a + 4, b + 4);
+    umma_bf16<1>(d, a + 6, b + 6);
 }
 
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -280,13 +316,10 @@ __device__ __forceinline__ float exp2_poly(float y) {
 #ifndef KVC_TC_POLY_EVERY
 #define KVC_TC_POLY_EVERY 0
 #endif
+__host__ __device__ constexpr bool poly_slot(int e) { return KVC_TC_POLY_EVERY > 0 && e % (KVC_TC_POLY_EVERY > 0 ? KVC_TC_POLY_EVERY : 1) == KVC_TC_POLY_EVERY - 1; }
 template <int E>
 __device__ __forceinline__ float exp2_mixed(float y) {
-    return (KVC_TC_POLY_EVERY > 0 && (E % KVC_TC_POLY_EVERY) == KVC_TC_POLY_EVERY - 1) ? exp2_poly(y) : ex2(y);
-}
-
-__device__ __forceinline__ void named_sync(int id, int n) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+    return poly_slot(E) ? exp2_poly(y) : ex2(y);
 }
 
 __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
@@ -347,12 +380,30 @@ __device__ __forceinline__ float prob_sum(const uint32_t (&x)[32], const float* 
 
 // ------------------------------------------------------------------------ the kernel
 
+// The CTA's local tiles i = 0, 1, ... are the global tiles cta + i * P; these helpers give
+// their unit and the local range of each unit.
+struct TileSeq {
+    int cta, P, T_u, n_local;
+    __device__ __forceinline__ int unit(int i) const { return (cta + i * P) / T_u; }
+    __device__ __forceinline__ int tile(int i) const { return cta + i * P - unit(i) * T_u; }
+    // first local tile whose global index is >= g
+    __device__ __forceinline__ int first_at(long long g) const {
+        const long long d = g - cta;
+        const long long i = d <= 0 ? 0 : (d + P - 1) / P;
+        return (int)(i < n_local ? i : n_local);
+    }
+    __device__ __forceinline__ int count(int u) const {
+        return first_at((long long)(u + 1) * T_u) - first_at((long long)u * T_u);
+    }
+};
+
 __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_constant__ TcArgs a) {
     extern __shared__ uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cta = blockIdx.x, P = a.P;
     const int n_local = cta < a.total_tiles ? (a.total_tiles - cta + P - 1) / P : 0;
+    const TileSeq seq{cta, P, a.T_u, n_local};
     volatile int* abort = &sm.abort;
 
     if (threadIdx.x == 0) {
@@ -366,17 +417,23 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
         }
         for (int b = 0; b < kQSlots; ++b) {
             mbar_init(&sm.qfull[b], 1);
-            mbar_init(&sm.qempty[b], 2);  // released by both MMA issuers
+            mbar_init(&sm.qempty[b], 1);
+        }
+        for (int b = 0; b < kAcc; ++b) {
+            mbar_init(&sm.accfull[b], 2);   // the issuer's arrive (job record) + the MMA commit
+            mbar_init(&sm.accempty[b], 4);  // one arrive per consumer warp
+        }
+        for (int b = 0; b < kRec; ++b) {
+            mbar_init(&sm.recfull[b], 4);
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&sm.d1full[b], 1);
-            mbar_init(&sm.d1empty[b], 4);
-            mbar_init(&sm.d2full[b], 1);
-            mbar_init(&sm.d2empty[b], 4);
-            mbar_init(&sm.pub_full[b], 2 * kQRows);
-            mbar_init(&sm.pub_empty[b], 1);
+            mbar_init(&sm.lsefull[b], 1);
+            sm.lse_done[b] = 0u;
         }
         sm.abort = 0;
+        sm.next_job = 0;
+        sm.jobs_started = 0;
+        sm.rec_consumed = 0;
         sm.p1_issued = 0;
         sm.p2_issued = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -408,31 +465,31 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             volatile int* other = ph == 0 ? &sm.p2_issued : &sm.p1_issued;
             int k = 0, qunit = -1, ord = -1;
             for (int i = 0; i < n_local && !*abort; ++i) {
-                const int t = cta + i * P, u = t / a.T_u, ti = t - u * a.T_u;
+                const int u = seq.unit(i), ti = seq.tile(i);
                 // phase 1 stays at most max_lead tiles ahead of phase 2 (L2 footprint);
                 // phase 2 never loads a tile before phase 1 has (so its read hits L2)
-                const long long t0 = globaltimer();
-                while (ph == 0 ? (i - *other >= a.max_lead) : (i >= *other)) {
-                    if (*abort) break;
-                    if (globaltimer() - t0 > kBarrierTimeoutNs) {
-                        atomicOr(a.err, kErrTimeout);
-                        *abort = 1;
-                        break;
+                if (ph == 0 ? (i - *other >= a.max_lead) : (i >= *other)) {
+                    const long long t0 = globaltimer();
+                    while (ph == 0 ? (i - *other >= a.max_lead) : (i >= *other)) {
+                        if (*abort) break;
+                        if (globaltimer() - t0 > kBarrierTimeoutNs) {
+                            atomicOr(a.err, kErrTimeout);
+                            *abort = 1;
+                            break;
+                        }
+                        __nanosleep(64);
                     }
-                    __nanosleep(128);
                 }
-                if (u != qunit) {
-                    // the CTA's ord-th unit: phase 1 loads its Q into slot ord % kQSlots once both
-                    // phases are done with the unit that used the slot kQSlots units ago
+                if (ph == 0 && u != qunit) {
+                    // the CTA's ord-th unit: load its Q into slot ord % kQSlots once phase 2
+                    // is done with the unit that used the slot kQSlots units ago
                     qunit = u;
                     ++ord;
-                    if (ph == 0) {
-                        const int slot = ord % kQSlots;
-                        if (ord >= kQSlots) mbar_wait(&sm.qempty[slot], ((ord / kQSlots) - 1) & 1, abort, a.err);
-                        mbar_expect_tx(&sm.qfull[slot], 2 * kBoxBytes);
-                        tma_load_2d(sm.q[slot], &a.tmap_q, &sm.qfull[slot], 0, u * kQRows);
-                        tma_load_2d(sm.q[slot] + kBoxBytes, &a.tmap_q, &sm.qfull[slot], 64, u * kQRows);
-                    }
+                    const int slot = ord % kQSlots;
+                    if (ord >= kQSlots) mbar_wait(&sm.qempty[slot], ((ord / kQSlots) - 1) & 1, abort, a.err);
+                    mbar_expect_tx(&sm.qfull[slot], 2 * kBoxBytes);
+                    tma_load_2d(sm.q[slot], &a.tmap_q, &sm.qfull[slot], 0, u * kQRows);
+                    tma_load_2d(sm.q[slot] + kBoxBytes, &a.tmap_q, &sm.qfull[slot], 64, u * kQRows);
                 }
                 for (int h = 0; h < 2; ++h, ++k) {
                     const int s = k % stages;
@@ -448,190 +505,263 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
         }
     } else if (warp == 1 || warp == 3) {
         // ------------------------------------------------------------ MMA issuers
+        // Warp 1 issues the phase-1 jobs, warp 3 the phase-2 jobs (a phase-2 tile once its
+        // unit's lse is in shared memory).  Each claims the next job number n when its job is
+        // ready and fills accumulator n % kAcc, so the consumers see one stream of jobs.  Two
+        // issuers keep the tensor pipe busy while either does its bookkeeping.
         if (lane == 0) {
             const int ph = warp == 1 ? 0 : 1;
-            uint8_t(*ring)[kBoxBytes] = ph == 0 ? sm.ringA : sm.ringB;
+            const int stages = ph == 0 ? kStagesA : kStagesB;
             uint64_t* full = ph == 0 ? sm.fullA : sm.fullB;
             uint64_t* empty = ph == 0 ? sm.emptyA : sm.emptyB;
-            uint64_t* dfull = ph == 0 ? sm.d1full : sm.d2full;
-            uint64_t* dempty = ph == 0 ? sm.d1empty : sm.d2empty;
-            const int stages = ph == 0 ? kStagesA : kStagesB;
-            const uint32_t dbase = tmem + (ph == 0 ? 0u : 256u);
-            int k = 0, qunit = -1, ord = -1;
-            const uint8_t* qtile = sm.q[0];
+            const uint64_t dK0 = sw128_desc(smem_u32(ph == 0 ? sm.ringA[0] : sm.ringB[0]));
+            const uint64_t dQ0 = sw128_desc(smem_u32(sm.q[0]));
+            constexpr uint64_t kBoxStep = kBoxBytes >> 4, kQStep = (2 * kBoxBytes) >> 4;
+            int u = cta / a.T_u, t = cta - (cta / a.T_u) * a.T_u;  // unit and tile of local tile i
+            int ord = 0, qslot = 0;                                 // unit ordinal, its Q slot
+            int s = 0;
+            uint32_t sph = 0;  // ring stage and phase
+            bool have_q = false;
             for (int i = 0; i < n_local && !*abort; ++i) {
-                const int t = cta + i * P, u = t / a.T_u;
-                if (u != qunit) {
-                    // this phase is done with the previous unit's Q slot once its MMAs finish
-                    if (ord >= 0) umma_commit(&sm.qempty[ord % kQSlots]);
-                    ++ord;
-                    mbar_wait(&sm.qfull[ord % kQSlots], (ord / kQSlots) & 1, abort, a.err);
-                    qtile = sm.q[ord % kQSlots];
-                    qunit = u;
+                if (!have_q) {
+                    // the unit's Q (its slot is not refilled before phase 2 releases it)
+                    mbar_wait(&sm.qfull[qslot], (ord / kQSlots) & 1, abort, a.err);
+                    have_q = true;
                 }
-                const int b = i & 1;
-                mbar_wait(&dempty[b], ((i >> 1) & 1) ^ 1, abort, a.err);
+                // phase 2 of a tile waits until its unit's lse is in shared memory
+                if (ph == 1) mbar_wait(&sm.lsefull[ord & 1], (ord >> 1) & 1, abort, a.err);
+                mbar_wait(&full[s], sph, abort, a.err);
+                const int n = atomicAdd(&sm.next_job, 1);
+                const int slot = n % kAcc;
+                // Accumulators are taken in job order: job n waits for the release of job
+                // n - kAcc only after job n - 1 has taken its own, so that the accumulator's
+                // barrier is never two phases behind this wait (a parity wait would pass).
+                spin_until_at_least(&sm.jobs_started, n, abort, a.err);
+                mbar_wait(&sm.accempty[slot], ((n / kAcc) & 1) ^ 1, abort, a.err);
                 tc_fence_after();
-                const uint32_t d = dbase + b * 128;
-                for (int h = 0; h < 2; ++h, ++k) {
-                    const int s = k % stages;
-                    mbar_wait(&full[s], (k / stages) & 1, abort, a.err);
+                *reinterpret_cast<volatile int*>(&sm.jobs_started) = n + 1;
+                sm.job[slot] = make_int4(ph, u, t, ph == 0 ? i : (ord & 1));
+                mbar_arrive(&sm.accfull[slot]);
+                const uint32_t d = tmem + slot * 128;
+                const uint64_t dq = dQ0 + (uint64_t)qslot * kQStep;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    if (h == 1) mbar_wait(&full[s], sph, abort, a.err);
                     tc_fence_after();
-                    const uint8_t* qbox = qtile + h * kBoxBytes;
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        if (ph == 0)
-                            umma_bf16(d, box_desc(qbox, kk), box_desc(ring[s], kk), (h | kk) != 0);
-                        else
-                            umma_bf16(d, box_desc(ring[s], kk), box_desc(qbox, kk), (h | kk) != 0);
-                    }
+                    const uint64_t dk = dK0 + (uint64_t)s * kBoxStep;
+                    if (ph == 0)
+                        umma_half(d, dq + h * kBoxStep, dk, h);
+                    else
+                        umma_half(d, dk, dq + h * kBoxStep, h);
                     umma_commit(&empty[s]);
+                    if (++s == stages) {
+                        s = 0;
+                        sph ^= 1u;
+                    }
                 }
-                umma_commit(&dfull[b]);
+                umma_commit(&sm.accfull[slot]);
+                // next tile; a new unit moves to the next Q slot (phase 2 releases the old one)
+                t += P;
+                int nu = u;
+                while (t >= a.T_u) {
+                    t -= a.T_u;
+                    ++nu;
+                }
+                if (nu != u) {
+                    if (ph == 1 && i + 1 < n_local) umma_commit(&sm.qempty[qslot]);
+                    u = nu;
+                    ++ord;
+                    if (++qslot == kQSlots) qslot = 0;
+                    have_q = false;
+                }
             }
         }
-    } else if (warp >= 4 && warp < 12) {
-        // ------------------------------------------------------------ phase 1: statistics
-        // warpgroup w takes the local tiles i with i % 2 == w (accumulator buffer w)
-        const int w = (warp - 4) >> 2;
-        const int r = threadIdx.x - 128 - 128 * w;  // query row == TMEM lane
-        const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + w * 128;
-        const int t_r = a.N - a.w + (r % a.w);  // last key this row sees
-        int cur = -1, npub = 0;
-        float m = -INFINITY, l = 0.f;
-        for (int i = 0; i <= n_local; ++i) {
-            const int t = cta + i * P;
-            const int u = i < n_local ? t / a.T_u : -2;
-            if (u != cur && cur >= 0) {
-                // hand this warpgroup's (max, sum) of unit `cur` to the publisher warp
-                const int slot = npub & 1;
-                mbar_wait(&sm.pub_empty[slot], ((npub >> 1) & 1) ^ 1, abort, a.err);
-                sm.pub[slot][w][r] = make_float2(m, l);
-                if (r == 0 && w == 0) sm.pub_unit[slot] = cur;
-                mbar_arrive(&sm.pub_full[slot]);
-                ++npub;
-            }
-            if (i == n_local) break;
-            if (u != cur) {
-                cur = u;
-                m = -INFINITY;
-                l = 0.f;
-            }
-            if ((i & 1) != w) continue;
-            const int ti = t - u * a.T_u;
-            mbar_wait(&sm.d1full[w], (i >> 1) & 1, abort, a.err);
-            tc_fence_after();
-            const bool full_tile = (ti + 1) * kTileKeys <= a.N - a.w + 1;
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                uint32_t x[32];
-                __syncwarp();
-                tmem_ld32(tl + c * 32, x);
-                tmem_wait32(x);
-                if (c == 3) {
-                    // the accumulator can take the next tile once it is in registers
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm.d1empty[w]);
-                }
-                if (!full_tile) {
-                    // causal mask: this row sees keys j <= t_r
-                    const int j0 = ti * kTileKeys + c * 32;
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (j0 + e > t_r) x[e] = __float_as_uint(-INFINITY);
-                }
-                stats_update(x, m, l);
-            }
-        }
-    } else if (warp >= 12 && warp < 20) {
-        // ------------------------------------------------------------ phase 2: scores
-        const int w = (warp - 12) >> 2;
-        const int r = threadIdx.x - 384 - 128 * w;  // key within the tile == TMEM lane
-        const uint32_t tl = tmem + 256 + ((uint32_t)(32 * (warp & 3)) << 16) + w * 128;
-        float* lse = sm.lse[w];
-        int cur = -1;
+    } else if (warp == 4) {
+        // ------------------------------------------------------------ lse of each unit
+        // lane l handles query rows l, l + 32, l + 64, l + 96
+        int cur = -1, ord = -1;
+        unsigned target[2] = {0u, 0u};
         bool gave_up = false;
-        for (int i = w; i < n_local; i += 2) {
-            const int t = cta + i * P, u = t / a.T_u, ti = t - u * a.T_u;
-            if (u != cur) {
-                named_sync(2 + w, 128);  // all threads are done with the previous unit's lse
-                if (r == 0) {
-                    // unit u is complete once every CTA holding tiles of it has added its part
-                    const unsigned* cnt = a.inject ? a.never : a.count + u;
-                    const unsigned n_contrib = (unsigned)min(a.T_u, a.P);
-                    bool ok = ld_acquire(cnt) >= n_contrib;
-                    for (long long spins = 0; !ok && !gave_up && spins < a.spin_limit; ++spins) {
-                        __nanosleep(64);
-                        ok = ld_acquire(cnt) >= n_contrib;
-                    }
-                    if (!ok) {
+        const unsigned n_contrib = (unsigned)min(a.T_u, a.P);
+        for (int i = 0; i < n_local && !*abort; ++i) {
+            const int u = seq.unit(i);
+            if (u == cur) continue;
+            cur = u;
+            ++ord;
+            const int slot = ord & 1;
+            // every phase-2 job of the unit that used this slot before has read it
+            if (lane == 0 && *reinterpret_cast<volatile unsigned*>(&sm.lse_done[slot]) < target[slot]) {
+                const long long t0 = globaltimer();
+                while (*reinterpret_cast<volatile unsigned*>(&sm.lse_done[slot]) < target[slot]) {
+                    if (*abort) break;
+                    if (globaltimer() - t0 > kBarrierTimeoutNs) {
                         atomicOr(a.err, kErrTimeout);
-                        gave_up = true;  // later units do not wait again
+                        *abort = 1;
+                        break;
                     }
-                    sm.flag2[w] = ok;
                 }
-                named_sync(2 + w, 128);
-                const bool ok = sm.flag2[w];
-                lse[r] = (ok && r < a.nq)
-                             ? (float)((double)__ldg(a.ref + (size_t)u * kQRows + r) + log2(__ldcg(a.sum + (size_t)u * kQRows + r)))
-                             : INFINITY;
-                named_sync(2 + w, 128);
-                cur = u;
             }
-            mbar_wait(&sm.d2full[w], (i >> 1) & 1, abort, a.err);
-            tc_fence_after();
-            const int j = ti * kTileKeys + r;
-            const bool full_tile = (ti + 1) * kTileKeys <= a.N - a.w + 1;
-            float s = 0.f;
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                uint32_t x[32];
-                __syncwarp();
-                tmem_ld32(tl + c * 32, x);
-                tmem_wait32(x);
-                if (c == 3) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm.d2empty[w]);
+            target[slot] += 4u * (unsigned)seq.count(u);
+            // unit u is complete once every CTA holding tiles of it has added its part
+            int ok = 0;
+            if (lane == 0) {
+                const unsigned* cnt = a.inject ? a.never : a.count + u;
+                bool done = ld_acquire(cnt) >= n_contrib;
+                for (long long spins = 0; !done && !gave_up && spins < a.spin_limit && !*abort; ++spins) {
+                    __nanosleep(32);
+                    done = ld_acquire(cnt) >= n_contrib;
                 }
-                if (!full_tile) {
-                    // causal mask: query row q (position N - w + q % w) sees this key iff j <= that
+                if (!done) {
+                    atomicOr(a.err, kErrTimeout);
+                    gave_up = true;  // later units do not wait again
+                }
+                ok = done;
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            __syncwarp();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (j > a.N - a.w + (c * 32 + e) % a.w) x[e] = __float_as_uint(-INFINITY);
-                }
-                s += prob_sum(x, lse + c * 32);
+            for (int rr = 0; rr < 4; ++rr) {
+                const int r = lane + 32 * rr;
+                sm.lse[slot][r] = (ok && r < a.nq)
+                                      ? (float)((double)__ldg(a.ref + (size_t)u * kQRows + r) +
+                                                log2(__ldcg(a.sum + (size_t)u * kQRows + r)))
+                                      : INFINITY;
             }
-            if (j < a.N) a.unit_scores[(size_t)u * a.N + j] = s;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.lsefull[slot]);
         }
-    } else if (warp >= 20) {
+    } else if (warp == 5) {
         // ------------------------------------------------------------ publisher
-        // one thread per query row; named barrier 4 spans these four warps
-        const int r = threadIdx.x - 640;
-        int npub = 0;
+        // lane l holds query rows l + 32 k; merges the phase-1 tile records in tile order and
+        // adds the CTA's part of each unit to the unit's total
+        float M[4], L[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            M[k] = -INFINITY;
+            L[k] = 0.f;
+        }
+        int u = cta / a.T_u, t = cta - (cta / a.T_u) * a.T_u;
         for (int i = 0; i < n_local; ++i) {
-            const int cur = (cta + i * P) / a.T_u;
-            const bool last_tile_of_unit = (i + 1 == n_local) || ((cta + (i + 1) * P) / a.T_u != cur);
-            if (!last_tile_of_unit) continue;
-            const int slot = npub & 1;
-            mbar_wait(&sm.pub_full[slot], (npub >> 1) & 1, abort, a.err);
-            const float2 p0 = sm.pub[slot][0][r], p1 = sm.pub[slot][1][r];
-            named_sync(4, 128);
-            if (r == 0) mbar_arrive(&sm.pub_empty[slot]);
-            ++npub;
-            // this CTA's sum over its keys of 2^(y - ref), added into the unit's fp64 total
-            const float M = fmaxf(p0.x, p1.x);
-            if (M != -INFINITY) {
-                float S = 0.f;
-                if (p0.x != -INFINITY) S += p0.y * ex2(p0.x - M);
-                if (p1.x != -INFINITY) S += p1.y * ex2(p1.x - M);
-                const double ref = (double)__ldg(a.ref + (size_t)cur * kQRows + r);
-                atomicAdd(a.sum + (size_t)cur * kQRows + r, (double)S * exp2((double)M - ref));
+            const int s = i % kRec;
+            mbar_wait(&sm.recfull[s], (i / kRec) & 1, abort, a.err);
+            if (*abort) break;
+            float2 v[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) v[k] = sm.rec[s][lane + 32 * k];
+            __syncwarp();
+            if (lane == 0) {
+                __threadfence_block();
+                *reinterpret_cast<volatile int*>(&sm.rec_consumed) = i + 1;
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                if (v[k].x != -INFINITY) {
+                    const float mn = fmaxf(M[k], v[k].x);
+                    L[k] = (M[k] == -INFINITY ? 0.f : L[k] * ex2(M[k] - mn)) + v[k].y * ex2(v[k].x - mn);
+                    M[k] = mn;
+                }
+            }
+            t += P;
+            int nu = u;
+            while (t >= a.T_u) {
+                t -= a.T_u;
+                ++nu;
+            }
+            if (nu == u && i + 1 < n_local) continue;
+            // last tile of unit u on this CTA
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int r = lane + 32 * k;
+                if (M[k] != -INFINITY) {
+                    const double ref = (double)__ldg(a.ref + (size_t)u * kQRows + r);
+                    atomicAdd(a.sum + (size_t)u * kQRows + r, (double)L[k] * exp2((double)M[k] - ref));
+                }
+                M[k] = -INFINITY;
+                L[k] = 0.f;
             }
             __threadfence();
-            named_sync(4, 128);
-            if (r == 0) atomicAdd(a.count + cur, 1u);
+            __syncwarp();
+            if (lane == 0) atomicAdd(a.count + u, 1u);
+            u = nu;
+        }
+    } else if (warp >= kConsumer0) {
+        // ------------------------------------------------------------ consumers
+        // warpgroup g drains accumulator g: jobs g, g + kAcc, ...; thread = TMEM lane, i.e.
+        // a query row for phase-1 jobs and a key of the tile for phase-2 jobs
+        const int g = (warp - kConsumer0) >> 2;
+        const int r = threadIdx.x - 32 * kConsumer0 - 128 * g;
+        const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + g * 128;
+        const int n_jobs = 2 * n_local;
+        for (int n = g; n < n_jobs; n += kAcc) {
+            mbar_wait(&sm.accfull[g], (n / kAcc) & 1, abort, a.err);
+            if (*abort) break;
+            tc_fence_after();
+            int4 jb;
+            asm volatile("ld.shared.v4.s32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(jb.x), "=r"(jb.y), "=r"(jb.z), "=r"(jb.w)
+                         : "r"(smem_u32(&sm.job[g]))
+                         : "memory");
+            const int u = jb.y, ti = jb.z;
+            const bool full_tile = (ti + 1) * kTileKeys <= a.N - a.w + 1;
+            if (jb.x == 0) {
+                // phase 1: this row's (max, sum of 2^(y - max)) over the tile's visible keys
+                const int t_r = a.N - a.w + (r % a.w);  // last key this row sees
+                float m = -INFINITY, l = 0.f;
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t x[32];
+                    __syncwarp();
+                    tmem_ld32(tl + c * 32, x);
+                    tmem_wait32(x);
+                    if (c == 3) {
+                        // the accumulator can take the next job once it is in registers
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&sm.accempty[g]);
+                    }
+                    if (!full_tile) {
+                        const int j0 = ti * kTileKeys + c * 32;
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (j0 + e > t_r) x[e] = __float_as_uint(-INFINITY);
+                    }
+                    stats_update(x, m, l);
+                }
+                // record slot i % kRec is free once the publisher has read record i - kRec
+                const int i = jb.w, s = i % kRec;
+                if (lane == 0) spin_until_at_least(&sm.rec_consumed, i - kRec + 1, abort, a.err);
+                __syncwarp();
+                sm.rec[s][r] = make_float2(m, l);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.recfull[s]);
+            } else {
+                // phase 2: this key's sum over the query rows of 2^(y - lse)
+                const float* lse = sm.lse[jb.w];
+                const int j = ti * kTileKeys + r;
+                float sc = 0.f;
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t x[32];
+                    __syncwarp();
+                    tmem_ld32(tl + c * 32, x);
+                    tmem_wait32(x);
+                    if (c == 3) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&sm.accempty[g]);
+                    }
+                    if (!full_tile) {
+                        // query row q (position N - w + q % w) sees this key iff j <= that
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (j > a.N - a.w + (c * 32 + e) % a.w) x[e] = __float_as_uint(-INFINITY);
+                    }
+                    sc += prob_sum(x, lse + c * 32);
+                }
+                if (j < a.N) a.unit_scores[(size_t)u * a.N + j] = sc;
+                __syncwarp();
+                if (lane == 0) atomicAdd(&sm.lse_done[jb.w], 1u);
+            }
         }
     }
 
