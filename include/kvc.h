@@ -258,14 +258,6 @@ KVC_API kvc_status kvc_poll_error(kvc_stream_t stream);
  */
 KVC_API uint64_t kvc_launch_count(void);
 
-/*
- * kvc_debug_exp2 -- diagnostics: out[i] = the software 2^y[i] that the tensor-core scoring
- * kernel evaluates on the FMA pipe for part of its exponentials (range reduction to
- * [-1/2, 1/2] plus a degree-5 minimax polynomial; relative error about 2.3e-7 for y in
- * [-125, 0], about 2^-125 for smaller y).  y, out: device, n floats.
- */
-KVC_API kvc_status kvc_debug_exp2(const float *y, float *out, int32_t n, kvc_stream_t stream);
-
 /* kvc_status_string -- static description of a status code (never NULL). */
 KVC_API const char *kvc_status_string(kvc_status status);
 

@@ -356,12 +356,6 @@ const char* kvc_status_string(kvc_status st) {
     return "unknown status";
 }
 
-kvc_status kvc_debug_exp2(const float* y, float* out, int32_t n, kvc_stream_t stream) {
-    if (!y || !out || n < 0) return KVC_ERR_ARG;
-    KVC_CUDA(kvc::debug_exp2(y, out, n, (cudaStream_t)stream));
-    return KVC_OK;
-}
-
 uint64_t kvc_launch_count(void) { return (uint64_t)g_launches.load(std::memory_order_relaxed); }
 
 const char* kvc_version(void) { return "kvc 0.1.0 sm_100a"; }

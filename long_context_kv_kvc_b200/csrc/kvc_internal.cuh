@@ -60,7 +60,6 @@ size_t tc_score_workspace(int U, int N, int nq);
 cudaError_t tc_score(const ScoreJob& job, cudaStream_t s);
 
 // the tensor-core kernel's software exp2, element-wise (diagnostics)
-cudaError_t debug_exp2(const float* y, float* out, int n, cudaStream_t s);
 
 // sums of unit scores over layers (and KV heads for the all-heads scope)
 cudaError_t reduce_units(const float* unit_scores, int L, int B, int Hkv, int N, int all_heads,

@@ -65,7 +65,7 @@ constexpr int kBoxBytes = kTileKeys * 64 * 2;          // a 128-row x 64-column 
 #define KVC_TC_Q_SLOTS 3
 #endif
 #ifndef KVC_TC_LEAD_SLACK
-#define KVC_TC_LEAD_SLACK 8
+#define KVC_TC_LEAD_SLACK 6
 #endif
 constexpr int kStagesA = KVC_TC_STAGES_A;              // phase-1 ring (HBM stream)
 constexpr int kStagesB = KVC_TC_STAGES_B;              // phase-2 ring (L2 re-read)
@@ -76,6 +76,10 @@ constexpr int kRec = 8;                // phase-1 tile records between consumers
 constexpr int kWarps = 24;
 constexpr int kThreads = kWarps * 32;
 constexpr int kConsumer0 = 8;          // first consumer warp
+#ifndef KVC_TC_SUM_COPIES
+#define KVC_TC_SUM_COPIES 8
+#endif
+constexpr int kSumCopies = KVC_TC_SUM_COPIES;  // copies of each unit's totals (CTA c adds to copy c % kSumCopies)
 constexpr int kMaxCtas = 160;                          // upper bound on the persistent grid
 constexpr uint32_t kTmemCols = 512;
 constexpr long long kBarrierTimeoutNs = 4000000000LL;  // hang guard for intra-CTA waits
@@ -89,7 +93,8 @@ struct TcArgs {
     CUtensorMap tmap_q;  // padded Q as [U*128][128] bf16, box 64 x 128, 128-byte swizzle
     float* unit_scores;  // [U][N]
     const float* ref;    // [U][128] per-row reference logit (base 2): the row's own-position key
-    double* sum;         // [U][128] sum over keys of 2^(y - ref), accumulated by all CTAs
+    double* sum;         // [U][kSumCopies][128] sums over keys of 2^(y - ref); CTA c adds into copy
+                         // c % kSumCopies, which spreads the atomics of the 148 CTAs over more addresses
     unsigned* count;     // [U] CTAs that have added their part of unit u
     unsigned* never;     // a counter nothing increments (wait-timeout injection)
     unsigned* err;
@@ -102,7 +107,7 @@ struct __align__(1024) Smem {
     uint8_t ringB[kStagesB][kBoxBytes];
     uint8_t q[kQSlots][2 * kBoxBytes];  // Q of the CTA's k-th unit in slot k % kQSlots (two boxes)
     float2 rec[kRec][kQRows];           // phase-1 tile i: per row (tile max, sum of 2^(y - max))
-    float lse[2][kQRows];               // lse of the CTA's k-th unit in slot k % 2
+    float nlse[2][kQRows];              // -lse of the CTA's k-th unit in slot k % 2
     int4 job[kAcc];                     // {kind, unit, tile within unit, record or lse slot}
     uint64_t fullA[kStagesA], emptyA[kStagesA], fullB[kStagesB], emptyB[kStagesB];
     uint64_t qfull[kQSlots], qempty[kQSlots];
@@ -290,36 +295,27 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// 2^y on the FMA pipe, for y <= ~0 (the kernel's arguments are logits minus a running
-// max or minus the log-sum-exp).  Cody-Waite range reduction y = n + f with n = round(y)
-// and f in [-1/2, 1/2]; 2^f from a degree-5 polynomial with equioscillating relative error
-// (Remez exchange, fitted by exp2_poly_fit.py next to this library, binary32 coefficients);
-// 2^n is added to the exponent field.  Arguments below -125 are clamped, which returns about
-// 2^-125 instead of 0 (absolute error below 3e-38).  Relative error about 2.3e-7 on [-125, 0].
-__device__ __forceinline__ float exp2_poly(float y) {
-    y = fmaxf(y, -125.0f);
-    const float t = y + 12582912.0f;  // 1.5 * 2^23: y rounded to an integer lands in t's low bits
-    const float n = t - 12582912.0f;
-    const float f = y - n;
-    float p = fmaf(f, 0.0013276472454890609f, 0.009675540961325169f);
-    p = fmaf(p, f, 0.05550713092088699f);
-    p = fmaf(p, f, 0.24022120237350464f);
-    p = fmaf(p, f, 0.6931469440460205f);
-    p = fmaf(p, f, 1.0000001192092896f);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+__device__ __forceinline__ float lg2(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
-// Exponentials of the fully visible tiles.  KVC_TC_POLY_EVERY = n > 0 sends one of every n
-// to the FMA-pipe polynomial; in this kernel all-MUFU measured fastest on B200 (the
-// polynomial costs about 13 issue slots, and the consumers are issue- and latency-bound
-// rather than MUFU-bound), so the default is 0.
-#ifndef KVC_TC_POLY_EVERY
-#define KVC_TC_POLY_EVERY 0
-#endif
-__host__ __device__ constexpr bool poly_slot(int e) { return KVC_TC_POLY_EVERY > 0 && e % (KVC_TC_POLY_EVERY > 0 ? KVC_TC_POLY_EVERY : 1) == KVC_TC_POLY_EVERY - 1; }
-template <int E>
-__device__ __forceinline__ float exp2_mixed(float y) {
-    return poly_slot(E) ? exp2_poly(y) : ex2(y);
+// x * 2^d in fp64 for fp32 x and finite d: 2^d = 2^e * 2^f with e = floor(d), f in [0, 1);
+// 2^f on the special-function unit (relative error ~2^-22), 2^e exact from its exponent bits.
+__device__ __forceinline__ double scale_exp2(float x, float d) {
+    const float e = floorf(d);
+    const int ei = (int)fminf(fmaxf(e, -1022.f), 1023.f);
+    return (double)(x * ex2(d - e)) * __longlong_as_double((long long)(ei + 1023) << 52);
+}
+
+// log2 of a positive normal fp64 value: its binary exponent plus log2 of the mantissa in
+// [1/2, 1) on the special-function unit (absolute error ~2^-22).
+__device__ __forceinline__ float log2_pos(double v) {
+    const long long b = __double_as_longlong(v);
+    const int e = (int)((b >> 52) & 0x7FF) - 1022;
+    const double m = __longlong_as_double((b & ~(0x7FFLL << 52)) | (1022LL << 52));
+    return (float)e + lg2((float)m);
 }
 
 __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
@@ -328,54 +324,78 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
     return v;
 }
 
-// Online (max, sum) update of one query row with 32 logits (invisible keys already set
-// to -inf).
-__device__ __forceinline__ void stats_update(const uint32_t (&x)[32], float& m, float& l) {
+// Largest of 32 logits.
+__device__ __forceinline__ float chunk_max(const uint32_t (&x)[32]) {
     float mx[8];
 #pragma unroll
     for (int g = 0; g < 8; ++g) mx[g] = __uint_as_float(x[g]);
 #pragma unroll
     for (int e = 8; e < 32; ++e) mx[e & 7] = fmaxf(mx[e & 7], __uint_as_float(x[e]));
-    const float cm =
-        fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-    if (cm == -INFINITY) return;
-    const float mn = fmaxf(m, cm * kLog2eOverSqrtD);
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+}
+
+// Packed fp32 pairs (Blackwell's f32x2 FMA/ADD): one instruction for two lanes' worth of
+// elementwise work.
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// 2^y for both halves of a pair (special-function unit)
+__device__ __forceinline__ uint64_t ex2_pair(uint64_t y) {
+    float a, b;
+    unpack2(y, a, b);
+    return pack2(ex2(a), ex2(b));
+}
+__device__ __forceinline__ float hsum2(uint64_t v) {
+    float a, b;
+    unpack2(v, a, b);
+    return a + b;
+}
+
+// Sum over 32 logits (invisible keys already set to -inf) of 2^(y - m) for a fixed m.
+__device__ __forceinline__ float sum_exp2_shifted(const uint32_t (&x)[32], float m) {
+    const uint64_t c2 = pack2(kLog2eOverSqrtD, kLog2eOverSqrtD), nm2 = pack2(-m, -m);
+    uint64_t acc0 = 0, acc1 = 0;  // (+0, +0) pairs
 #pragma unroll
-    for (int e = 0; e < 32; e += 8) {
-        acc[0] += exp2_mixed<0>(fmaf(__uint_as_float(x[e + 0]), kLog2eOverSqrtD, -mn));
-        acc[1] += exp2_mixed<1>(fmaf(__uint_as_float(x[e + 1]), kLog2eOverSqrtD, -mn));
-        acc[2] += exp2_mixed<2>(fmaf(__uint_as_float(x[e + 2]), kLog2eOverSqrtD, -mn));
-        acc[3] += exp2_mixed<3>(fmaf(__uint_as_float(x[e + 3]), kLog2eOverSqrtD, -mn));
-        acc[4] += exp2_mixed<4>(fmaf(__uint_as_float(x[e + 4]), kLog2eOverSqrtD, -mn));
-        acc[5] += exp2_mixed<5>(fmaf(__uint_as_float(x[e + 5]), kLog2eOverSqrtD, -mn));
-        acc[6] += exp2_mixed<6>(fmaf(__uint_as_float(x[e + 6]), kLog2eOverSqrtD, -mn));
-        acc[7] += exp2_mixed<7>(fmaf(__uint_as_float(x[e + 7]), kLog2eOverSqrtD, -mn));
+    for (int e = 0; e < 32; e += 4) {
+        const uint64_t y0 = fma2(pack2(__uint_as_float(x[e]), __uint_as_float(x[e + 1])), c2, nm2);
+        const uint64_t y1 = fma2(pack2(__uint_as_float(x[e + 2]), __uint_as_float(x[e + 3])), c2, nm2);
+        acc0 = add2(acc0, ex2_pair(y0));
+        acc1 = add2(acc1, ex2_pair(y1));
     }
-    const float sum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-    l = (m == -INFINITY ? 0.f : l * ex2(m - mn)) + sum;
-    m = mn;
+    return hsum2(add2(acc0, acc1));
 }
 
 // Sum over 32 query rows (invisible ones already set to -inf) of 2^(y - lse) for this
-// thread's key.
-__device__ __forceinline__ float prob_sum(const uint32_t (&x)[32], const float* lse) {
-    const float4* L4 = reinterpret_cast<const float4*>(lse);
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+// thread's key; nlse holds -lse per row.
+__device__ __forceinline__ float prob_sum(const uint32_t (&x)[32], const float* nlse) {
+    const uint64_t c2 = pack2(kLog2eOverSqrtD, kLog2eOverSqrtD);
+    const ulonglong2* L = reinterpret_cast<const ulonglong2*>(nlse);
+    uint64_t acc0 = 0, acc1 = 0;
 #pragma unroll
-    for (int e8 = 0; e8 < 4; ++e8) {
-        const float4 La = L4[2 * e8], Lb = L4[2 * e8 + 1];
-        const int e = 8 * e8;
-        acc[0] += exp2_mixed<0>(fmaf(__uint_as_float(x[e + 0]), kLog2eOverSqrtD, -La.x));
-        acc[1] += exp2_mixed<1>(fmaf(__uint_as_float(x[e + 1]), kLog2eOverSqrtD, -La.y));
-        acc[2] += exp2_mixed<2>(fmaf(__uint_as_float(x[e + 2]), kLog2eOverSqrtD, -La.z));
-        acc[3] += exp2_mixed<3>(fmaf(__uint_as_float(x[e + 3]), kLog2eOverSqrtD, -La.w));
-        acc[4] += exp2_mixed<4>(fmaf(__uint_as_float(x[e + 4]), kLog2eOverSqrtD, -Lb.x));
-        acc[5] += exp2_mixed<5>(fmaf(__uint_as_float(x[e + 5]), kLog2eOverSqrtD, -Lb.y));
-        acc[6] += exp2_mixed<6>(fmaf(__uint_as_float(x[e + 6]), kLog2eOverSqrtD, -Lb.z));
-        acc[7] += exp2_mixed<7>(fmaf(__uint_as_float(x[e + 7]), kLog2eOverSqrtD, -Lb.w));
+    for (int e4 = 0; e4 < 8; ++e4) {
+        const ulonglong2 l = L[e4];
+        const int e = 4 * e4;
+        const uint64_t y0 = fma2(pack2(__uint_as_float(x[e]), __uint_as_float(x[e + 1])), c2, l.x);
+        const uint64_t y1 = fma2(pack2(__uint_as_float(x[e + 2]), __uint_as_float(x[e + 3])), c2, l.y);
+        acc0 = add2(acc0, ex2_pair(y0));
+        acc1 = add2(acc1, ex2_pair(y1));
     }
-    return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+    return hsum2(add2(acc0, acc1));
 }
 
 // ------------------------------------------------------------------------ the kernel
@@ -619,13 +639,20 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             }
             ok = __shfl_sync(0xffffffffu, ok, 0);
             __syncwarp();
+            // the unit's total per row: the copies added in a fixed order
+            double tot[4] = {0.0, 0.0, 0.0, 0.0};
+            const double* su = a.sum + (size_t)u * kSumCopies * kQRows;
+#pragma unroll
+            for (int c = 0; c < kSumCopies; ++c)
+#pragma unroll
+                for (int rr = 0; rr < 4; ++rr) tot[rr] += __ldcg(su + c * kQRows + lane + 32 * rr);
 #pragma unroll
             for (int rr = 0; rr < 4; ++rr) {
                 const int r = lane + 32 * rr;
-                sm.lse[slot][r] = (ok && r < a.nq)
-                                      ? (float)((double)__ldg(a.ref + (size_t)u * kQRows + r) +
-                                                log2(__ldcg(a.sum + (size_t)u * kQRows + r)))
-                                      : INFINITY;
+                // the total is >= ~1: it holds the row's own-position key, whose logit is ref
+                sm.nlse[slot][r] = (ok && r < a.nq && tot[rr] > 0.0)
+                                       ? -(__ldg(a.ref + (size_t)u * kQRows + r) + log2_pos(tot[rr]))
+                                       : -INFINITY;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.lsefull[slot]);
@@ -672,10 +699,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const int r = lane + 32 * k;
-                if (M[k] != -INFINITY) {
-                    const double ref = (double)__ldg(a.ref + (size_t)u * kQRows + r);
-                    atomicAdd(a.sum + (size_t)u * kQRows + r, (double)L[k] * exp2((double)M[k] - ref));
-                }
+                if (M[k] != -INFINITY)
+                    atomicAdd(a.sum + ((size_t)u * kSumCopies + cta % kSumCopies) * kQRows + r,
+                              scale_exp2(L[k], M[k] - __ldg(a.ref + (size_t)u * kQRows + r)));
                 M[k] = -INFINITY;
                 L[k] = 0.f;
             }
@@ -704,9 +730,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             const int u = jb.y, ti = jb.z;
             const bool full_tile = (ti + 1) * kTileKeys <= a.N - a.w + 1;
             if (jb.x == 0) {
-                // phase 1: this row's (max, sum of 2^(y - max)) over the tile's visible keys
+                // phase 1: this row's (m, sum of 2^(y - m)) over the tile's visible keys.  m is
+                // the row's reference logit (its own-position key), so no running max is
+                // needed; a chunk whose sum is not below 2^100 (a logit ~100 above the
+                // reference) is redone with its exact max.
                 const int t_r = a.N - a.w + (r % a.w);  // last key this row sees
-                float m = -INFINITY, l = 0.f;
+                float m = __ldg(a.ref + (size_t)u * kQRows + r), l = 0.f;
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     uint32_t x[32];
@@ -725,7 +754,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                         for (int e = 0; e < 32; ++e)
                             if (j0 + e > t_r) x[e] = __float_as_uint(-INFINITY);
                     }
-                    stats_update(x, m, l);
+                    const float cs = sum_exp2_shifted(x, m);
+                    if (cs < 0x1p100f) {
+                        l += cs;
+                    } else {
+                        const float mn = fmaxf(m, chunk_max(x) * kLog2eOverSqrtD);
+                        l = l * ex2(m - mn) + sum_exp2_shifted(x, mn);
+                        m = mn;
+                    }
                 }
                 // record slot i % kRec is free once the publisher has read record i - kRec
                 const int i = jb.w, s = i % kRec;
@@ -736,7 +772,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                 if (lane == 0) mbar_arrive(&sm.recfull[s]);
             } else {
                 // phase 2: this key's sum over the query rows of 2^(y - lse)
-                const float* lse = sm.lse[jb.w];
+                const float* nlse = sm.nlse[jb.w];
                 const int j = ti * kTileKeys + r;
                 float sc = 0.f;
 #pragma unroll 1
@@ -756,7 +792,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                         for (int e = 0; e < 32; ++e)
                             if (j > a.N - a.w + (c * 32 + e) % a.w) x[e] = __float_as_uint(-INFINITY);
                     }
-                    sc += prob_sum(x, lse + c * 32);
+                    sc += prob_sum(x, nlse + c * 32);
                 }
                 if (j < a.N) a.unit_scores[(size_t)u * a.N + j] = sc;
                 __syncwarp();
@@ -802,15 +838,13 @@ __global__ void tc_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_b
             for (int d = 0; d < kHeadDim; ++d) x = fmaf(__bfloat162float(qr[d]), __bfloat162float(kr[d]), x);
         }
         ref[e] = x * kLog2eOverSqrtD;
-        sum[e] = 0.0;
     }
+    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < (long long)U * kSumCopies * kQRows;
+         e += (long long)gridDim.x * blockDim.x)
+        sum[e] = 0.0;
     for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n_flags;
          e += (long long)gridDim.x * blockDim.x)
         flags[e] = 0u;
-}
-
-__global__ void exp2_poly_kernel(const float* __restrict__ y, float* __restrict__ out, int n) {
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) out[i] = exp2_poly(y[i]);
 }
 
 // ------------------------------------------------------------------------ host side
@@ -829,7 +863,7 @@ TcLayout tc_layout(int U) {
     L.ref = off;
     off = a256(off + (size_t)U * kQRows * sizeof(float));
     L.sum = off;
-    off = a256(off + (size_t)U * kQRows * sizeof(double));
+    off = a256(off + (size_t)U * kSumCopies * kQRows * sizeof(double));
     L.flags = off;  // count[U], never
     L.n_flags = (size_t)U + 1;
     off = a256(off + L.n_flags * sizeof(unsigned));
@@ -862,13 +896,6 @@ int sm_count() {
 }
 
 }  // namespace
-
-cudaError_t debug_exp2(const float* y, float* out, int n, cudaStream_t s) {
-    if (n <= 0) return cudaSuccess;
-    exp2_poly_kernel<<<std::min((n + 255) / 256, 148 * 4), 256, 0, s>>>(y, out, n);
-    count_launches(1);
-    return cudaGetLastError();
-}
 
 bool tc_score_supported(const ScoreJob& j) {
     return j.dtype == KVC_BF16 && j.nq >= 1 && j.nq <= kQRows && j.N >= 1 && j.U >= 1 &&

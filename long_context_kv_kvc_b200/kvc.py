@@ -24,7 +24,7 @@ KVC_STAGE_SCORE, KVC_STAGE_SELECT, KVC_STAGE_GATHER, KVC_STAGE_COUNT = 0, 1, 2, 
 
 EXPORTED = ("kvc_workspace_size", "kvc_score", "kvc_accumulate", "kvc_pool", "kvc_topk_workspace_size",
             "kvc_topk", "kvc_gather", "kvc_compress", "kvc_tsp_count", "kvc_poll_error",
-            "kvc_status_string", "kvc_version", "kvc_launch_count", "kvc_score_noalloc", "kvc_debug_exp2")
+            "kvc_status_string", "kvc_version", "kvc_launch_count", "kvc_score_noalloc")
 
 
 class KvcError(RuntimeError):
@@ -64,7 +64,6 @@ def _load():
         "kvc_version": (ctypes.c_char_p, []),
         "kvc_launch_count": (ctypes.c_uint64, []),
         "kvc_score_noalloc": (st, [P, vp, vp, vp, vp]),
-        "kvc_debug_exp2": (st, [vp, vp, i32, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -198,10 +197,6 @@ def kvc_poll_error(stream=None) -> int:
 
 def kvc_status_string(st: int) -> str:
     return lib.kvc_status_string(st).decode()
-
-
-def kvc_debug_exp2(y, out, stream=None):
-    _check(lib.kvc_debug_exp2(_ptr(y), _ptr(out), y.numel(), _stream(stream)), "kvc_debug_exp2")
 
 
 def kvc_launch_count() -> int:
