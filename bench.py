@@ -79,6 +79,9 @@ def tsp_count(wl) -> int:
     return sel + wl.n_sink + wl.window if sel >= 1 else 0
 
 
+L2_BYTES = 126 * 2**20  # B200 L2
+
+
 def measured_peaks() -> tuple:
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -224,7 +227,14 @@ def config_of(wl, world) -> dict:
             "Hkv": wl.Hkv, "N": wl.N, "D": wl.D, "window": wl.window, "n_layers": wl.n_layers,
             "kv_budget": wl.kv_budget, "pool_kernel": wl.pool_kernel, "n_sink": wl.n_sink,
             "tsp_rate": wl.tsp_rate, "parallelism": f"batch-sharded replicas x{world} (no collective)",
-            "l2": "inputs larger than L2 (1 GiB of K per GPU), no flush"}
+            "l2": l2_note(wl)}
+
+
+def l2_note(wl) -> str:
+    k_bytes = wl.n_layers * wl.B * wl.Hkv * wl.N * wl.D * (2 if wl.dtype == "bf16" else 4)
+    if k_bytes > L2_BYTES:
+        return f"inputs larger than L2 ({k_bytes / 2**30:.2f} GiB of K per GPU), no flush"
+    return f"K ({k_bytes / 2**20:.0f} MiB per GPU) fits in L2: timed steps re-read it from L2"
 
 
 # ----------------------------------------------------------------------------- GPU leg

@@ -827,17 +827,30 @@ __global__ void tc_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_b
         if (r < nq) v = *reinterpret_cast<const uint4*>(q + ((u * nq + r) * kHeadDim + piece * 8));
         *reinterpret_cast<uint4*>(qpad + (row * kHeadDim + piece * 8)) = v;
     }
-    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < (long long)U * kQRows;
-         e += (long long)gridDim.x * blockDim.x) {
+    // one warp per (unit, row): lane l takes dimensions 4l .. 4l + 3 (8-byte loads), then a
+    // butterfly sum
+    const int lane = threadIdx.x & 31;
+    const long long n_warps = (long long)gridDim.x * blockDim.x / 32;
+    for (long long e = (blockIdx.x * (long long)blockDim.x + threadIdx.x) / 32; e < (long long)U * kQRows;
+         e += n_warps) {
         const int r = (int)(e % kQRows);
         const long long u = e / kQRows;
         float x = 0.f;
         if (r < nq) {
-            const __nv_bfloat16* qr = q + (u * nq + r) * kHeadDim;
-            const __nv_bfloat16* kr = k + (u * N + (N - w + r % w)) * kHeadDim;
-            for (int d = 0; d < kHeadDim; ++d) x = fmaf(__bfloat162float(qr[d]), __bfloat162float(kr[d]), x);
+            const uint2 qv = *reinterpret_cast<const uint2*>(q + (u * nq + r) * kHeadDim + 4 * lane);
+            const uint2 kv = *reinterpret_cast<const uint2*>(k + (u * N + (N - w + r % w)) * kHeadDim + 4 * lane);
+            const __nv_bfloat162* qh = reinterpret_cast<const __nv_bfloat162*>(&qv);
+            const __nv_bfloat162* kh = reinterpret_cast<const __nv_bfloat162*>(&kv);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float2 qf = __bfloat1622float2(qh[h]), kf = __bfloat1622float2(kh[h]);
+                x = fmaf(qf.x, kf.x, x);
+                x = fmaf(qf.y, kf.y, x);
+            }
         }
-        ref[e] = x * kLog2eOverSqrtD;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+        if (lane == 0) ref[e] = x * kLog2eOverSqrtD;
     }
     for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < (long long)U * kSumCopies * kQRows;
          e += (long long)gridDim.x * blockDim.x)
