@@ -29,6 +29,13 @@
  *           "Inferentie Pipeline", Preservation; FastKV page, sec. 2A: the selected
  *           tokens plus a window of the newest tokens are propagated).
  *   gather  Row r of the compact cache is the source row idx[r], byte for byte.
+ *   pivot metrics
+ *           StructKV watches attention entropy, sparsity and variance during the first
+ *           pass to find the layer where attention settles (StructKV page, sec. 2
+ *           "Dynamische Pivot Detectie"); the page gives no formulas.  Read here as: the
+ *           Shannon entropy (nats) of each window query's attention row; the share of a
+ *           score row's mass that the kept positions hold; the population variance of a
+ *           score row over the candidates C.
  *
  * Everything is done in double precision with plain loops; inputs arrive as raw fp32 or
  * bf16 bytes and are widened exactly.  Parallelism, where present, is only over
@@ -309,4 +316,130 @@ int oracle_tsp_count(int N, int w, int S, double rate)
     if (sel > n_c) sel = n_c;
     if (sel < 1) return 0; /* nothing to select: not a valid TSP configuration */
     return (int)(sel + S + w);
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* pivot metrics                                                                         */
+/* ------------------------------------------------------------------------------------ */
+
+typedef struct {
+    int B, Hq, Hkv, N, D, w, dtype;
+    const void *q, *k;
+    const int32_t *rows;
+    int n_rows, next;
+    double *out;
+    pthread_mutex_t lock;
+} entropy_job;
+
+/* H = -sum_j p_j ln p_j over the keys j <= t that flat query row r sees. */
+static double row_entropy(const entropy_job *J, int r, double *x)
+{
+    const int N = J->N, D = J->D, w = J->w, G = J->Hq / J->Hkv;
+    const int i = r % w;
+    const int g = (r / w) % J->Hq;
+    const int lb = r / (w * J->Hq); /* layer * B + b */
+    const int h = g / G;
+    const double scale = 1.0 / sqrt((double)J->D);
+    const size_t q_base = (size_t)r * D;
+    const size_t k_base = ((size_t)lb * J->Hkv + h) * (size_t)N * D;
+    const int last = N - w + i; /* the row's position: keys 0..last are visible */
+    double m = -INFINITY;
+    for (int j = 0; j <= last; ++j) {
+        double acc = 0.0;
+        for (int d = 0; d < D; ++d)
+            acc += widen(J->q, J->dtype, q_base + d) * widen(J->k, J->dtype, k_base + (size_t)j * D + d);
+        x[j] = acc * scale;
+        if (x[j] > m) m = x[j];
+    }
+    double l = 0.0;
+    for (int j = 0; j <= last; ++j) l += exp(x[j] - m);
+    double H = 0.0;
+    for (int j = 0; j <= last; ++j) {
+        const double p = exp(x[j] - m) / l;
+        if (p > 0.0) H -= p * log(p);
+    }
+    return H;
+}
+
+static void *entropy_worker(void *arg)
+{
+    entropy_job *J = (entropy_job *)arg;
+    double *x = (double *)malloc(sizeof(double) * (size_t)J->N);
+    if (!x) return (void *)1;
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        int n = J->next++;
+        pthread_mutex_unlock(&J->lock);
+        if (n >= J->n_rows) break;
+        J->out[n] = row_entropy(J, J->rows[n], x);
+    }
+    free(x);
+    return NULL;
+}
+
+/*
+ * oracle_entropy -- attention entropy (nats) of window query rows.
+ *   q [L, B, Hq, w, D], k [L, B, Hkv, N, D] (dtype as in oracle_score); rows[n] is a flat
+ *   query-row index ((layer * B + b) * Hq + g) * w + i; out[n] = -sum_j p_j ln p_j of that
+ *   row's causal window softmax.
+ */
+int oracle_entropy(int B, int Hq, int Hkv, int N, int D, int w, int L, const void *q, const void *k,
+                   int dtype, const int32_t *rows, int n_rows, double *out, int n_threads)
+{
+    if (B < 1 || Hkv < 1 || Hq < Hkv || Hq % Hkv || N < 1 || D < 1 || w < 1 || w > N || L < 1 || n_rows < 0)
+        return -1;
+    for (int n = 0; n < n_rows; ++n)
+        if (rows[n] < 0 || rows[n] >= L * B * Hq * w) return -1;
+    entropy_job J;
+    J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.N = N; J.D = D; J.w = w; J.dtype = dtype;
+    J.q = q; J.k = k; J.rows = rows; J.n_rows = n_rows; J.next = 0; J.out = out;
+    pthread_mutex_init(&J.lock, NULL);
+    if (n_threads < 1) n_threads = 1;
+    if (n_threads > n_rows) n_threads = n_rows > 0 ? n_rows : 1;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)n_threads);
+    int rc = 0;
+    for (int t = 1; t < n_threads; ++t) pthread_create(&th[t], NULL, entropy_worker, &J);
+    if (entropy_worker(&J)) rc = -1;
+    for (int t = 1; t < n_threads; ++t) {
+        void *r;
+        pthread_join(th[t], &r);
+        if (r) rc = -1;
+    }
+    free(th);
+    pthread_mutex_destroy(&J.lock);
+    return rc;
+}
+
+/*
+ * oracle_row_stats -- per score row s (rows of length N):
+ *   kept_mass[row] = sum of s over the row's `budget` positions in idx / sum_{j < N} s
+ *                    (skipped when idx is NULL)
+ *   cand_var[row]  = (1/n) sum_{j in C} (s_j - mean_C)^2 over the n = N - w - S candidates
+ *                    C = [S, N - w), mean_C their mean (two passes)
+ */
+int oracle_row_stats(const double *scores, int rows, int N, int S, int w, const int32_t *idx, int budget,
+                     double *kept_mass, double *cand_var)
+{
+    if (rows < 1 || N < 1 || S < 0 || w < 0 || S + w >= N || (idx && (budget < 1 || budget > N))) return -1;
+    const int n_c = N - w - S;
+    for (int row = 0; row < rows; ++row) {
+        const double *s = scores + (size_t)row * N;
+        if (idx) {
+            double total = 0.0, kept = 0.0;
+            for (int j = 0; j < N; ++j) total += s[j];
+            for (int t = 0; t < budget; ++t) {
+                const int j = idx[(size_t)row * budget + t];
+                if (j < 0 || j >= N) return -1;
+                kept += s[j];
+            }
+            kept_mass[row] = kept / total;
+        }
+        double mean = 0.0;
+        for (int j = S; j < N - w; ++j) mean += s[j];
+        mean /= n_c;
+        double var = 0.0;
+        for (int j = S; j < N - w; ++j) var += (s[j] - mean) * (s[j] - mean);
+        cand_var[row] = var / n_c;
+    }
+    return 0;
 }

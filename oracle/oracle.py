@@ -6,7 +6,8 @@ CUDA library package.
 
 All arithmetic lives in kvc_oracle.c (fp64, plain loops).  This file only marshals
 arguments and composes the steps in the order the method takes them:
-score -> aggregate -> pool -> select -> gather (+ the TSP branch).
+score -> aggregate -> pool -> select -> gather (+ the TSP branch), plus the pivot metrics
+(attention entropy of the window rows, kept mass and candidate variance of score rows).
 """
 from __future__ import annotations
 
@@ -44,8 +45,10 @@ def _load(so_path: str):
     L.oracle_select.argtypes = [p, i, i, i, i, i, i, p]
     L.oracle_gather.argtypes = [p, i, i, i, sz, p, i, i, p]
     L.oracle_tsp_count.argtypes = [i, i, i, d]
+    L.oracle_entropy.argtypes = [i, i, i, i, i, i, i, p, p, i, p, i, p, i]
+    L.oracle_row_stats.argtypes = [p, i, i, i, i, p, i, p, p]
     for f in ("oracle_score", "oracle_accumulate", "oracle_pool", "oracle_select",
-              "oracle_gather", "oracle_tsp_count"):
+              "oracle_gather", "oracle_tsp_count", "oracle_entropy", "oracle_row_stats"):
         getattr(L, f).restype = ctypes.c_int
     return L
 
@@ -168,6 +171,47 @@ def gather(src: torch.Tensor, idx: np.ndarray) -> torch.Tensor:
 
 def tsp_count(N: int, window: int, n_sink: int, rate: float) -> int:
     return int(lib().oracle_tsp_count(N, window, n_sink, float(rate)))
+
+
+def entropy(q, k, *, window: int, rows=None, threads: int = 0) -> np.ndarray:
+    """Attention entropy (nats) of window query rows, fp64.
+
+    q [L, B, Hq, w, D] (or [B, Hq, w, D]), k [L, B, Hkv, N, D] (or [B, Hkv, N, D]).  Returns
+    [L, B, Hq, w], or, with `rows` (flat indices into that shape), the listed rows only.
+    """
+    if q.dim() == 4:
+        q, k = q.unsqueeze(0), k.unsqueeze(0)
+    L, B, Hq, w, D = q.shape
+    _, _, Hkv, N, _ = k.shape
+    assert w == window and k.shape[0] == L and k.shape[1] == B and k.shape[4] == D
+    qb, qd = _as_buffer(q)
+    kb, kd = _as_buffer(k)
+    assert qd == kd
+    all_rows = rows is None
+    r = np.arange(L * B * Hq * w, dtype=np.int32) if all_rows else np.ascontiguousarray(rows, dtype=np.int32)
+    out = np.zeros(r.size, dtype=np.float64)
+    threads = threads or (os.cpu_count() or 1)
+    rc = lib().oracle_entropy(B, Hq, Hkv, N, D, w, L, qb.ctypes.data, kb.ctypes.data, qd, r.ctypes.data, r.size,
+                              out.ctypes.data, threads)
+    _check(rc, "entropy")
+    return out.reshape(L, B, Hq, w) if all_rows else out
+
+
+def row_stats(scores: np.ndarray, n_sink: int, window: int, idx: np.ndarray = None):
+    """(kept_mass, cand_var) per score row of scores [B, H, N] (kept_mass None without idx)."""
+    s = np.ascontiguousarray(scores, dtype=np.float64)
+    B, H, N = s.shape
+    km = np.zeros((B, H), dtype=np.float64)
+    cv = np.zeros((B, H), dtype=np.float64)
+    ip, budget = None, 0
+    if idx is not None:
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+        budget = idx.shape[-1]
+        ip = idx.ctypes.data
+    rc = lib().oracle_row_stats(s.ctypes.data, B * H, N, n_sink, window, ip, budget, km.ctypes.data,
+                                cv.ctypes.data)
+    _check(rc, "row_stats")
+    return (km if idx is not None else None), cv
 
 
 def compress(q, k, v, *, window: int, n_sink: int, pool_kernel: int, kv_budget: int,

@@ -36,6 +36,13 @@ MUTANTS = [
      "for (int j = N - w; j < N - 1; ++j) kept[n++] = j;\n        kept[n++] = c[k_sel].j;"),
     ("layers not summed", "for (int layer = 0; layer < L; ++layer)\n        for (int b = 0; b < B; ++b)",
      "for (int layer = L - 1; layer < L; ++layer)\n        for (int b = 0; b < B; ++b)"),
+    ("entropy logit scale 1/D", "1.0 / sqrt((double)J->D)", "1.0 / (double)J->D"),
+    ("entropy in bits", "if (p > 0.0) H -= p * log(p);", "if (p > 0.0) H -= p * log2(p);"),
+    ("entropy row's keys one short", "for (int j = 0; j <= last; ++j) {\n        double acc",
+     "for (int j = 0; j < last; ++j) {\n        double acc"),
+    ("sample variance", "cand_var[row] = var / n_c;", "cand_var[row] = var / (n_c - 1);"),
+    ("kept mass over the candidates only", "for (int j = 0; j < N; ++j) total += s[j];",
+     "for (int j = S; j < N - w; ++j) total += s[j];"),
 ]
 
 PIN_TESTS = [
@@ -53,6 +60,10 @@ PIN_TESTS = [
     pins.test_select_brute_force_with_ties,
     pins.test_select_matches_library_sort_and_invariants,
     pins.test_select_all_equal_takes_lowest_indices,
+    lambda: [pins.test_entropy_equal_logits_is_log_of_visible_count(*a) for a in [(17, 3, 2), (40, 8, 4)]],
+    pins.test_entropy_two_keys_is_binary_entropy,
+    pins.test_entropy_dominant_key_is_zero_and_matches_library,
+    pins.test_row_stats_against_definitions,
 ]
 
 

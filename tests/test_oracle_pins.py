@@ -306,3 +306,79 @@ def test_compress_composition_invariants():
         assert torch.equal(out["hidden_out"][b], hidden[b, torch.from_numpy(out["tsp_idx"][b, 0]).long()])
         for h in range(2):
             assert torch.equal(out["k_out"][b, h], k[0, b, h, torch.from_numpy(out["idx"][b, h]).long()])
+
+
+# ------------------------------------------------------------------- pivot metrics
+
+@pytest.mark.parametrize("N,w,G", [(17, 3, 2), (40, 8, 4)])
+def test_entropy_equal_logits_is_log_of_visible_count(N, w, G):
+    # K == 0: every row's softmax is uniform over its t_i + 1 visible keys, so its entropy
+    # is ln(t_i + 1) in nats (pins the mask, the normalisation and the natural log).
+    q, k = _zeros_case(2, 2 * G, 2, N, 16, w, L=2)
+    H = O.entropy(q, k, window=w)
+    for i in range(w):
+        np.testing.assert_allclose(H[..., i], math.log(N - w + i + 1), rtol=0, atol=1e-13)
+
+
+def test_entropy_two_keys_is_binary_entropy():
+    # One query seeing two keys with logits x0, x1: the binary entropy of expit(x0 - x1)
+    # (pins the 1/sqrt(D) scale inside the entropy).
+    D = 16
+    for a, b0, b1 in [(2.0, 3.0, -1.0), (0.5, -4.0, 6.0), (8.0, 1.0, 1.25)]:
+        q = torch.zeros(1, 1, 1, 1, D, dtype=torch.float64)
+        k = torch.zeros(1, 1, 1, 2, D, dtype=torch.float64)
+        q[..., 0] = a
+        k[0, 0, 0, 0, 0] = b0
+        k[0, 0, 0, 1, 0] = b1
+        p = scipy.special.expit((a * b0 - a * b1) / math.sqrt(D))
+        want = -(p * math.log(p) + (1 - p) * math.log(1 - p))
+        assert O.entropy(q, k, window=1)[0, 0, 0, 0] == pytest.approx(want, abs=1e-14)
+
+
+def test_entropy_dominant_key_is_zero_and_matches_library():
+    # A key with a logit gap of ~1000 takes all the mass: entropy 0 (also pins the max
+    # shift, exp(1000) overflows); random rows against torch's float64 softmax entropy.
+    q = torch.zeros(1, 1, 2, 2, 8, dtype=torch.float64)
+    k = torch.randn(1, 1, 1, 12, 8, dtype=torch.float64, generator=torch.Generator().manual_seed(5)) * 0.01
+    q[..., 0] = 200.0
+    k[0, 0, 0, 3, 0] = 40.0
+    assert np.all(np.abs(O.entropy(q, k, window=2)) < 1e-12)
+    g = torch.Generator().manual_seed(6)
+    L, B, Hq, Hkv, N, D, w = 2, 2, 4, 2, 37, 16, 5
+    q = torch.randn(L, B, Hq, w, D, dtype=torch.float64, generator=g)
+    k = torch.randn(L, B, Hkv, N, D, dtype=torch.float64, generator=g)
+    H = O.entropy(q, k, window=w)
+    G = Hq // Hkv
+    for layer in range(L):
+        for b in range(B):
+            for hq in range(Hq):
+                x = q[layer, b, hq] @ k[layer, b, hq // G].T / math.sqrt(D)
+                for i in range(w):
+                    lp = torch.log_softmax(x[i, : N - w + i + 1], dim=0)
+                    want = float(-(lp.exp() * lp).sum())
+                    assert H[layer, b, hq, i] == pytest.approx(want, abs=1e-12)
+    rows = np.array([0, 7, 31, L * B * Hq * w - 1], dtype=np.int32)
+    np.testing.assert_array_equal(O.entropy(q, k, window=w, rows=rows), H.reshape(-1)[rows])
+
+
+def test_row_stats_against_definitions():
+    # kept mass against a brute-force sum; candidate variance against numpy's population
+    # variance over [S, N - w); a constant row has variance 0; a full budget keeps mass 1.
+    g = np.random.default_rng(8)
+    B, H, N, S, w = 2, 3, 50, 2, 5
+    s = g.random((B, H, N))
+    idx = np.stack([np.sort(g.choice(N, 20, replace=False)) for _ in range(B * H)]).reshape(B, H, 20)
+    km, cv = O.row_stats(s, S, w, idx)
+    for b in range(B):
+        for h in range(H):
+            assert km[b, h] == pytest.approx(s[b, h, idx[b, h]].sum() / s[b, h].sum(), rel=1e-14)
+            assert cv[b, h] == pytest.approx(np.var(s[b, h, S:N - w]), rel=1e-12)
+    km_full, _ = O.row_stats(s, S, w, np.tile(np.arange(N, dtype=np.int32), (B, H, 1)))
+    np.testing.assert_allclose(km_full, 1.0, rtol=1e-15)
+    _, cv_const = O.row_stats(np.full((1, 1, N), 0.37), S, w)
+    assert cv_const[0, 0] < 1e-30
+    # variance over C only: values outside C do not move it
+    s2 = s.copy()
+    s2[..., :S] = 1e6
+    s2[..., N - w:] = -1e6
+    np.testing.assert_allclose(O.row_stats(s2, S, w)[1], cv, rtol=1e-13)
