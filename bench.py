@@ -247,6 +247,8 @@ def main():
     ap.add_argument("--impl", default="kvc", choices=["kvc", "reference"])
     ap.add_argument("--workload", default=synth.LLAMA8B_128K_B4.name, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--pivot-steps", type=int, default=5,
+                    help="calls timed for the pivot metrics (entropy pass, row statistics); 0 skips")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--flags", type=int, default=0, help="kvc_params.flags (1 = CUDA-core scoring)")
     ap.add_argument("--no-clocks", action="store_true",
@@ -368,6 +370,35 @@ def main():
         e2e = {"value": tokens / (float(te.item()) / args.e2e_steps / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
+    # the pivot-detection metrics (StructKV sec. 2): cost of the entropy in the scoring pass
+    # and of the per-row kept mass / candidate variance, outside the timed region
+    pivot = None
+    if args.pivot_steps > 0:
+        Hs = wl.Hkv if wl.scope == kvc.KVC_SCOPE_PER_KV_HEAD else 1
+        sc = torch.empty((wl.B, Hs, wl.N), dtype=torch.float32, device="cuda")
+        ent = torch.empty((wl.n_layers, wl.B, wl.Hq, wl.window), dtype=torch.float32, device="cuda")
+        km = torch.empty((wl.B, Hs), dtype=torch.float32, device="cuda")
+        cv = torch.empty((wl.B, Hs), dtype=torch.float32, device="cuda")
+
+        def timed(fn):
+            fn()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(args.pivot_steps):
+                fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            return a.elapsed_time(b) / args.pivot_steps
+
+        t_plain = timed(lambda: kvc.kvc_score(p, dev["q"], dev["k"], sc, comp.ws))
+        t_ent = timed(lambda: kvc.kvc_score_entropy(p, dev["q"], dev["k"], sc, ent, comp.ws))
+        t_rs = timed(lambda: kvc.kvc_row_stats(sc, wl.n_sink, wl.window, cv, idx=comp.out["idx_out"], kept_mass=km))
+        if kvc.kvc_poll_error() != kvc.KVC_OK:
+            raise RuntimeError("device-side error in the pivot-metric calls")
+        pivot = {"score_ms": t_plain, "score_with_entropy_ms": t_ent, "row_stats_ms": t_rs,
+                 "calls": args.pivot_steps}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         threads = min(wl.Hkv, os.cpu_count() or 1)
@@ -388,6 +419,7 @@ def main():
                          "peak_source": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": traffic, "algorithmic_bytes_per_launch": ab["score"]},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
+            "pivot_metrics": pivot,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -219,6 +219,40 @@ KVC_API kvc_status kvc_compress(const kvc_params *p, const void *q, const void *
                         kvc_stream_t stream);
 
 /*
+ * kvc_score_entropy -- kvc_score plus the attention entropy of every window query row,
+ * taken in the same pass.  StructKV watches attention entropy (with sparsity and variance,
+ * see kvc_row_stats) during the first pass to find the layer where attention settles
+ * (StructKV page, sec. 2 "Dynamische Pivot Detectie"); the page gives no formula, so the
+ * entropy here is Shannon's, in nats, of each window query's causal softmax row:
+ * H = -sum_j p_j ln p_j over the keys j <= N - window + i that query i sees.
+ *   q, k, scores, ws  as in kvc_score (same results in `scores`).
+ *   entropy  device, [n_layers, B, Hq, window] fp32 (4-byte aligned), written; row order as
+ *            in q.
+ * Cost: one extra multiply-add per logit and one more fp64 total per query row.
+ */
+KVC_API kvc_status kvc_score_entropy(const kvc_params *p, const void *q, const void *k, float *scores,
+                                     float *entropy, void *workspace, size_t workspace_bytes,
+                                     kvc_stream_t stream);
+
+/*
+ * kvc_row_stats -- the other two pivot-detection signals (StructKV page, sec. 2), per score
+ * row: the share of the row's mass held by its kept positions (sparsity) and the population
+ * variance of the row over the candidates C = [n_sink, N - window).
+ *   scores     device, [rows, N] fp32 (e.g. kvc_score's [B, Hs, N] with rows = B * Hs).
+ *   idx        device, [rows, budget] int32 kept positions (kvc_topk's output), or NULL to
+ *              skip the kept mass.  An index outside [0, N) is left out of the sum and sets
+ *              KVC_ERR_INDEX for kvc_poll_error.
+ *   kept_mass  device, [rows] fp32: sum of s over idx / sum of s over [0, N) (unused when
+ *              idx is NULL).
+ *   cand_var   device, [rows] fp32: (1/n) sum over C of (s - mean_C)^2, n = |C|.
+ * Requires n_sink + window < N and, with idx, 1 <= budget <= N.  fp64 sums in a fixed
+ * order, so results are deterministic.
+ */
+KVC_API kvc_status kvc_row_stats(const float *scores, int32_t rows, int32_t N, int32_t n_sink, int32_t window,
+                                 const int32_t *idx, int32_t budget, float *kept_mass, float *cand_var,
+                                 kvc_stream_t stream);
+
+/*
  * kvc_score_noalloc -- kvc_score for callers that cannot allocate device memory.  The
  * pages have no counterpart: it exists for engines that have already given all device
  * memory to their own pool, or plugin interfaces that forbid cudaMalloc/cudaFree during a

@@ -46,7 +46,7 @@ struct Plan {
     bool units = false;  // unit scores need a reduction (several layers or all heads)
     bool use_tc = false;
     int n_chunks = 0, chunk = 0;
-    size_t off_partial = 0, off_lse = 0, off_units = 0, off_scores = 0, off_pooled = 0;
+    size_t off_partial = 0, off_partial_t = 0, off_lse = 0, off_units = 0, off_scores = 0, off_pooled = 0;
     size_t off_tsp_scores = 0, off_tsp_pooled = 0, off_tc = 0, tc_bytes = 0, total = 0;
 };
 
@@ -107,6 +107,8 @@ void make_plan(const kvc_params* p, bool compress, Plan* pl) {
         const size_t pb = simt_score_workspace(P.U, p->N, P.nq, &P.n_chunks, &P.chunk);
         P.off_partial = off;
         off = align_up(off + pb);
+        P.off_partial_t = off;  // the entropy's third statistic, half the size of (m, l)
+        off = align_up(off + pb / 2);
     }
     P.off_lse = off;
     off = align_up(off + (size_t)P.U * P.nq * sizeof(float));
@@ -133,8 +135,9 @@ void make_plan(const kvc_params* p, bool compress, Plan* pl) {
 
 // Runs the scoring stage: unit scores (and their reduction) into `scores` [B, Hs, N].
 kvc_status run_score(const kvc_params* p, const Plan& P, const void* q, const void* k, float* scores,
-                     char* ws, cudaStream_t s) {
+                     char* ws, cudaStream_t s, float* entropy = nullptr) {
     ScoreJob job = make_job(p, q, k);
+    job.entropy = entropy;
     job.unit_scores = P.units ? (float*)(ws + P.off_units) : scores;
     job.lse = (float*)(ws + P.off_lse);
     job.err = device_error_word();
@@ -146,6 +149,7 @@ kvc_status run_score(const kvc_params* p, const Plan& P, const void* q, const vo
         e = tc_score(job, s);
     } else {
         job.partial = (float2*)(ws + P.off_partial);
+        job.partial_t = (float*)(ws + P.off_partial_t);
         job.n_chunks = P.n_chunks;
         job.chunk = P.chunk;
         e = simt_score(job, s);
@@ -197,6 +201,32 @@ kvc_status kvc_score(const kvc_params* p, const void* q, const void* k, float* s
     make_plan(p, false, &P);
     if (ws_bytes < P.total) return KVC_ERR_WORKSPACE;
     return run_score(p, P, q, k, scores, (char*)ws, (cudaStream_t)stream);
+}
+
+kvc_status kvc_score_entropy(const kvc_params* p, const void* q, const void* k, float* scores, float* entropy,
+                             void* ws, size_t ws_bytes, kvc_stream_t stream) {
+    KVC_TRY(check_params(p));
+    if (!q || !k || !scores || !entropy || !ws) return KVC_ERR_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(scores) || ((uintptr_t)entropy & 3u) ||
+        ((uintptr_t)ws & (kAlign - 1)))
+        return KVC_ERR_ALIGN;
+    Plan P;
+    make_plan(p, false, &P);
+    if (ws_bytes < P.total) return KVC_ERR_WORKSPACE;
+    return run_score(p, P, q, k, scores, (char*)ws, (cudaStream_t)stream, entropy);
+}
+
+kvc_status kvc_row_stats(const float* scores, int32_t rows, int32_t N, int32_t n_sink, int32_t window,
+                         const int32_t* idx, int32_t budget, float* kept_mass, float* cand_var,
+                         kvc_stream_t stream) {
+    if (!scores || !cand_var || rows < 1 || N < 1 || n_sink < 0 || window < 0) return KVC_ERR_ARG;
+    if ((long long)n_sink + window >= N) return KVC_ERR_ARG;
+    if (idx && (!kept_mass || budget < 1 || budget > N)) return KVC_ERR_ARG;
+    unsigned* err = device_error_word();
+    if (!err) return KVC_ERR_CUDA;
+    KVC_CUDA(kvc::row_stats(scores, rows, N, n_sink, window, idx, idx ? budget : 0, kept_mass, cand_var, err,
+                            (cudaStream_t)stream));
+    return KVC_OK;
 }
 
 kvc_status kvc_accumulate(float* acc, const float* src, int32_t B, int32_t Hi, int32_t Ho, int32_t N,

@@ -37,8 +37,10 @@ struct ScoreJob {
     int G;
     int nq;       // G * window query rows per unit
     float* unit_scores;  // [U][N] fp32 output (sum over the unit's query rows)
+    float* entropy;      // [U][nq] attention entropy per window row (nats), or null
     // workspace
     float2* partial;     // SIMT: [U][n_chunks][nq] (m, l) partial softmax stats
+    float* partial_t;    // SIMT with entropy: [U][n_chunks][nq] sum 2^(y - m) (y - m)
     float* lse;          // [U][nq] log2-sum-exp per query row
     int n_chunks;
     int chunk;
@@ -78,5 +80,10 @@ cudaError_t topk_fused(const float* scores, int rows, int N, int n_sink, int win
 cudaError_t gather(const void* src0, void* dst0, const void* src1, void* dst1, int B, int Hsrc,
                    int N, size_t row_bytes, const int32_t* idx, int Hidx, int K, unsigned* err,
                    cudaStream_t s);
+
+// per score row: share of mass at the kept positions (when idx is not null) and population
+// variance over the candidates [S, N - w)
+cudaError_t row_stats(const float* scores, int rows, int N, int S, int w, const int32_t* idx, int budget,
+                      float* kept_mass, float* cand_var, unsigned* err, cudaStream_t s);
 
 }  // namespace kvc

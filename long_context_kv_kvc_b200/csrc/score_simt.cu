@@ -9,6 +9,9 @@
 //   2. combine: per (unit, query row) lse = M + log2(sum_c l_c 2^(m_c - M)), fixed order;
 //   3. scores:  per key j, s_j = sum over query rows r of 2^(y_rj - lse_r), masked for keys
 //               after the row's position (causal window).
+// With an entropy output the statistics carry t = sum 2^(y - m) (y - m) as well, and the
+// combine step writes each row's attention entropy ln2 (log2 l - t / l) in nats (StructKV
+// page, sec. 2: attention entropy is one of the signals watched for the pivot layer).
 // The definition is the plain window softmax: the FastKV page (sec. 2A) selects tokens by
 // a saliency score, and the SnapKV scoring it names uses the softmaxed attention of the
 // observation window; all sums run in a fixed order so results are deterministic.
@@ -48,10 +51,25 @@ __device__ __forceinline__ void merge_stats(float& m, float& l, float m2, float 
     m = M;
 }
 
-template <typename T>
+// The same merge for (m, l, t) with t = sum 2^(y - m) (y - m): moving the reference from m
+// to M scales the sums by 2^(m - M) and shifts each y - m by m - M.  l is formed by the very
+// expression of merge_stats, so the entropy pass leaves the statistics (and the scores)
+// bit-identical.
+__device__ __forceinline__ void merge_stats3(float& m, float& l, float& t, float m2, float l2, float t2) {
+    const float M = fmaxf(m, m2);
+    if (M == -INFINITY) return;
+    float T = 0.f;
+    if (m != -INFINITY) T += exp2f(m - M) * (t + (m - M) * l);
+    if (m2 != -INFINITY) T += exp2f(m2 - M) * (t2 + (m2 - M) * l2);
+    l = (m == -INFINITY ? 0.f : l * exp2f(m - M)) + (m2 == -INFINITY ? 0.f : l2 * exp2f(m2 - M));
+    m = M;
+    t = T;
+}
+
+template <typename T, bool ENT>
 __global__ void __launch_bounds__(kThreads)
 stats_kernel(const T* __restrict__ q, const T* __restrict__ k, int N, int w, int nq, int chunk,
-             int n_chunks, float2* __restrict__ partial) {
+             int n_chunks, float2* __restrict__ partial, float* __restrict__ partial_t) {
     __shared__ float Qs[kQB][D + 1];
     __shared__ float Ks[kKT][D + 1];
     const int u = blockIdx.y, c = blockIdx.x;
@@ -65,7 +83,7 @@ stats_kernel(const T* __restrict__ q, const T* __restrict__ k, int N, int w, int
         stage_rows(Qs, qu + (size_t)qb * D, kQB, nq - qb);
         const int r = qb + qi;
         const int t_r = r < nq ? N - w + r % w : -1;  // position of window query r
-        float m = -INFINITY, l = 0.f;
+        float m = -INFINITY, l = 0.f, tt = 0.f;
         for (int jt = j0; jt < j1; jt += kKT) {
             __syncthreads();
             stage_rows(Ks, ku + (size_t)jt * D, kKT, j1 - jt);
@@ -85,10 +103,19 @@ stats_kernel(const T* __restrict__ q, const T* __restrict__ k, int N, int w, int
                 if (j < j1 && j <= t_r) {
                     const float y = acc[t] * kLog2eOverSqrtD;
                     if (y > m) {
-                        l = (m == -INFINITY ? 0.f : l * exp2f(m - y)) + 1.f;
+                        if (m == -INFINITY) {
+                            l = 1.f;
+                            tt = 0.f;
+                        } else {
+                            const float f = exp2f(m - y);
+                            if (ENT) tt = f * (tt + (m - y) * l);
+                            l = l * f + 1.f;
+                        }
                         m = y;
                     } else {
-                        l += exp2f(y - m);
+                        const float e = exp2f(y - m);
+                        l += e;
+                        if (ENT) tt = fmaf(e, y - m, tt);
                     }
                 }
             }
@@ -98,25 +125,41 @@ stats_kernel(const T* __restrict__ q, const T* __restrict__ k, int N, int w, int
         for (int off = 1; off < 8; off <<= 1) {
             const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
             const float l2 = __shfl_xor_sync(0xffffffffu, l, off);
-            merge_stats(m, l, m2, l2);
+            if (ENT) {
+                const float t2 = __shfl_xor_sync(0xffffffffu, tt, off);
+                merge_stats3(m, l, tt, m2, l2, t2);
+            } else {
+                merge_stats(m, l, m2, l2);
+            }
         }
-        if (kj == 0 && r < nq) partial[((size_t)u * n_chunks + c) * nq + r] = make_float2(m, l);
+        if (kj == 0 && r < nq) {
+            partial[((size_t)u * n_chunks + c) * nq + r] = make_float2(m, l);
+            if (ENT) partial_t[((size_t)u * n_chunks + c) * nq + r] = tt;
+        }
     }
 }
 
-__global__ void combine_kernel(const float2* __restrict__ partial, int n_chunks, int nq,
-                               float* __restrict__ lse) {
+// lse per row; with `entropy`, also each row's attention entropy in nats: with the chunks'
+// (m, l, t) moved to the common reference M, E[y] = M + T / L and lse = M + log2 L, so
+// -sum p ln p = ln2 (lse - E[y]) = ln2 (log2 L - T / L).
+__global__ void combine_kernel(const float2* __restrict__ partial, const float* __restrict__ partial_t,
+                               int n_chunks, int nq, float* __restrict__ lse, float* __restrict__ entropy) {
     const int u = blockIdx.x;
     for (int r = threadIdx.x; r < nq; r += blockDim.x) {
         const float2* p = partial + (size_t)u * n_chunks * nq + r;
         float M = -INFINITY;
         for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, p[(size_t)c * nq].x);
-        float S = 0.f;
+        float S = 0.f, T = 0.f;
         for (int c = 0; c < n_chunks; ++c) {
             const float2 v = p[(size_t)c * nq];
-            if (v.x != -INFINITY) S += v.y * exp2f(v.x - M);
+            if (v.x != -INFINITY) {
+                const float f = exp2f(v.x - M);
+                S += v.y * f;
+                if (entropy) T += f * (partial_t[((size_t)u * n_chunks + c) * nq + r] + (v.x - M) * v.y);
+            }
         }
         lse[(size_t)u * nq + r] = M + log2f(S);
+        if (entropy) entropy[(size_t)u * nq + r] = 0.69314718055994531f * (log2f(S) - T / S);
     }
 }
 
@@ -184,6 +227,8 @@ scores_kernel(const T* __restrict__ q, const T* __restrict__ k, int N, int w, in
 
 }  // namespace
 
+// partial (m, l) per (unit, chunk, row); the entropy's t per (unit, chunk, row) is a separate
+// array of half that size (ScoreJob::partial_t)
 size_t simt_score_workspace(int U, int N, int nq, int* n_chunks_out, int* chunk_out) {
     // enough CTAs to fill the GPU about twice, chunks of at most kChunkMax keys
     long long target = 148LL * 2;
@@ -200,17 +245,28 @@ size_t simt_score_workspace(int U, int N, int nq, int* n_chunks_out, int* chunk_
 cudaError_t simt_score(const ScoreJob& j, cudaStream_t s) {
     dim3 grid(j.n_chunks, j.U);
     count_launches(3);
+    float* partial_t = j.partial_t;
+    const bool ent = j.entropy != nullptr;
     if (j.dtype == KVC_F32) {
-        stats_kernel<float><<<grid, kThreads, 0, s>>>((const float*)j.q, (const float*)j.k, j.N,
-                                                       j.window, j.nq, j.chunk, j.n_chunks, j.partial);
+        if (ent)
+            stats_kernel<float, true><<<grid, kThreads, 0, s>>>((const float*)j.q, (const float*)j.k, j.N, j.window,
+                                                                 j.nq, j.chunk, j.n_chunks, j.partial, partial_t);
+        else
+            stats_kernel<float, false><<<grid, kThreads, 0, s>>>((const float*)j.q, (const float*)j.k, j.N, j.window,
+                                                                  j.nq, j.chunk, j.n_chunks, j.partial, partial_t);
     } else {
-        stats_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(
-            (const __nv_bfloat16*)j.q, (const __nv_bfloat16*)j.k, j.N, j.window, j.nq, j.chunk,
-            j.n_chunks, j.partial);
+        if (ent)
+            stats_kernel<__nv_bfloat16, true><<<grid, kThreads, 0, s>>>(
+                (const __nv_bfloat16*)j.q, (const __nv_bfloat16*)j.k, j.N, j.window, j.nq, j.chunk, j.n_chunks,
+                j.partial, partial_t);
+        else
+            stats_kernel<__nv_bfloat16, false><<<grid, kThreads, 0, s>>>(
+                (const __nv_bfloat16*)j.q, (const __nv_bfloat16*)j.k, j.N, j.window, j.nq, j.chunk, j.n_chunks,
+                j.partial, partial_t);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    combine_kernel<<<j.U, 128, 0, s>>>(j.partial, j.n_chunks, j.nq, j.lse);
+    combine_kernel<<<j.U, 128, 0, s>>>(j.partial, partial_t, j.n_chunks, j.nq, j.lse, j.entropy);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (j.dtype == KVC_F32) {
         scores_kernel<float><<<grid, kThreads, 0, s>>>((const float*)j.q, (const float*)j.k, j.N,

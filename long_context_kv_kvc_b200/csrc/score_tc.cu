@@ -95,6 +95,8 @@ struct TcArgs {
     const float* ref;    // [U][128] per-row reference logit (base 2): the row's own-position key
     double* sum;         // [U][kSumCopies][128] sums over keys of 2^(y - ref); CTA c adds into copy
                          // c % kSumCopies, which spreads the atomics of the 148 CTAs over more addresses
+    double* sum_t;       // [U][kSumCopies][128] sums of 2^(y - ref) (y - ref), for the entropy
+    float* entropy;      // [U][nq] attention entropy (nats) per window row, or null
     unsigned* count;     // [U] CTAs that have added their part of unit u
     unsigned* never;     // a counter nothing increments (wait-timeout injection)
     unsigned* err;
@@ -106,7 +108,8 @@ struct __align__(1024) Smem {
     uint8_t ringA[kStagesA][kBoxBytes];
     uint8_t ringB[kStagesB][kBoxBytes];
     uint8_t q[kQSlots][2 * kBoxBytes];  // Q of the CTA's k-th unit in slot k % kQSlots (two boxes)
-    float2 rec[kRec][kQRows];           // phase-1 tile i: per row (tile max, sum of 2^(y - max))
+    float2 rec[kRec][kQRows];           // phase-1 tile i: per row (m, sum of 2^(y - m))
+    float rec_t[kRec][kQRows];          // with the entropy: sum of 2^(y - m) (y - m)
     float nlse[2][kQRows];              // -lse of the CTA's k-th unit in slot k % 2
     int4 job[kAcc];                     // {kind, unit, tile within unit, record or lse slot}
     uint64_t fullA[kStagesA], emptyA[kStagesA], fullB[kStagesB], emptyB[kStagesB];
@@ -366,17 +369,26 @@ __device__ __forceinline__ float hsum2(uint64_t v) {
     return a + b;
 }
 
-// Sum over 32 logits (invisible keys already set to -inf) of 2^(y - m) for a fixed m.
-__device__ __forceinline__ float sum_exp2_shifted(const uint32_t (&x)[32], float m) {
+// Sum over 32 logits (invisible keys already set to kMasked) of 2^(y - m) for a fixed m;
+// with ENT also tsum = sum of 2^(y - m) (y - m).
+constexpr float kMasked = -3.0e38f;  // a masked logit: 2^(y - m) is 0 and so is its product with y - m
+template <bool ENT>
+__device__ __forceinline__ float sum_exp2_shifted(const uint32_t (&x)[32], float m, float& tsum) {
     const uint64_t c2 = pack2(kLog2eOverSqrtD, kLog2eOverSqrtD), nm2 = pack2(-m, -m);
-    uint64_t acc0 = 0, acc1 = 0;  // (+0, +0) pairs
+    uint64_t acc0 = 0, acc1 = 0, at0 = 0, at1 = 0;  // (+0, +0) pairs
 #pragma unroll
     for (int e = 0; e < 32; e += 4) {
         const uint64_t y0 = fma2(pack2(__uint_as_float(x[e]), __uint_as_float(x[e + 1])), c2, nm2);
         const uint64_t y1 = fma2(pack2(__uint_as_float(x[e + 2]), __uint_as_float(x[e + 3])), c2, nm2);
-        acc0 = add2(acc0, ex2_pair(y0));
-        acc1 = add2(acc1, ex2_pair(y1));
+        const uint64_t e0 = ex2_pair(y0), e1 = ex2_pair(y1);
+        acc0 = add2(acc0, e0);
+        acc1 = add2(acc1, e1);
+        if (ENT) {
+            at0 = fma2(e0, y0, at0);
+            at1 = fma2(e1, y1, at1);
+        }
     }
+    if (ENT) tsum = hsum2(add2(at0, at1));
     return hsum2(add2(acc0, acc1));
 }
 
@@ -417,6 +429,7 @@ struct TileSeq {
     }
 };
 
+template <bool ENT>
 __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_constant__ TcArgs a) {
     extern __shared__ uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -640,12 +653,26 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             ok = __shfl_sync(0xffffffffu, ok, 0);
             __syncwarp();
             // the unit's total per row: the copies added in a fixed order
-            double tot[4] = {0.0, 0.0, 0.0, 0.0};
+            double tot[4] = {0.0, 0.0, 0.0, 0.0}, tott[4] = {0.0, 0.0, 0.0, 0.0};
             const double* su = a.sum + (size_t)u * kSumCopies * kQRows;
+            const double* st = a.sum_t + (size_t)u * kSumCopies * kQRows;
 #pragma unroll
             for (int c = 0; c < kSumCopies; ++c)
 #pragma unroll
-                for (int rr = 0; rr < 4; ++rr) tot[rr] += __ldcg(su + c * kQRows + lane + 32 * rr);
+                for (int rr = 0; rr < 4; ++rr) {
+                    tot[rr] += __ldcg(su + c * kQRows + lane + 32 * rr);
+                    if (ENT) tott[rr] += __ldcg(st + c * kQRows + lane + 32 * rr);
+                }
+            if (ENT && ok) {
+                // entropy (nats) = ln2 (lse - E[y]) = ln2 (log2 total - E[y - ref])
+#pragma unroll
+                for (int rr = 0; rr < 4; ++rr) {
+                    const int r = lane + 32 * rr;
+                    if (r < a.nq && tot[rr] > 0.0)
+                        a.entropy[(size_t)u * a.nq + r] =
+                            (float)(0.69314718055994531 * ((double)log2_pos(tot[rr]) - tott[rr] / tot[rr]));
+                }
+            }
 #pragma unroll
             for (int rr = 0; rr < 4; ++rr) {
                 const int r = lane + 32 * rr;
@@ -661,11 +688,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
         // ------------------------------------------------------------ publisher
         // lane l holds query rows l + 32 k; merges the phase-1 tile records in tile order and
         // adds the CTA's part of each unit to the unit's total
-        float M[4], L[4];
+        float M[4], L[4], T[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             M[k] = -INFINITY;
             L[k] = 0.f;
+            T[k] = 0.f;
         }
         int u = cta / a.T_u, t = cta - (cta / a.T_u) * a.T_u;
         for (int i = 0; i < n_local; ++i) {
@@ -673,8 +701,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             mbar_wait(&sm.recfull[s], (i / kRec) & 1, abort, a.err);
             if (*abort) break;
             float2 v[4];
+            float vt[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int k = 0; k < 4; ++k) v[k] = sm.rec[s][lane + 32 * k];
+            for (int k = 0; k < 4; ++k) {
+                v[k] = sm.rec[s][lane + 32 * k];
+                if (ENT) vt[k] = sm.rec_t[s][lane + 32 * k];
+            }
             __syncwarp();
             if (lane == 0) {
                 __threadfence_block();
@@ -684,7 +716,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             for (int k = 0; k < 4; ++k) {
                 if (v[k].x != -INFINITY) {
                     const float mn = fmaxf(M[k], v[k].x);
-                    L[k] = (M[k] == -INFINITY ? 0.f : L[k] * ex2(M[k] - mn)) + v[k].y * ex2(v[k].x - mn);
+                    const float fa = M[k] == -INFINITY ? 0.f : ex2(M[k] - mn), fb = ex2(v[k].x - mn);
+                    if (ENT)
+                        T[k] = (M[k] == -INFINITY ? 0.f : fa * (T[k] + (M[k] - mn) * L[k])) +
+                               fb * (vt[k] + (v[k].x - mn) * v[k].y);
+                    L[k] = (M[k] == -INFINITY ? 0.f : L[k] * fa) + v[k].y * fb;
                     M[k] = mn;
                 }
             }
@@ -699,11 +735,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const int r = lane + 32 * k;
-                if (M[k] != -INFINITY)
-                    atomicAdd(a.sum + ((size_t)u * kSumCopies + cta % kSumCopies) * kQRows + r,
-                              scale_exp2(L[k], M[k] - __ldg(a.ref + (size_t)u * kQRows + r)));
+                if (M[k] != -INFINITY) {
+                    const size_t at = ((size_t)u * kSumCopies + cta % kSumCopies) * kQRows + r;
+                    const float d = M[k] - __ldg(a.ref + (size_t)u * kQRows + r);
+                    atomicAdd(a.sum + at, scale_exp2(L[k], d));
+                    // sum of 2^(y - ref) (y - ref) = 2^d (T + d L)
+                    if (ENT) atomicAdd(a.sum_t + at, scale_exp2(fmaf(d, L[k], T[k]), d));
+                }
                 M[k] = -INFINITY;
                 L[k] = 0.f;
+                T[k] = 0.f;
             }
             __threadfence();
             __syncwarp();
@@ -735,7 +776,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                 // needed; a chunk whose sum is not below 2^100 (a logit ~100 above the
                 // reference) is redone with its exact max.
                 const int t_r = a.N - a.w + (r % a.w);  // last key this row sees
-                float m = __ldg(a.ref + (size_t)u * kQRows + r), l = 0.f;
+                float m = __ldg(a.ref + (size_t)u * kQRows + r), l = 0.f, t = 0.f;
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     uint32_t x[32];
@@ -752,14 +793,21 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                         const int j0 = ti * kTileKeys + c * 32;
 #pragma unroll
                         for (int e = 0; e < 32; ++e)
-                            if (j0 + e > t_r) x[e] = __float_as_uint(-INFINITY);
+                            if (j0 + e > t_r) x[e] = __float_as_uint(kMasked);
                     }
-                    const float cs = sum_exp2_shifted(x, m);
+                    float ct = 0.f;
+                    const float cs = sum_exp2_shifted<ENT>(x, m, ct);
                     if (cs < 0x1p100f) {
                         l += cs;
+                        if (ENT) t += ct;
                     } else {
+                        // move the reference to the chunk's max: sums scale by 2^(m - mn), each
+                        // y - m shifts by m - mn
                         const float mn = fmaxf(m, chunk_max(x) * kLog2eOverSqrtD);
-                        l = l * ex2(m - mn) + sum_exp2_shifted(x, mn);
+                        const float f = ex2(m - mn);
+                        if (ENT) t = f * (t + (m - mn) * l);
+                        l = l * f + sum_exp2_shifted<ENT>(x, mn, ct);
+                        if (ENT) t += ct;
                         m = mn;
                     }
                 }
@@ -768,6 +816,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                 if (lane == 0) spin_until_at_least(&sm.rec_consumed, i - kRec + 1, abort, a.err);
                 __syncwarp();
                 sm.rec[s][r] = make_float2(m, l);
+                if (ENT) sm.rec_t[s][r] = t;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.recfull[s]);
             } else {
@@ -852,7 +901,7 @@ __global__ void tc_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_b
         for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
         if (lane == 0) ref[e] = x * kLog2eOverSqrtD;
     }
-    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < (long long)U * kSumCopies * kQRows;
+    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < 2LL * U * kSumCopies * kQRows;
          e += (long long)gridDim.x * blockDim.x)
         sum[e] = 0.0;
     for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n_flags;
@@ -875,8 +924,8 @@ TcLayout tc_layout(int U) {
     off = a256(off + (size_t)U * kQRows * kHeadDim * 2);
     L.ref = off;
     off = a256(off + (size_t)U * kQRows * sizeof(float));
-    L.sum = off;
-    off = a256(off + (size_t)U * kSumCopies * kQRows * sizeof(double));
+    L.sum = off;  // the totals, then the entropy's totals
+    off = a256(off + 2 * (size_t)U * kSumCopies * kQRows * sizeof(double));
     L.flags = off;  // count[U], never
     L.n_flags = (size_t)U + 1;
     off = a256(off + L.n_flags * sizeof(unsigned));
@@ -928,6 +977,8 @@ cudaError_t tc_score(const ScoreJob& j, cudaStream_t s) {
     a.unit_scores = j.unit_scores;
     a.ref = (const float*)(ws + L.ref);
     a.sum = (double*)(ws + L.sum);
+    a.sum_t = a.sum + (size_t)j.U * kSumCopies * kQRows;
+    a.entropy = j.entropy;
     a.count = flags;
     a.never = flags + j.U;
     a.err = j.err;
@@ -979,13 +1030,15 @@ cudaError_t tc_score(const ScoreJob& j, cudaStream_t s) {
     if (e != cudaSuccess) return e;
 
     const size_t smem = sizeof(Smem) + 1024;
-    static std::atomic<bool> attr_set[64];
+    const bool ent = j.entropy != nullptr;
+    static std::atomic<bool> attr_set[2][64];
     int dev = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if (dev >= 64 || !attr_set[dev].load()) {
-        e = cudaFuncSetAttribute(tc_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (dev >= 64 || !attr_set[ent][dev].load()) {
+        e = ent ? cudaFuncSetAttribute(tc_score_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
+                : cudaFuncSetAttribute(tc_score_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        if (dev < 64) attr_set[dev].store(true);
+        if (dev < 64) attr_set[ent][dev].store(true);
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.P);
@@ -997,7 +1050,7 @@ cudaError_t tc_score(const ScoreJob& j, cudaStream_t s) {
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, tc_score_kernel, a);
+    e = ent ? cudaLaunchKernelEx(&cfg, tc_score_kernel<true>, a) : cudaLaunchKernelEx(&cfg, tc_score_kernel<false>, a);
     count_launches(1);
     return e;
 }

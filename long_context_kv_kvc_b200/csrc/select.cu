@@ -394,6 +394,67 @@ topk_cluster_kernel(const float* __restrict__ scores, int N, int S, int w, int b
     cluster.sync();  // siblings may still read this CTA's counts until here
 }
 
+// --------------------------------------------------------------- row statistics
+//
+// Two of the signals StructKV watches to find its pivot layer (StructKV page, sec. 2
+// "Dynamische Pivot Detectie": sparsity and variance of the attention), per score row:
+// the share of the row's mass held by its kept positions, and the population variance of
+// the row over the candidates C = [S, N - w).  One CTA per row, fp64 partial sums in a
+// fixed order (deterministic).
+
+constexpr int kRsThreads = 1024;
+
+__device__ __forceinline__ double block_sum(double v, double* red) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __syncthreads();  // red may still be read by a previous call
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    double t = 0.0;
+    for (int i = 0; i < kRsThreads / 32; ++i) t += red[i];
+    return t;
+}
+
+__global__ void __launch_bounds__(kRsThreads)
+row_stats_kernel(const float* __restrict__ scores, int N, int S, int w, const int32_t* __restrict__ idx,
+                 int budget, float* __restrict__ kept_mass, float* __restrict__ cand_var, unsigned* err) {
+    __shared__ double red[kRsThreads / 32];
+    const int row = blockIdx.x;
+    const float* s = scores + (size_t)row * N;
+    const int lo = S, hi = N - w;
+    double tot = 0.0, csum = 0.0;
+    for (int j = threadIdx.x; j < N; j += kRsThreads) {
+        const double v = s[j];
+        tot += v;
+        if (j >= lo && j < hi) csum += v;
+    }
+    tot = block_sum(tot, red);
+    csum = block_sum(csum, red);
+    const double mean = csum / (hi - lo);
+    double var = 0.0;
+    for (int j = lo + threadIdx.x; j < hi; j += kRsThreads) {
+        const double d = s[j] - mean;
+        var += d * d;
+    }
+    var = block_sum(var, red);
+    double kept = 0.0;
+    if (idx) {
+        for (int t = threadIdx.x; t < budget; t += kRsThreads) {
+            const int j = idx[(size_t)row * budget + t];
+            if (j >= 0 && j < N)
+                kept += s[j];
+            else
+                atomicOr(err, kErrIndex);
+        }
+        kept = block_sum(kept, red);
+    }
+    if (threadIdx.x == 0) {
+        cand_var[row] = (float)(var / (hi - lo));
+        if (idx) kept_mass[row] = (float)(kept / tot);
+    }
+}
+
 int grid_for(long long total, int threads) {
     long long g = (total + threads - 1) / threads;
     if (g > 148LL * 32) g = 148LL * 32;
@@ -458,6 +519,13 @@ cudaError_t topk(const float* pooled, int rows, int N, int n_sink, int window, i
                  int32_t* idx, cudaStream_t s) {
     if (rows == 0) return cudaSuccess;
     topk_kernel<<<rows, kTopkThreads, 0, s>>>(pooled, N, n_sink, window, budget, idx);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t row_stats(const float* scores, int rows, int N, int S, int w, const int32_t* idx, int budget,
+                      float* kept_mass, float* cand_var, unsigned* err, cudaStream_t s) {
+    row_stats_kernel<<<rows, kRsThreads, 0, s>>>(scores, N, S, w, idx, budget, kept_mass, cand_var, err);
     count_launches(1);
     return cudaGetLastError();
 }

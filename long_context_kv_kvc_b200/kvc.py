@@ -24,7 +24,8 @@ KVC_STAGE_SCORE, KVC_STAGE_SELECT, KVC_STAGE_GATHER, KVC_STAGE_COUNT = 0, 1, 2, 
 
 EXPORTED = ("kvc_workspace_size", "kvc_score", "kvc_accumulate", "kvc_pool", "kvc_topk_workspace_size",
             "kvc_topk", "kvc_gather", "kvc_compress", "kvc_tsp_count", "kvc_poll_error",
-            "kvc_status_string", "kvc_version", "kvc_launch_count", "kvc_score_noalloc")
+            "kvc_status_string", "kvc_version", "kvc_launch_count", "kvc_score_noalloc", "kvc_score_entropy",
+            "kvc_row_stats")
 
 
 class KvcError(RuntimeError):
@@ -64,6 +65,8 @@ def _load():
         "kvc_version": (ctypes.c_char_p, []),
         "kvc_launch_count": (ctypes.c_uint64, []),
         "kvc_score_noalloc": (st, [P, vp, vp, vp, vp]),
+        "kvc_score_entropy": (st, [P, vp, vp, vp, vp, vp, sz, vp]),
+        "kvc_row_stats": (st, [vp, i32, i32, i32, i32, vp, i32, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -145,6 +148,24 @@ def kvc_score_noalloc(p: Params, q, k, scores, stream=None):
     library's fixed 4 MiB per-device scratch array stands in for it (see include/kvc.h)."""
     _check(lib.kvc_score_noalloc(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(scores), _stream(stream)),
            "kvc_score_noalloc")
+
+
+def kvc_score_entropy(p: Params, q, k, scores, entropy, ws, stream=None):
+    """kvc_score plus the attention entropy (nats) of every window query row, in one pass;
+    entropy is [n_layers, B, Hq, window] fp32."""
+    _check(lib.kvc_score_entropy(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(scores), _ptr(entropy), _ptr(ws),
+                                 ws.numel() * ws.element_size(), _stream(stream)), "kvc_score_entropy")
+
+
+def kvc_row_stats(scores, n_sink, window, cand_var, idx=None, kept_mass=None, stream=None):
+    """Per score row of scores [..., N]: population variance over [n_sink, N - window) into
+    cand_var, and (with idx [..., budget]) the share of the row's mass at idx into kept_mass."""
+    N = scores.shape[-1]
+    rows = scores.numel() // N
+    budget = idx.shape[-1] if idx is not None else 0
+    _check(lib.kvc_row_stats(_ptr(scores), rows, N, n_sink, window, _ptr(idx) if idx is not None else None,
+                             budget, _ptr(kept_mass) if kept_mass is not None else None, _ptr(cand_var),
+                             _stream(stream)), "kvc_row_stats")
 
 
 def kvc_accumulate(acc, src, stream=None):
