@@ -443,3 +443,172 @@ int oracle_row_stats(const double *scores, int rows, int N, int S, int w, const 
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------------------ */
+/* Chunked Soft Matching (CentroidKV)                                                    */
+/* ------------------------------------------------------------------------------------ */
+
+/*
+ * CentroidKV clusters KV states instead of evicting them (CentroidKV page, sec. 3 "Chunked
+ * Soft Matching" and sec. 4 "Aggregatie"):
+ *   chunks     the candidates C = [S, N - w) are cut into chunks of `chunk` tokens (sinks and
+ *              the recent window stay as they are: sec. 2, Preservation);
+ *   partition  inside a chunk, tokens alternate between set A (even offset) and set B (odd);
+ *   matching   each A token's match is the B token of its chunk with the largest cosine
+ *              similarity of the key states (ties: lower position; a zero key has
+ *              similarity 0); an A token alone in its chunk has no match;
+ *   merge      the matches are ranked by similarity and only the top fraction merges:
+ *              m = min(floor(r * |C|), matchable A tokens) of them (ties: lower position);
+ *   aggregate  a B token and the A tokens merged into it become their degree-weighted
+ *              mean, K and V alike; degrees add (sec. 4: n_t counts the merged tokens).
+ * The cache keeps every token except the merged A tokens, in position order.
+ */
+
+static double key_dot(const void *k, int dtype, size_t ra, size_t rb, int D)
+{
+    double s = 0.0;
+    for (int d = 0; d < D; ++d) s += widen(k, dtype, ra * D + d) * widen(k, dtype, rb * D + d);
+    return s;
+}
+
+/* Rounds v to the element type (bf16: round to nearest even; f32: nearest) and stores it. */
+static void store_elem(void *dst, int dtype, size_t i, double v)
+{
+    if (dtype == OR_F64) { ((double *)dst)[i] = v; return; }
+    float f = (float)v;
+    if (dtype == OR_F32) { ((float *)dst)[i] = f; return; }
+    uint32_t bits;
+    memcpy(&bits, &f, sizeof bits);
+    if ((bits & 0x7F800000u) == 0x7F800000u && (bits & 0x007FFFFFu)) { /* NaN stays NaN */
+        ((uint16_t *)dst)[i] = (uint16_t)((bits >> 16) | 0x40u);
+        return;
+    }
+    /* v -> float may already round; redo from v in double for an exact bf16 RNE */
+    double av = fabs(v);
+    if (av == 0.0) { ((uint16_t *)dst)[i] = (uint16_t)(bits >> 16); return; }
+    int e;
+    frexp(av, &e);                                  /* av = f * 2^e, f in [0.5, 1) */
+    double ulp = ldexp(1.0, (e < -125 ? -125 : e) - 8); /* bf16 spacing at av */
+    double q = nearbyint(av / ulp) * ulp;           /* round half to even (default mode) */
+    float qf = (float)(v < 0 ? -q : q);
+    memcpy(&bits, &qf, sizeof bits);
+    ((uint16_t *)dst)[i] = (uint16_t)(bits >> 16);
+}
+
+/* Merges m of a row's A tokens; see above.  Outputs per row: best[N] (match position or -1),
+ * sim[N] (match similarity, -inf when there is none), merged[N] (0/1), and the kept rows. */
+static int csm_row(const void *k, const void *v, int dtype, const int32_t *deg, int N, int D, int S, int w,
+                   int chunk, int m, int32_t *best, double *sim, unsigned char *merged,
+                   void *k_out, void *v_out, int32_t *deg_out, int32_t *pos_out)
+{
+    const int lo = S, hi = N - w;
+    for (int j = 0; j < N; ++j) { best[j] = -1; sim[j] = -INFINITY; merged[j] = 0; }
+    for (int c0 = lo; c0 < hi; c0 += chunk) {
+        const int c1 = c0 + chunk < hi ? c0 + chunk : hi;
+        for (int a = c0; a < c1; a += 2) {
+            const double na = sqrt(key_dot(k, dtype, a, a, D));
+            for (int b = c0 + 1; b < c1; b += 2) {
+                const double nb = sqrt(key_dot(k, dtype, b, b, D));
+                const double s = (na > 0.0 && nb > 0.0) ? key_dot(k, dtype, a, b, D) / (na * nb) : 0.0;
+                if (best[a] < 0 || s > sim[a]) { best[a] = b; sim[a] = s; }
+            }
+        }
+    }
+    /* the m matches with the largest similarity, ties to the lower position */
+    int n_a = 0;
+    for (int j = lo; j < hi; ++j)
+        if (best[j] >= 0) ++n_a;
+    cand *c = (cand *)malloc(sizeof(cand) * (size_t)(n_a > 0 ? n_a : 1));
+    if (!c) return -1;
+    int t = 0;
+    for (int j = lo; j < hi; ++j)
+        if (best[j] >= 0) { c[t].v = sim[j]; c[t].j = j; ++t; }
+    qsort(c, (size_t)n_a, sizeof(cand), cand_cmp);
+    for (int q = 0; q < m && q < n_a; ++q) merged[c[q].j] = 1;
+    free(c);
+    /* kept rows in position order; a B token absorbs the A tokens merged into it */
+    double *acc_k = (double *)malloc(sizeof(double) * (size_t)D), *acc_v = (double *)malloc(sizeof(double) * (size_t)D);
+    if (!acc_k || !acc_v) { free(acc_k); free(acc_v); return -1; }
+    int o = 0;
+    for (int j = 0; j < N; ++j) {
+        if (merged[j]) continue;
+        long long n = deg[j];
+        for (int d = 0; d < D; ++d) {
+            acc_k[d] = (double)deg[j] * widen(k, dtype, (size_t)j * D + d);
+            acc_v[d] = (double)deg[j] * widen(v, dtype, (size_t)j * D + d);
+        }
+        if (j >= lo && j < hi && (j - lo) % chunk % 2 == 1) {
+            const int c0 = lo + (j - lo) / chunk * chunk;
+            const int c1 = c0 + chunk < hi ? c0 + chunk : hi;
+            for (int a = c0; a < c1; a += 2)
+                if (merged[a] && best[a] == j) {
+                    n += deg[a];
+                    for (int d = 0; d < D; ++d) {
+                        acc_k[d] += (double)deg[a] * widen(k, dtype, (size_t)a * D + d);
+                        acc_v[d] += (double)deg[a] * widen(v, dtype, (size_t)a * D + d);
+                    }
+                }
+        }
+        for (int d = 0; d < D; ++d) {
+            store_elem(k_out, dtype, (size_t)o * D + d, acc_k[d] / (double)n);
+            store_elem(v_out, dtype, (size_t)o * D + d, acc_v[d] / (double)n);
+        }
+        deg_out[o] = (int32_t)n;
+        pos_out[o] = j;
+        ++o;
+    }
+    free(acc_k);
+    free(acc_v);
+    return o;
+}
+
+/*
+ * oracle_csm_merges -- m = min(floor(r * |C|), matchable A tokens) for a row of N tokens.
+ * An A token is matchable when its chunk holds a B token: every A token except one alone in
+ * the last chunk.
+ */
+int oracle_csm_merges(int N, int S, int w, int chunk, double r)
+{
+    if (N < 1 || S < 0 || w < 0 || S + w > N || chunk < 2 || chunk % 2 || !(r >= 0.0 && r <= 0.5)) return -1;
+    const int n_c = N - w - S;
+    int n_a = 0;
+    for (int c0 = 0; c0 < n_c; c0 += chunk) {
+        const int len = c0 + chunk < n_c ? chunk : n_c - c0;
+        if (len >= 2) n_a += (len + 1) / 2;
+    }
+    const long m = (long)floor(r * (double)n_c);
+    return (int)(m < n_a ? m : n_a);
+}
+
+/*
+ * oracle_csm -- one Chunked Soft Matching round over rows of [rows, N, D] K and V (dtype as
+ * in oracle_score; fp64 arithmetic, outputs rounded to the same dtype) with degrees
+ * deg[rows][N].  Outputs per row: best, sim, merged as in csm_row; k_out, v_out
+ * [rows][N - m][D], deg_out and pos_out [rows][N - m].  Returns N - m, or -1 on bad
+ * arguments.
+ */
+int oracle_csm(const void *k, const void *v, int dtype, const int32_t *deg, int rows, int N, int D, int S, int w,
+               int chunk, double r, int32_t *best, double *sim, unsigned char *merged, void *k_out, void *v_out,
+               int32_t *deg_out, int32_t *pos_out)
+{
+    const int m = oracle_csm_merges(N, S, w, chunk, r);
+    if (m < 0 || rows < 1 || D < 1) return -1;
+    const size_t esz = dtype == OR_F32 ? 4 : dtype == OR_F64 ? 8 : 2;
+    const int n_out = N - m;
+    for (int row = 0; row < rows; ++row) {
+        const size_t in = (size_t)row * N, out = (size_t)row * n_out;
+        const int o = csm_row((const char *)k + in * D * esz, (const char *)v + in * D * esz, dtype, deg + in, N, D,
+                              S, w, chunk, m, best + in, sim + in, merged + in, (char *)k_out + out * D * esz,
+                              (char *)v_out + out * D * esz, deg_out + out, pos_out + out);
+        if (o != n_out) return -1;
+    }
+    return n_out;
+}
+
+/* The progressive schedule of the merge ratio over rounds (CentroidKV page, sec. 3):
+ * r_j = r_init - j * delta, not below 0. */
+double oracle_csm_ratio(double r_init, double delta, int round)
+{
+    const double r = r_init - (double)round * delta;
+    return r > 0.0 ? r : 0.0;
+}

@@ -47,8 +47,13 @@ def _load(so_path: str):
     L.oracle_tsp_count.argtypes = [i, i, i, d]
     L.oracle_entropy.argtypes = [i, i, i, i, i, i, i, p, p, i, p, i, p, i]
     L.oracle_row_stats.argtypes = [p, i, i, i, i, p, i, p, p]
+    L.oracle_csm_merges.argtypes = [i, i, i, i, d]
+    L.oracle_csm.argtypes = [p, p, i, p, i, i, i, i, i, i, d, p, p, p, p, p, p, p]
+    L.oracle_csm_ratio.argtypes = [d, d, i]
+    L.oracle_csm_ratio.restype = d
     for f in ("oracle_score", "oracle_accumulate", "oracle_pool", "oracle_select",
-              "oracle_gather", "oracle_tsp_count", "oracle_entropy", "oracle_row_stats"):
+              "oracle_gather", "oracle_tsp_count", "oracle_entropy", "oracle_row_stats",
+              "oracle_csm_merges", "oracle_csm"):
         getattr(L, f).restype = ctypes.c_int
     return L
 
@@ -212,6 +217,53 @@ def row_stats(scores: np.ndarray, n_sink: int, window: int, idx: np.ndarray = No
                                 cv.ctypes.data)
     _check(rc, "row_stats")
     return (km if idx is not None else None), cv
+
+
+def csm_merges(N: int, n_sink: int, window: int, chunk: int, ratio: float) -> int:
+    m = int(lib().oracle_csm_merges(N, n_sink, window, chunk, float(ratio)))
+    _check(0 if m >= 0 else -1, "csm_merges")
+    return m
+
+
+def csm_ratio(r_init: float, delta: float, round_: int) -> float:
+    return float(lib().oracle_csm_ratio(float(r_init), float(delta), int(round_)))
+
+
+def csm(k, v, deg, *, n_sink: int, window: int, chunk: int, ratio: float) -> dict:
+    """One Chunked Soft Matching round (fp64) over k, v [..., N, D] (fp32 / bf16 / fp64 tensors)
+    with degrees deg [..., N] int32.  Returns best, sim, merged [..., N] and the kept
+    k_out, v_out [..., N - m, D] (input dtype), deg_out, pos_out [..., N - m]."""
+    k = k.detach().cpu().contiguous()
+    v = v.detach().cpu().contiguous()
+    lead, (N, D) = tuple(k.shape[:-2]), tuple(k.shape[-2:])
+    rows = int(np.prod(lead)) if lead else 1
+    kb, kd = _as_buffer(k)
+    vb, vd = _as_buffer(v)
+    assert kd == vd and v.shape == k.shape
+    dg = np.ascontiguousarray(np.asarray(deg, dtype=np.int32).reshape(rows, N))
+    m = csm_merges(N, n_sink, window, chunk, ratio)
+    n_out = N - m
+    best = np.empty((rows, N), dtype=np.int32)
+    sim = np.empty((rows, N), dtype=np.float64)
+    merged = np.empty((rows, N), dtype=np.uint8)
+    k_out = torch.empty(lead + (n_out, D), dtype=k.dtype)
+    v_out = torch.empty(lead + (n_out, D), dtype=k.dtype)
+    ko, _ = _as_buffer(k_out)
+    vo, _ = _as_buffer(v_out)
+    deg_out = np.empty((rows, n_out), dtype=np.int32)
+    pos_out = np.empty((rows, n_out), dtype=np.int32)
+    rc = lib().oracle_csm(kb.ctypes.data, vb.ctypes.data, kd, dg.ctypes.data, rows, N, D, n_sink, window, chunk,
+                          float(ratio), best.ctypes.data, sim.ctypes.data, merged.ctypes.data, ko.ctypes.data,
+                          vo.ctypes.data, deg_out.ctypes.data, pos_out.ctypes.data)
+    _check(0 if rc == n_out else -1, "csm")
+    # the buffers handed to C were views of k_out / v_out (bf16 through an int16 view)
+    if k.dtype == torch.bfloat16:
+        k_out = torch.from_numpy(ko).view(torch.bfloat16).reshape(k_out.shape)
+        v_out = torch.from_numpy(vo).view(torch.bfloat16).reshape(v_out.shape)
+    shp = lead if lead else ()
+    return {"best": best.reshape(shp + (N,)), "sim": sim.reshape(shp + (N,)), "merged": merged.reshape(shp + (N,)),
+            "k_out": k_out, "v_out": v_out, "deg_out": deg_out.reshape(shp + (n_out,)),
+            "pos_out": pos_out.reshape(shp + (n_out,)), "m": m}
 
 
 def compress(q, k, v, *, window: int, n_sink: int, pool_kernel: int, kv_budget: int,

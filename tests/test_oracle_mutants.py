@@ -41,6 +41,15 @@ MUTANTS = [
     ("entropy row's keys one short", "for (int j = 0; j <= last; ++j) {\n        double acc",
      "for (int j = 0; j < last; ++j) {\n        double acc"),
     ("sample variance", "cand_var[row] = var / n_c;", "cand_var[row] = var / (n_c - 1);"),
+    ("csm: dot product instead of cosine", "? key_dot(k, dtype, a, b, D) / (na * nb) : 0.0",
+     "? key_dot(k, dtype, a, b, D) : 0.0"),
+    ("csm: partition A odd", "for (int a = c0; a < c1; a += 2) {\n            const double na",
+     "for (int a = c0 + 1; a < c1; a += 2) {\n            const double na"),
+    ("csm: match ties to the higher position", "if (best[a] < 0 || s > sim[a])", "if (best[a] < 0 || s >= sim[a])"),
+    ("csm: merge count rounds up", "const long m = (long)floor(r * (double)n_c);", "const long m = (long)ceil(r * (double)n_c);"),
+    ("csm: unweighted mean", "acc_k[d] += (double)deg[a] * widen(k, dtype, (size_t)a * D + d);",
+     "acc_k[d] += (double)deg[j] * widen(k, dtype, (size_t)a * D + d);"),
+    ("csm: degrees not accumulated", "                    n += deg[a];\n", ""),
     ("kept mass over the candidates only", "for (int j = 0; j < N; ++j) total += s[j];",
      "for (int j = S; j < N - w; ++j) total += s[j];"),
 ]
@@ -64,6 +73,12 @@ PIN_TESTS = [
     pins.test_entropy_two_keys_is_binary_entropy,
     pins.test_entropy_dominant_key_is_zero_and_matches_library,
     pins.test_row_stats_against_definitions,
+    pins.test_csm_merge_count,
+    lambda: [pins.test_csm_matches_brute_force(*a) for a in [(23, 1, 3, 4, 0.5), (40, 0, 0, 6, 0.3), (31, 2, 5, 8, 0.45),
+                                                             (12, 1, 1, 2, 0.5)]],
+    pins.test_csm_invariants_and_closed_forms,
+    pins.test_csm_bf16_output_rounding,
+    pins.test_csm_ties_go_to_lower_position,
 ]
 
 

@@ -382,3 +382,124 @@ def test_row_stats_against_definitions():
     s2[..., :S] = 1e6
     s2[..., N - w:] = -1e6
     np.testing.assert_allclose(O.row_stats(s2, S, w)[1], cv, rtol=1e-13)
+
+
+# ------------------------------------------------------------------- Chunked Soft Matching
+
+def _csm_brute(k, deg, S, w, chunk, m, v=None):
+    """Plain-Python restatement for tiny inputs: matches, the m merged A tokens, kept rows
+    (of k, or of v when given, with k's matches)."""
+    N = k.shape[0]
+    kk = k.double().numpy()
+    best, sim = {}, {}
+    for c0 in range(S, N - w, chunk):
+        c1 = min(c0 + chunk, N - w)
+        A, B = list(range(c0, c1, 2)), list(range(c0 + 1, c1, 2))
+        for a in A:
+            if not B:
+                continue
+            sims = []
+            for b in B:
+                na, nb = np.linalg.norm(kk[a]), np.linalg.norm(kk[b])
+                sims.append(float(kk[a] @ kk[b] / (na * nb)) if na > 0 and nb > 0 else 0.0)
+            i = int(np.argmax(sims))  # first maximum: the lower position
+            best[a], sim[a] = B[i], sims[i]
+    order = sorted(best, key=lambda a: (-sim[a], a))
+    merged = set(order[:m])
+    src = kk if v is None else v.double().numpy()
+    rows, degs, pos = [], [], []
+    for j in range(N):
+        if j in merged:
+            continue
+        parts = [j] + [a for a in sorted(merged) if best[a] == j]
+        n = sum(int(deg[x]) for x in parts)
+        rows.append(sum(int(deg[x]) * src[x] for x in parts) / n)
+        degs.append(n)
+        pos.append(j)
+    return best, sim, merged, np.array(rows), np.array(degs), np.array(pos)
+
+
+def test_csm_merge_count():
+    # C = [1, 8) in chunks of 4: [1, 5) holds 2 A tokens, [5, 8) holds 2 -> 4 matchable
+    assert O.csm_merges(10, 1, 2, 4, 0.5) == 3            # floor(0.5 * 7)
+    assert O.csm_merges(10, 1, 2, 4, 0.25) == 1
+    assert O.csm_merges(10, 1, 2, 4, 0.0) == 0
+    assert O.csm_merges(9, 0, 0, 4, 0.5) == 4             # [0,4) [4,8) [8,9): the lone A is unmatchable
+    assert O.csm_merges(5, 0, 0, 2, 0.5) == 2             # chunks [0,2) [2,4) [4,5)
+    assert O.csm_ratio(0.5, 0.1, 0) == 0.5 and O.csm_ratio(0.5, 0.1, 2) == pytest.approx(0.3)
+    assert O.csm_ratio(0.5, 0.2, 9) == 0.0
+
+
+@pytest.mark.parametrize("N,S,w,chunk,r", [(23, 1, 3, 4, 0.5), (40, 0, 0, 6, 0.3), (31, 2, 5, 8, 0.45),
+                                           (12, 1, 1, 2, 0.5)])
+def test_csm_matches_brute_force(N, S, w, chunk, r):
+    g = torch.Generator().manual_seed(N + chunk)
+    k = torch.randn(N, 6, dtype=torch.float64, generator=g)
+    k[S + 3] = 0.0  # a zero key: similarity 0 to everything
+    v = torch.randn(N, 6, dtype=torch.float64, generator=g)
+    deg = torch.randint(1, 5, (N,), generator=g).numpy().astype(np.int32)
+    m = O.csm_merges(N, S, w, chunk, r)
+    out = O.csm(k, v, deg, n_sink=S, window=w, chunk=chunk, ratio=r)
+    best, sim, merged, rows, degs, pos = _csm_brute(k, deg, S, w, chunk, m)
+    for a in range(N):
+        if a in best:
+            assert out["best"][a] == best[a] and out["sim"][a] == pytest.approx(sim[a], abs=1e-13)
+        else:
+            assert out["best"][a] == -1
+    assert set(np.nonzero(out["merged"])[0].tolist()) == merged
+    np.testing.assert_array_equal(out["pos_out"], pos)
+    np.testing.assert_array_equal(out["deg_out"], degs)
+    np.testing.assert_allclose(out["k_out"].numpy(), rows, rtol=1e-13, atol=1e-13)
+    vrows = _csm_brute(k, deg, S, w, chunk, m, v=v)[3]
+    np.testing.assert_allclose(out["v_out"].numpy(), vrows, rtol=1e-13, atol=1e-13)
+
+
+def test_csm_invariants_and_closed_forms():
+    # identical directions merge first (cosine 1); a B token absorbing an A token of the
+    # same direction gives the degree-weighted mean; sinks, window and unmerged rows are
+    # unchanged bit for bit; degrees are conserved; r = 0 is the identity
+    N, D = 16, 8
+    g = torch.Generator().manual_seed(21)
+    k = torch.randn(N, D, dtype=torch.float32, generator=g)
+    v = torch.randn(N, D, dtype=torch.float32, generator=g)
+    k[5] = 2.0 * k[4]                      # chunk [4, 8) with S=0, chunk 4: A = {4, 6}, B = {5, 7}
+    deg = np.array([1, 2, 1, 1, 3, 1, 2, 1, 1, 1, 4, 1, 1, 1, 1, 1], dtype=np.int32)
+    out = O.csm(k, v, deg, n_sink=0, window=0, chunk=4, ratio=1 / 16)  # m = 1
+    assert out["m"] == 1 and out["merged"][4] == 1 and out["best"][4] == 5
+    assert out["sim"][4] == pytest.approx(1.0, abs=1e-7)
+    j = list(out["pos_out"]).index(5)
+    want = (3 * k[4].double() + 1 * k[5].double()) / 4
+    np.testing.assert_allclose(out["k_out"][j].double().numpy(), want.numpy(), rtol=1e-6)
+    assert out["deg_out"][j] == 4 and out["deg_out"].sum() == deg.sum()
+    for o, p in enumerate(out["pos_out"]):
+        if p != 5:
+            assert torch.equal(out["k_out"][o], k[p]) and torch.equal(out["v_out"][o], v[p])
+    ident = O.csm(k, v, deg, n_sink=2, window=3, chunk=4, ratio=0.0)
+    assert torch.equal(ident["k_out"], k) and np.array_equal(ident["pos_out"], np.arange(N))
+    big = O.csm(k, v, deg, n_sink=2, window=3, chunk=4, ratio=0.5)
+    assert set(range(2)) <= set(big["pos_out"].tolist()) and set(range(N - 3, N)) <= set(big["pos_out"].tolist())
+    assert big["deg_out"].sum() == deg.sum() and len(big["pos_out"]) == N - big["m"]
+    assert np.all(np.diff(big["pos_out"]) > 0)
+
+
+def test_csm_bf16_output_rounding():
+    # merged rows are rounded to bf16 to nearest, ties to even: 1 and 1 + 2^-7 (degrees 1, 1)
+    # average to 1 + 2^-8, a tie that rounds to 1; 1 and 1 + 3 * 2^-7 give 1 + 3 * 2^-8, which
+    # rounds up to 1 + 2^-6
+    D = 2
+    for hi, want in [(1 + 2 ** -7, 1.0), (1 + 3 * 2 ** -7, 1 + 2 ** -6)]:
+        k = torch.tensor([[1.0, 1.0], [hi, hi]], dtype=torch.bfloat16)
+        out = O.csm(k, k, np.ones(2, np.int32), n_sink=0, window=0, chunk=2, ratio=0.5)
+        assert out["m"] == 1 and out["k_out"].shape == (1, D)
+        assert out["k_out"][0, 0].item() == want
+
+
+def test_csm_ties_go_to_lower_position():
+    # two B tokens with the same key: every A token of the chunk matches the lower one, and
+    # equal similarities merge in position order
+    a, b = [1.0, 0.2, 0.0], [0.3, 1.0, 0.5]
+    k = torch.tensor([a, b, a, b, a, b, a, b], dtype=torch.float64)
+    out = O.csm(k, k, np.ones(8, np.int32), n_sink=0, window=0, chunk=8, ratio=0.25)
+    assert out["best"][0] == 1 and out["best"][2] == 1 and out["best"][4] == 1 and out["best"][6] == 1
+    # all four A tokens tie; two merges take positions 0 and 2
+    assert out["m"] == 2 and np.nonzero(out["merged"])[0].tolist() == [0, 2]
