@@ -399,6 +399,22 @@ def main():
         pivot = {"score_ms": t_plain, "score_with_entropy_ms": t_ent, "row_stats_ms": t_rs,
                  "calls": args.pivot_steps}
 
+        # one CentroidKV Chunked Soft Matching round over the last layer's K and V (r = 0.25,
+        # chunks of 64): algorithmic bytes = K read to match + K and V read and the kept rows
+        # (K, V, degree, position) written
+        if wl.D == 128:
+            kl, vl = dev["k"][-1], dev["v"]
+            r, ch = 0.25, 64
+            m = kvc.kvc_csm_merges(wl.N, wl.n_sink, wl.window, ch, r)
+            csm_out = kvc.kvc_csm(kl, vl, wl.n_sink, wl.window, ch, r)
+            t_csm = timed(lambda: kvc.kvc_csm(kl, vl, wl.n_sink, wl.window, ch, r, out=csm_out))
+            if kvc.kvc_poll_error() != kvc.KVC_OK:
+                raise RuntimeError("device-side error in the clustering round")
+            row = wl.D * kl.element_size()
+            nbytes = wl.B * wl.Hkv * (3 * wl.N * row + (wl.N - m) * (2 * row + 8))  # + degree, position
+            pivot["csm"] = {"ratio": r, "chunk": ch, "ms": t_csm, "gbs": nbytes / (t_csm * 1e-3) / 1e9,
+                            "algorithmic_bytes": nbytes, "frac_of_peak": nbytes / (t_csm * 1e-3) / 1e9 / peak}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         threads = min(wl.Hkv, os.cpu_count() or 1)

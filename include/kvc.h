@@ -253,6 +253,51 @@ KVC_API kvc_status kvc_row_stats(const float *scores, int32_t rows, int32_t N, i
                                  kvc_stream_t stream);
 
 /*
+ * Chunked Soft Matching -- CentroidKV clusters KV states instead of evicting them (CentroidKV
+ * page, sec. 3 "Chunked Soft Matching", sec. 4 "Aggregatie").  One round over rows (batch,
+ * KV head) of N cached tokens with degrees n_t:
+ *   - the candidates C = [n_sink, N - window) are cut into chunks of `chunk` tokens; sinks and
+ *     the recent window stay as they are (sec. 2, Preservation);
+ *   - in a chunk, the tokens at even offsets form set A and the odd ones set B; each A token
+ *     is matched with the B token of its chunk whose key is the most cosine-similar (ties:
+ *     lower position; a zero key has similarity 0); an A token alone in its chunk has no
+ *     match;
+ *   - the m = kvc_csm_merges(...) matches with the largest similarity merge (ties: lower
+ *     position): a B token and the A tokens merged into it become their degree-weighted mean
+ *     (keys and values alike, fp32 arithmetic rounded once to the element type) and their
+ *     degrees add; every other kept row is copied bit for bit;
+ *   - the output keeps every token except the merged A tokens, in position order.
+ * The ratio r is at most 0.5 (at most half of the cache per round); CentroidKV lowers it
+ * over rounds, see kvc_csm_ratio.
+ */
+
+/* kvc_csm_merges -- m = min(floor(ratio * |C|), matchable A tokens); -1 for invalid
+ * arguments (chunk even in [2, 128], 0 <= ratio <= 0.5, n_sink + window <= N).  Host only. */
+KVC_API int32_t kvc_csm_merges(int32_t N, int32_t n_sink, int32_t window, int32_t chunk, float ratio);
+
+/* kvc_csm_ratio -- the progressive schedule of the merge ratio (CentroidKV page, sec. 3):
+ * r_round = r_init - round * delta, not below 0.  Host only. */
+KVC_API float kvc_csm_ratio(float r_init, float delta, int32_t round);
+
+/* kvc_csm_workspace_size -- bytes of device workspace kvc_csm needs for B * H rows. */
+KVC_API kvc_status kvc_csm_workspace_size(int32_t B, int32_t H, int32_t N, int32_t n_sink, int32_t window,
+                                          int32_t chunk, float ratio, size_t *bytes);
+
+/*
+ * kvc_csm -- one Chunked Soft Matching round.
+ *   k, v      device, [B, H, N, D] dtype (KVC_F32 or KVC_BF16), D = 128, 16-byte aligned.
+ *   deg       device, [B, H, N] int32 degrees (>= 1), or NULL for all ones (a first round).
+ *   k_out, v_out  device, [B, H, N - m, D] dtype, written (16-byte aligned).
+ *   deg_out   device, [B, H, N - m] int32 degrees of the kept tokens, written.
+ *   pos_out   device, [B, H, N - m] int32 original positions of the kept tokens, ascending.
+ *   ws        device workspace of >= kvc_csm_workspace_size(...) bytes.
+ */
+KVC_API kvc_status kvc_csm(const void *k, const void *v, const int32_t *deg, int32_t B, int32_t H, int32_t N,
+                           int32_t D, int32_t dtype, int32_t n_sink, int32_t window, int32_t chunk, float ratio,
+                           void *k_out, void *v_out, int32_t *deg_out, int32_t *pos_out, void *workspace,
+                           size_t workspace_bytes, kvc_stream_t stream);
+
+/*
  * kvc_score_noalloc -- kvc_score for callers that cannot allocate device memory.  The
  * pages have no counterpart: it exists for engines that have already given all device
  * memory to their own pool, or plugin interfaces that forbid cudaMalloc/cudaFree during a

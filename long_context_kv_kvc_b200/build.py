@@ -16,7 +16,7 @@ INCLUDE = os.path.join(ROOT, "include")
 OBJ = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libkvc.so")
 
-SOURCES = ["api.cu", "score_simt.cu", "score_tc.cu", "select.cu", "gather.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "score_simt.cu", "score_tc.cu", "select.cu", "gather.cu", "noalloc.cu", "csm.cu"]
 HEADERS = ["kvc_internal.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

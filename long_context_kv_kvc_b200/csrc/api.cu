@@ -229,6 +229,49 @@ kvc_status kvc_row_stats(const float* scores, int32_t rows, int32_t N, int32_t n
     return KVC_OK;
 }
 
+namespace {
+kvc_status check_csm(int32_t N, int32_t D, int32_t n_sink, int32_t window, int32_t chunk, float ratio) {
+    if (N < 1 || n_sink < 0 || window < 0 || (long long)n_sink + window > N) return KVC_ERR_ARG;
+    if (chunk < 2 || chunk > 128 || chunk % 2 || !(ratio >= 0.f && ratio <= 0.5f)) return KVC_ERR_ARG;
+    if (D != kHeadDim) return KVC_ERR_UNSUPPORTED;
+    return KVC_OK;
+}
+}  // namespace
+
+int32_t kvc_csm_merges(int32_t N, int32_t n_sink, int32_t window, int32_t chunk, float ratio) {
+    if (check_csm(N, kHeadDim, n_sink, window, chunk, ratio) != KVC_OK) return -1;
+    return kvc::csm_merges(N, n_sink, window, chunk, ratio);
+}
+
+float kvc_csm_ratio(float r_init, float delta, int32_t round) {
+    const float r = r_init - (float)round * delta;
+    return r > 0.f ? r : 0.f;
+}
+
+kvc_status kvc_csm_workspace_size(int32_t B, int32_t H, int32_t N, int32_t n_sink, int32_t window, int32_t chunk,
+                                  float ratio, size_t* bytes) {
+    if (!bytes || B < 1 || H < 1) return KVC_ERR_ARG;
+    KVC_TRY(check_csm(N, kHeadDim, n_sink, window, chunk, ratio));
+    *bytes = kvc::csm_workspace(B * H, N, kvc::csm_merges(N, n_sink, window, chunk, ratio));
+    return KVC_OK;
+}
+
+kvc_status kvc_csm(const void* k, const void* v, const int32_t* deg, int32_t B, int32_t H, int32_t N, int32_t D,
+                   int32_t dtype, int32_t n_sink, int32_t window, int32_t chunk, float ratio, void* k_out, void* v_out,
+                   int32_t* deg_out, int32_t* pos_out, void* ws, size_t ws_bytes, kvc_stream_t stream) {
+    if (!k || !v || !k_out || !v_out || !deg_out || !pos_out || !ws || B < 1 || H < 1) return KVC_ERR_ARG;
+    if (dtype != KVC_F32 && dtype != KVC_BF16) return KVC_ERR_UNSUPPORTED;
+    KVC_TRY(check_csm(N, D, n_sink, window, chunk, ratio));
+    if (!aligned16(k) || !aligned16(v) || !aligned16(k_out) || !aligned16(v_out) || ((uintptr_t)ws & (kAlign - 1)))
+        return KVC_ERR_ALIGN;
+    if ((long long)B * H * N > (1LL << 31) - 1) return KVC_ERR_ARG;
+    const int m = kvc::csm_merges(N, n_sink, window, chunk, ratio);
+    if (ws_bytes < kvc::csm_workspace(B * H, N, m)) return KVC_ERR_WORKSPACE;
+    KVC_CUDA(kvc::csm(k, v, dtype, deg, B * H, N, n_sink, window, chunk, m, k_out, v_out, deg_out, pos_out, ws,
+                      (cudaStream_t)stream));
+    return KVC_OK;
+}
+
 kvc_status kvc_accumulate(float* acc, const float* src, int32_t B, int32_t Hi, int32_t Ho, int32_t N,
                           kvc_stream_t stream) {
     if (!acc || !src || B < 1 || Hi < 1 || Ho < 1 || N < 0 || Hi % Ho) return KVC_ERR_ARG;

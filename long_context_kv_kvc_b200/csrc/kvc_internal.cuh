@@ -86,4 +86,11 @@ cudaError_t gather(const void* src0, void* dst0, const void* src1, void* dst1, i
 cudaError_t row_stats(const float* scores, int rows, int N, int S, int w, const int32_t* idx, int budget,
                       float* kept_mass, float* cand_var, unsigned* err, cudaStream_t s);
 
+// CentroidKV Chunked Soft Matching (csm.cu): merges m = csm_merges(...) A tokens per row
+int csm_merges(int N, int S, int w, int chunk, float ratio);
+size_t csm_workspace(int rows, int N, int m);
+cudaError_t csm(const void* k, const void* v, int dtype, const int32_t* deg, int rows, int N, int S, int w,
+                int chunk, int m, void* k_out, void* v_out, int32_t* deg_out, int32_t* pos_out, void* ws,
+                cudaStream_t s);
+
 }  // namespace kvc

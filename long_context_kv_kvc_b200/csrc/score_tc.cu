@@ -48,6 +48,7 @@
 #include <atomic>
 
 #include "kvc_internal.cuh"
+#include "tc_ptx.cuh"
 
 namespace kvc {
 namespace {
@@ -82,11 +83,6 @@ constexpr int kConsumer0 = 8;          // first consumer warp
 constexpr int kSumCopies = KVC_TC_SUM_COPIES;  // copies of each unit's totals (CTA c adds to copy c % kSumCopies)
 constexpr int kMaxCtas = 160;                          // upper bound on the persistent grid
 constexpr uint32_t kTmemCols = 512;
-constexpr long long kBarrierTimeoutNs = 4000000000LL;  // hang guard for intra-CTA waits
-
-// tcgen05 instruction descriptor, kind::f16: fp32 accumulate (bits 4-5 = 1), A and B bf16
-// (bits 7-9, 10-12 = 1), both K-major, N = 128 (bits 17-22 = N/8), M = 128 (bits 24-28 = M/16)
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 
 struct TcArgs {
     CUtensorMap tmap_k;  // K as [U][N][128] bf16, box 64 x 128 x 1, 128-byte swizzle
@@ -125,172 +121,6 @@ struct __align__(1024) Smem {
     int abort;
     int p1_issued, p2_issued;  // tiles whose loads each producer has issued (L2 lead control)
 };
-
-// ------------------------------------------------------------------------ PTX wrappers
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ long long globaltimer() {
-    long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Bounded wait for the phase of `bar` with the given parity.  On time-out (a broken
-// pipeline, never a normal run) it records the error, puts the CTA in fail-fast mode and
-// returns, so that the kernel always terminates.
-__device__ __forceinline__ void mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, unsigned* err) {
-    if (mbar_try_wait(bar, parity)) return;
-    const long long t0 = globaltimer();
-    while (!mbar_try_wait(bar, parity)) {
-        if (*abort) return;
-        if (globaltimer() - t0 > kBarrierTimeoutNs) {
-            atomicOr(err, kErrTimeout);
-            *abort = 1;
-            return;
-        }
-    }
-}
-
-// Bounded wait until the shared counter *c (written by other warps of the CTA) reaches v.
-__device__ __forceinline__ void spin_until_at_least(int* c, int v, volatile int* abort, unsigned* err) {
-    volatile int* vc = c;
-    if (*vc >= v) return;
-    const long long t0 = globaltimer();
-    while (*vc < v) {
-        if (*abort) return;
-        if (globaltimer() - t0 > kBarrierTimeoutNs) {
-            atomicOr(err, kErrTimeout);
-            *abort = 1;
-            return;
-        }
-    }
-    __threadfence_block();
-}
-
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
-                                            int z) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
-        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
-        : "memory");
-}
-
-// Same, with an L2 eviction-policy hint (a createpolicy value).
-__device__ __forceinline__ void tma_load_3d_hint(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
-                                                 int z, uint64_t policy) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1, {%3, %4, %5}], [%2], %6;"
-        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z),
-          "l"(policy)
-        : "memory");
-}
-
-__device__ __forceinline__ uint64_t policy_evict_first() {
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
-        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
-        : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// Shared-memory matrix descriptor for a K-major operand in the 128-byte swizzled layout
-// that TMA writes: rows of 128 bytes, 8-row (1024-byte) swizzle atoms stacked along M/N.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-    uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);  // start address
-    d |= (uint64_t)1u << 16;                          // leading-dimension offset (unused here)
-    d |= (uint64_t)(1024u >> 4) << 32;                // stride between 8-row atoms
-    d |= (uint64_t)1u << 46;                          // descriptor version (sm_100)
-    d |= (uint64_t)2u << 61;                          // 128-byte swizzle
-    return d;
-}
-
-template <int ACC>
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(a), "l"(b), "r"(kIdesc), "n"(ACC)
-        : "memory");
-}
-
-// The 8 MMAs (K = 128 in slices of 16) of one 128 x 128 x 128 product; the operands are the
-// two 64-column halves (h) of A and B, given as descriptors of half 0 and the half stride.
-__device__ __forceinline__ void umma_half(uint32_t d, uint64_t a, uint64_t b, int h) {
-    if (h == 0) umma_bf16<0>(d, a, b);
-    else umma_bf16<1>(d, a, b);
-    umma_bf16<1>(d, a + 2, b + 2);
-    umma_bf16<1>(d, a + 4, b + 4);
-    umma_bf16<1>(d, a + 6, b + 6);
-}
-
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
-}
-
-// 32 consecutive fp32 columns of this thread's TMEM lane (one tcgen05.ld).  The values are
-// only valid after tmem_wait32, which takes them as in/out operands so that no use can be
-// scheduled before the wait.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {"
-        "%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31"
-        "}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr)
-        : "memory");
-}
-
-__device__ __forceinline__ void tmem_wait32(uint32_t (&r)[32]) {
-    asm volatile("tcgen05.wait::ld.sync.aligned;"
-                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
-                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
-                   "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
-                   "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
-                 :
-                 : "memory");
-}
 
 __device__ __forceinline__ float ex2(float x) {
     float y;
@@ -933,6 +763,8 @@ TcLayout tc_layout(int U) {
     return L;
 }
 
+}  // namespace
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static std::atomic<void*> fn{nullptr};
     void* f = fn.load();
@@ -956,8 +788,6 @@ int sm_count() {
     if (dev < 64) cache[dev].store(n);
     return n;
 }
-
-}  // namespace
 
 bool tc_score_supported(const ScoreJob& j) {
     return j.dtype == KVC_BF16 && j.nq >= 1 && j.nq <= kQRows && j.N >= 1 && j.U >= 1 &&

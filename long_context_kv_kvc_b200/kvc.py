@@ -25,7 +25,7 @@ KVC_STAGE_SCORE, KVC_STAGE_SELECT, KVC_STAGE_GATHER, KVC_STAGE_COUNT = 0, 1, 2, 
 EXPORTED = ("kvc_workspace_size", "kvc_score", "kvc_accumulate", "kvc_pool", "kvc_topk_workspace_size",
             "kvc_topk", "kvc_gather", "kvc_compress", "kvc_tsp_count", "kvc_poll_error",
             "kvc_status_string", "kvc_version", "kvc_launch_count", "kvc_score_noalloc", "kvc_score_entropy",
-            "kvc_row_stats")
+            "kvc_row_stats", "kvc_csm_merges", "kvc_csm_ratio", "kvc_csm_workspace_size", "kvc_csm")
 
 
 class KvcError(RuntimeError):
@@ -67,6 +67,11 @@ def _load():
         "kvc_score_noalloc": (st, [P, vp, vp, vp, vp]),
         "kvc_score_entropy": (st, [P, vp, vp, vp, vp, vp, sz, vp]),
         "kvc_row_stats": (st, [vp, i32, i32, i32, i32, vp, i32, vp, vp, vp]),
+        "kvc_csm_merges": (i32, [i32, i32, i32, i32, ctypes.c_float]),
+        "kvc_csm_ratio": (ctypes.c_float, [ctypes.c_float, ctypes.c_float, i32]),
+        "kvc_csm_workspace_size": (st, [i32, i32, i32, i32, i32, i32, ctypes.c_float, ctypes.POINTER(sz)]),
+        "kvc_csm": (st, [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, ctypes.c_float, vp, vp, vp, vp, vp, sz,
+                         vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -166,6 +171,39 @@ def kvc_row_stats(scores, n_sink, window, cand_var, idx=None, kept_mass=None, st
     _check(lib.kvc_row_stats(_ptr(scores), rows, N, n_sink, window, _ptr(idx) if idx is not None else None,
                              budget, _ptr(kept_mass) if kept_mass is not None else None, _ptr(cand_var),
                              _stream(stream)), "kvc_row_stats")
+
+
+def kvc_csm_merges(N, n_sink, window, chunk, ratio) -> int:
+    m = int(lib.kvc_csm_merges(N, n_sink, window, chunk, ratio))
+    if m < 0:
+        raise KvcError(KVC_ERR_ARG, "kvc_csm_merges: invalid arguments")
+    return m
+
+
+def kvc_csm_ratio(r_init, delta, round_) -> float:
+    return float(lib.kvc_csm_ratio(r_init, delta, round_))
+
+
+def kvc_csm(k, v, n_sink, window, chunk, ratio, deg=None, out=None, ws=None, stream=None) -> dict:
+    """One Chunked Soft Matching round over k, v [B, H, N, D]; returns (and fills, when given
+    as `out`) k_out, v_out [B, H, N - m, D], deg_out and pos_out [B, H, N - m]."""
+    B, H, N, D = k.shape
+    dt = KVC_BF16 if k.dtype == torch.bfloat16 else KVC_F32
+    m = kvc_csm_merges(N, n_sink, window, chunk, ratio)
+    if out is None:
+        out = {"k_out": torch.empty((B, H, N - m, D), dtype=k.dtype, device=k.device),
+               "v_out": torch.empty((B, H, N - m, D), dtype=k.dtype, device=k.device),
+               "deg_out": torch.empty((B, H, N - m), dtype=torch.int32, device=k.device),
+               "pos_out": torch.empty((B, H, N - m), dtype=torch.int32, device=k.device)}
+    if ws is None:
+        n = ctypes.c_size_t(0)
+        _check(lib.kvc_csm_workspace_size(B, H, N, n_sink, window, chunk, ratio, ctypes.byref(n)),
+               "kvc_csm_workspace_size")
+        ws = torch.empty(max(n.value, 256), dtype=torch.uint8, device=k.device)
+    _check(lib.kvc_csm(_ptr(k), _ptr(v), _ptr(deg) if deg is not None else None, B, H, N, D, dt, n_sink, window,
+                       chunk, ratio, _ptr(out["k_out"]), _ptr(out["v_out"]), _ptr(out["deg_out"]),
+                       _ptr(out["pos_out"]), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "kvc_csm")
+    return out
 
 
 def kvc_accumulate(acc, src, stream=None):

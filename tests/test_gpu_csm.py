@@ -1,0 +1,190 @@
+"""Parity of Chunked Soft Matching (kvc_csm) through the C ABI with the fp64 oracle.
+
+Cosine similarities are fp32 on the GPU and fp64 in the oracle, so the decisions they take
+follow the band rule used for the top-k: a match whose oracle similarity is clearly above
+(below) the m-th best must (must not) merge; only matches within 1e-5 of it may differ.
+Given the GPU's merge set, every kept row must equal the oracle's degree-weighted mean of
+the same tokens up to fp32 summation error (2e-6 of the summands' magnitude) plus, for bf16
+outputs, one unit in the last place; every unmerged row must be a bit-exact copy, and
+degrees and positions must be exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+
+pytestmark = pytest.mark.gpu
+
+BAND = 1e-5
+
+
+@pytest.fixture(scope="module")
+def K():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from long_context_kv_kvc_b200 import build
+    build.build()
+    from long_context_kv_kvc_b200 import kvc
+    torch.cuda.set_device(0)
+    return kvc
+
+
+def make_kv(B, H, N, dtype, seed, dup=0, zero=0):
+    g = torch.Generator().manual_seed(seed)
+    k = torch.randn(B, H, N, 128, generator=g)
+    v = torch.randn(B, H, N, 128, generator=g)
+    if dup:
+        # planted near-duplicates: some tokens repeat their left neighbour's key direction
+        idx = torch.randint(1, N - 1, (dup,), generator=g)
+        k[:, :, idx] = 1.5 * k[:, :, idx - 1]
+    if zero:
+        # zero keys: similarity 0 with every token
+        k[:, :, torch.randint(0, N, (zero,), generator=g)] = 0.0
+    return k.to(dtype), v.to(dtype)
+
+
+def check_row(kr, vr, dr, out_k, out_v, out_d, out_p, S, w, chunk, ratio, dtype):
+    """One row: band rule on the merge set, then the kept rows given the GPU's merges."""
+    N = kr.shape[0]
+    ref = O.csm(kr, vr, dr, n_sink=S, window=w, chunk=chunk, ratio=ratio)
+    m = ref["m"]
+    pos = np.asarray(out_p, dtype=np.int64)
+    assert pos.size == N - m and np.all(np.diff(pos) > 0)
+    is_merged = np.ones(N, dtype=bool)
+    is_merged[pos] = False
+    merged = np.nonzero(is_merged)[0]
+    assert merged.size == m
+    sim, best = ref["sim"], ref["best"]
+    assert np.all(best[merged] >= 0), "a token without a match was merged"
+    if m:
+        T = np.sort(sim[best >= 0])[::-1][m - 1]
+        must = (best >= 0) & (sim > T + BAND)
+        mustnot = (best >= 0) & (sim < T - BAND)
+        assert not np.any(must & ~is_merged), f"{int((must & ~is_merged).sum())} clearly better matches not merged"
+        assert not np.any(mustnot & is_merged), "clearly worse matches merged"
+    # the B token each merged A joins: the best match in fp64, unless the runner-up is within
+    # the band (then neither candidate row is checked)
+    kk, vv = kr.double().numpy(), vr.double().numpy()
+    nrm = np.linalg.norm(kk, axis=1)
+    unit = np.divide(kk, nrm[:, None], out=np.zeros_like(kk), where=nrm[:, None] > 0)
+    owner = np.full(N, -1, dtype=np.int64)
+    ambiguous = np.zeros(N, dtype=bool)
+    for c0 in range(S, N - w, chunk):
+        c1 = min(c0 + chunk, N - w)
+        A = np.arange(c0, c1, 2)
+        Bs = np.arange(c0 + 1, c1, 2)
+        A = A[is_merged[A]]
+        if A.size == 0 or Bs.size == 0:
+            continue
+        sm = unit[A] @ unit[Bs].T
+        order = np.argsort(-sm, axis=1, kind="stable")
+        owner[A] = Bs[order[:, 0]]
+        if Bs.size > 1:
+            gap = sm[np.arange(A.size), order[:, 0]] - sm[np.arange(A.size), order[:, 1]]
+            close = gap < BAND
+            ambiguous[Bs[order[close, 0]]] = True
+            ambiguous[Bs[order[close, 1]]] = True
+    # expected rows of the kept tokens: degree-weighted sums over the token and its absorbed ones
+    d = np.asarray(dr, dtype=np.float64)
+    n = d.copy()
+    sk, sv = d[:, None] * kk, d[:, None] * vv
+    ak, av = np.abs(sk), np.abs(sv)  # magnitude of the summands: the scale of the rounding error
+    src = merged
+    np.add.at(n, owner[src], d[src])
+    np.add.at(sk, owner[src], d[src, None] * kk[src])
+    np.add.at(sv, owner[src], d[src, None] * vv[src])
+    np.add.at(ak, owner[src], d[src, None] * np.abs(kk[src]))
+    np.add.at(av, owner[src], d[src, None] * np.abs(vv[src]))
+    has = np.zeros(N, dtype=bool)
+    has[owner[src]] = True
+    check = ~ambiguous[pos]
+    np.testing.assert_array_equal(np.asarray(out_d)[check], n[pos][check].astype(np.int64))
+    single = check & ~has[pos]
+    assert torch.equal(out_k[torch.from_numpy(single)], kr[torch.from_numpy(pos[single])]), "unmerged rows not copied"
+    assert torch.equal(out_v[torch.from_numpy(single)], vr[torch.from_numpy(pos[single])]), "unmerged rows not copied"
+    multi = check & has[pos]
+    tol = 2.0 ** -7 if dtype == torch.bfloat16 else 2e-6
+    for s_, a_, got in ((sk, ak, out_k), (sv, av, out_v)):
+        want = s_[pos[multi]] / n[pos[multi], None]
+        scale = a_[pos[multi]] / n[pos[multi], None]
+        g = got[torch.from_numpy(multi)].double().numpy()
+        err = np.abs(g - want)
+        # fp32 sums: error below ~2^-23 of the summands' magnitude; bf16 adds half a unit of
+        # the result's last place
+        bound = 2e-6 * scale + (tol * np.abs(want) if dtype == torch.bfloat16 else 0.0) + 1e-30
+        assert np.all(err <= bound), f"merged rows off by {(err / np.maximum(scale, 1e-30)).max():.2e} of their scale"
+
+
+# bf16 keys take the tensor-core match (128-token tiles holding whole chunks: 128 for chunk
+# 2, 64 and 128, 126 for chunk 6, 96 for chunk 48), fp32 keys the CUDA-core one
+CASES = [
+    dict(B=1, H=2, N=1000, S=1, w=32, chunk=64, ratio=0.25, dtype=torch.bfloat16, deg=False, dup=40, zero=0),
+    dict(B=2, H=1, N=777, S=0, w=0, chunk=2, ratio=0.5, dtype=torch.float32, deg=True, dup=0, zero=0),
+    dict(B=1, H=3, N=2053, S=4, w=16, chunk=128, ratio=0.1, dtype=torch.bfloat16, deg=True, dup=100, zero=0),
+    dict(B=1, H=1, N=515, S=1, w=3, chunk=6, ratio=0.45, dtype=torch.float32, deg=False, dup=20, zero=6),
+    dict(B=1, H=2, N=700, S=3, w=5, chunk=6, ratio=0.3, dtype=torch.bfloat16, deg=True, dup=30, zero=8),
+    dict(B=2, H=1, N=1500, S=0, w=0, chunk=48, ratio=0.2, dtype=torch.bfloat16, deg=False, dup=50, zero=0),
+    dict(B=1, H=1, N=401, S=2, w=7, chunk=2, ratio=0.5, dtype=torch.bfloat16, deg=True, dup=0, zero=0),
+    dict(B=1, H=1, N=300, S=130, w=140, chunk=16, ratio=0.5, dtype=torch.bfloat16, deg=False, dup=5, zero=0),
+]
+
+
+@pytest.mark.parametrize("case", range(len(CASES)))
+def test_csm_matches_oracle(K, case):
+    c = CASES[case]
+    B, H, N = c["B"], c["H"], c["N"]
+    k, v = make_kv(B, H, N, c["dtype"], 30 + case, dup=c["dup"], zero=c["zero"])
+    deg = (torch.randint(1, 6, (B, H, N), generator=torch.Generator().manual_seed(case), dtype=torch.int32)
+           if c["deg"] else torch.ones((B, H, N), dtype=torch.int32))
+    out = K.kvc_csm(k.cuda(), v.cuda(), c["S"], c["w"], c["chunk"], c["ratio"],
+                    deg=deg.cuda() if c["deg"] else None)
+    assert K.kvc_poll_error() == K.KVC_OK
+    for b in range(B):
+        for h in range(H):
+            check_row(k[b, h], v[b, h], deg[b, h].numpy(), out["k_out"][b, h].cpu(), out["v_out"][b, h].cpu(),
+                      out["deg_out"][b, h].cpu().numpy(), out["pos_out"][b, h].cpu().numpy(), c["S"], c["w"],
+                      c["chunk"], c["ratio"], c["dtype"])
+
+
+def test_csm_identity_and_arguments(K):
+    k, v = make_kv(1, 2, 300, torch.bfloat16, 7)
+    out = K.kvc_csm(k.cuda(), v.cuda(), 1, 8, 16, 0.0)
+    assert torch.equal(out["k_out"].cpu(), k) and torch.equal(out["v_out"].cpu(), v)
+    assert torch.equal(out["pos_out"].cpu(), torch.arange(300, dtype=torch.int32).expand(1, 2, 300))
+    assert torch.all(out["deg_out"] == 1)
+    assert K.kvc_csm_merges(10, 1, 2, 4, 0.5) == O.csm_merges(10, 1, 2, 4, 0.5) == 3
+    assert K.kvc_csm_merges(9, 0, 0, 4, 0.5) == O.csm_merges(9, 0, 0, 4, 0.5) == 4
+    assert K.kvc_csm_ratio(0.5, 0.1, 2) == pytest.approx(O.csm_ratio(0.5, 0.1, 2))
+    for bad in [dict(chunk=3), dict(chunk=130), dict(ratio=0.6)]:
+        a = dict(chunk=16, ratio=0.25)
+        a.update(bad)
+        with pytest.raises(K.KvcError):
+            K.kvc_csm(k.cuda(), v.cuda(), 1, 8, a["chunk"], a["ratio"])
+    assert K.kvc_poll_error() == K.KVC_OK
+
+
+def test_csm_full_size_128k_batch4(K):
+    """The 8B shape at 128K x 4 (bf16 K and V, 32 rows): invariants on every row, the band
+    rule and the kept rows against the oracle on two sampled rows."""
+    B, H, N, S, w, chunk, ratio = 4, 8, 131072, 1, 32, 64, 0.25
+    k, v = make_kv(B, H, N, torch.bfloat16, 99, dup=2000)
+    kd, vd = k.cuda(), v.cuda()
+    out = K.kvc_csm(kd, vd, S, w, chunk, ratio)
+    assert K.kvc_poll_error() == K.KVC_OK
+    m = O.csm_merges(N, S, w, chunk, ratio)
+    n_out = N - m
+    pos = out["pos_out"]
+    assert pos.shape == (B, H, n_out)
+    assert torch.all(pos[..., 1:] > pos[..., :-1])
+    assert torch.all(out["deg_out"].sum(dim=-1) == N)
+    assert torch.all(pos[..., :S] == torch.arange(S, device="cuda"))
+    assert torch.all(pos[..., -w:] == torch.arange(N - w, N, device="cuda", dtype=torch.int32))
+    # rows of degree 1 are exact copies of their source rows
+    single = out["deg_out"] == 1
+    src = torch.gather(kd, 2, pos.long().unsqueeze(-1).expand(-1, -1, -1, 128))
+    assert torch.equal(out["k_out"][single], src[single])
+    for b, h in [(0, 0), (3, 7)]:
+        check_row(k[b, h], v[b, h], np.ones(N, np.int32), out["k_out"][b, h].cpu(), out["v_out"][b, h].cpu(),
+                  out["deg_out"][b, h].cpu().numpy(), out["pos_out"][b, h].cpu().numpy(), S, w, chunk, ratio,
+                  torch.bfloat16)
