@@ -343,8 +343,9 @@ def main():
     ab = algorithmic_bytes(wl)
     peak, peak_kind = measured_peaks()
     achieved = ab["score"] / (score_ms / 1e3) / 1e9
-    digest = source_digest("score_tc.cu" if not (args.flags & 1) and wl.dtype == "bf16" else "score_simt.cu")
-    kernel_name = "score_tc" if not (args.flags & 1) and wl.dtype == "bf16" else "score_simt"
+    tc_path = not (args.flags & 1) and wl.dtype == "bf16"
+    digest = source_digest("score_tc.cu", "tc_ptx.cuh") if tc_path else source_digest("score_simt.cu")
+    kernel_name = "score_tc" if tc_path else "score_simt"
     traffic = recorded_traffic(kernel_name, wl.name, digest)
 
     # end to end through the public API: pinned host inputs -> device -> compact cache -> host

@@ -22,10 +22,11 @@
 //   2. the m best matches per row: the radix top-k over a row of match scores (-inf where
 //      there is no match), then merge flags and per-chunk merge counts, and a per-row scan
 //      of the kept tokens per chunk that gives every chunk its first output slot;
-//   3. write: one CTA per chunk (or per 128 sink / window tokens) stages the chunk's merged
-//      A rows in shared memory, then streams every kept row with all of its loads in flight,
-//      forming the merged means in fp32 (rounded once to the element type) and copying every
-//      other row bit for bit.
+//   3. write: one CTA per chunk (or per 128 sink / window tokens) brings the block's K and V
+//      rows into shared memory with two bulk copies (a block's rows are contiguous), forms
+//      the merged means there in fp32 (rounded once to the element type), and sends every
+//      run of consecutive kept rows to its output slots with one bulk store per tensor;
+//      every other row is thus copied bit for bit.
 #include <math.h>
 
 #include <algorithm>
@@ -41,35 +42,26 @@ constexpr int D = kHeadDim;
 constexpr int kMatchThreads = 256;
 constexpr int kKS = D + 4;  // shared-memory row stride of a staged fp32 key (16-byte aligned rows)
 constexpr int kScanThreads = 1024;
-constexpr int kWriteThreads = 256;
+constexpr int kWriteThreads = 128;  // one thread per token of a block
 constexpr int kSeg = 128;  // sink / window tokens per write CTA
 
 // tensor-core match
 constexpr int kTileTok = 128;                // Gram tile: MMA M = N = 128 tokens, K = 128 dimensions
 constexpr int kHalfBytes = kTileTok * 64 * 2;  // one 64-dimension half of a tile: 16 KiB
 constexpr int kTcStages = 5;
-constexpr int kTcThreads = 6 * 32;           // warp 0 TMA, 1 MMA + TMEM owner, 2-5 epilogue
+constexpr int kTcAcc = 4;                    // TMEM accumulators = epilogue warpgroups
+constexpr int kTcThreads = (2 + 4 * kTcAcc) * 32;  // warp 0 TMA, 1 MMA + TMEM owner, 2.. epilogue
 constexpr int kTcMaxCtas = 160;
-constexpr uint32_t kTcCols = 256;            // two 128-column accumulators
+constexpr uint32_t kTcCols = 128 * kTcAcc;
 
 // ------------------------------------------------------------------------ row pieces
-// A lane moves 8 elements of a row: one 16-byte vector for bf16, two for fp32.
+// A lane handles 8 elements of a row: one 16-byte vector for bf16, two for fp32.
 
 template <typename T>
 struct Vec {
     static constexpr int n = sizeof(T) / 2;
 };
 
-template <typename T>
-__device__ __forceinline__ void ld_piece(const T* p, uint4 (&r)[Vec<T>::n]) {
-#pragma unroll
-    for (int i = 0; i < Vec<T>::n; ++i) r[i] = __ldcs(reinterpret_cast<const uint4*>(p) + i);
-}
-template <typename T>
-__device__ __forceinline__ void st_piece(T* p, const uint4 (&r)[Vec<T>::n]) {
-#pragma unroll
-    for (int i = 0; i < Vec<T>::n; ++i) reinterpret_cast<uint4*>(p)[i] = r[i];
-}
 __device__ __forceinline__ void to_f8(const uint4 (&r)[1], float (&x)[8]) {
     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&r[0]);
 #pragma unroll
@@ -210,8 +202,8 @@ struct TcMatchArgs {
 
 struct __align__(1024) MatchSmem {
     uint8_t ring[kTcStages][2][kHalfBytes];  // a tile = two 64-dimension halves
-    float inv[2][kTileTok];                  // 1/|k| of the tile's tokens, double-buffered by tile
-    uint64_t full[kTcStages], empty[kTcStages], accfull[2], accempty[2];
+    float inv[kTcAcc][2][kTileTok];          // per warpgroup: 1/|k| of the tile's tokens, double-buffered
+    uint64_t full[kTcStages], empty[kTcStages], accfull[kTcAcc], accempty[kTcAcc];
     uint32_t tmem_base;
     int abort;
 };
@@ -243,7 +235,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) csm_match_tc_kernel(const __gri
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kTcAcc; ++i) {
             mbar_init(&sm.accfull[i], 1);
             mbar_init(&sm.accempty[i], 4);
         }
@@ -287,9 +279,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) csm_match_tc_kernel(const __gri
         if (lane == 0) {
             int last = -1;
             for (int i = 0; i < n_local && !*abort; ++i) {
-                const int s = i % kTcStages, acc = i & 1;
+                const int s = i % kTcStages, acc = i % kTcAcc;
                 mbar_wait(&sm.full[s], (i / kTcStages) & 1, abort, a.err);
-                mbar_wait(&sm.accempty[acc], ((i >> 1) & 1) ^ 1, abort, a.err);
+                mbar_wait(&sm.accempty[acc], ((i / kTcAcc) & 1) ^ 1, abort, a.err);
                 if (*abort) break;
                 tc_fence_after();
                 const uint32_t d = tmem + acc * kTileTok;
@@ -301,36 +293,44 @@ __global__ void __launch_bounds__(kTcThreads, 1) csm_match_tc_kernel(const __gri
                 last = i;
             }
             // the last products have completed before TMEM is released
-            if (last >= 0) mbar_drain(&sm.accfull[last & 1], (last >> 1) & 1, a.err);
+            if (last >= 0) mbar_drain(&sm.accfull[last % kTcAcc], (last / kTcAcc) & 1, a.err);
         }
     } else {
-        // ------------------------------------------------------------ epilogue (warps 2-5)
-        // Thread r = TMEM lane = the tile's token r.  Every warp runs every iteration (the
-        // waits return at once after an abort), so the named barrier always sees all four.
-        const int qd = warp & 3;
+        // ------------------------------------------------------------ epilogue
+        // Warpgroup g (warps 2 + 4g .. 5 + 4g) takes the tiles i = g, g + 4, ... from
+        // accumulator g.  Thread r = TMEM lane = the tile's token r.  Every warp of a group
+        // runs every one of its iterations (the waits return at once after an abort), so
+        // the group's named barrier always sees all four warps.
+        const int grp = (warp - 2) >> 2, qd = warp & 3;
         const int r = 32 * qd + lane;
-        const uint32_t lane_base = tmem + ((uint32_t)(32 * qd) << 16);
-        for (int i = 0; i < n_local; ++i) {
+        const uint32_t lane_base = tmem + ((uint32_t)(32 * qd) << 16) + grp * kTileTok;
+        for (int i = grp, it = 0; i < n_local; i += kTcAcc, ++it) {
             const int g = cta + i * P;
             const int u = g / a.tiles_per_row, tau = g - u * a.tiles_per_row;
             const int t0 = a.S + tau * a.tt;
             const int valid = min(a.tt, a.N - a.w - t0);
-            const int acc = i & 1;
-            mbar_wait(&sm.accfull[acc], (i >> 1) & 1, abort, a.err);
+            mbar_wait(&sm.accfull[grp], it & 1, abort, a.err);
             tc_fence_after();
-            const uint32_t tl = lane_base + acc * kTileTok;
-            uint32_t x[32];
-            // the diagonal: this thread's column r sits in column block qd, register lane
-            tmem_ld32(tl + 32 * qd, x);
+            uint32_t x[32], y[32];
+            // the diagonal: this thread's column r sits in column block qd, register `lane`
+            // (a select tree over the lane's bits)
+            tmem_ld32(lane_base + 32 * qd, x);
             tmem_wait32(x);
-            float gd = 0.f;
+            float v16[16];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) gd = e == lane ? __uint_as_float(x[e]) : gd;
-            float* inv = sm.inv[i & 1];
+            for (int e = 0; e < 16; ++e) v16[e] = __uint_as_float((lane & 1) ? x[2 * e + 1] : x[2 * e]);
+#pragma unroll
+            for (int lv = 1; lv < 5; ++lv) {
+#pragma unroll
+                for (int e = 0; e < (16 >> lv); ++e) v16[e] = ((lane >> lv) & 1) ? v16[2 * e + 1] : v16[2 * e];
+            }
+            const float gd = v16[0];
+            float* inv = sm.inv[grp][it & 1];
             inv[r] = gd > 0.f ? rsqrtf(gd) : 0.f;
-            asm volatile("bar.sync 1, 128;" ::: "memory");
+            asm volatile("bar.sync %0, 128;" ::"r"(1 + grp) : "memory");
             // A tokens (even offsets of a chunk): argmax over the chunk's B columns (odd
-            // offsets; chunk starts are even), ascending so that ties keep the lower column
+            // offsets; chunk starts are even), ascending so that ties keep the lower column.
+            // Column blocks come in pairs with one comparison chain each.
             const int cs = (r / a.chunk) * a.chunk, ce = min(cs + a.chunk, valid);
             const bool is_a = r < valid && ((r - cs) & 1) == 0;
             const float ir = inv[r];
@@ -338,25 +338,44 @@ __global__ void __launch_bounds__(kTcThreads, 1) csm_match_tc_kernel(const __gri
             int bb = -1;
             const int r_lo = 32 * qd, r_hi = min(32 * qd + 31, valid - 1);
             if (r_lo <= r_hi) {
-                const int col_lo = (r_lo / a.chunk) * a.chunk;
-                const int col_hi = min((r_hi / a.chunk) * a.chunk + a.chunk, valid);
-                for (int cb = col_lo >> 5; cb * 32 < col_hi; ++cb) {
-                    tmem_ld32(tl + 32 * cb, x);
+                const int cb_lo = ((r_lo / a.chunk) * a.chunk) >> 5;
+                const int cb_hi = (min((r_hi / a.chunk) * a.chunk + a.chunk, valid) + 31) >> 5;  // exclusive
+                for (int cb = cb_lo; cb < cb_hi; cb += 2) {
+                    const bool two = cb + 1 < cb_hi;
+                    tmem_ld32(lane_base + 32 * cb, x);
+                    if (two) tmem_ld32(lane_base + 32 * (cb + 1), y);
                     tmem_wait32(x);
+                    if (two) tmem_wait32(y);
+                    float s0 = -INFINITY, s1 = -INFINITY;
+                    int b0 = -1, b1 = -1;
 #pragma unroll
                     for (int e = 1; e < 32; e += 2) {
-                        const int j = 32 * cb + e;
-                        const float sv = __uint_as_float(x[e]) * ir * inv[j];
-                        if (is_a && j > cs && j < ce && (bb < 0 || sv > bs)) {
-                            bs = sv;
-                            bb = j;
+                        const int j0 = 32 * cb + e, j1 = j0 + 32;
+                        const float v0 = __uint_as_float(x[e]) * ir * inv[j0];
+                        const float v1 = __uint_as_float(y[e]) * ir * inv[two ? j1 : j0];
+                        if (j0 > cs && j0 < ce && (b0 < 0 || v0 > s0)) {
+                            s0 = v0;
+                            b0 = j0;
                         }
+                        if (two && j1 > cs && j1 < ce && (b1 < 0 || v1 > s1)) {
+                            s1 = v1;
+                            b1 = j1;
+                        }
+                    }
+                    // merge: the earlier (lower) columns win ties
+                    if (b1 >= 0 && (b0 < 0 || s1 > s0)) {
+                        s0 = s1;
+                        b0 = b1;
+                    }
+                    if (b0 >= 0 && (bb < 0 || s0 > bs)) {
+                        bs = s0;
+                        bb = b0;
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.accempty[acc]);
+            if (lane == 0) mbar_arrive(&sm.accempty[grp]);
             float* sr = a.score + (size_t)u * a.N;
             if (r < valid) {
                 sr[t0 + r] = is_a && bb >= 0 ? bs : -INFINITY;
@@ -431,9 +450,23 @@ csm_base_kernel(int N, int S, int w, int chunk, int n_chunks, int32_t* __restric
 
 // ------------------------------------------------------------------------ write
 
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(dst)), "l"((uint64_t)__cvta_generic_to_global(src)), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 ::"l"((uint64_t)__cvta_generic_to_global(dst)), "r"(smem_u32(src)), "r"(bytes)
+                 : "memory");
+}
+
 // blockIdx.x = row * n_blk + b: b < n_chunks is chunk b, then ceil(S / 128) sink segments,
-// then ceil(w / 128) window segments.  Lane l of a warp moves elements 8 (l % 16) .. +7 of
-// the K row (lanes 0-15) or the V row (lanes 16-31); a warp handles rows warp, warp + 8, ...
+// then ceil(w / 128) window segments.  A block's K and V rows are contiguous in HBM: two
+// bulk copies bring them into shared memory while the merge flags load; merged means are
+// formed in place (a warp per B token: lanes 0-15 its K row, 16-31 its V row, 8 elements
+// each); every run of consecutive kept rows then leaves with one bulk store per tensor
+// (consecutive kept rows have consecutive output slots).
 template <typename T>
 __global__ void __launch_bounds__(kWriteThreads)
 csm_write_kernel(const T* __restrict__ k, const T* __restrict__ v, const int32_t* __restrict__ deg, int N, int S,
@@ -442,12 +475,13 @@ csm_write_kernel(const T* __restrict__ k, const T* __restrict__ v, const int32_t
                  T* __restrict__ k_out, T* __restrict__ v_out, int32_t* __restrict__ deg_out,
                  int32_t* __restrict__ pos_out, unsigned* __restrict__ err) {
     constexpr int V = Vec<T>::n;
-    constexpr int R = 8 / V;                       // rows in flight per warp
-    extern __shared__ __align__(16) uint4 stage[];  // [chunk / 2][32 lanes][V]: the merged A rows
+    extern __shared__ __align__(128) uint8_t wsm[];  // K rows, then V rows, of this block
+    __shared__ uint64_t bar;
+    __shared__ int failed;
     __shared__ unsigned char mg[128];
     __shared__ int32_t dg[128], ns[128];
-    __shared__ uint32_t amask[64][2];              // per B token (offset / 2): its merged A tokens (offset / 2)
-    __shared__ uint32_t mword[4];                  // merged flags, 32 tokens per word
+    __shared__ uint32_t amask[64][2];  // per B token (offset / 2): its merged A tokens (offset / 2)
+    __shared__ uint32_t mword[4];      // merged flags, 32 tokens per word
     const int row = blockIdx.x / n_blk, b = blockIdx.x - row * n_blk;
     const int hi = N - w;
     const int n_sblk = (S + kSeg - 1) / kSeg;
@@ -470,16 +504,25 @@ csm_write_kernel(const T* __restrict__ k, const T* __restrict__ v, const int32_t
     }
     const size_t rN = (size_t)row * N;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t tensor_bytes = (uint32_t)n * D * sizeof(T);
+    T* sk = reinterpret_cast<T*>(wsm);
+    T* sv = sk + (size_t)n * D;
 
-    if (tid < 128) {
-        amask[tid >> 1][tid & 1] = 0u;
-        if (tid < n) {
-            mg[tid] = in_c ? merged[rN + p0 + tid] : 0;
-            dg[tid] = deg ? deg[rN + p0 + tid] : 1;
-        }
+    if (tid == 0) {
+        failed = 0;
+        mbar_init(&bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        mbar_expect_tx(&bar, 2 * tensor_bytes);
+        bulk_load(sk, k + (rN + p0) * D, tensor_bytes, &bar);
+        bulk_load(sv, v + (rN + p0) * D, tensor_bytes, &bar);
+    }
+    amask[tid >> 1][tid & 1] = 0u;
+    if (tid < n) {
+        mg[tid] = in_c ? merged[rN + p0 + tid] : 0;
+        dg[tid] = deg ? deg[rN + p0 + tid] : 1;
     }
     __syncthreads();
-    if (tid < 128) {
+    {
         const bool m = tid < n && mg[tid];
         const unsigned bits = __ballot_sync(0xffffffffu, m);
         if (lane == 0) mword[warp] = bits;
@@ -510,72 +553,71 @@ csm_write_kernel(const T* __restrict__ k, const T* __restrict__ v, const int32_t
         deg_out[o] = nsum;
         pos_out[o] = p0 + tid;
     }
-    const T* src = (lane < 16 ? k : v) + rN * D + 8 * (lane & 15);
-    T* dst = (lane < 16 ? k_out : v_out) + (size_t)row * n_out * D + 8 * (lane & 15);
-    // pass 1: merged A rows into shared memory
-    if (in_c) {
-        for (int t0 = warp; t0 < n; t0 += 8 * R) {
-            uint4 raw[R][V];
-#pragma unroll
-            for (int i = 0; i < R; ++i) {
-                const int t = t0 + 8 * i;
-                if (t < n && mg[t]) ld_piece(src + (size_t)(p0 + t) * D, raw[i]);
-            }
-#pragma unroll
-            for (int i = 0; i < R; ++i) {
-                const int t = t0 + 8 * i;
-                if (t < n && mg[t]) {
-#pragma unroll
-                    for (int j = 0; j < V; ++j) stage[((t >> 1) * 32 + lane) * V + j] = raw[i][j];
-                }
+    // the rows have landed (bounded wait; a copy that never lands is reported, not used)
+    if (!mbar_try_wait(&bar, 0)) {
+        const long long t0 = globaltimer();
+        while (!mbar_try_wait(&bar, 0)) {
+            if (globaltimer() - t0 > kBarrierTimeoutNs) {
+                atomicOr(err, kErrTimeout);
+                failed = 1;
+                break;
             }
         }
     }
     __syncthreads();
-    // pass 2: every kept row
-    for (int t0 = warp; t0 < n; t0 += 8 * R) {
-        uint4 raw[R][V];
+    if (failed) return;
+    // merged means in place: the B row first, then its A rows by position, in fp32
+    for (int t = 2 * warp + 1; t < n; t += 2 * (kWriteThreads / 32)) {
+        const uint32_t m0 = amask[t >> 1][0], m1 = amask[t >> 1][1];
+        if (!(m0 | m1)) continue;
+        T* base = (lane < 16 ? sk : sv) + 8 * (lane & 15);
+        uint4 r[V];
+        float acc[8], x[8];
 #pragma unroll
-        for (int i = 0; i < R; ++i) {
-            const int t = t0 + 8 * i;
-            if (t < n && !mg[t]) ld_piece(src + (size_t)(p0 + t) * D, raw[i]);
-        }
+        for (int j = 0; j < V; ++j) r[j] = reinterpret_cast<const uint4*>(base + (size_t)t * D)[j];
+        to_f8(r, x);
+        const float db = (float)dg[t];
 #pragma unroll
-        for (int i = 0; i < R; ++i) {
-            const int t = t0 + 8 * i;
-            if (t >= n || mg[t]) continue;
-            T* out = dst + (size_t)slot_of(t) * D;
-            const uint32_t m0 = (t & 1) ? amask[t >> 1][0] : 0u, m1 = (t & 1) ? amask[t >> 1][1] : 0u;
-            if (m0 | m1) {
-                // degree-weighted mean: the B row first, then its A rows by position
-                float acc[8], x[8];
-                to_f8(raw[i], x);
-                const float db = (float)dg[t];
+        for (int e = 0; e < 8; ++e) acc[e] = db * x[e];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) acc[e] = db * x[e];
+        for (int wd = 0; wd < 2; ++wd) {
+            for (uint32_t mm = wd ? m1 : m0; mm; mm &= mm - 1u) {
+                const int ta = 2 * (32 * wd + __ffs(mm) - 1);
 #pragma unroll
-                for (int wd = 0; wd < 2; ++wd) {
-                    for (uint32_t mm = wd ? m1 : m0; mm; mm &= mm - 1u) {
-                        const int ia = 32 * wd + __ffs(mm) - 1;
-                        uint4 ra[V];
+                for (int j = 0; j < V; ++j) r[j] = reinterpret_cast<const uint4*>(base + (size_t)ta * D)[j];
+                to_f8(r, x);
+                const float da = (float)dg[ta];
 #pragma unroll
-                        for (int j = 0; j < V; ++j) ra[j] = stage[(ia * 32 + lane) * V + j];
-                        to_f8(ra, x);
-                        const float da = (float)dg[2 * ia];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) acc[e] = fmaf(da, x[e], acc[e]);
-                    }
-                }
-                const float inv = 1.f / (float)ns[t];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[e] *= inv;
-                uint4 ro[V];
-                from_f8(acc, ro);
-                st_piece(out, ro);
-            } else {
-                st_piece(out, raw[i]);
+                for (int e = 0; e < 8; ++e) acc[e] = fmaf(da, x[e], acc[e]);
             }
         }
+        const float inv = 1.f / (float)ns[t];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] *= inv;
+        from_f8(acc, r);
+#pragma unroll
+        for (int j = 0; j < V; ++j) reinterpret_cast<uint4*>(base + (size_t)t * D)[j] = r[j];
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
+    // one bulk store per tensor for each run of kept rows, issued by the thread of its first row
+    if (tid < n && !mg[tid] && (tid == 0 || mg[tid - 1])) {
+        int e = n;
+        for (int wd = (tid + 1) >> 5; wd < 4; ++wd) {
+            uint32_t mm = mword[wd];
+            if (wd == ((tid + 1) >> 5)) mm &= ~0u << ((tid + 1) & 31);
+            if (mm) {
+                e = min(n, 32 * wd + __ffs(mm) - 1);
+                break;
+            }
+        }
+        const size_t o = (size_t)row * n_out + slot_of(tid);
+        const uint32_t bytes = (uint32_t)(e - tid) * D * sizeof(T);
+        bulk_store(k_out + o * D, sk + (size_t)tid * D, bytes);
+        bulk_store(v_out + o * D, sv + (size_t)tid * D, bytes);
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        // shared memory stays valid until the stores have read it
+        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
     }
 }
 
@@ -710,12 +752,27 @@ cudaError_t csm(const void* k, const void* v, int dtype, const int32_t* deg, int
     const int n_blk = n_chunks + (S + kSeg - 1) / kSeg + (w + kSeg - 1) / kSeg;
     const long long grid = (long long)rows * n_blk;
     if (grid > (1LL << 31) - 1) return cudaErrorInvalidValue;
+    // rows of the longest block (a chunk, or a sink / window segment), K and V
+    const int max_rows = std::max(n_chunks > 0 ? chunk : 0, std::max(std::min(S, kSeg), std::min(w, kSeg)));
+    const size_t esz = dtype == KVC_BF16 ? 2 : 4;
+    const size_t smem = 2 * (size_t)max_rows * D * esz;
+    static std::atomic<bool> attr_set[2][64];
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    const int ti = dtype == KVC_BF16;
+    if (dev >= 64 || !attr_set[ti][dev].load()) {
+        const int lim = 2 * kSeg * D * 4;
+        e = ti ? cudaFuncSetAttribute(csm_write_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim)
+               : cudaFuncSetAttribute(csm_write_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+        if (e != cudaSuccess) return e;
+        if (dev < 64) attr_set[ti][dev].store(true);
+    }
     if (dtype == KVC_BF16)
-        csm_write_kernel<__nv_bfloat16><<<(unsigned)grid, kWriteThreads, (size_t)(chunk / 2) * 32 * 16, s>>>(
+        csm_write_kernel<__nv_bfloat16><<<(unsigned)grid, kWriteThreads, smem, s>>>(
             (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, deg, N, S, w, chunk, n_chunks, n_blk, best, merged, cb,
             n_out, (__nv_bfloat16*)k_out, (__nv_bfloat16*)v_out, deg_out, pos_out, err);
     else
-        csm_write_kernel<float><<<(unsigned)grid, kWriteThreads, (size_t)(chunk / 2) * 32 * 32, s>>>(
+        csm_write_kernel<float><<<(unsigned)grid, kWriteThreads, smem, s>>>(
             (const float*)k, (const float*)v, deg, N, S, w, chunk, n_chunks, n_blk, best, merged, cb, n_out,
             (float*)k_out, (float*)v_out, deg_out, pos_out, err);
     count_launches(1);
