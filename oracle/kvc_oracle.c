@@ -36,6 +36,10 @@
  *           Shannon entropy (nats) of each window query's attention row; the share of a
  *           score row's mass that the kept positions hold; the population variance of a
  *           score row over the candidates C.
+ *   clustering and decode attention
+ *           CentroidKV merges similar tokens into degree-weighted centroids instead of
+ *           evicting them (Chunked Soft Matching, CentroidKV page, sec. 3-4) and attends to
+ *           the centroids with the log of their degree added to the logits (sec. 4).
  *
  * Everything is done in double precision with plain loops; inputs arrive as raw fp32 or
  * bf16 bytes and are widened exactly.  Parallelism, where present, is only over
@@ -611,4 +615,56 @@ double oracle_csm_ratio(double r_init, double delta, int round)
 {
     const double r = r_init - (double)round * delta;
     return r > 0.0 ? r : 0.0;
+}
+
+/* ------------------------------------------------------------------------------------ */
+/* Decode attention over a clustered cache (CentroidKV)                                  */
+/* ------------------------------------------------------------------------------------ */
+
+/*
+ * oracle_centroid_attention -- attention of decode queries over a cache of centroids whose
+ * degrees enter the softmax as a log term (CentroidKV page, sec. 4 "Aggregatie": the
+ * cluster degree is added to the softmax as a log-term so that attention over a centroid
+ * approximates attention over the tokens it replaced).  Read as: a centroid of degree n
+ * weighs like n copies of itself, i.e. its logit gains ln n:
+ *     x_t = q . k_t / sqrt(D) + ln n_t,   p = softmax_t(x),   out = sum_t p_t v_t
+ * over all n cached rows (no mask: every cached row precedes the decode queries).
+ * Layouts: q [B][Hq][nq][D], k and v [B][Hkv][n][D] (kv_dtype), deg [B][Hkv][n] or NULL
+ * (all degrees 1: plain attention), out [B][Hq][nq][D] fp64.  Query head g reads KV head
+ * g / (Hq / Hkv).  Returns 0, or -1 on bad arguments.
+ */
+int oracle_centroid_attention(const void *q, int q_dtype, const void *k, const void *v, int kv_dtype,
+                              const int32_t *deg, int B, int Hq, int Hkv, int nq, int n, int D, double *out)
+{
+    if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || nq < 1 || n < 1 || D < 1) return -1;
+    const int G = Hq / Hkv;
+    const double sqrt_d = sqrt((double)D);
+    double *x = (double *)malloc(sizeof(double) * (size_t)n);
+    if (!x) return -1;
+    for (int b = 0; b < B; ++b)
+        for (int g = 0; g < Hq; ++g) {
+            const int kvh = g / G;
+            const size_t kv_row0 = ((size_t)b * Hkv + kvh) * n;
+            for (int i = 0; i < nq; ++i) {
+                const size_t q0 = (((size_t)b * Hq + g) * nq + i) * D;
+                double m = -INFINITY;
+                for (int t = 0; t < n; ++t) {
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d)
+                        dot += widen(q, q_dtype, q0 + d) * widen(k, kv_dtype, (kv_row0 + t) * D + d);
+                    x[t] = dot / sqrt_d + (deg ? log((double)deg[kv_row0 + t]) : 0.0);
+                    if (x[t] > m) m = x[t];
+                }
+                double l = 0.0;
+                for (int t = 0; t < n; ++t) l += exp(x[t] - m);
+                double *o = out + q0;
+                for (int d = 0; d < D; ++d) o[d] = 0.0;
+                for (int t = 0; t < n; ++t) {
+                    const double p = exp(x[t] - m) / l;
+                    for (int d = 0; d < D; ++d) o[d] += p * widen(v, kv_dtype, (kv_row0 + t) * D + d);
+                }
+            }
+        }
+    free(x);
+    return 0;
 }

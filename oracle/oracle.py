@@ -7,7 +7,8 @@ CUDA library package.
 All arithmetic lives in kvc_oracle.c (fp64, plain loops).  This file only marshals
 arguments and composes the steps in the order the method takes them:
 score -> aggregate -> pool -> select -> gather (+ the TSP branch), plus the pivot metrics
-(attention entropy of the window rows, kept mass and candidate variance of score rows).
+(attention entropy of the window rows, kept mass and candidate variance of score rows),
+CentroidKV's Chunked Soft Matching round and decode attention over its centroids.
 """
 from __future__ import annotations
 
@@ -50,10 +51,11 @@ def _load(so_path: str):
     L.oracle_csm_merges.argtypes = [i, i, i, i, d]
     L.oracle_csm.argtypes = [p, p, i, p, i, i, i, i, i, i, d, p, p, p, p, p, p, p]
     L.oracle_csm_ratio.argtypes = [d, d, i]
+    L.oracle_centroid_attention.argtypes = [p, i, p, p, i, p, i, i, i, i, i, i, p]
     L.oracle_csm_ratio.restype = d
     for f in ("oracle_score", "oracle_accumulate", "oracle_pool", "oracle_select",
               "oracle_gather", "oracle_tsp_count", "oracle_entropy", "oracle_row_stats",
-              "oracle_csm_merges", "oracle_csm"):
+              "oracle_csm_merges", "oracle_csm", "oracle_centroid_attention"):
         getattr(L, f).restype = ctypes.c_int
     return L
 
@@ -264,6 +266,25 @@ def csm(k, v, deg, *, n_sink: int, window: int, chunk: int, ratio: float) -> dic
     return {"best": best.reshape(shp + (N,)), "sim": sim.reshape(shp + (N,)), "merged": merged.reshape(shp + (N,)),
             "k_out": k_out, "v_out": v_out, "deg_out": deg_out.reshape(shp + (n_out,)),
             "pos_out": pos_out.reshape(shp + (n_out,)), "m": m}
+
+
+def centroid_attention(q, k, v, deg=None) -> np.ndarray:
+    """Decode attention (fp64) of q [B, Hq, nq, D] over a cache k, v [B, Hkv, n, D] whose
+    degrees deg [B, Hkv, n] (None: all 1) add ln(deg) to the logits.  Returns
+    [B, Hq, nq, D] float64."""
+    qb, qd = _as_buffer(q)
+    kb, kd = _as_buffer(k)
+    vb, vd = _as_buffer(v)
+    assert kd == vd
+    B, Hq, nq, D = q.shape
+    _, Hkv, n, _ = k.shape
+    dg = None if deg is None else np.ascontiguousarray(np.asarray(deg, dtype=np.int32).reshape(B, Hkv, n))
+    out = np.empty((B, Hq, nq, D), dtype=np.float64)
+    rc = lib().oracle_centroid_attention(qb.ctypes.data, qd, kb.ctypes.data, vb.ctypes.data, kd,
+                                         None if dg is None else dg.ctypes.data, B, Hq, Hkv, nq, n, D,
+                                         out.ctypes.data)
+    _check(rc, "centroid_attention")
+    return out
 
 
 def compress(q, k, v, *, window: int, n_sink: int, pool_kernel: int, kv_budget: int,

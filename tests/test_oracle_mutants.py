@@ -50,6 +50,14 @@ MUTANTS = [
     ("csm: unweighted mean", "acc_k[d] += (double)deg[a] * widen(k, dtype, (size_t)a * D + d);",
      "acc_k[d] += (double)deg[j] * widen(k, dtype, (size_t)a * D + d);"),
     ("csm: degrees not accumulated", "                    n += deg[a];\n", ""),
+    ("decode: log2 of the degree", "x[t] = dot / sqrt_d + (deg ? log((double)deg[kv_row0 + t]) : 0.0);",
+     "x[t] = dot / sqrt_d + (deg ? log2((double)deg[kv_row0 + t]) : 0.0);"),
+    ("decode: degree term subtracted", "x[t] = dot / sqrt_d + (deg ? log((double)deg[kv_row0 + t]) : 0.0);",
+     "x[t] = dot / sqrt_d - (deg ? log((double)deg[kv_row0 + t]) : 0.0);"),
+    ("decode: degree ignored", "x[t] = dot / sqrt_d + (deg ? log((double)deg[kv_row0 + t]) : 0.0);",
+     "x[t] = dot / sqrt_d;"),
+    ("decode: no logit scale", "x[t] = dot / sqrt_d + (deg ?", "x[t] = dot + (deg ?"),
+    ("decode: GQA interleaved", "const int kvh = g / G;", "const int kvh = g % Hkv;"),
     ("kept mass over the candidates only", "for (int j = 0; j < N; ++j) total += s[j];",
      "for (int j = S; j < N - w; ++j) total += s[j];"),
 ]
@@ -79,6 +87,11 @@ PIN_TESTS = [
     pins.test_csm_invariants_and_closed_forms,
     pins.test_csm_bf16_output_rounding,
     pins.test_csm_ties_go_to_lower_position,
+    lambda: [pins.test_centroid_attention_unit_degrees_is_library_attention(*a)
+             for a in [(1, 4, 1, 1, 37, __import__("torch").float64), (2, 8, 2, 3, 70, __import__("torch").float32)]],
+    pins.test_centroid_attention_degree_is_replication,
+    pins.test_centroid_attention_closed_forms,
+    pins.test_centroid_attention_gqa_groups,
 ]
 
 

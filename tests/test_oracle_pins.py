@@ -503,3 +503,83 @@ def test_csm_ties_go_to_lower_position():
     assert out["best"][0] == 1 and out["best"][2] == 1 and out["best"][4] == 1 and out["best"][6] == 1
     # all four A tokens tie; two merges take positions 0 and 2
     assert out["m"] == 2 and np.nonzero(out["merged"])[0].tolist() == [0, 2]
+
+
+# ---------------------------------------------------------------- decode attention (CentroidKV sec. 4)
+
+def _sdpa_gqa(q, k, v):
+    """torch's float64 scaled-dot-product attention with each KV head serving its group."""
+    G = q.shape[1] // k.shape[1]
+    return torch.nn.functional.scaled_dot_product_attention(
+        q.double(), k.double().repeat_interleave(G, dim=1), v.double().repeat_interleave(G, dim=1)).numpy()
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,nq,n,dtype", [(1, 4, 1, 1, 37, torch.float64), (2, 8, 2, 3, 70, torch.float32),
+                                                  (1, 6, 3, 2, 129, torch.bfloat16)])
+def test_centroid_attention_unit_degrees_is_library_attention(B, Hq, Hkv, nq, n, dtype):
+    g = torch.Generator().manual_seed(n)
+    q = torch.randn(B, Hq, nq, 128, generator=g).to(dtype)
+    k = torch.randn(B, Hkv, n, 128, generator=g).to(dtype)
+    v = torch.randn(B, Hkv, n, 128, generator=g).to(dtype)
+    ref = _sdpa_gqa(q, k, v)
+    np.testing.assert_allclose(O.centroid_attention(q, k, v), ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(O.centroid_attention(q, k, v, deg=np.ones((B, Hkv, n), np.int32)), ref, rtol=0,
+                               atol=1e-12)
+
+
+def test_centroid_attention_degree_is_replication():
+    # a centroid of degree n attends exactly like n copies of itself with degree 1
+    g = torch.Generator().manual_seed(5)
+    B, Hq, Hkv, nq, n = 2, 4, 2, 2, 23
+    q = torch.randn(B, Hq, nq, 128, generator=g, dtype=torch.float64)
+    k = torch.randn(B, Hkv, n, 128, generator=g, dtype=torch.float64)
+    v = torch.randn(B, Hkv, n, 128, generator=g, dtype=torch.float64)
+    deg = torch.randint(1, 5, (B, Hkv, n), generator=g, dtype=torch.int32)
+    got = O.centroid_attention(q, k, v, deg=deg.numpy())
+    for b in range(B):
+        for h in range(Hkv):
+            reps = deg[b, h].long()
+            kr = k[b, h].repeat_interleave(reps, dim=0)[None, None]
+            vr = v[b, h].repeat_interleave(reps, dim=0)[None, None]
+            want = O.centroid_attention(q[b:b + 1, 2 * h:2 * h + 2], kr, vr)
+            np.testing.assert_allclose(got[b, 2 * h:2 * h + 2], want[0], rtol=0, atol=1e-12)
+
+
+def test_centroid_attention_closed_forms():
+    g = torch.Generator().manual_seed(9)
+    q = torch.randn(1, 2, 1, 128, generator=g, dtype=torch.float64)
+    # one cached row: the output is its value whatever the degree
+    k1 = torch.randn(1, 1, 1, 128, generator=g, dtype=torch.float64)
+    v1 = torch.randn(1, 1, 1, 128, generator=g, dtype=torch.float64)
+    for d in (1, 7):
+        np.testing.assert_allclose(O.centroid_attention(q, k1, v1, deg=np.full((1, 1, 1), d, np.int32)),
+                                   v1.expand(1, 2, 1, 128).numpy(), rtol=0, atol=1e-14)
+    # two rows: the weight of row 0 is the logistic function of the scaled logit gap plus
+    # ln(n0 / n1)
+    k2 = torch.randn(1, 1, 2, 128, generator=g, dtype=torch.float64)
+    v2 = torch.randn(1, 1, 2, 128, generator=g, dtype=torch.float64)
+    n0, n1 = 5, 2
+    got = O.centroid_attention(q, k2, v2, deg=np.array([[[n0, n1]]], np.int32))
+    for hq in range(2):
+        gap = float((q[0, hq, 0] @ (k2[0, 0, 0] - k2[0, 0, 1])) / math.sqrt(128)) + math.log(n0 / n1)
+        p0 = scipy.special.expit(gap)
+        want = p0 * v2[0, 0, 0].numpy() + (1 - p0) * v2[0, 0, 1].numpy()
+        np.testing.assert_allclose(got[0, hq, 0], want, rtol=0, atol=1e-13)
+    # scaling every degree by the same factor changes nothing (softmax shift invariance)
+    k = torch.randn(1, 1, 30, 128, generator=g, dtype=torch.float64)
+    v = torch.randn(1, 1, 30, 128, generator=g, dtype=torch.float64)
+    deg = torch.randint(1, 4, (1, 1, 30), generator=g, dtype=torch.int32).numpy()
+    np.testing.assert_allclose(O.centroid_attention(q, k, v, deg=3 * deg), O.centroid_attention(q, k, v, deg=deg),
+                               rtol=0, atol=1e-13)
+
+
+def test_centroid_attention_gqa_groups():
+    # KV head h holds the constant value h + 1: query head g must read KV head g // G
+    g = torch.Generator().manual_seed(2)
+    Hq, Hkv, n = 6, 3, 11
+    q = torch.randn(1, Hq, 2, 128, generator=g, dtype=torch.float64)
+    k = torch.randn(1, Hkv, n, 128, generator=g, dtype=torch.float64)
+    v = (torch.arange(Hkv, dtype=torch.float64) + 1).view(1, Hkv, 1, 1).expand(1, Hkv, n, 128).contiguous()
+    got = O.centroid_attention(q, k, v, deg=torch.randint(1, 9, (1, Hkv, n), generator=g).numpy())
+    for hq in range(Hq):
+        np.testing.assert_allclose(got[0, hq], hq // (Hq // Hkv) + 1.0, rtol=0, atol=1e-13)
