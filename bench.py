@@ -373,7 +373,7 @@ def main():
 
     # the pivot-detection metrics (StructKV sec. 2): cost of the entropy in the scoring pass
     # and of the per-row kept mass / candidate variance, outside the timed region
-    pivot = None
+    pivot = csm_round = decode_att = None
     if args.pivot_steps > 0:
         Hs = wl.Hkv if wl.scope == kvc.KVC_SCOPE_PER_KV_HEAD else 1
         sc = torch.empty((wl.B, Hs, wl.N), dtype=torch.float32, device="cuda")
@@ -402,7 +402,8 @@ def main():
 
         # one CentroidKV Chunked Soft Matching round over the last layer's K and V (r = 0.25,
         # chunks of 64): algorithmic bytes = K read to match + K and V read and the kept rows
-        # (K, V, degree, position) written
+        # (K, V, degree, position) written; then one decode step's attention (one query per
+        # query head) over the centroids with their log-degrees: K, V and degrees read
         if wl.D == 128:
             kl, vl = dev["k"][-1], dev["v"]
             r, ch = 0.25, 64
@@ -413,8 +414,21 @@ def main():
                 raise RuntimeError("device-side error in the clustering round")
             row = wl.D * kl.element_size()
             nbytes = wl.B * wl.Hkv * (3 * wl.N * row + (wl.N - m) * (2 * row + 8))  # + degree, position
-            pivot["csm"] = {"ratio": r, "chunk": ch, "ms": t_csm, "gbs": nbytes / (t_csm * 1e-3) / 1e9,
-                            "algorithmic_bytes": nbytes, "frac_of_peak": nbytes / (t_csm * 1e-3) / 1e9 / peak}
+            csm_round = {"ratio": r, "chunk": ch, "ms": t_csm, "gbs": nbytes / (t_csm * 1e-3) / 1e9,
+                         "algorithmic_bytes": nbytes, "frac_of_peak": nbytes / (t_csm * 1e-3) / 1e9 / peak}
+            n_c = wl.N - m
+            qd = torch.randn((wl.B, wl.Hq, 1, wl.D), generator=torch.Generator().manual_seed(5)).to(kl.dtype).cuda()
+            att = torch.empty((wl.B, wl.Hq, 1, wl.D), dtype=torch.float32, device="cuda")
+            att_ws = torch.empty(kvc.kvc_decode_attention_workspace_size(wl.B, wl.Hq, wl.Hkv, 1, n_c),
+                                 dtype=torch.uint8, device="cuda")
+            t_dec = timed(lambda: kvc.kvc_decode_attention(qd, csm_out["k_out"], csm_out["v_out"],
+                                                           deg=csm_out["deg_out"], out=att, ws=att_ws))
+            if kvc.kvc_poll_error() != kvc.KVC_OK:
+                raise RuntimeError("device-side error in the decode attention")
+            dbytes = wl.B * wl.Hkv * n_c * (2 * row + 4) + wl.B * wl.Hq * wl.D * (kl.element_size() + 4)  # + q, out
+            decode_att = {"cached_rows": n_c, "query_heads": wl.Hq, "ms": t_dec,
+                          "gbs": dbytes / (t_dec * 1e-3) / 1e9, "algorithmic_bytes": dbytes,
+                          "frac_of_peak": dbytes / (t_dec * 1e-3) / 1e9 / peak}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -437,6 +451,8 @@ def main():
                          "traffic": traffic, "algorithmic_bytes_per_launch": ab["score"]},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
             "pivot_metrics": pivot,
+            "csm_round": csm_round,
+            "decode_attention": decode_att,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -285,17 +285,69 @@ KVC_API kvc_status kvc_csm_workspace_size(int32_t B, int32_t H, int32_t N, int32
 
 /*
  * kvc_csm -- one Chunked Soft Matching round.
- *   k, v      device, [B, H, N, D] dtype (KVC_F32 or KVC_BF16), D = 128, 16-byte aligned.
- *   deg       device, [B, H, N] int32 degrees (>= 1), or NULL for all ones (a first round).
- *   k_out, v_out  device, [B, H, N - m, D] dtype, written (16-byte aligned).
- *   deg_out   device, [B, H, N - m] int32 degrees of the kept tokens, written.
- *   pos_out   device, [B, H, N - m] int32 original positions of the kept tokens, ascending.
+ *   k, v      device, rows (b, h) of N tokens at a stride of ld_in tokens: row (b, h) starts
+ *             at (b * H + h) * ld_in * D elements; dtype KVC_F32 or KVC_BF16, D = 128,
+ *             16-byte aligned.  ld_in = 0 means N (dense [B, H, N, D]).
+ *   deg       device, same row layout, int32 degrees (>= 1), or NULL for all ones (a
+ *             first round).
+ *   pos       device, same row layout, int32 positions carried into pos_out, or NULL for
+ *             the row index 0..N-1.
+ *   k_out, v_out  device, rows of N - m tokens at a stride of ld_out tokens (0 means
+ *             N - m), written; must not be k or v (a round is never in place).
+ *   deg_out   device, [B, H] x ld_out int32 degrees of the kept tokens, written.
+ *   pos_out   device, [B, H] x ld_out int32 positions of the kept tokens (pos[...] of the
+ *             input row, or its index), in ascending input order.
  *   ws        device workspace of >= kvc_csm_workspace_size(...) bytes.
+ * Errors: KVC_ERR_ARG (null pointers, in-place outputs, chunk/ratio/n_sink/window out of
+ * range, ld_in < N, ld_out < N - m), KVC_ERR_UNSUPPORTED (dtype, D), KVC_ERR_ALIGN,
+ * KVC_ERR_WORKSPACE.  A malformed selection inside the kernels (never for valid inputs)
+ * sets KVC_ERR_INDEX in kvc_poll_error.
  */
-KVC_API kvc_status kvc_csm(const void *k, const void *v, const int32_t *deg, int32_t B, int32_t H, int32_t N,
-                           int32_t D, int32_t dtype, int32_t n_sink, int32_t window, int32_t chunk, float ratio,
-                           void *k_out, void *v_out, int32_t *deg_out, int32_t *pos_out, void *workspace,
-                           size_t workspace_bytes, kvc_stream_t stream);
+KVC_API kvc_status kvc_csm(const void *k, const void *v, const int32_t *deg, const int32_t *pos, int32_t B,
+                           int32_t H, int32_t N, int32_t ld_in, int32_t D, int32_t dtype, int32_t n_sink,
+                           int32_t window, int32_t chunk, float ratio, void *k_out, void *v_out, int32_t *deg_out,
+                           int32_t *pos_out, int32_t ld_out, void *workspace, size_t workspace_bytes,
+                           kvc_stream_t stream);
+
+/*
+ * kvc_append -- appends t_new decode tokens to every (b, h) row of a cache (CentroidKV page,
+ * sec. 2 Inferentie Pipeline, Decoding: the cache grows by one token per step between
+ * clustering rounds).
+ *   k_cache, v_cache  device, rows of capacity ld tokens holding n tokens; rows n .. n +
+ *             t_new - 1 are written from k_new, v_new [B, H, t_new, D] (device).
+ *   deg_cache, pos_cache  device int32 caches of the same row layout, or NULL; the new
+ *             slots get degree 1 and positions pos0 .. pos0 + t_new - 1.
+ * Errors: KVC_ERR_ARG (null pointers, n + t_new > ld), KVC_ERR_UNSUPPORTED (dtype, D),
+ * KVC_ERR_ALIGN (16-byte).
+ */
+KVC_API kvc_status kvc_append(void *k_cache, void *v_cache, int32_t *deg_cache, int32_t *pos_cache, int32_t B,
+                              int32_t H, int32_t ld, int32_t n, const void *k_new, const void *v_new,
+                              int32_t t_new, int32_t pos0, int32_t D, int32_t dtype, kvc_stream_t stream);
+
+/* kvc_decode_attention_workspace_size -- bytes of device workspace kvc_decode_attention
+ * needs for these shapes (G * nq = Hq / Hkv * nq <= 8). */
+KVC_API kvc_status kvc_decode_attention_workspace_size(int32_t B, int32_t Hq, int32_t Hkv, int32_t nq, int32_t n,
+                                                       size_t *bytes);
+
+/*
+ * kvc_decode_attention -- attention of decode queries over a clustered cache (CentroidKV
+ * page, sec. 4 Aggregatie: the cluster degree enters the softmax as a log term, so that
+ * a centroid of degree n weighs like n copies of itself):
+ *     out[b, g, i, :] = sum_t softmax_t(q[b, g, i] . k[b, h, t] / sqrt(D) + ln deg[b, h, t]) v[b, h, t, :]
+ * over the n cached rows t of KV head h = g / (Hq / Hkv); no mask.
+ *   q         device, [B, Hq, nq, D] dtype (the cache's dtype), 16-byte aligned.
+ *   k, v      device, rows (b, h) of capacity ld tokens (0 means n) holding n tokens.
+ *   deg       device int32 degrees (>= 1) in the same row layout, or NULL (plain attention).
+ *   out       device, [B, Hq, nq, D] fp32, written.
+ *   ws        device workspace of >= kvc_decode_attention_workspace_size(...) bytes.
+ * Errors: KVC_ERR_ARG (null pointers, Hq % Hkv, n < 1, ld < n), KVC_ERR_UNSUPPORTED
+ * (Hq / Hkv * nq > 8, dtype, D), KVC_ERR_ALIGN, KVC_ERR_WORKSPACE.  A degree below 1 is
+ * read as 1 and sets KVC_ERR_INDEX in kvc_poll_error.
+ */
+KVC_API kvc_status kvc_decode_attention(const void *q, const void *k, const void *v, const int32_t *deg, int32_t B,
+                                        int32_t Hq, int32_t Hkv, int32_t nq, int32_t n, int32_t ld, int32_t D,
+                                        int32_t dtype, float *out, void *workspace, size_t workspace_bytes,
+                                        kvc_stream_t stream);
 
 /*
  * kvc_score_noalloc -- kvc_score for callers that cannot allocate device memory.  The

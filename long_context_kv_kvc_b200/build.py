@@ -16,8 +16,8 @@ INCLUDE = os.path.join(ROOT, "include")
 OBJ = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libkvc.so")
 
-SOURCES = ["api.cu", "score_simt.cu", "score_tc.cu", "select.cu", "gather.cu", "noalloc.cu", "csm.cu"]
-HEADERS = ["kvc_internal.cuh"]
+SOURCES = ["api.cu", "score_simt.cu", "score_tc.cu", "select.cu", "gather.cu", "noalloc.cu", "csm.cu", "decode.cu"]
+HEADERS = ["kvc_internal.cuh", "tc_ptx.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",

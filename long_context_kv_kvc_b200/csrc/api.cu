@@ -1,5 +1,6 @@
 // api.cu -- the C ABI of libkvc.so: argument validation, workspace layout and the
 // launch sequence of each entry point.  See include/kvc.h for the contracts.
+#include <algorithm>
 #include <math.h>
 #include <stdio.h>
 #include <string.h>
@@ -256,19 +257,70 @@ kvc_status kvc_csm_workspace_size(int32_t B, int32_t H, int32_t N, int32_t n_sin
     return KVC_OK;
 }
 
-kvc_status kvc_csm(const void* k, const void* v, const int32_t* deg, int32_t B, int32_t H, int32_t N, int32_t D,
-                   int32_t dtype, int32_t n_sink, int32_t window, int32_t chunk, float ratio, void* k_out, void* v_out,
-                   int32_t* deg_out, int32_t* pos_out, void* ws, size_t ws_bytes, kvc_stream_t stream) {
+kvc_status kvc_csm(const void* k, const void* v, const int32_t* deg, const int32_t* pos, int32_t B, int32_t H,
+                   int32_t N, int32_t ld_in, int32_t D, int32_t dtype, int32_t n_sink, int32_t window, int32_t chunk,
+                   float ratio, void* k_out, void* v_out, int32_t* deg_out, int32_t* pos_out, int32_t ld_out,
+                   void* ws, size_t ws_bytes, kvc_stream_t stream) {
     if (!k || !v || !k_out || !v_out || !deg_out || !pos_out || !ws || B < 1 || H < 1) return KVC_ERR_ARG;
+    if (k_out == k || v_out == v || k_out == v || v_out == k) return KVC_ERR_ARG;  // no in-place round
     if (dtype != KVC_F32 && dtype != KVC_BF16) return KVC_ERR_UNSUPPORTED;
     KVC_TRY(check_csm(N, D, n_sink, window, chunk, ratio));
+    const int m = kvc::csm_merges(N, n_sink, window, chunk, ratio);
+    if (ld_in == 0) ld_in = N;
+    if (ld_out == 0) ld_out = N - m;
+    if (ld_in < N || ld_out < N - m) return KVC_ERR_ARG;
     if (!aligned16(k) || !aligned16(v) || !aligned16(k_out) || !aligned16(v_out) || ((uintptr_t)ws & (kAlign - 1)))
         return KVC_ERR_ALIGN;
-    if ((long long)B * H * N > (1LL << 31) - 1) return KVC_ERR_ARG;
-    const int m = kvc::csm_merges(N, n_sink, window, chunk, ratio);
+    if ((long long)B * H * std::max(ld_in, N) > (1LL << 31) - 1) return KVC_ERR_ARG;
     if (ws_bytes < kvc::csm_workspace(B * H, N, m)) return KVC_ERR_WORKSPACE;
-    KVC_CUDA(kvc::csm(k, v, dtype, deg, B * H, N, n_sink, window, chunk, m, k_out, v_out, deg_out, pos_out, ws,
-                      (cudaStream_t)stream));
+    KVC_CUDA(kvc::csm(k, v, dtype, deg, pos, B * H, N, ld_in, n_sink, window, chunk, m, k_out, v_out, deg_out,
+                      pos_out, ld_out, ws, (cudaStream_t)stream));
+    return KVC_OK;
+}
+
+kvc_status kvc_append(void* k_cache, void* v_cache, int32_t* deg_cache, int32_t* pos_cache, int32_t B, int32_t H,
+                      int32_t ld, int32_t n, const void* k_new, const void* v_new, int32_t t_new, int32_t pos0,
+                      int32_t D, int32_t dtype, kvc_stream_t stream) {
+    if (!k_cache || !v_cache || !k_new || !v_new || B < 1 || H < 1 || n < 0 || t_new < 0) return KVC_ERR_ARG;
+    if ((long long)n + t_new > ld || (long long)B * H * ld > (1LL << 31) - 1) return KVC_ERR_ARG;
+    if (dtype != KVC_F32 && dtype != KVC_BF16) return KVC_ERR_UNSUPPORTED;
+    if (D != kHeadDim) return KVC_ERR_UNSUPPORTED;
+    if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_new) || !aligned16(v_new)) return KVC_ERR_ALIGN;
+    KVC_CUDA(kvc::append_rows(k_cache, v_cache, deg_cache, pos_cache, dtype, B * H, ld, n, k_new, v_new, t_new, pos0,
+                              (cudaStream_t)stream));
+    return KVC_OK;
+}
+
+namespace {
+kvc_status check_decode(int32_t B, int32_t Hq, int32_t Hkv, int32_t nq, int32_t n) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || nq < 1 || n < 1 || Hq % Hkv) return KVC_ERR_ARG;
+    if (!kvc::decode_rows_supported(Hq / Hkv * nq)) return KVC_ERR_UNSUPPORTED;
+    return KVC_OK;
+}
+}  // namespace
+
+kvc_status kvc_decode_attention_workspace_size(int32_t B, int32_t Hq, int32_t Hkv, int32_t nq, int32_t n,
+                                               size_t* bytes) {
+    if (!bytes) return KVC_ERR_ARG;
+    KVC_TRY(check_decode(B, Hq, Hkv, nq, n));
+    *bytes = kvc::decode_workspace(B * Hkv, Hq / Hkv * nq, n);
+    return KVC_OK;
+}
+
+kvc_status kvc_decode_attention(const void* q, const void* k, const void* v, const int32_t* deg, int32_t B,
+                                int32_t Hq, int32_t Hkv, int32_t nq, int32_t n, int32_t ld, int32_t D, int32_t dtype,
+                                float* out, void* ws, size_t ws_bytes, kvc_stream_t stream) {
+    if (!q || !k || !v || !out || !ws) return KVC_ERR_ARG;
+    KVC_TRY(check_decode(B, Hq, Hkv, nq, n));
+    if (ld == 0) ld = n;
+    if (ld < n || (long long)B * Hkv * ld > (1LL << 31) - 1) return KVC_ERR_ARG;
+    if (dtype != KVC_F32 && dtype != KVC_BF16) return KVC_ERR_UNSUPPORTED;
+    if (D != kHeadDim) return KVC_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || ((uintptr_t)ws & (kAlign - 1)))
+        return KVC_ERR_ALIGN;
+    const int U = B * Hkv, Rv = Hq / Hkv * nq;
+    if (ws_bytes < kvc::decode_workspace(U, Rv, n)) return KVC_ERR_WORKSPACE;
+    KVC_CUDA(kvc::decode_attention(q, k, v, deg, dtype, U, Rv, n, ld, out, ws, (cudaStream_t)stream));
     return KVC_OK;
 }
 

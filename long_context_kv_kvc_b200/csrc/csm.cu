@@ -99,7 +99,7 @@ __device__ __forceinline__ void from_f8(const float (&x)[8], uint4 (&r)[2]) {
 // and last chunk, at the sinks and the window); best[pos] = the matched B position.  The
 // keys are staged in shared memory; each thread forms a 2 x 2 block of A-B dot products.
 __global__ void __launch_bounds__(kMatchThreads)
-csm_match_f32_kernel(const float* __restrict__ k, int N, int S, int w, int chunk, int n_chunks,
+csm_match_f32_kernel(const float* __restrict__ k, int N, long long ld, int S, int w, int chunk, int n_chunks,
                      float* __restrict__ score, int32_t* __restrict__ best) {
     extern __shared__ __align__(16) float ks[];  // [chunk][kKS]
     __shared__ float inv_norm[128];
@@ -108,7 +108,7 @@ csm_match_f32_kernel(const float* __restrict__ k, int N, int S, int w, int chunk
     const int hi = N - w;
     const int c0 = S + q * chunk, c1 = min(c0 + chunk, hi);
     const int len = c1 - c0;
-    const float* kr = k + (size_t)row * N * D;
+    const float* kr = k + (size_t)row * ld * D;
     float* sr = score + (size_t)row * N;
     int32_t* br = best + (size_t)row * N;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -469,11 +469,12 @@ __device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t 
 // (consecutive kept rows have consecutive output slots).
 template <typename T>
 __global__ void __launch_bounds__(kWriteThreads)
-csm_write_kernel(const T* __restrict__ k, const T* __restrict__ v, const int32_t* __restrict__ deg, int N, int S,
-                 int w, int chunk, int n_chunks, int n_blk, const int32_t* __restrict__ best,
-                 const unsigned char* __restrict__ merged, const int32_t* __restrict__ cb, int n_out,
-                 T* __restrict__ k_out, T* __restrict__ v_out, int32_t* __restrict__ deg_out,
-                 int32_t* __restrict__ pos_out, unsigned* __restrict__ err) {
+csm_write_kernel(const T* __restrict__ k, const T* __restrict__ v, const int32_t* __restrict__ deg,
+                 const int32_t* __restrict__ pos, int N, long long ld_in, int S, int w, int chunk, int n_chunks,
+                 int n_blk, const int32_t* __restrict__ best, const unsigned char* __restrict__ merged,
+                 const int32_t* __restrict__ cb, int n_out, long long ld_out, T* __restrict__ k_out,
+                 T* __restrict__ v_out, int32_t* __restrict__ deg_out, int32_t* __restrict__ pos_out,
+                 unsigned* __restrict__ err) {
     constexpr int V = Vec<T>::n;
     extern __shared__ __align__(128) uint8_t wsm[];  // K rows, then V rows, of this block
     __shared__ uint64_t bar;
@@ -502,7 +503,8 @@ csm_write_kernel(const T* __restrict__ k, const T* __restrict__ v, const int32_t
         n = min(kSeg, w - off);
         o0 = cb[(size_t)row * (n_chunks + 1) + n_chunks] + off;
     }
-    const size_t rN = (size_t)row * N;
+    const size_t rN = (size_t)row * N;     // workspace rows (dense)
+    const size_t rI = (size_t)row * ld_in;  // input cache rows
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t tensor_bytes = (uint32_t)n * D * sizeof(T);
     T* sk = reinterpret_cast<T*>(wsm);
@@ -513,13 +515,13 @@ csm_write_kernel(const T* __restrict__ k, const T* __restrict__ v, const int32_t
         mbar_init(&bar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         mbar_expect_tx(&bar, 2 * tensor_bytes);
-        bulk_load(sk, k + (rN + p0) * D, tensor_bytes, &bar);
-        bulk_load(sv, v + (rN + p0) * D, tensor_bytes, &bar);
+        bulk_load(sk, k + (rI + p0) * D, tensor_bytes, &bar);
+        bulk_load(sv, v + (rI + p0) * D, tensor_bytes, &bar);
     }
     amask[tid >> 1][tid & 1] = 0u;
     if (tid < n) {
         mg[tid] = in_c ? merged[rN + p0 + tid] : 0;
-        dg[tid] = deg ? deg[rN + p0 + tid] : 1;
+        dg[tid] = deg ? deg[rI + p0 + tid] : 1;
     }
     __syncthreads();
     {
@@ -549,9 +551,9 @@ csm_write_kernel(const T* __restrict__ k, const T* __restrict__ v, const int32_t
                 for (uint32_t mm = amask[tid >> 1][wd]; mm; mm &= mm - 1u) nsum += dg[2 * (32 * wd + __ffs(mm) - 1)];
         }
         ns[tid] = nsum;
-        const size_t o = (size_t)row * n_out + slot_of(tid);
+        const size_t o = (size_t)row * ld_out + slot_of(tid);
         deg_out[o] = nsum;
-        pos_out[o] = p0 + tid;
+        pos_out[o] = pos ? pos[rI + p0 + tid] : p0 + tid;
     }
     // the rows have landed (bounded wait; a copy that never lands is reported, not used)
     if (!mbar_try_wait(&bar, 0)) {
@@ -611,7 +613,7 @@ csm_write_kernel(const T* __restrict__ k, const T* __restrict__ v, const int32_t
                 break;
             }
         }
-        const size_t o = (size_t)row * n_out + slot_of(tid);
+        const size_t o = (size_t)row * ld_out + slot_of(tid);
         const uint32_t bytes = (uint32_t)(e - tid) * D * sizeof(T);
         bulk_store(k_out + o * D, sk + (size_t)tid * D, bytes);
         bulk_store(v_out + o * D, sv + (size_t)tid * D, bytes);
@@ -644,8 +646,8 @@ size_t csm_workspace(int rows, int N, int m) {
 
 namespace {
 
-cudaError_t match_tc(const void* k, int rows, int N, int S, int w, int chunk, float* score, int32_t* best,
-                     cudaStream_t s) {
+cudaError_t match_tc(const void* k, int rows, int N, long long ld, int S, int w, int chunk, float* score,
+                     int32_t* best, cudaStream_t s) {
     TcMatchArgs a{};
     a.score = score;
     a.best = best;
@@ -662,7 +664,7 @@ cudaError_t match_tc(const void* k, int rows, int N, int S, int w, int chunk, fl
     auto encode = encode_fn();
     if (!encode) return cudaErrorNotSupported;
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)rows};
-    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)N * D * 2};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)ld * D * 2};
     cuuint32_t box[3] = {64, kTileTok, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     if (encode(&a.tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(k), dims, strides, box, estr,
@@ -688,8 +690,8 @@ cudaError_t match_tc(const void* k, int rows, int N, int S, int w, int chunk, fl
     return cudaGetLastError();
 }
 
-cudaError_t match_f32(const float* k, int rows, int N, int S, int w, int chunk, int n_chunks, float* score,
-                      int32_t* best, cudaStream_t s) {
+cudaError_t match_f32(const float* k, int rows, int N, long long ld, int S, int w, int chunk, int n_chunks,
+                      float* score, int32_t* best, cudaStream_t s) {
     static std::atomic<bool> attr_set[64];
     int dev = 0;
     cudaError_t e;
@@ -703,16 +705,16 @@ cudaError_t match_f32(const float* k, int rows, int N, int S, int w, int chunk, 
     const long long grid = (long long)rows * n_chunks;
     if (grid > (1LL << 31) - 1) return cudaErrorInvalidValue;
     csm_match_f32_kernel<<<(unsigned)grid, kMatchThreads, (size_t)chunk * kKS * sizeof(float), s>>>(
-        k, N, S, w, chunk, n_chunks, score, best);
+        k, N, ld, S, w, chunk, n_chunks, score, best);
     count_launches(1);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t csm(const void* k, const void* v, int dtype, const int32_t* deg, int rows, int N, int S, int w,
-                int chunk, int m, void* k_out, void* v_out, int32_t* deg_out, int32_t* pos_out, void* ws,
-                cudaStream_t s) {
+cudaError_t csm(const void* k, const void* v, int dtype, const int32_t* deg, const int32_t* pos, int rows, int N,
+                long long ld_in, int S, int w, int chunk, int m, void* k_out, void* v_out, int32_t* deg_out,
+                int32_t* pos_out, long long ld_out, void* ws, cudaStream_t s) {
     const size_t rn = (size_t)rows * N;
     char* p = (char*)ws;
     float* score = (float*)p;
@@ -733,8 +735,8 @@ cudaError_t csm(const void* k, const void* v, int dtype, const int32_t* deg, int
     if ((e = cudaMemsetAsync(merged, 0, rn, s)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(cb, 0, (size_t)rows * (n_chunks + 1) * sizeof(int32_t), s)) != cudaSuccess) return e;
     if (m > 0 && n_chunks > 0) {
-        e = dtype == KVC_BF16 ? match_tc(k, rows, N, S, w, chunk, score, best, s)
-                              : match_f32((const float*)k, rows, N, S, w, chunk, n_chunks, score, best, s);
+        e = dtype == KVC_BF16 ? match_tc(k, rows, N, ld_in, S, w, chunk, score, best, s)
+                              : match_f32((const float*)k, rows, N, ld_in, S, w, chunk, n_chunks, score, best, s);
         if (e != cudaSuccess) return e;
         // the m best matches (ties to the lower position), ascending
         e = topk_fused_fits(N, 0, 0) ? topk_fused(score, rows, N, 0, 0, m, 1, sel, s)
@@ -769,12 +771,12 @@ cudaError_t csm(const void* k, const void* v, int dtype, const int32_t* deg, int
     }
     if (dtype == KVC_BF16)
         csm_write_kernel<__nv_bfloat16><<<(unsigned)grid, kWriteThreads, smem, s>>>(
-            (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, deg, N, S, w, chunk, n_chunks, n_blk, best, merged, cb,
-            n_out, (__nv_bfloat16*)k_out, (__nv_bfloat16*)v_out, deg_out, pos_out, err);
+            (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, deg, pos, N, ld_in, S, w, chunk, n_chunks, n_blk, best,
+            merged, cb, n_out, ld_out, (__nv_bfloat16*)k_out, (__nv_bfloat16*)v_out, deg_out, pos_out, err);
     else
         csm_write_kernel<float><<<(unsigned)grid, kWriteThreads, smem, s>>>(
-            (const float*)k, (const float*)v, deg, N, S, w, chunk, n_chunks, n_blk, best, merged, cb, n_out,
-            (float*)k_out, (float*)v_out, deg_out, pos_out, err);
+            (const float*)k, (const float*)v, deg, pos, N, ld_in, S, w, chunk, n_chunks, n_blk, best, merged, cb,
+            n_out, ld_out, (float*)k_out, (float*)v_out, deg_out, pos_out, err);
     count_launches(1);
     return cudaGetLastError();
 }

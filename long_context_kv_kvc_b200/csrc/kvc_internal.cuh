@@ -89,8 +89,18 @@ cudaError_t row_stats(const float* scores, int rows, int N, int S, int w, const 
 // CentroidKV Chunked Soft Matching (csm.cu): merges m = csm_merges(...) A tokens per row
 int csm_merges(int N, int S, int w, int chunk, float ratio);
 size_t csm_workspace(int rows, int N, int m);
-cudaError_t csm(const void* k, const void* v, int dtype, const int32_t* deg, int rows, int N, int S, int w,
-                int chunk, int m, void* k_out, void* v_out, int32_t* deg_out, int32_t* pos_out, void* ws,
-                cudaStream_t s);
+cudaError_t csm(const void* k, const void* v, int dtype, const int32_t* deg, const int32_t* pos, int rows, int N,
+                long long ld_in, int S, int w, int chunk, int m, void* k_out, void* v_out, int32_t* deg_out,
+                int32_t* pos_out, long long ld_out, void* ws, cudaStream_t s);
+
+// decode attention over a (clustered) cache (decode.cu): U = B * Hkv units of Rv = G * nq
+// query rows each, n cached rows at a row stride of ld tokens; out [U * Rv][128] fp32
+bool decode_rows_supported(int rows_per_kv_head);
+size_t decode_workspace(int U, int Rv, int n);
+cudaError_t decode_attention(const void* q, const void* k, const void* v, const int32_t* deg, int dtype, int U,
+                             int Rv, int n, long long ld, float* out, void* ws, cudaStream_t s);
+// appends t_new rows per unit to caches of row stride ld holding n rows (decode.cu)
+cudaError_t append_rows(void* k_cache, void* v_cache, int32_t* deg_cache, int32_t* pos_cache, int dtype, int U,
+                        long long ld, int n, const void* k_new, const void* v_new, int t_new, int pos0, cudaStream_t s);
 
 }  // namespace kvc

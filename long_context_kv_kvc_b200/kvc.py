@@ -25,7 +25,8 @@ KVC_STAGE_SCORE, KVC_STAGE_SELECT, KVC_STAGE_GATHER, KVC_STAGE_COUNT = 0, 1, 2, 
 EXPORTED = ("kvc_workspace_size", "kvc_score", "kvc_accumulate", "kvc_pool", "kvc_topk_workspace_size",
             "kvc_topk", "kvc_gather", "kvc_compress", "kvc_tsp_count", "kvc_poll_error",
             "kvc_status_string", "kvc_version", "kvc_launch_count", "kvc_score_noalloc", "kvc_score_entropy",
-            "kvc_row_stats", "kvc_csm_merges", "kvc_csm_ratio", "kvc_csm_workspace_size", "kvc_csm")
+            "kvc_row_stats", "kvc_csm_merges", "kvc_csm_ratio", "kvc_csm_workspace_size", "kvc_csm", "kvc_append",
+            "kvc_decode_attention_workspace_size", "kvc_decode_attention")
 
 
 class KvcError(RuntimeError):
@@ -70,8 +71,11 @@ def _load():
         "kvc_csm_merges": (i32, [i32, i32, i32, i32, ctypes.c_float]),
         "kvc_csm_ratio": (ctypes.c_float, [ctypes.c_float, ctypes.c_float, i32]),
         "kvc_csm_workspace_size": (st, [i32, i32, i32, i32, i32, i32, ctypes.c_float, ctypes.POINTER(sz)]),
-        "kvc_csm": (st, [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, ctypes.c_float, vp, vp, vp, vp, vp, sz,
-                         vp]),
+        "kvc_csm": (st, [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, i32, ctypes.c_float, vp, vp, vp, vp,
+                         i32, vp, sz, vp]),
+        "kvc_append": (st, [vp, vp, vp, vp, i32, i32, i32, i32, vp, vp, i32, i32, i32, i32, vp]),
+        "kvc_decode_attention_workspace_size": (st, [i32, i32, i32, i32, i32, ctypes.POINTER(sz)]),
+        "kvc_decode_attention": (st, [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -184,25 +188,74 @@ def kvc_csm_ratio(r_init, delta, round_) -> float:
     return float(lib.kvc_csm_ratio(r_init, delta, round_))
 
 
-def kvc_csm(k, v, n_sink, window, chunk, ratio, deg=None, out=None, ws=None, stream=None) -> dict:
-    """One Chunked Soft Matching round over k, v [B, H, N, D]; returns (and fills, when given
-    as `out`) k_out, v_out [B, H, N - m, D], deg_out and pos_out [B, H, N - m]."""
-    B, H, N, D = k.shape
+def kvc_csm_workspace_size(B, H, N, n_sink, window, chunk, ratio) -> int:
+    nb = ctypes.c_size_t(0)
+    _check(lib.kvc_csm_workspace_size(B, H, N, n_sink, window, chunk, ratio, ctypes.byref(nb)), "kvc_csm_workspace_size")
+    return nb.value
+
+
+def kvc_csm(k, v, n_sink, window, chunk, ratio, deg=None, out=None, ws=None, stream=None, n=None, pos=None,
+            ld_out=None) -> dict:
+    """One Chunked Soft Matching round over the first n (default: all) rows of k, v
+    [B, H, cap, D]; returns (and fills, when given as `out`) k_out, v_out [B, H, cap_out, D],
+    deg_out and pos_out [B, H, cap_out] whose first N - m rows are the kept tokens.  deg and
+    pos (nullable) share k's row layout; without `out` the outputs are dense (cap_out =
+    N - m) unless ld_out is given."""
+    B, H, cap, D = k.shape
+    N = cap if n is None else n
     dt = KVC_BF16 if k.dtype == torch.bfloat16 else KVC_F32
     m = kvc_csm_merges(N, n_sink, window, chunk, ratio)
     if out is None:
-        out = {"k_out": torch.empty((B, H, N - m, D), dtype=k.dtype, device=k.device),
-               "v_out": torch.empty((B, H, N - m, D), dtype=k.dtype, device=k.device),
-               "deg_out": torch.empty((B, H, N - m), dtype=torch.int32, device=k.device),
-               "pos_out": torch.empty((B, H, N - m), dtype=torch.int32, device=k.device)}
+        co = N - m if ld_out is None else ld_out
+        out = {"k_out": torch.empty((B, H, co, D), dtype=k.dtype, device=k.device),
+               "v_out": torch.empty((B, H, co, D), dtype=k.dtype, device=k.device),
+               "deg_out": torch.empty((B, H, co), dtype=torch.int32, device=k.device),
+               "pos_out": torch.empty((B, H, co), dtype=torch.int32, device=k.device)}
+    cap_out = out["k_out"].shape[2]
     if ws is None:
-        n = ctypes.c_size_t(0)
-        _check(lib.kvc_csm_workspace_size(B, H, N, n_sink, window, chunk, ratio, ctypes.byref(n)),
-               "kvc_csm_workspace_size")
-        ws = torch.empty(max(n.value, 256), dtype=torch.uint8, device=k.device)
-    _check(lib.kvc_csm(_ptr(k), _ptr(v), _ptr(deg) if deg is not None else None, B, H, N, D, dt, n_sink, window,
-                       chunk, ratio, _ptr(out["k_out"]), _ptr(out["v_out"]), _ptr(out["deg_out"]),
-                       _ptr(out["pos_out"]), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "kvc_csm")
+        ws = torch.empty(max(kvc_csm_workspace_size(B, H, N, n_sink, window, chunk, ratio), 256), dtype=torch.uint8,
+                         device=k.device)
+    _check(lib.kvc_csm(_ptr(k), _ptr(v), _ptr(deg) if deg is not None else None,
+                       _ptr(pos) if pos is not None else None, B, H, N, cap, D, dt, n_sink, window, chunk, ratio,
+                       _ptr(out["k_out"]), _ptr(out["v_out"]), _ptr(out["deg_out"]), _ptr(out["pos_out"]), cap_out,
+                       _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "kvc_csm")
+    return out
+
+
+def kvc_append(k_cache, v_cache, n, k_new, v_new, deg_cache=None, pos_cache=None, pos0=0, stream=None):
+    """Writes k_new, v_new [B, H, t_new, D] into rows n .. n + t_new - 1 of the caches
+    [B, H, cap, D] (degrees 1, positions pos0 ..)."""
+    B, H, cap, D = k_cache.shape
+    t_new = k_new.shape[2]
+    dt = KVC_BF16 if k_cache.dtype == torch.bfloat16 else KVC_F32
+    _check(lib.kvc_append(_ptr(k_cache), _ptr(v_cache), _ptr(deg_cache) if deg_cache is not None else None,
+                          _ptr(pos_cache) if pos_cache is not None else None, B, H, cap, n, _ptr(k_new), _ptr(v_new),
+                          t_new, pos0, D, dt, _stream(stream)), "kvc_append")
+
+
+def kvc_decode_attention_workspace_size(B, Hq, Hkv, nq, n) -> int:
+    nb = ctypes.c_size_t(0)
+    _check(lib.kvc_decode_attention_workspace_size(B, Hq, Hkv, nq, n, ctypes.byref(nb)),
+           "kvc_decode_attention_workspace_size")
+    return nb.value
+
+
+def kvc_decode_attention(q, k, v, deg=None, n=None, out=None, ws=None, stream=None):
+    """Attention of q [B, Hq, nq, D] over the first n (default: all) rows of the cache
+    k, v [B, Hkv, cap, D] with ln(deg) added to the logits (deg [B, Hkv, cap] or None);
+    returns out [B, Hq, nq, D] fp32."""
+    B, Hq, nq, D = q.shape
+    _, Hkv, cap, _ = k.shape
+    n = cap if n is None else n
+    dt = KVC_BF16 if k.dtype == torch.bfloat16 else KVC_F32
+    if out is None:
+        out = torch.empty((B, Hq, nq, D), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = torch.empty(max(kvc_decode_attention_workspace_size(B, Hq, Hkv, nq, n), 256), dtype=torch.uint8,
+                         device=q.device)
+    _check(lib.kvc_decode_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(deg) if deg is not None else None, B, Hq, Hkv,
+                                    nq, n, cap, D, dt, _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
+                                    _stream(stream)), "kvc_decode_attention")
     return out
 
 

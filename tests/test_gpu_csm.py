@@ -13,11 +13,9 @@ import pytest
 import torch
 
 from oracle import oracle as O
+from parity_util import check_csm_row as check_row
 
 pytestmark = pytest.mark.gpu
-
-BAND = 1e-5
-
 
 @pytest.fixture(scope="module")
 def K():
@@ -42,78 +40,6 @@ def make_kv(B, H, N, dtype, seed, dup=0, zero=0):
         # zero keys: similarity 0 with every token
         k[:, :, torch.randint(0, N, (zero,), generator=g)] = 0.0
     return k.to(dtype), v.to(dtype)
-
-
-def check_row(kr, vr, dr, out_k, out_v, out_d, out_p, S, w, chunk, ratio, dtype):
-    """One row: band rule on the merge set, then the kept rows given the GPU's merges."""
-    N = kr.shape[0]
-    ref = O.csm(kr, vr, dr, n_sink=S, window=w, chunk=chunk, ratio=ratio)
-    m = ref["m"]
-    pos = np.asarray(out_p, dtype=np.int64)
-    assert pos.size == N - m and np.all(np.diff(pos) > 0)
-    is_merged = np.ones(N, dtype=bool)
-    is_merged[pos] = False
-    merged = np.nonzero(is_merged)[0]
-    assert merged.size == m
-    sim, best = ref["sim"], ref["best"]
-    assert np.all(best[merged] >= 0), "a token without a match was merged"
-    if m:
-        T = np.sort(sim[best >= 0])[::-1][m - 1]
-        must = (best >= 0) & (sim > T + BAND)
-        mustnot = (best >= 0) & (sim < T - BAND)
-        assert not np.any(must & ~is_merged), f"{int((must & ~is_merged).sum())} clearly better matches not merged"
-        assert not np.any(mustnot & is_merged), "clearly worse matches merged"
-    # the B token each merged A joins: the best match in fp64, unless the runner-up is within
-    # the band (then neither candidate row is checked)
-    kk, vv = kr.double().numpy(), vr.double().numpy()
-    nrm = np.linalg.norm(kk, axis=1)
-    unit = np.divide(kk, nrm[:, None], out=np.zeros_like(kk), where=nrm[:, None] > 0)
-    owner = np.full(N, -1, dtype=np.int64)
-    ambiguous = np.zeros(N, dtype=bool)
-    for c0 in range(S, N - w, chunk):
-        c1 = min(c0 + chunk, N - w)
-        A = np.arange(c0, c1, 2)
-        Bs = np.arange(c0 + 1, c1, 2)
-        A = A[is_merged[A]]
-        if A.size == 0 or Bs.size == 0:
-            continue
-        sm = unit[A] @ unit[Bs].T
-        order = np.argsort(-sm, axis=1, kind="stable")
-        owner[A] = Bs[order[:, 0]]
-        if Bs.size > 1:
-            gap = sm[np.arange(A.size), order[:, 0]] - sm[np.arange(A.size), order[:, 1]]
-            close = gap < BAND
-            ambiguous[Bs[order[close, 0]]] = True
-            ambiguous[Bs[order[close, 1]]] = True
-    # expected rows of the kept tokens: degree-weighted sums over the token and its absorbed ones
-    d = np.asarray(dr, dtype=np.float64)
-    n = d.copy()
-    sk, sv = d[:, None] * kk, d[:, None] * vv
-    ak, av = np.abs(sk), np.abs(sv)  # magnitude of the summands: the scale of the rounding error
-    src = merged
-    np.add.at(n, owner[src], d[src])
-    np.add.at(sk, owner[src], d[src, None] * kk[src])
-    np.add.at(sv, owner[src], d[src, None] * vv[src])
-    np.add.at(ak, owner[src], d[src, None] * np.abs(kk[src]))
-    np.add.at(av, owner[src], d[src, None] * np.abs(vv[src]))
-    has = np.zeros(N, dtype=bool)
-    has[owner[src]] = True
-    check = ~ambiguous[pos]
-    np.testing.assert_array_equal(np.asarray(out_d)[check], n[pos][check].astype(np.int64))
-    single = check & ~has[pos]
-    assert torch.equal(out_k[torch.from_numpy(single)], kr[torch.from_numpy(pos[single])]), "unmerged rows not copied"
-    assert torch.equal(out_v[torch.from_numpy(single)], vr[torch.from_numpy(pos[single])]), "unmerged rows not copied"
-    multi = check & has[pos]
-    tol = 2.0 ** -7 if dtype == torch.bfloat16 else 2e-6
-    for s_, a_, got in ((sk, ak, out_k), (sv, av, out_v)):
-        want = s_[pos[multi]] / n[pos[multi], None]
-        scale = a_[pos[multi]] / n[pos[multi], None]
-        g = got[torch.from_numpy(multi)].double().numpy()
-        err = np.abs(g - want)
-        # fp32 sums: error below ~2^-23 of the summands' magnitude; bf16 adds half a unit of
-        # the result's last place
-        bound = 2e-6 * scale + (tol * np.abs(want) if dtype == torch.bfloat16 else 0.0) + 1e-30
-        assert np.all(err <= bound), f"merged rows off by {(err / np.maximum(scale, 1e-30)).max():.2e} of their scale"
 
 
 # bf16 keys take the tensor-core match (128-token tiles holding whole chunks: 128 for chunk
