@@ -350,6 +350,67 @@ KVC_API kvc_status kvc_decode_attention(const void *q, const void *k, const void
                                         kvc_stream_t stream);
 
 /*
+ * Sequence sharding (one GPU per contiguous block of the sequence, for contexts beyond one
+ * GPU's memory).  The exchange steps between the calls below are the caller's (collectives
+ * of a few KiB): an all-gather of every shard's (m, l), a halo of (pool_kernel - 1) / 2
+ * scores at each block edge for the pool, a sum of the radix-select histograms per digit,
+ * and a count of the ties each shard holds.  Supported for the per-KV-head budget:
+ * p->n_layers = 1 and p->scope = KVC_SCOPE_PER_KV_HEAD; p->N is the whole sequence's length.
+ * Scoring runs on the CUDA cores.
+ */
+
+/* kvc_shard_workspace_size -- device workspace of kvc_shard_stats / kvc_shard_scores for a
+ * block of n_local keys. */
+KVC_API kvc_status kvc_shard_workspace_size(const kvc_params *p, int32_t n_local, size_t *bytes);
+
+/*
+ * kvc_shard_stats -- this block's part of each window row's softmax normaliser.
+ *   q        device, [B, Hq, window, D] (all window queries; every shard holds them).
+ *   k_local  device, [B, Hkv, n_local, D]: keys key_offset .. key_offset + n_local - 1.
+ *   ml       device, [B * Hkv][G * window][2] fp32, written: (m, l) = (max y, sum 2^(y - m))
+ *            over the block's keys that the row sees (y = q.k log2(e) / sqrt(D); window row
+ *            i sits at position N - window + i); (-inf, 0) when it sees none.
+ */
+KVC_API kvc_status kvc_shard_stats(const kvc_params *p, const void *q, const void *k_local, int32_t n_local,
+                                   int32_t key_offset, float *ml, void *workspace, size_t workspace_bytes,
+                                   kvc_stream_t stream);
+
+/*
+ * kvc_shard_scores -- the block's saliency scores given every shard's (m, l).
+ *   ml_all   device, [n_shards][B * Hkv][G * window][2]: the shards' kvc_shard_stats
+ *            outputs in shard order; merged in that order into each row's log-sum-exp, so
+ *            every shard uses the same value.
+ *   scores   device, [B, Hkv, n_local] fp32, written.
+ */
+KVC_API kvc_status kvc_shard_scores(const kvc_params *p, const void *q, const void *k_local, int32_t n_local,
+                                    int32_t key_offset, const float *ml_all, int32_t n_shards, float *scores,
+                                    void *workspace, size_t workspace_bytes, kvc_stream_t stream);
+
+/*
+ * kvc_select_hist -- one digit of a radix select spread over shards: for each row of pooled
+ * [rows, n] (fp32, device), hist[row][d] (device, [rows][1 << digit_bits] uint32, written)
+ * counts the candidates j in [lo, hi) whose order key (a monotone map of the fp32 value to
+ * uint32, -0.0 read as +0.0; larger value, larger key) has its top prefix_bits equal to
+ * prefix[row]'s (device uint32 [rows]) and the next digit_bits equal to d.
+ * 1 <= digit_bits <= 12, prefix_bits + digit_bits <= 32.
+ */
+KVC_API kvc_status kvc_select_hist(const float *pooled, int32_t rows, int32_t n, int32_t lo, int32_t hi,
+                                   const uint32_t *prefix, int32_t prefix_bits, int32_t digit_bits, uint32_t *hist,
+                                   kvc_stream_t stream);
+
+/*
+ * kvc_select_emit -- the shard's part of the selection once the threshold key is known:
+ * for each row writes, in position order, pos_offset + j for the candidates j in [lo, hi)
+ * whose key is above thr[row] and for the first ties[row] candidates whose key equals it
+ * (ties go to the lower positions) into out[row][0 .. cap) (device int32), and the number
+ * written into count[row].  More than cap sets KVC_ERR_INDEX in kvc_poll_error.  pos_offset
+ * may be negative (a block's row can start with a halo) as long as pos_offset + lo >= 0.
+ */
+KVC_API kvc_status kvc_select_emit(const float *pooled, int32_t rows, int32_t n, int32_t lo, int32_t hi,
+                                   const uint32_t *thr, const int32_t *ties, int32_t pos_offset, int32_t *out,
+                                   int32_t cap, int32_t *count, kvc_stream_t stream);
+
+/*
  * kvc_score_noalloc -- kvc_score for callers that cannot allocate device memory.  The
  * pages have no counterpart: it exists for engines that have already given all device
  * memory to their own pool, or plugin interfaces that forbid cudaMalloc/cudaFree during a

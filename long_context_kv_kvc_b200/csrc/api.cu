@@ -324,6 +324,103 @@ kvc_status kvc_decode_attention(const void* q, const void* k, const void* v, con
     return KVC_OK;
 }
 
+namespace {
+// sequence sharding supports the per-KV-head budget (one layer, per-KV-head scope); the block
+// of keys [key_offset, key_offset + n_local) lies inside the sequence of p->N keys
+kvc_status check_shard(const kvc_params* p, int32_t n_local, int32_t key_offset) {
+    KVC_TRY(check_params(p));
+    if (p->n_layers != 1 || p->scope != KVC_SCOPE_PER_KV_HEAD) return KVC_ERR_UNSUPPORTED;
+    if (n_local < 1 || key_offset < 0 || (long long)key_offset + n_local > p->N) return KVC_ERR_ARG;
+    return KVC_OK;
+}
+
+struct ShardPlan {
+    int n_chunks, chunk;
+    size_t off_partial, off_lse, total;
+};
+
+ShardPlan shard_plan(const kvc_params* p, int n_local) {
+    ShardPlan P{};
+    const ScoreJob job = make_job(p, nullptr, nullptr);
+    const size_t pb = simt_score_workspace(job.U, n_local, job.nq, &P.n_chunks, &P.chunk);
+    P.off_partial = 0;
+    P.off_lse = align_up(pb);
+    P.total = align_up(P.off_lse + (size_t)job.U * job.nq * sizeof(float));
+    return P;
+}
+
+ScoreJob shard_job(const kvc_params* p, const ShardPlan& P, const void* q, const void* k, int n_local, int key_offset,
+                   char* ws) {
+    ScoreJob job = make_job(p, q, k);
+    job.N = n_local;
+    job.key_off = key_offset;
+    job.n_total = p->N;
+    job.partial = (float2*)(ws + P.off_partial);
+    job.lse = (float*)(ws + P.off_lse);
+    job.n_chunks = P.n_chunks;
+    job.chunk = P.chunk;
+    return job;
+}
+}  // namespace
+
+kvc_status kvc_shard_workspace_size(const kvc_params* p, int32_t n_local, size_t* bytes) {
+    if (!bytes) return KVC_ERR_ARG;
+    KVC_TRY(check_shard(p, n_local, 0));
+    *bytes = shard_plan(p, n_local).total;
+    return KVC_OK;
+}
+
+kvc_status kvc_shard_stats(const kvc_params* p, const void* q, const void* k_local, int32_t n_local,
+                           int32_t key_offset, float* ml, void* ws, size_t ws_bytes, kvc_stream_t stream) {
+    KVC_TRY(check_shard(p, n_local, key_offset));
+    if (!q || !k_local || !ml || !ws) return KVC_ERR_ARG;
+    if (!aligned16(q) || !aligned16(k_local) || ((uintptr_t)ml & 7u) || ((uintptr_t)ws & (kAlign - 1)))
+        return KVC_ERR_ALIGN;
+    const ShardPlan P = shard_plan(p, n_local);
+    if (ws_bytes < P.total) return KVC_ERR_WORKSPACE;
+    const ScoreJob job = shard_job(p, P, q, k_local, n_local, key_offset, (char*)ws);
+    KVC_CUDA(kvc::simt_shard_stats(job, (float2*)ml, (cudaStream_t)stream));
+    return KVC_OK;
+}
+
+kvc_status kvc_shard_scores(const kvc_params* p, const void* q, const void* k_local, int32_t n_local,
+                            int32_t key_offset, const float* ml_all, int32_t n_shards, float* scores, void* ws,
+                            size_t ws_bytes, kvc_stream_t stream) {
+    KVC_TRY(check_shard(p, n_local, key_offset));
+    if (!q || !k_local || !ml_all || !scores || !ws || n_shards < 1) return KVC_ERR_ARG;
+    if (!aligned16(q) || !aligned16(k_local) || ((uintptr_t)ml_all & 7u) || ((uintptr_t)scores & 3u) ||
+        ((uintptr_t)ws & (kAlign - 1)))
+        return KVC_ERR_ALIGN;
+    const ShardPlan P = shard_plan(p, n_local);
+    if (ws_bytes < P.total) return KVC_ERR_WORKSPACE;
+    ScoreJob job = shard_job(p, P, q, k_local, n_local, key_offset, (char*)ws);
+    job.unit_scores = scores;
+    KVC_CUDA(kvc::simt_shard_scores(job, (const float2*)ml_all, n_shards, (cudaStream_t)stream));
+    return KVC_OK;
+}
+
+kvc_status kvc_select_hist(const float* pooled, int32_t rows, int32_t n, int32_t lo, int32_t hi,
+                           const uint32_t* prefix, int32_t prefix_bits, int32_t digit_bits, uint32_t* hist,
+                           kvc_stream_t stream) {
+    if (!pooled || !prefix || !hist || rows < 1 || n < 1) return KVC_ERR_ARG;
+    if (lo < 0 || hi > n || lo > hi || digit_bits < 1 || digit_bits > 12 || prefix_bits < 0 ||
+        prefix_bits + digit_bits > 32)
+        return KVC_ERR_ARG;
+    KVC_CUDA(kvc::select_hist(pooled, rows, n, lo, hi, prefix, prefix_bits, digit_bits, hist, (cudaStream_t)stream));
+    return KVC_OK;
+}
+
+kvc_status kvc_select_emit(const float* pooled, int32_t rows, int32_t n, int32_t lo, int32_t hi, const uint32_t* thr,
+                           const int32_t* ties, int32_t pos_offset, int32_t* out, int32_t cap, int32_t* count,
+                           kvc_stream_t stream) {
+    if (!pooled || !thr || !ties || !out || !count || rows < 1 || n < 1 || cap < 0) return KVC_ERR_ARG;
+    if (lo < 0 || hi > n || lo > hi || (long long)pos_offset + hi > (1LL << 31) - 1 ||
+        (hi > lo && (long long)pos_offset + lo < 0))
+        return KVC_ERR_ARG;
+    KVC_CUDA(kvc::select_emit(pooled, rows, n, lo, hi, thr, ties, pos_offset, out, cap, count, (cudaStream_t)stream));
+    return KVC_OK;
+}
+
 kvc_status kvc_accumulate(float* acc, const float* src, int32_t B, int32_t Hi, int32_t Ho, int32_t N,
                           kvc_stream_t stream) {
     if (!acc || !src || B < 1 || Hi < 1 || Ho < 1 || N < 0 || Hi % Ho) return KVC_ERR_ARG;

@@ -32,7 +32,9 @@ struct ScoreJob {
     const void* k;
     int dtype;
     int U;        // units = n_layers * B * Hkv
-    int N;
+    int N;        // keys per unit in k
+    int key_off;  // sequence sharding: position of k's first key in the whole sequence
+    int n_total;  // sequence sharding: keys of the whole sequence (0: N)
     int window;
     int G;
     int nq;       // G * window query rows per unit
@@ -55,6 +57,10 @@ struct ScoreJob {
 // CUDA-core (FFMA) scoring, fp32 or bf16 inputs
 size_t simt_score_workspace(int U, int N, int nq, int* n_chunks, int* chunk);
 cudaError_t simt_score(const ScoreJob& job, cudaStream_t s);
+// sequence sharding: this block of keys' (m, l) per (unit, window row); then the scores of the
+// block's keys given every shard's (m, l) [W][U * nq] (merged into job.lse in shard order)
+cudaError_t simt_shard_stats(const ScoreJob& job, float2* ml, cudaStream_t s);
+cudaError_t simt_shard_scores(const ScoreJob& job, const float2* ml_all, int W, cudaStream_t s);
 
 // tensor-core scoring (bf16, tcgen05 + TMA); returns false if the shape is not supported
 bool tc_score_supported(const ScoreJob& job);
@@ -74,6 +80,11 @@ cudaError_t topk(const float* pooled, int rows, int N, int n_sink, int window, i
 // pool (odd width `kernel` over [n_sink, N - window)) and top-k in one launch, one 8-CTA
 // cluster per row; for rows whose candidates fit the clusters' shared memory
 bool topk_fused_fits(int N, int n_sink, int window);
+// distributed radix select over a sharded score row (select.cu)
+cudaError_t select_hist(const float* pooled, int rows, int n, int lo, int hi, const uint32_t* prefix, int prefix_bits,
+                        int digit_bits, uint32_t* hist, cudaStream_t s);
+cudaError_t select_emit(const float* pooled, int rows, int n, int lo, int hi, const uint32_t* thr, const int32_t* ties,
+                        int pos_offset, int32_t* out, int cap, int32_t* count, cudaStream_t s);
 cudaError_t topk_fused(const float* scores, int rows, int N, int n_sink, int window, int budget, int kernel,
                        int32_t* idx, cudaStream_t s);
 // two gathers of the same shape in one launch (src1/dst1 may be null)

@@ -68,8 +68,8 @@ __device__ __forceinline__ void merge_stats3(float& m, float& l, float& t, float
 
 template <typename T, bool ENT>
 __global__ void __launch_bounds__(kThreads)
-stats_kernel(const T* __restrict__ q, const T* __restrict__ k, int N, int w, int nq, int chunk,
-             int n_chunks, float2* __restrict__ partial, float* __restrict__ partial_t) {
+stats_kernel(const T* __restrict__ q, const T* __restrict__ k, int N, int key_off, int n_total, int w, int nq,
+             int chunk, int n_chunks, float2* __restrict__ partial, float* __restrict__ partial_t) {
     __shared__ float Qs[kQB][D + 1];
     __shared__ float Ks[kKT][D + 1];
     const int u = blockIdx.y, c = blockIdx.x;
@@ -82,7 +82,8 @@ stats_kernel(const T* __restrict__ q, const T* __restrict__ k, int N, int w, int
         __syncthreads();
         stage_rows(Qs, qu + (size_t)qb * D, kQB, nq - qb);
         const int r = qb + qi;
-        const int t_r = r < nq ? N - w + r % w : -1;  // position of window query r
+        // position of window query r, in this block of keys (which starts at key_off of n_total)
+        const int t_r = r < nq ? n_total - w + r % w - key_off : -1;
         float m = -INFINITY, l = 0.f, tt = 0.f;
         for (int jt = j0; jt < j1; jt += kKT) {
             __syncthreads();
@@ -163,10 +164,43 @@ __global__ void combine_kernel(const float2* __restrict__ partial, const float* 
     }
 }
 
+// Sequence sharding: this block's (m, l) per (unit, row), the chunk partials merged in
+// chunk order (M = -inf, l = 0 when the block holds no key the row sees).
+__global__ void shard_ml_kernel(const float2* __restrict__ partial, int n_chunks, int nq, float2* __restrict__ ml) {
+    const int u = blockIdx.x;
+    for (int r = threadIdx.x; r < nq; r += blockDim.x) {
+        const float2* p = partial + (size_t)u * n_chunks * nq + r;
+        float M = -INFINITY;
+        for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, p[(size_t)c * nq].x);
+        float S = 0.f;
+        if (M != -INFINITY)
+            for (int c = 0; c < n_chunks; ++c) {
+                const float2 v = p[(size_t)c * nq];
+                if (v.x != -INFINITY) S += v.y * exp2f(v.x - M);
+            }
+        ml[(size_t)u * nq + r] = make_float2(M, S);
+    }
+}
+
+// lse per row from every shard's (m, l), merged in shard order (so every shard computes the
+// same value): ml_all [W][rows].
+__global__ void shard_lse_kernel(const float2* __restrict__ ml_all, int W, int rows, float* __restrict__ lse) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < rows; i += gridDim.x * blockDim.x) {
+        float M = -INFINITY;
+        for (int w = 0; w < W; ++w) M = fmaxf(M, ml_all[(size_t)w * rows + i].x);
+        float S = 0.f;
+        for (int w = 0; w < W; ++w) {
+            const float2 v = ml_all[(size_t)w * rows + i];
+            if (v.x != -INFINITY) S += v.y * exp2f(v.x - M);
+        }
+        lse[i] = M + log2f(S);
+    }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
-scores_kernel(const T* __restrict__ q, const T* __restrict__ k, int N, int w, int nq, int chunk,
-              const float* __restrict__ lse, float* __restrict__ out) {
+scores_kernel(const T* __restrict__ q, const T* __restrict__ k, int N, int key_off, int n_total, int w, int nq,
+              int chunk, const float* __restrict__ lse, float* __restrict__ out) {
     __shared__ float Qs[kQB][D + 1];
     __shared__ float Ks[kKT][D + 1];
     __shared__ float Ls[kQB];
@@ -184,7 +218,7 @@ scores_kernel(const T* __restrict__ q, const T* __restrict__ k, int N, int w, in
         stage_rows(Qs, qu + (size_t)qb * D, kQB, nq - qb);
         if (tid < kQB) Ls[tid] = qb + tid < nq ? lse[(size_t)u * nq + qb + tid] : INFINITY;
         const int r = qb + qi;
-        const int t_r = r < nq ? N - w + r % w : -1;
+        const int t_r = r < nq ? n_total - w + r % w - key_off : -1;
         for (int jt = j0; jt < j1; jt += kKT) {
             __syncthreads();
             stage_rows(Ks, ku + (size_t)jt * D, kKT, j1 - jt);
@@ -242,41 +276,75 @@ size_t simt_score_workspace(int U, int N, int nq, int* n_chunks_out, int* chunk_
     return (size_t)U * n_chunks * nq * sizeof(float2);
 }
 
-cudaError_t simt_score(const ScoreJob& j, cudaStream_t s) {
+namespace {
+
+cudaError_t launch_stats(const ScoreJob& j, cudaStream_t s) {
     dim3 grid(j.n_chunks, j.U);
-    count_launches(3);
+    const int n_total = j.n_total > 0 ? j.n_total : j.N;
     float* partial_t = j.partial_t;
     const bool ent = j.entropy != nullptr;
     if (j.dtype == KVC_F32) {
         if (ent)
-            stats_kernel<float, true><<<grid, kThreads, 0, s>>>((const float*)j.q, (const float*)j.k, j.N, j.window,
-                                                                 j.nq, j.chunk, j.n_chunks, j.partial, partial_t);
+            stats_kernel<float, true><<<grid, kThreads, 0, s>>>((const float*)j.q, (const float*)j.k, j.N, j.key_off,
+                                                                 n_total, j.window, j.nq, j.chunk, j.n_chunks,
+                                                                 j.partial, partial_t);
         else
-            stats_kernel<float, false><<<grid, kThreads, 0, s>>>((const float*)j.q, (const float*)j.k, j.N, j.window,
-                                                                  j.nq, j.chunk, j.n_chunks, j.partial, partial_t);
+            stats_kernel<float, false><<<grid, kThreads, 0, s>>>((const float*)j.q, (const float*)j.k, j.N,
+                                                                  j.key_off, n_total, j.window, j.nq, j.chunk,
+                                                                  j.n_chunks, j.partial, partial_t);
     } else {
         if (ent)
             stats_kernel<__nv_bfloat16, true><<<grid, kThreads, 0, s>>>(
-                (const __nv_bfloat16*)j.q, (const __nv_bfloat16*)j.k, j.N, j.window, j.nq, j.chunk, j.n_chunks,
-                j.partial, partial_t);
+                (const __nv_bfloat16*)j.q, (const __nv_bfloat16*)j.k, j.N, j.key_off, n_total, j.window, j.nq,
+                j.chunk, j.n_chunks, j.partial, partial_t);
         else
             stats_kernel<__nv_bfloat16, false><<<grid, kThreads, 0, s>>>(
-                (const __nv_bfloat16*)j.q, (const __nv_bfloat16*)j.k, j.N, j.window, j.nq, j.chunk, j.n_chunks,
-                j.partial, partial_t);
+                (const __nv_bfloat16*)j.q, (const __nv_bfloat16*)j.k, j.N, j.key_off, n_total, j.window, j.nq,
+                j.chunk, j.n_chunks, j.partial, partial_t);
     }
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    combine_kernel<<<j.U, 128, 0, s>>>(j.partial, partial_t, j.n_chunks, j.nq, j.lse, j.entropy);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scores(const ScoreJob& j, cudaStream_t s) {
+    dim3 grid(j.n_chunks, j.U);
+    const int n_total = j.n_total > 0 ? j.n_total : j.N;
     if (j.dtype == KVC_F32) {
-        scores_kernel<float><<<grid, kThreads, 0, s>>>((const float*)j.q, (const float*)j.k, j.N,
+        scores_kernel<float><<<grid, kThreads, 0, s>>>((const float*)j.q, (const float*)j.k, j.N, j.key_off, n_total,
                                                         j.window, j.nq, j.chunk, j.lse, j.unit_scores);
     } else {
         scores_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(
-            (const __nv_bfloat16*)j.q, (const __nv_bfloat16*)j.k, j.N, j.window, j.nq, j.chunk,
+            (const __nv_bfloat16*)j.q, (const __nv_bfloat16*)j.k, j.N, j.key_off, n_total, j.window, j.nq, j.chunk,
             j.lse, j.unit_scores);
     }
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t simt_score(const ScoreJob& j, cudaStream_t s) {
+    count_launches(3);
+    cudaError_t e = launch_stats(j, s);
+    if (e != cudaSuccess) return e;
+    combine_kernel<<<j.U, 128, 0, s>>>(j.partial, j.partial_t, j.n_chunks, j.nq, j.lse, j.entropy);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    return launch_scores(j, s);
+}
+
+cudaError_t simt_shard_stats(const ScoreJob& j, float2* ml, cudaStream_t s) {
+    count_launches(2);
+    cudaError_t e = launch_stats(j, s);
+    if (e != cudaSuccess) return e;
+    shard_ml_kernel<<<j.U, 128, 0, s>>>(j.partial, j.n_chunks, j.nq, ml);
+    return cudaGetLastError();
+}
+
+cudaError_t simt_shard_scores(const ScoreJob& j, const float2* ml_all, int W, cudaStream_t s) {
+    count_launches(2);
+    const int rows = j.U * j.nq;
+    shard_lse_kernel<<<(rows + 255) / 256, 256, 0, s>>>(ml_all, W, rows, j.lse);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_scores(j, s);
 }
 
 }  // namespace kvc

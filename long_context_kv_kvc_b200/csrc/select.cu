@@ -461,6 +461,94 @@ int grid_for(long long total, int threads) {
     return (int)(g < 1 ? 1 : g);
 }
 
+// ------------------------------------------------------------------------ distributed select
+// Sequence sharding splits a score row across GPUs; the radix select then runs digit by
+// digit over all shards: each shard histograms the digit of its candidates that match the
+// prefix found so far (the histograms are summed across shards), and once the threshold key
+// is known each shard writes its candidates above it plus its share of the ties.
+
+constexpr int kHistThreads = 256;
+constexpr int kHistBlocksPerRow = 16;
+
+// hist[row][d] += #candidates j in [lo, hi) of the row whose key's top prefix_bits equal
+// prefix[row]'s and whose next digit_bits are d.
+__global__ void __launch_bounds__(kHistThreads)
+select_hist_kernel(const float* __restrict__ v, int n, int lo, int hi, const uint32_t* __restrict__ prefix,
+                   int prefix_bits, int digit_bits, uint32_t* __restrict__ hist) {
+    extern __shared__ uint32_t h[];
+    const int row = blockIdx.y, nb = 1 << digit_bits;
+    for (int i = threadIdx.x; i < nb; i += kHistThreads) h[i] = 0u;
+    __syncthreads();
+    const uint32_t want = prefix[row];
+    const int shift = 32 - prefix_bits - digit_bits;
+    const float* vr = v + (size_t)row * n;
+    const int span = (hi - lo + gridDim.x - 1) / gridDim.x;
+    const int j0 = lo + blockIdx.x * span, j1 = min(hi, j0 + span);
+    for (int j = j0 + threadIdx.x; j < j1; j += kHistThreads) {
+        const uint32_t key = order_key(vr[j]);
+        const bool match = prefix_bits == 0 || (key >> (32 - prefix_bits)) == (want >> (32 - prefix_bits));
+        if (match) atomicAdd(&h[(key >> shift) & (nb - 1)], 1u);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < nb; i += kHistThreads)
+        if (h[i]) atomicAdd(&hist[(size_t)row * nb + i], h[i]);
+}
+
+// One CTA per row: writes, in position order, pos_offset + j for the candidates j in [lo, hi)
+// with key > thr[row] and for the first ties[row] candidates with key == thr[row]; count[row]
+// = the number written (at most cap; more sets KVC_ERR_INDEX and is not written).
+__global__ void __launch_bounds__(kTopkThreads)
+select_emit_kernel(const float* __restrict__ v, int n, int lo, int hi, const uint32_t* __restrict__ thr,
+                   const int32_t* __restrict__ ties, int pos_offset, int32_t* __restrict__ out, int cap,
+                   int32_t* __restrict__ count, unsigned* __restrict__ err) {
+    __shared__ int wsel[kWarps], weq[kWarps];
+    __shared__ int base_sel, base_eq;
+    const int row = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const float* vr = v + (size_t)row * n;
+    int32_t* o = out + (size_t)row * cap;
+    const uint32_t T = thr[row];
+    const int take = ties[row];
+    if (tid == 0) {
+        base_sel = 0;
+        base_eq = 0;
+    }
+    __syncthreads();
+    for (int j0 = lo; j0 < hi; j0 += kTopkThreads) {
+        const int j = j0 + tid;
+        const uint32_t key = j < hi ? order_key(vr[j]) : 0u;
+        const bool gt = j < hi && key > T, eq = j < hi && key == T;
+        const unsigned beq = __ballot_sync(0xffffffffu, eq);
+        if (lane == 0) weq[warp] = __popc(beq);
+        __syncthreads();
+        int eq_before = base_eq;  // ties before j, in position order
+        for (int i = 0; i < warp; ++i) eq_before += weq[i];
+        eq_before += __popc(beq & lanemask_lt());
+        const bool sel = gt || (eq && eq_before < take);
+        const unsigned bsel = __ballot_sync(0xffffffffu, sel);
+        if (lane == 0) wsel[warp] = __popc(bsel);
+        __syncthreads();
+        int at = base_sel;
+        for (int i = 0; i < warp; ++i) at += wsel[i];
+        at += __popc(bsel & lanemask_lt());
+        if (sel) {
+            if (at < cap) o[at] = pos_offset + j;
+            else atomicOr(err, kErrIndex);
+        }
+        __syncthreads();
+        if (tid == 0) {
+            int a = 0, b = 0;
+            for (int i = 0; i < kWarps; ++i) {
+                a += wsel[i];
+                b += weq[i];
+            }
+            base_sel += a;
+            base_eq += b;
+        }
+        __syncthreads();
+    }
+    if (tid == 0) count[row] = min(base_sel, cap);
+}
+
 }  // namespace
 
 cudaError_t reduce_units(const float* units, int L, int B, int Hkv, int N, int all_heads, float* out,
@@ -526,6 +614,26 @@ cudaError_t topk(const float* pooled, int rows, int N, int n_sink, int window, i
 cudaError_t row_stats(const float* scores, int rows, int N, int S, int w, const int32_t* idx, int budget,
                       float* kept_mass, float* cand_var, unsigned* err, cudaStream_t s) {
     row_stats_kernel<<<rows, kRsThreads, 0, s>>>(scores, N, S, w, idx, budget, kept_mass, cand_var, err);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t select_hist(const float* pooled, int rows, int n, int lo, int hi, const uint32_t* prefix, int prefix_bits,
+                        int digit_bits, uint32_t* hist, cudaStream_t s) {
+    const int nb = 1 << digit_bits;
+    cudaError_t e = cudaMemsetAsync(hist, 0, (size_t)rows * nb * sizeof(uint32_t), s);
+    if (e != cudaSuccess || hi <= lo) return e;
+    dim3 grid(kHistBlocksPerRow, rows);
+    select_hist_kernel<<<grid, kHistThreads, nb * sizeof(uint32_t), s>>>(pooled, n, lo, hi, prefix, prefix_bits,
+                                                                          digit_bits, hist);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t select_emit(const float* pooled, int rows, int n, int lo, int hi, const uint32_t* thr, const int32_t* ties,
+                        int pos_offset, int32_t* out, int cap, int32_t* count, cudaStream_t s) {
+    select_emit_kernel<<<rows, kTopkThreads, 0, s>>>(pooled, n, lo, hi, thr, ties, pos_offset, out, cap, count,
+                                                     device_error_word());
     count_launches(1);
     return cudaGetLastError();
 }

@@ -26,7 +26,8 @@ EXPORTED = ("kvc_workspace_size", "kvc_score", "kvc_accumulate", "kvc_pool", "kv
             "kvc_topk", "kvc_gather", "kvc_compress", "kvc_tsp_count", "kvc_poll_error",
             "kvc_status_string", "kvc_version", "kvc_launch_count", "kvc_score_noalloc", "kvc_score_entropy",
             "kvc_row_stats", "kvc_csm_merges", "kvc_csm_ratio", "kvc_csm_workspace_size", "kvc_csm", "kvc_append",
-            "kvc_decode_attention_workspace_size", "kvc_decode_attention")
+            "kvc_decode_attention_workspace_size", "kvc_decode_attention", "kvc_shard_workspace_size",
+            "kvc_shard_stats", "kvc_shard_scores", "kvc_select_hist", "kvc_select_emit")
 
 
 class KvcError(RuntimeError):
@@ -76,6 +77,11 @@ def _load():
         "kvc_append": (st, [vp, vp, vp, vp, i32, i32, i32, i32, vp, vp, i32, i32, i32, i32, vp]),
         "kvc_decode_attention_workspace_size": (st, [i32, i32, i32, i32, i32, ctypes.POINTER(sz)]),
         "kvc_decode_attention": (st, [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp, vp, sz, vp]),
+        "kvc_shard_workspace_size": (st, [P, i32, ctypes.POINTER(sz)]),
+        "kvc_shard_stats": (st, [P, vp, vp, i32, i32, vp, vp, sz, vp]),
+        "kvc_shard_scores": (st, [P, vp, vp, i32, i32, vp, i32, vp, vp, sz, vp]),
+        "kvc_select_hist": (st, [vp, i32, i32, i32, i32, vp, i32, i32, vp, vp]),
+        "kvc_select_emit": (st, [vp, i32, i32, i32, i32, vp, vp, i32, vp, i32, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -257,6 +263,37 @@ def kvc_decode_attention(q, k, v, deg=None, n=None, out=None, ws=None, stream=No
                                     nq, n, cap, D, dt, _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
                                     _stream(stream)), "kvc_decode_attention")
     return out
+
+
+def kvc_shard_workspace_size(p, n_local) -> int:
+    nb = ctypes.c_size_t(0)
+    _check(lib.kvc_shard_workspace_size(ctypes.byref(p), n_local, ctypes.byref(nb)), "kvc_shard_workspace_size")
+    return nb.value
+
+
+def kvc_shard_stats(p, q, k_local, key_offset, ml, ws, stream=None):
+    n_local = k_local.shape[-2]
+    _check(lib.kvc_shard_stats(ctypes.byref(p), _ptr(q), _ptr(k_local), n_local, key_offset, _ptr(ml), _ptr(ws),
+                               ws.numel() * ws.element_size(), _stream(stream)), "kvc_shard_stats")
+
+
+def kvc_shard_scores(p, q, k_local, key_offset, ml_all, scores, ws, stream=None):
+    n_local = k_local.shape[-2]
+    _check(lib.kvc_shard_scores(ctypes.byref(p), _ptr(q), _ptr(k_local), n_local, key_offset, _ptr(ml_all),
+                                ml_all.shape[0], _ptr(scores), _ptr(ws), ws.numel() * ws.element_size(),
+                                _stream(stream)), "kvc_shard_scores")
+
+
+def kvc_select_hist(pooled, lo, hi, prefix, prefix_bits, digit_bits, hist, stream=None):
+    rows, n = pooled.shape[0] * pooled.shape[1], pooled.shape[-1]
+    _check(lib.kvc_select_hist(_ptr(pooled), rows, n, lo, hi, _ptr(prefix), prefix_bits, digit_bits, _ptr(hist),
+                               _stream(stream)), "kvc_select_hist")
+
+
+def kvc_select_emit(pooled, lo, hi, thr, ties, pos_offset, out, count, stream=None):
+    rows, n = pooled.shape[0] * pooled.shape[1], pooled.shape[-1]
+    _check(lib.kvc_select_emit(_ptr(pooled), rows, n, lo, hi, _ptr(thr), _ptr(ties), pos_offset, _ptr(out),
+                               out.shape[-1], _ptr(count), _stream(stream)), "kvc_select_emit")
 
 
 def kvc_accumulate(acc, src, stream=None):

@@ -75,7 +75,7 @@ CSM_BAND = 1e-5  # cosine band inside which fp32 (GPU) and fp64 (oracle) merge d
 
 
 def check_csm_row(kr, vr, dr, out_k, out_v, out_d, out_p, S, w, chunk, ratio, dtype):
-    """One Chunked Soft Matching row against the oracle: the band rule (CSM_CSM_BAND) on the merge
+    """One Chunked Soft Matching row against the oracle: the band rule (CSM_BAND) on the merge
     set, then every kept row given the GPU's merges (out_p: indices of the kept input rows)."""
     N = kr.shape[0]
     ref = O.csm(kr, vr, dr, n_sink=S, window=w, chunk=chunk, ratio=ratio)
