@@ -18,13 +18,16 @@ void count_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::me
 
 unsigned int* device_error_word() {
     // one address per device; cudaGetSymbolAddress is cheap but not free
-    static unsigned int* cache[64] = {nullptr};
+    static std::atomic<unsigned int*> cache[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return nullptr;
-    if (dev < 64 && cache[dev]) return cache[dev];
+    if (dev < 64) {
+        unsigned int* c = cache[dev].load();
+        if (c) return c;
+    }
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
-    if (dev < 64) cache[dev] = (unsigned int*)p;
+    if (dev < 64) cache[dev].store((unsigned int*)p);
     return (unsigned int*)p;
 }
 

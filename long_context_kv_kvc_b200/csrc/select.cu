@@ -11,6 +11,8 @@
 // block-wide steps are the digit search and one scan of per-warp counts.
 #include <cooperative_groups.h>
 
+#include <atomic>
+
 #include "kvc_internal.cuh"
 
 namespace cg = cooperative_groups;
@@ -588,14 +590,14 @@ cudaError_t topk_fused(const float* scores, int rows, int N, int n_sink, int win
     const int seg = (n_c + kClusterCtas - 1) / kClusterCtas;
     if (seg > kSegMax) return cudaErrorInvalidValue;
     const size_t smem = sizeof(TopkSmem) - sizeof(uint32_t) * (size_t)(kSegMax - seg);
-    static bool attr_done[64] = {false};
+    static std::atomic<bool> attr_done[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev >= 64 || !attr_done[dev]) {
+    if (dev >= 64 || !attr_done[dev].load()) {
         e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(TopkSmem));
         if (e != cudaSuccess) return e;
-        if (dev < 64) attr_done[dev] = true;
+        if (dev < 64) attr_done[dev].store(true);
     }
     topk_cluster_kernel<<<rows * kClusterCtas, kCtThreads, smem, s>>>(scores, N, n_sink, window, budget,
                                                                      (kernel - 1) / 2, seg, idx);
