@@ -73,6 +73,35 @@ def test_csm_matches_oracle(K, case):
                       c["chunk"], c["ratio"], c["dtype"])
 
 
+EDGE_CASES = [
+    # sinks and window cover the row: no candidate, the round is the identity
+    dict(N=40, S=5, w=35, chunk=16, ratio=0.5),
+    # one chunk shorter than the chunk size, odd length
+    dict(N=50, S=2, w=9, chunk=64, ratio=0.3),
+    # every matchable A token merges (m = n_A: even |C|, chunks of 2, r = 0.5)
+    dict(N=130, S=1, w=1, chunk=2, ratio=0.5),
+    # every A merges with chunks of 128 (one ragged last chunk)
+    dict(N=400, S=0, w=3, chunk=128, ratio=0.5),
+]
+
+
+@pytest.mark.parametrize("case", range(len(EDGE_CASES)))
+def test_csm_edge_cases(K, case):
+    c = EDGE_CASES[case]
+    N, S, w, chunk, ratio = c["N"], c["S"], c["w"], c["chunk"], c["ratio"]
+    for dtype in (torch.bfloat16, torch.float32):
+        k, v = make_kv(1, 2, N, dtype, 50 + case, dup=5)
+        deg = torch.randint(1, 4, (1, 2, N), generator=torch.Generator().manual_seed(case), dtype=torch.int32)
+        out = K.kvc_csm(k.cuda(), v.cuda(), S, w, chunk, ratio, deg=deg.cuda())
+        assert K.kvc_poll_error() == K.KVC_OK
+        m = O.csm_merges(N, S, w, chunk, K.kvc_csm_ratio(ratio, 0.0, 0))
+        assert out["pos_out"].shape[-1] == N - m
+        for h in range(2):
+            check_row(k[0, h], v[0, h], deg[0, h].numpy(), out["k_out"][0, h].cpu(), out["v_out"][0, h].cpu(),
+                      out["deg_out"][0, h].cpu().numpy(), out["pos_out"][0, h].cpu().numpy(), S, w, chunk, ratio,
+                      dtype)
+
+
 def test_csm_identity_and_arguments(K):
     k, v = make_kv(1, 2, 300, torch.bfloat16, 7)
     out = K.kvc_csm(k.cuda(), v.cuda(), 1, 8, 16, 0.0)
