@@ -514,7 +514,10 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
 }
 
 // One warp per (unit, query row): merges the (range, warp) partials of every range that
-// touches the unit, in range and warp order.
+// touches the unit.  The partials' (max, sum) are read 32 at a time, one per lane (the max
+// and the weighted sum are warp reductions); each lane accumulates its 4 dimensions over
+// the partials in order with kCombineDepth loads in flight, the weights broadcast by shuffles.
+constexpr int kCombineDepth = 8;
 __global__ void __launch_bounds__(256)
 decode_tc_combine_kernel(const float2* __restrict__ part_ml, const float* __restrict__ part_o, int U, int Rv, int P,
                          long long X, int T_u, float* __restrict__ out) {
@@ -535,24 +538,45 @@ decode_tc_combine_kernel(const float2* __restrict__ part_ml, const float* __rest
         if (item_start(mid, P, X) < hi) a0 = mid;
         else c_hi = mid - 1;
     }
+    // slot s = 0 .. n_slots - 1 is partial (c_lo + u) * kDtEpiWarps + s (ranges and warps in order)
+    const int n_slots = (c_hi - c_lo + 1) * kDtEpiWarps;
+    const size_t slot0 = ((size_t)(c_lo + u)) * kDtEpiWarps;
     float M = -INFINITY;
-    for (int c = c_lo; c <= c_hi; ++c)
-        for (int w = 0; w < kDtEpiWarps; ++w) M = fmaxf(M, part_ml[((size_t)(c + u) * kDtEpiWarps + w) * 8 + r].x);
+    for (int s0 = 0; s0 < n_slots; s0 += 32) {
+        const int sl = s0 + lane;
+        if (sl < n_slots) M = fmaxf(M, part_ml[(slot0 + sl) * 8 + r].x);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
     float L = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int c = c_lo; c <= c_hi; ++c) {
-        for (int w = 0; w < kDtEpiWarps; ++w) {
-            const size_t i = ((size_t)(c + u) * kDtEpiWarps + w) * 8 + r;
-            const float2 ml = part_ml[i];
-            if (ml.y == 0.f) continue;  // an empty state
-            const float wgt = exp2f(ml.x - M);
-            L = fmaf(ml.y, wgt, L);
-            const float4 ov = *reinterpret_cast<const float4*>(part_o + i * D + 4 * lane);
-            acc[0] = fmaf(ov.x, wgt, acc[0]);
-            acc[1] = fmaf(ov.y, wgt, acc[1]);
-            acc[2] = fmaf(ov.z, wgt, acc[2]);
-            acc[3] = fmaf(ov.w, wgt, acc[3]);
+    const float* po = part_o + (slot0 * 8 + r) * D + 4 * lane;
+    for (int s0 = 0; s0 < n_slots; s0 += 32) {
+        // lane t holds the weight of slot s0 + t (0 past the end and for empty states)
+        const int sl = s0 + lane;
+        const float2 ml = sl < n_slots ? part_ml[(slot0 + sl) * 8 + r] : make_float2(-INFINITY, 0.f);
+        const float wt = ml.y == 0.f ? 0.f : exp2f(ml.x - M);
+        L = fmaf(ml.y, wt, L);
+        const int cnt = min(32, n_slots - s0);
+        for (int t0 = 0; t0 < cnt; t0 += kCombineDepth) {
+            float4 ov[kCombineDepth];
+            float wg[kCombineDepth];
+#pragma unroll
+            for (int t = 0; t < kCombineDepth; ++t) {
+                wg[t] = __shfl_sync(kFull, wt, (t0 + t) & 31);
+                ov[t] = wg[t] != 0.f ? *reinterpret_cast<const float4*>(po + (size_t)(s0 + t0 + t) * 8 * D)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int t = 0; t < kCombineDepth; ++t) {
+                acc[0] = fmaf(ov[t].x, wg[t], acc[0]);
+                acc[1] = fmaf(ov[t].y, wg[t], acc[1]);
+                acc[2] = fmaf(ov[t].z, wg[t], acc[2]);
+                acc[3] = fmaf(ov[t].w, wg[t], acc[3]);
+            }
         }
     }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(kFull, L, off);
     const float inv = 1.f / L;
     *reinterpret_cast<float4*>(out + (size_t)gw * D + 4 * lane) =
         make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);

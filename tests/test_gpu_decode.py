@@ -73,6 +73,7 @@ CASES = [  # B, Hq, Hkv, nq, n, ld, dtype, degrees
     (1, 12, 4, 1, 257, 260, torch.bfloat16, False),  # 3 rows, padded to 4
     (1, 8, 1, 1, 1, 1, torch.bfloat16, True),       # a single cached row
     (1, 4, 4, 1, 4133, 4133, torch.float32, True),  # G = 1
+    (1, 4, 1, 1, 20000, 20000, torch.bfloat16, True),  # one unit over every CTA's range
 ]
 
 
