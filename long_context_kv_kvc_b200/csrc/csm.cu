@@ -19,9 +19,10 @@
 //      products of bf16 values are exact); its diagonal gives the norms, and the thread that
 //      owns an A token's TMEM lane takes the argmax over its chunk's B columns.  fp32 keys
 //      use a CUDA-core kernel over the chunk staged in shared memory;
-//   2. the m best matches per row: the radix top-k over a row of match scores (-inf where
-//      there is no match), then merge flags and per-chunk merge counts, and a per-row scan
-//      of the kept tokens per chunk that gives every chunk its first output slot;
+//   2. the m best matches per row: the radix top-k over the row's A-token match scores (the
+//      A tokens are S + 2i because chunks are even; -inf where there is no match), then merge
+//      flags and per-chunk merge counts, and a per-row scan of the kept tokens per chunk that
+//      gives every chunk its first output slot;
 //   3. write: one CTA per chunk (or per 128 sink / window tokens) brings the block's K and V
 //      rows into shared memory with two bulk copies (a block's rows are contiguous), forms
 //      the merged means there in fp32 (rounded once to the element type), and sends every
@@ -94,13 +95,14 @@ __device__ __forceinline__ void from_f8(const float (&x)[8], uint4 (&r)[2]) {
 
 // ------------------------------------------------------------------------ match, fp32 keys
 
-// One CTA per (row, chunk), blockIdx.x = row * n_chunks + chunk.  score[pos] = the match
-// similarity at A positions with a match, -inf elsewhere in the chunk (and, from the first
-// and last chunk, at the sinks and the window); best[pos] = the matched B position.  The
-// keys are staged in shared memory; each thread forms a 2 x 2 block of A-B dot products.
+// One CTA per (row, chunk), blockIdx.x = row * n_chunks + chunk.  Chunks start at even
+// offsets from S (chunk is even), so the A tokens are the positions S + 2i: score[i] = the
+// match similarity of A token i (-inf without a match), a row of n_A = ceil(|C| / 2) entries;
+// best[pos] = the matched B position.  The keys are staged in shared memory; each thread
+// forms a 2 x 2 block of A-B dot products.
 __global__ void __launch_bounds__(kMatchThreads)
 csm_match_f32_kernel(const float* __restrict__ k, int N, long long ld, int S, int w, int chunk, int n_chunks,
-                     float* __restrict__ score, int32_t* __restrict__ best) {
+                     int n_a_row, float* __restrict__ score, int32_t* __restrict__ best) {
     extern __shared__ __align__(16) float ks[];  // [chunk][kKS]
     __shared__ float inv_norm[128];
     __shared__ float sim[64][65];                // [A index][B index]
@@ -109,7 +111,7 @@ csm_match_f32_kernel(const float* __restrict__ k, int N, long long ld, int S, in
     const int c0 = S + q * chunk, c1 = min(c0 + chunk, hi);
     const int len = c1 - c0;
     const float* kr = k + (size_t)row * ld * D;
-    float* sr = score + (size_t)row * N;
+    float* sr = score + (size_t)row * n_a_row + (c0 - S) / 2;  // A token 0 of this chunk
     int32_t* br = best + (size_t)row * N;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int kW = kMatchThreads / 32;
@@ -118,11 +120,6 @@ csm_match_f32_kernel(const float* __restrict__ k, int N, long long ld, int S, in
         const int t = e / (D / 4), d = (e - t * (D / 4)) * 4;
         *reinterpret_cast<float4*>(ks + t * kKS + d) = __ldcs(reinterpret_cast<const float4*>(kr + (size_t)(c0 + t) * D + d));
     }
-    if (q == 0)
-        for (int j = threadIdx.x; j < S; j += kMatchThreads) sr[j] = -INFINITY;
-    if (c1 == hi)
-        for (int j = hi + threadIdx.x; j < N; j += kMatchThreads) sr[j] = -INFINITY;
-    for (int t = 1 + 2 * threadIdx.x; t < len; t += 2 * kMatchThreads) sr[c0 + t] = -INFINITY;
     __syncthreads();
     // 1 / |k| (0 for a zero key, which makes its similarity 0)
     for (int t = warp; t < len; t += kW) {
@@ -181,7 +178,7 @@ csm_match_f32_kernel(const float* __restrict__ k, int N, long long ld, int S, in
             }
         }
         if (lane == 0) {
-            sr[c0 + 2 * ia] = bb >= 0 ? bs : -INFINITY;
+            sr[ia] = bb >= 0 ? bs : -INFINITY;
             br[c0 + 2 * ia] = bb >= 0 ? c0 + 2 * bb + 1 : -1;
         }
     }
@@ -198,6 +195,7 @@ struct TcMatchArgs {
     int tt;             // tokens per tile: a whole number of chunks, <= 128
     int tiles_per_row;  // ceil(|C| / tt)
     int total_tiles;
+    int n_a_row;        // A tokens per row: score row length
 };
 
 struct __align__(1024) MatchSmem {
@@ -222,6 +220,7 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, unsig
 // Persistent: CTA c takes the global tiles c, c + P, ...  (row-major over (row, tile)).
 // Tile (u, tau) covers tokens t0 = S + tau * tt .. t0 + 127 of row u (tokens past the tile's
 // chunks are loaded and ignored; past N they read as 0).  D[r][j] = k_{t0+r} . k_{t0+j}.
+// Writes score[u][i] for the row's A tokens S + 2i and best[u][pos] at A positions.
 __global__ void __launch_bounds__(kTcThreads, 1) csm_match_tc_kernel(const __grid_constant__ TcMatchArgs a) {
     extern __shared__ uint8_t smem_raw[];
     MatchSmem& sm = *reinterpret_cast<MatchSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -376,15 +375,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) csm_match_tc_kernel(const __gri
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.accempty[grp]);
-            float* sr = a.score + (size_t)u * a.N;
-            if (r < valid) {
-                sr[t0 + r] = is_a && bb >= 0 ? bs : -INFINITY;
-                if (is_a) a.best[(size_t)u * a.N + t0 + r] = bb >= 0 ? t0 + bb : -1;
+            if (is_a) {  // A token (t0 + r - S) / 2 of the row (tiles start at even offsets)
+                a.score[(size_t)u * a.n_a_row + (t0 + r - a.S) / 2] = bb >= 0 ? bs : -INFINITY;
+                a.best[(size_t)u * a.N + t0 + r] = bb >= 0 ? t0 + bb : -1;
             }
-            if (tau == 0)
-                for (int j = r; j < a.S; j += kTileTok) sr[j] = -INFINITY;
-            if (tau == a.tiles_per_row - 1)
-                for (int j = a.N - a.w + r; j < a.N; j += kTileTok) sr[j] = -INFINITY;
         }
     }
 
@@ -399,7 +393,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) csm_match_tc_kernel(const __gri
 
 // ------------------------------------------------------------------------ selection bookkeeping
 
-// merged[pos] = 1 for the selected A positions; cb[row][c] counts the merges of chunk c.
+// merged[pos] = 1 for the selected A tokens (sel holds A indices i, position S + 2i);
+// cb[row][c] counts the merges of chunk c.
 __global__ void csm_mark_kernel(const int32_t* __restrict__ sel, int rows, int N, int S, int w, int chunk, int m,
                                 int n_chunks, unsigned char* __restrict__ merged, int32_t* __restrict__ cb,
                                 unsigned* __restrict__ err) {
@@ -407,8 +402,8 @@ __global__ void csm_mark_kernel(const int32_t* __restrict__ sel, int rows, int N
     for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
          e += (long long)gridDim.x * blockDim.x) {
         const long long row = e / m;
-        const int p = sel[e];
-        if (p < S || p >= N - w) {  // never for a well-formed selection
+        const int p = S + 2 * sel[e];  // A token sel[e] of the row
+        if (sel[e] < 0 || p >= N - w) {  // never for a well-formed selection
             atomicOr(err, kErrIndex);
             continue;
         }
@@ -658,6 +653,7 @@ cudaError_t match_tc(const void* k, int rows, int N, long long ld, int S, int w,
     a.chunk = chunk;
     a.tt = (kTileTok / chunk) * chunk;
     a.tiles_per_row = (N - w - S + a.tt - 1) / a.tt;
+    a.n_a_row = (N - w - S + 1) / 2;
     const long long total = (long long)rows * a.tiles_per_row;
     if (total > (1LL << 31) - 1) return cudaErrorInvalidValue;
     a.total_tiles = (int)total;
@@ -691,7 +687,7 @@ cudaError_t match_tc(const void* k, int rows, int N, long long ld, int S, int w,
 }
 
 cudaError_t match_f32(const float* k, int rows, int N, long long ld, int S, int w, int chunk, int n_chunks,
-                      float* score, int32_t* best, cudaStream_t s) {
+                      int n_a_row, float* score, int32_t* best, cudaStream_t s) {
     static std::atomic<bool> attr_set[64];
     int dev = 0;
     cudaError_t e;
@@ -705,7 +701,7 @@ cudaError_t match_f32(const float* k, int rows, int N, long long ld, int S, int 
     const long long grid = (long long)rows * n_chunks;
     if (grid > (1LL << 31) - 1) return cudaErrorInvalidValue;
     csm_match_f32_kernel<<<(unsigned)grid, kMatchThreads, (size_t)chunk * kKS * sizeof(float), s>>>(
-        k, N, ld, S, w, chunk, n_chunks, score, best);
+        k, N, ld, S, w, chunk, n_chunks, n_a_row, score, best);
     count_launches(1);
     return cudaGetLastError();
 }
@@ -735,12 +731,14 @@ cudaError_t csm(const void* k, const void* v, int dtype, const int32_t* deg, con
     if ((e = cudaMemsetAsync(merged, 0, rn, s)) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(cb, 0, (size_t)rows * (n_chunks + 1) * sizeof(int32_t), s)) != cudaSuccess) return e;
     if (m > 0 && n_chunks > 0) {
-        e = dtype == KVC_BF16 ? match_tc(k, rows, N, ld_in, S, w, chunk, score, best, s)
-                              : match_f32((const float*)k, rows, N, ld_in, S, w, chunk, n_chunks, score, best, s);
+        const int n_a_row = (hi - S + 1) / 2;  // A tokens S, S + 2, ... of C
+        e = dtype == KVC_BF16
+                ? match_tc(k, rows, N, ld_in, S, w, chunk, score, best, s)
+                : match_f32((const float*)k, rows, N, ld_in, S, w, chunk, n_chunks, n_a_row, score, best, s);
         if (e != cudaSuccess) return e;
-        // the m best matches (ties to the lower position), ascending
-        e = topk_fused_fits(N, 0, 0) ? topk_fused(score, rows, N, 0, 0, m, 1, sel, s)
-                                     : topk(score, rows, N, 0, 0, m, sel, s);
+        // the m best matches over the row of A scores (ties to the lower position), ascending
+        e = topk_fused_fits(n_a_row, 0, 0) ? topk_fused(score, rows, n_a_row, 0, 0, m, 1, sel, s)
+                                           : topk(score, rows, n_a_row, 0, 0, m, sel, s);
         if (e != cudaSuccess) return e;
         const long long total = (long long)rows * m;
         csm_mark_kernel<<<(int)std::min<long long>((total + 255) / 256, 148LL * 8), 256, 0, s>>>(
