@@ -248,13 +248,20 @@ topk_cluster_kernel(const float* __restrict__ scores, int N, int S, int w, int b
         for (int i = tid; i < S; i += kCtThreads) out[i] = i;
         for (int i = tid; i < w; i += kCtThreads) out[budget - w + i] = N - w + i;
     }
-    // pooled keys of this CTA's candidates (max over the clipped window of raw scores)
+    // pooled keys of this CTA's candidates (max over the clipped window of raw scores); the
+    // first digit's histogram (the top 11 bits of every key) is counted as they are formed
+    for (int i = tid; i < kBins; i += kCtThreads) sm.hist[i] = 0u;
+    __syncthreads();
     for (int e = tid; e < n_mine; e += kCtThreads) {
         const int j = s0 + e;
         const int t0 = max(lo, j - radius), t1 = min(hi - 1, j + radius);
         float m = __ldg(v + t0);
         for (int t = t0 + 1; t <= t1; ++t) m = fmaxf(m, __ldg(v + t));
-        sm.keys[e] = order_key(m);
+        const uint32_t key = order_key(m);
+        sm.keys[e] = key;
+        const unsigned digit = key >> 21;
+        const unsigned peers = __match_any_sync(__activemask(), digit);
+        if (lane == __ffs(peers) - 1) atomicAdd(&sm.hist[digit], (unsigned)__popc(peers));
     }
 
     uint32_t prefix = 0, mask = 0;
@@ -264,14 +271,16 @@ topk_cluster_kernel(const float* __restrict__ scores, int N, int S, int w, int b
     for (int pass = 0; pass < 3; ++pass) {
         const int shift = shifts[pass];
         const uint32_t dmask = (1u << widths[pass]) - 1u;
-        for (int i = tid; i < kBins; i += kCtThreads) sm.hist[i] = 0u;
-        __syncthreads();
-        for (int e = tid; e < n_mine; e += kCtThreads) {
-            const uint32_t key = sm.keys[e];
-            if ((key & mask) == prefix) {
-                const unsigned digit = (key >> shift) & dmask;
-                const unsigned peers = __match_any_sync(__activemask(), digit);
-                if (lane == __ffs(peers) - 1) atomicAdd(&sm.hist[digit], (unsigned)__popc(peers));
+        if (pass > 0) {  // the first pass's histogram was built with the keys
+            for (int i = tid; i < kBins; i += kCtThreads) sm.hist[i] = 0u;
+            __syncthreads();
+            for (int e = tid; e < n_mine; e += kCtThreads) {
+                const uint32_t key = sm.keys[e];
+                if ((key & mask) == prefix) {
+                    const unsigned digit = (key >> shift) & dmask;
+                    const unsigned peers = __match_any_sync(__activemask(), digit);
+                    if (lane == __ffs(peers) - 1) atomicAdd(&sm.hist[digit], (unsigned)__popc(peers));
+                }
             }
         }
         cluster.sync();  // every CTA's histogram is complete
