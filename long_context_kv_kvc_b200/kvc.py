@@ -208,6 +208,8 @@ def kvc_csm(k, v, n_sink, window, chunk, ratio, deg=None, out=None, ws=None, str
     pos (nullable) share k's row layout; without `out` the outputs are dense (cap_out =
     N - m) unless ld_out is given."""
     B, H, cap, D = k.shape
+    if v.dtype != k.dtype or v.shape != k.shape:
+        raise KvcError(KVC_ERR_ARG, "kvc_csm: k and v must have the same shape and dtype")
     N = cap if n is None else n
     dt = KVC_BF16 if k.dtype == torch.bfloat16 else KVC_F32
     m = kvc_csm_merges(N, n_sink, window, chunk, ratio)
@@ -233,6 +235,8 @@ def kvc_append(k_cache, v_cache, n, k_new, v_new, deg_cache=None, pos_cache=None
     [B, H, cap, D] (degrees 1, positions pos0 ..)."""
     B, H, cap, D = k_cache.shape
     t_new = k_new.shape[2]
+    if not (k_new.dtype == v_new.dtype == v_cache.dtype == k_cache.dtype):
+        raise KvcError(KVC_ERR_ARG, "kvc_append: caches and new rows must share one dtype")
     dt = KVC_BF16 if k_cache.dtype == torch.bfloat16 else KVC_F32
     _check(lib.kvc_append(_ptr(k_cache), _ptr(v_cache), _ptr(deg_cache) if deg_cache is not None else None,
                           _ptr(pos_cache) if pos_cache is not None else None, B, H, cap, n, _ptr(k_new), _ptr(v_new),
@@ -252,6 +256,8 @@ def kvc_decode_attention(q, k, v, deg=None, n=None, out=None, ws=None, stream=No
     returns out [B, Hq, nq, D] fp32."""
     B, Hq, nq, D = q.shape
     _, Hkv, cap, _ = k.shape
+    if q.dtype != k.dtype or v.dtype != k.dtype or v.shape != k.shape:
+        raise KvcError(KVC_ERR_ARG, "kvc_decode_attention: q, k and v must share one dtype; k and v one shape")
     n = cap if n is None else n
     dt = KVC_BF16 if k.dtype == torch.bfloat16 else KVC_F32
     if out is None:
