@@ -140,3 +140,74 @@ def test_status_strings(K):
         assert len(K.kvc_status_string(st)) >= 2
     assert "unknown" in K.kvc_status_string(99)
     assert K.kvc_version().startswith("kvc ")
+
+
+def test_next_rows_validate_on_host(K, oracle_lib):
+    # every call below fails validation on the host: none reaches a launch with the fake pointers
+    L = K.lib
+    F2 = ctypes.c_void_p((1 << 20) + 4096)  # a second distinct fake buffer
+    sz = ctypes.c_size_t
+    # Chunked Soft Matching: merge count, workspace, argument checks
+    for args in [(1000, 1, 32, 64, 0.25), (777, 0, 0, 2, 0.5), (515, 1, 3, 6, 0.45), (40, 5, 35, 16, 0.5),
+                 (130, 1, 1, 2, 0.5), (9, 0, 0, 4, 0.5)]:
+        assert K.kvc_csm_merges(*args) == oracle_lib.csm_merges(*args)
+    assert L.kvc_csm_merges(100, 1, 8, 3, 0.25) == -1      # odd chunk
+    assert L.kvc_csm_merges(100, 1, 8, 130, 0.25) == -1    # chunk > 128
+    assert L.kvc_csm_merges(100, 1, 8, 16, 0.6) == -1      # ratio > 0.5
+    n = sz()
+    assert L.kvc_csm_workspace_size(1, 2, 1000, 1, 32, 64, ctypes.c_float(0.25), ctypes.byref(n)) == K.KVC_OK
+    assert n.value > 0
+    def csm(k=FAKE, v=F2, ko=ctypes.c_void_p(1 << 22), vo=ctypes.c_void_p(1 << 23), N=1000, ld_in=0, ld_out=0,
+            D=128, dtype=K.KVC_BF16, chunk=64, ratio=0.25, ws_bytes=1 << 40):
+        return L.kvc_csm(k, v, None, None, 1, 2, N, ld_in, D, dtype, 1, 32, chunk, ctypes.c_float(ratio), ko, vo,
+                         FAKE, FAKE, ld_out, FAKE, ws_bytes, None)
+    assert csm(k=None) == K.KVC_ERR_ARG
+    assert csm(ko=FAKE) == K.KVC_ERR_ARG                   # in place
+    assert csm(chunk=7) == K.KVC_ERR_ARG
+    assert csm(ld_in=999) == K.KVC_ERR_ARG                 # capacity below N
+    assert csm(D=64) == K.KVC_ERR_UNSUPPORTED
+    assert csm(dtype=9) == K.KVC_ERR_UNSUPPORTED
+    assert csm(k=ctypes.c_void_p((1 << 20) + 8)) == K.KVC_ERR_ALIGN
+    assert csm(ws_bytes=10) == K.KVC_ERR_WORKSPACE
+    # append
+    assert L.kvc_append(FAKE, F2, None, None, 1, 2, 100, 90, FAKE, F2, 11, 0, 128, K.KVC_BF16, None) == K.KVC_ERR_ARG
+    assert L.kvc_append(FAKE, F2, None, None, 1, 2, 100, 90, FAKE, F2, 5, 0, 64, K.KVC_BF16, None) == \
+        K.KVC_ERR_UNSUPPORTED
+    # decode attention
+    def dec(q=FAKE, Hq=32, Hkv=8, nq=1, n=1000, ld=0, D=128, dtype=K.KVC_BF16, ws_bytes=1 << 40):
+        return L.kvc_decode_attention(q, FAKE, F2, None, 1, Hq, Hkv, nq, n, ld, D, dtype, FAKE, FAKE, ws_bytes, None)
+    assert dec(q=None) == K.KVC_ERR_ARG
+    assert dec(Hq=30) == K.KVC_ERR_ARG                     # Hq % Hkv
+    assert dec(nq=3) == K.KVC_ERR_UNSUPPORTED              # 12 query rows per KV head
+    assert dec(ld=999) == K.KVC_ERR_ARG                    # capacity below n
+    assert dec(D=64) == K.KVC_ERR_UNSUPPORTED
+    assert dec(q=ctypes.c_void_p((1 << 20) + 8)) == K.KVC_ERR_ALIGN
+    assert dec(ws_bytes=10) == K.KVC_ERR_WORKSPACE
+    small, big = K.kvc_decode_attention_workspace_size(1, 32, 8, 1, 1000), \
+        K.kvc_decode_attention_workspace_size(4, 32, 8, 1, 98313)
+    assert 0 < small <= big
+    # sequence sharding and the distributed select
+    p = _p(K)
+    assert L.kvc_shard_workspace_size(ctypes.byref(_p(K, scope=K.KVC_SCOPE_ALL_HEADS)), 100, ctypes.byref(n)) == \
+        K.KVC_ERR_UNSUPPORTED
+    assert L.kvc_shard_workspace_size(ctypes.byref(p), 100, ctypes.byref(n)) == K.KVC_OK and n.value > 0
+    assert L.kvc_shard_stats(ctypes.byref(p), FAKE, FAKE, 100, 4000, FAKE, FAKE, 1 << 40, None) == K.KVC_ERR_ARG
+    assert L.kvc_shard_stats(ctypes.byref(p), FAKE, FAKE, 100, 0, FAKE, FAKE, 10, None) == K.KVC_ERR_WORKSPACE
+    assert L.kvc_shard_scores(ctypes.byref(p), FAKE, FAKE, 100, 0, FAKE, 0, FAKE, FAKE, 1 << 40, None) == \
+        K.KVC_ERR_ARG                                      # no shards
+    assert L.kvc_select_hist(FAKE, 2, 100, 0, 100, FAKE, 0, 13, FAKE, None) == K.KVC_ERR_ARG  # 13-bit digit
+    assert L.kvc_select_hist(FAKE, 2, 100, 0, 100, FAKE, 22, 11, FAKE, None) == K.KVC_ERR_ARG  # 33 bits
+    assert L.kvc_select_hist(FAKE, 2, 100, 50, 40, FAKE, 0, 11, FAKE, None) == K.KVC_ERR_ARG   # lo > hi
+    assert L.kvc_select_emit(FAKE, 2, 100, 0, 100, FAKE, FAKE, -1, FAKE, 100, FAKE, None) == K.KVC_ERR_ARG
+
+
+def test_binding_rejects_mixed_dtypes(K):
+    import torch
+    q = torch.zeros(1, 4, 1, 128, dtype=torch.float32)
+    k = torch.zeros(1, 1, 10, 128, dtype=torch.bfloat16)
+    with pytest.raises(K.KvcError):
+        K.kvc_decode_attention(q, k, k)
+    with pytest.raises(K.KvcError):
+        K.kvc_csm(k, k.float(), 1, 2, 4, 0.25)
+    with pytest.raises(K.KvcError):
+        K.kvc_append(k, k, 0, k.float(), k.float())
