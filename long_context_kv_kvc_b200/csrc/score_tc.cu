@@ -35,10 +35,12 @@
 //   * an lse warp waits for each unit's count, turns the totals into lse = ref + log2(total)
 //     in shared memory and releases the unit's phase-2 jobs; a phase-2 job gives each key
 //     of the tile its sum over the query rows of 2^(y - lse).
-// Two TMA producers with their own shared-memory rings (16 KiB half-tiles of 64 columns,
-// the 128-byte swizzle atom) keep the HBM stream independent of phase-2 waits.  Warps:
-// 0 phase-1 TMA, 1 TMEM owner + phase-1 MMA, 2 phase-2 TMA, 3 phase-2 MMA, 4 lse,
-// 5 publisher, 6-7 idle, 8-23 consumers (four warpgroups, one per accumulator).  Every
+// Phase 1 streams each 128-key tile from HBM as one 32 KiB TMA op (both 64-column halves, the
+// 128-byte swizzle atom) into a 2-tile ring; phase 2 re-reads each tile as two 16 KiB halves,
+// issued by two threads, into a 3-stage ring (a single issuing thread completes TMA ops at a
+// roughly fixed rate, so large ops and several issuers stream faster).  Warps: 0 phase-1 TMA,
+// 1 TMEM owner + phase-1 MMA, 2 and 6 phase-2 TMA (halves 0 and 1), 3 phase-2 MMA, 4 lse,
+// 5 publisher, 7 idle, 8-23 consumers (four warpgroups, one per accumulator).  Every
 // wait is bounded: a wait that runs out sets the per-device error word and the kernel
 // still ends.
 #include <cuda.h>
@@ -68,7 +70,8 @@ constexpr int kBoxBytes = kTileKeys * 64 * 2;          // a 128-row x 64-column 
 #ifndef KVC_TC_LEAD_SLACK
 #define KVC_TC_LEAD_SLACK 6
 #endif
-constexpr int kStagesA = KVC_TC_STAGES_A;              // phase-1 ring (HBM stream)
+constexpr int kStagesA = KVC_TC_STAGES_A;              // phase-1 ring, in 16 KiB halves (HBM stream)
+constexpr int kTilesA = kStagesA / 2;                  // the same ring in whole tiles (one op each)
 constexpr int kStagesB = KVC_TC_STAGES_B;              // phase-2 ring (L2 re-read)
 constexpr int kQSlots = KVC_TC_Q_SLOTS;                // Q of the CTA's last units, by unit ordinal
 constexpr int kLeadSlack = KVC_TC_LEAD_SLACK;          // phase-1 lead beyond one unit, in tiles
@@ -85,7 +88,9 @@ constexpr int kMaxCtas = 160;                          // upper bound on the per
 constexpr uint32_t kTmemCols = 512;
 
 struct TcArgs {
-    CUtensorMap tmap_k;  // K as [U][N][128] bf16, box 64 x 128 x 1, 128-byte swizzle
+    CUtensorMap tmap_k;  // K as [U][N][128] bf16, box 64 x 128 x 1, 128-byte swizzle (a half tile)
+    CUtensorMap tmap_k4; // K as [U][2 halves][N][64] (strides: key 256 B, half 128 B), box 64 x 128 x 2 x 1,
+                         // 128-byte swizzle: a whole tile in one op, the two halves one after the other
     CUtensorMap tmap_q;  // padded Q as [U*128][128] bf16, box 64 x 128, 128-byte swizzle
     float* unit_scores;  // [U][N]
     const float* ref;    // [U][128] per-row reference logit (base 2): the row's own-position key
@@ -121,6 +126,51 @@ struct __align__(1024) Smem {
     int abort;
     int p1_issued, p2_issued;  // tiles whose loads each producer has issued (L2 lead control)
 };
+
+// Spinning bounded wait (no suspension) for the single-thread roles, which must react fast.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ void mbar_spin(uint64_t* bar, uint32_t parity, volatile int* abort, unsigned* err) {
+    if (mbar_test(bar, parity)) return;
+    const long long t0 = globaltimer();
+    while (!mbar_test(bar, parity)) {
+        if (*abort) return;
+        if (globaltimer() - t0 > kBarrierTimeoutNs) {
+            atomicOr(err, kErrTimeout);
+            *abort = 1;
+            return;
+        }
+    }
+}
+
+// Bounded wait that ignores the fail-fast flag: after a time-out elsewhere, the producers
+// wait for their own copies still in flight before the CTA exits.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsigned* err) {
+    const long long t0 = globaltimer();
+    while (!mbar_test(bar, parity)) {
+        if (globaltimer() - t0 > kBarrierTimeoutNs) {
+            atomicOr(err, kErrTimeout);
+            return;
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z,
+                                            int w) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], [%2];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "r"(w)
+        : "memory");
+}
 
 __device__ __forceinline__ float ex2(float x) {
     float y;
@@ -313,21 +363,20 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
 
-    if (warp == 0 || warp == 2) {
+    if (warp == 0 || warp == 2 || warp == 6) {
         // ------------------------------------------------------------ TMA producers
+        // Warp 0 streams the phase-1 tiles from HBM, one 32 KiB op per tile (both 64-column
+        // halves); warps 2 and 6 issue the phase-2 re-reads, half 0 and half 1 of every tile.
+        // A single issuing thread completes TMA ops at a roughly fixed rate, so the phase-1
+        // stream uses large ops and the phase-2 stream two threads.
         if (lane == 0) {
-            const int ph = warp == 0 ? 0 : 1;
-            const CUtensorMap* mk = &a.tmap_k;
+            const int ph = warp == 0 ? 0 : 1, hh = warp == 6 ? 1 : 0;
+            const CUtensorMap* mk = ph == 0 ? &a.tmap_k4 : &a.tmap_k;
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(mk)) : "memory");
             const uint64_t evict_first = policy_evict_first();
-            uint8_t(*ring)[kBoxBytes] = ph == 0 ? sm.ringA : sm.ringB;
-            uint64_t* full = ph == 0 ? sm.fullA : sm.fullB;
-            uint64_t* empty = ph == 0 ? sm.emptyA : sm.emptyB;
-            const int stages = ph == 0 ? kStagesA : kStagesB;
-            volatile int* mine = ph == 0 ? &sm.p1_issued : &sm.p2_issued;
             volatile int* other = ph == 0 ? &sm.p2_issued : &sm.p1_issued;
-            int k = 0, qunit = -1, ord = -1;
-            for (int i = 0; i < n_local && !*abort; ++i) {
+            int qunit = -1, ord = -1, i = 0;
+            for (; i < n_local && !*abort; ++i) {
                 const int u = seq.unit(i), ti = seq.tile(i);
                 // phase 1 stays at most max_lead tiles ahead of phase 2 (L2 footprint);
                 // phase 2 never loads a tile before phase 1 has (so its read hits L2)
@@ -340,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                             *abort = 1;
                             break;
                         }
-                        __nanosleep(64);
+                        __nanosleep(32);
                     }
                 }
                 if (ph == 0 && u != qunit) {
@@ -349,21 +398,38 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                     qunit = u;
                     ++ord;
                     const int slot = ord % kQSlots;
-                    if (ord >= kQSlots) mbar_wait(&sm.qempty[slot], ((ord / kQSlots) - 1) & 1, abort, a.err);
+                    if (ord >= kQSlots) mbar_spin(&sm.qempty[slot], ((ord / kQSlots) - 1) & 1, abort, a.err);
                     mbar_expect_tx(&sm.qfull[slot], 2 * kBoxBytes);
                     tma_load_2d(sm.q[slot], &a.tmap_q, &sm.qfull[slot], 0, u * kQRows);
                     tma_load_2d(sm.q[slot] + kBoxBytes, &a.tmap_q, &sm.qfull[slot], 64, u * kQRows);
                 }
-                for (int h = 0; h < 2; ++h, ++k) {
-                    const int s = k % stages;
-                    mbar_wait(&empty[s], ((k / stages) & 1) ^ 1, abort, a.err);
-                    mbar_expect_tx(&full[s], kBoxBytes);
-                    if (ph == 0)
-                        tma_load_3d(ring[s], mk, &full[s], 64 * h, ti * kTileKeys, u);
-                    else
-                        tma_load_3d_hint(ring[s], mk, &full[s], 64 * h, ti * kTileKeys, u, evict_first);
+                if (ph == 0) {
+                    const int st = i % kTilesA;
+                    mbar_spin(&sm.emptyA[st], ((i / kTilesA) & 1) ^ 1, abort, a.err);
+                    mbar_expect_tx(&sm.fullA[st], 2 * kBoxBytes);
+                    tma_load_4d(sm.ringA[2 * st], mk, &sm.fullA[st], 0, ti * kTileKeys, 0, u);
+                    *reinterpret_cast<volatile int*>(&sm.p1_issued) = i + 1;
+                } else {
+                    const int k = 2 * i + hh, st = k % kStagesB;
+                    mbar_spin(&sm.emptyB[st], ((k / kStagesB) & 1) ^ 1, abort, a.err);
+                    mbar_expect_tx(&sm.fullB[st], kBoxBytes);
+                    tma_load_3d_hint(sm.ringB[st], mk, &sm.fullB[st], 64 * hh, ti * kTileKeys, u, evict_first);
+                    if (hh == 0) *reinterpret_cast<volatile int*>(&sm.p2_issued) = i + 1;
                 }
-                *mine = i + 1;
+            }
+            if (*abort) {
+                // copies still in flight land before the CTA exits
+                if (ph == 0) {
+                    for (int n = std::max(0, i - kTilesA); n < i; ++n)
+                        drain_wait(&sm.fullA[n % kTilesA], (n / kTilesA) & 1, a.err);
+                    for (int o = std::max(0, ord - kQSlots + 1); o <= ord; ++o)
+                        drain_wait(&sm.qfull[o % kQSlots], (o / kQSlots) & 1, a.err);
+                } else {
+                    for (int n = std::max(0, i - 2); n < i; ++n) {
+                        const int k = 2 * n + hh;
+                        drain_wait(&sm.fullB[k % kStagesB], (k / kStagesB) & 1, a.err);
+                    }
+                }
             }
         }
     } else if (warp == 1 || warp == 3) {
@@ -374,52 +440,58 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
         // issuers keep the tensor pipe busy while either does its bookkeeping.
         if (lane == 0) {
             const int ph = warp == 1 ? 0 : 1;
-            const int stages = ph == 0 ? kStagesA : kStagesB;
-            uint64_t* full = ph == 0 ? sm.fullA : sm.fullB;
-            uint64_t* empty = ph == 0 ? sm.emptyA : sm.emptyB;
             const uint64_t dK0 = sw128_desc(smem_u32(ph == 0 ? sm.ringA[0] : sm.ringB[0]));
             const uint64_t dQ0 = sw128_desc(smem_u32(sm.q[0]));
             constexpr uint64_t kBoxStep = kBoxBytes >> 4, kQStep = (2 * kBoxBytes) >> 4;
             int u = cta / a.T_u, t = cta - (cta / a.T_u) * a.T_u;  // unit and tile of local tile i
             int ord = 0, qslot = 0;                                 // unit ordinal, its Q slot
             int s = 0;
-            uint32_t sph = 0;  // ring stage and phase
+            uint32_t sph = 0;  // phase-2 ring stage and phase
             bool have_q = false;
             for (int i = 0; i < n_local && !*abort; ++i) {
                 if (!have_q) {
                     // the unit's Q (its slot is not refilled before phase 2 releases it)
-                    mbar_wait(&sm.qfull[qslot], (ord / kQSlots) & 1, abort, a.err);
+                    mbar_spin(&sm.qfull[qslot], (ord / kQSlots) & 1, abort, a.err);
                     have_q = true;
                 }
                 // phase 2 of a tile waits until its unit's lse is in shared memory
-                if (ph == 1) mbar_wait(&sm.lsefull[ord & 1], (ord >> 1) & 1, abort, a.err);
-                mbar_wait(&full[s], sph, abort, a.err);
+                if (ph == 1) mbar_spin(&sm.lsefull[ord & 1], (ord >> 1) & 1, abort, a.err);
+                if (ph == 0)
+                    mbar_spin(&sm.fullA[i % kTilesA], (i / kTilesA) & 1, abort, a.err);
+                else
+                    mbar_spin(&sm.fullB[s], sph, abort, a.err);
                 const int n = atomicAdd(&sm.next_job, 1);
                 const int slot = n % kAcc;
                 // Accumulators are taken in job order: job n waits for the release of job
                 // n - kAcc only after job n - 1 has taken its own, so that the accumulator's
                 // barrier is never two phases behind this wait (a parity wait would pass).
                 spin_until_at_least(&sm.jobs_started, n, abort, a.err);
-                mbar_wait(&sm.accempty[slot], ((n / kAcc) & 1) ^ 1, abort, a.err);
+                mbar_spin(&sm.accempty[slot], ((n / kAcc) & 1) ^ 1, abort, a.err);
                 tc_fence_after();
                 *reinterpret_cast<volatile int*>(&sm.jobs_started) = n + 1;
                 sm.job[slot] = make_int4(ph, u, t, ph == 0 ? i : (ord & 1));
                 mbar_arrive(&sm.accfull[slot]);
                 const uint32_t d = tmem + slot * 128;
                 const uint64_t dq = dQ0 + (uint64_t)qslot * kQStep;
+                if (ph == 0) {
+                    // both halves of the tile arrived with one op
+                    const int st = i % kTilesA;
+                    const uint64_t dk = dK0 + (uint64_t)(2 * st) * kBoxStep;
+                    umma_half(d, dq, dk, 0);
+                    umma_half(d, dq + kBoxStep, dk + kBoxStep, 1);
+                    umma_commit(&sm.emptyA[st]);
+                } else {
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    if (h == 1) mbar_wait(&full[s], sph, abort, a.err);
-                    tc_fence_after();
-                    const uint64_t dk = dK0 + (uint64_t)s * kBoxStep;
-                    if (ph == 0)
-                        umma_half(d, dq + h * kBoxStep, dk, h);
-                    else
+                    for (int h = 0; h < 2; ++h) {
+                        if (h == 1) mbar_spin(&sm.fullB[s], sph, abort, a.err);
+                        tc_fence_after();
+                        const uint64_t dk = dK0 + (uint64_t)s * kBoxStep;
                         umma_half(d, dk, dq + h * kBoxStep, h);
-                    umma_commit(&empty[s]);
-                    if (++s == stages) {
-                        s = 0;
-                        sph ^= 1u;
+                        umma_commit(&sm.emptyB[s]);
+                        if (++s == kStagesB) {
+                            s = 0;
+                            sph ^= 1u;
+                        }
                     }
                 }
                 umma_commit(&sm.accfull[slot]);
@@ -830,6 +902,16 @@ cudaError_t tc_score(const ScoreJob& j, cudaStream_t s) {
     auto encode = encode_fn();
     if (!encode) return cudaErrorNotSupported;
     {
+        // K as [U][2 halves][N][64]: a box of 64 x 128 x 2 lands the tile's two 64-column halves
+        // one after the other, each in the 128-byte-swizzled layout the MMA reads
+        cuuint64_t dims4[4] = {64, (cuuint64_t)j.N, 2, (cuuint64_t)j.U};
+        cuuint64_t strides4[3] = {(cuuint64_t)kHeadDim * 2, 128, (cuuint64_t)j.N * kHeadDim * 2};
+        cuuint32_t box4[4] = {64, kTileKeys, 2, 1};
+        cuuint32_t estr4[4] = {1, 1, 1, 1};
+        if (encode(&a.tmap_k4, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(j.k), dims4, strides4, box4,
+                   estr4, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
         cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)j.N, (cuuint64_t)j.U};
         cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)j.N * kHeadDim * 2};
         cuuint32_t box[3] = {64, kTileKeys, 1};
