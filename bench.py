@@ -178,21 +178,28 @@ def summarize_clocks(rows) -> dict:
 
 # ----------------------------------------------------------------------------- CPU legs
 
-def oracle_sample(wl: synth.Workload, inputs: dict, heads: int, threads: int) -> tuple:
-    """Runs the fp64 oracle on sequence 0, KV heads [0, heads) (the sample) and returns
-    (seconds, equivalent context tokens = N * heads / Hkv)."""
+def oracle_units(wl: synth.Workload) -> tuple:
+    """The CPU sample: as many (sequence, KV head) units as the host has cores (the oracle
+    runs one unit per thread), whole sequences first; returns (sequences, KV heads each)."""
+    cores = os.cpu_count() or 1
+    if cores >= wl.Hkv:
+        return max(1, min(wl.B, cores // wl.Hkv)), wl.Hkv
+    return 1, cores
+
+
+def oracle_sample(wl: synth.Workload, inputs: dict, n_seq: int, heads: int) -> tuple:
+    """Runs the fp64 oracle on sequences [0, n_seq), KV heads [0, heads) of each (the
+    sample), one thread per unit; returns (seconds, equivalent context tokens)."""
     from oracle import oracle as O
     G = wl.G
-    q = inputs["q"][:, :1, :heads * G]
-    k = inputs["k"][:, :1, :heads]
-    v = inputs["v"][:1, :heads]
-    wsub = wl.replace(B=1, Hq=heads * G, Hkv=heads)
+    q = inputs["q"][:, :n_seq, :heads * G]
+    k = inputs["k"][:, :n_seq, :heads]
+    v = inputs["v"][:n_seq, :heads]
     t0 = time.perf_counter()
     O.compress(q, k, v, window=wl.window, n_sink=wl.n_sink, pool_kernel=wl.pool_kernel,
-               kv_budget=wl.kv_budget, scope=wl.scope, threads=threads)
+               kv_budget=wl.kv_budget, scope=wl.scope, threads=n_seq * heads)
     dt = time.perf_counter() - t0
-    del wsub
-    return dt, wl.N * heads / wl.Hkv
+    return dt, wl.N * n_seq * heads / wl.Hkv
 
 
 def run_reference(args, wl, rank, world):
@@ -201,21 +208,22 @@ def run_reference(args, wl, rank, world):
         return 0
     inputs = synth.make_inputs(wl, seeds=rank_seeds(wl, 0), with_hidden=False)
     cores = os.cpu_count() or 1
-    heads = 1
+    n_seq, heads = oracle_units(wl)
     for _ in range(max(args.warmup, 0)):
-        oracle_sample(wl, inputs, heads, 1)
+        oracle_sample(wl, inputs, n_seq, heads)
     total_t, total_tok = 0.0, 0.0
     for _ in range(args.steps):
-        dt, tok = oracle_sample(wl, inputs, heads, 1)
+        dt, tok = oracle_sample(wl, inputs, n_seq, heads)
         total_t += dt
         total_tok += tok
     value = total_tok / total_t
-    sample = f"sequence 0, KV head 0 of {wl.Hkv} ({wl.N} tokens x 1/{wl.Hkv} of the heads) per step"
+    sample = (f"sequences 0-{n_seq - 1} of {wl.B}, KV heads 0-{heads - 1} of {wl.Hkv} ({wl.N} tokens each), "
+              f"one oracle thread per (sequence, KV head), per step")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": config_of(wl, world),
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": n_seq * heads, "kind": "oracle",
                              "sample": sample, "host_cores": cores},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -239,6 +247,84 @@ def l2_note(wl) -> str:
 
 # ----------------------------------------------------------------------------- GPU leg
 
+OTHER_CONFIGS = ("llama8b-32k", "structkv-8layer-32k", "fastkv-tsp20-64k")
+
+
+def time_sharded_scoring(wl, p, dev, steps: int, stream) -> dict:
+    import torch
+    from long_context_kv_kvc_b200 import kvc
+    q, k = dev["q"][0], dev["k"][0]
+    U, nq = wl.B * wl.Hkv, wl.G * wl.window
+    cuts = (0, wl.N // 2, wl.N)
+    blocks = []
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        kb = k[:, :, a:b].contiguous()
+        ws = torch.empty(kvc.kvc_shard_workspace_size(p, b - a), dtype=torch.uint8, device="cuda")
+        ml = torch.empty((U, nq, 2), dtype=torch.float32, device="cuda")
+        sc = torch.empty((wl.B, wl.Hkv, b - a), dtype=torch.float32, device="cuda")
+        blocks.append((a, kb, ws, ml, sc))
+    ml_all = torch.empty((len(blocks), U, nq, 2), dtype=torch.float32, device="cuda")
+    whole = torch.empty((wl.B, wl.Hkv, wl.N), dtype=torch.float32, device="cuda")
+    ws_whole = torch.empty(kvc.kvc_workspace_size(p), dtype=torch.uint8, device="cuda")
+
+    def run_blocks():
+        for i, (a, kb, ws, ml, sc) in enumerate(blocks):
+            kvc.kvc_shard_stats(p, q, kb, a, ml_all[i], ws)
+        for a, kb, ws, ml, sc in blocks:
+            kvc.kvc_shard_scores(p, q, kb, a, ml_all, sc, ws)
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    t_blocks = timed(run_blocks)
+    t_whole = timed(lambda: kvc.kvc_score(p, q, k, whole, ws_whole))
+    return {"blocks": len(blocks), "shard_stats_and_scores_ms": t_blocks, "kvc_score_ms": t_whole,
+            "ratio": t_blocks / t_whole, "calls": steps}
+
+
+def time_config(wl, rank: int, steps: int, peak: float) -> dict:
+    """Mean time of one kvc_compress step of workload `wl` over `steps` CUDA-event-timed
+    steps (after 3 warm-up steps), with enough rotating input copies that the inputs of a
+    step are not in L2 from the step before; GB/s against the algorithmic bytes."""
+    import torch
+    from long_context_kv_kvc_b200 import kvc
+    inputs = synth.make_inputs(wl, seeds=rank_seeds(wl, rank))
+    e = 2 if wl.dtype == "bf16" else 4
+    in_bytes = (wl.n_layers + 1) * wl.B * wl.Hkv * wl.N * wl.D * e
+    copies = max(1, -(-3 * L2_BYTES // in_bytes))
+    dev = [{k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inputs.items()}]
+    for _ in range(copies - 1):
+        dev.append({k: (v.clone() if isinstance(v, torch.Tensor) else v) for k, v in dev[0].items()})
+    comp = kvc.Compressor(kvc.params_for(wl))
+    stream = torch.cuda.current_stream()
+    for i in range(3):
+        d = dev[i % copies]
+        comp.run_device(d["q"], d["k"], d["v"], d.get("hidden"))
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        d = dev[i % copies]
+        ev[i][0].record(stream)
+        comp.run_device(d["q"], d["k"], d["v"], d.get("hidden"))
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    ab = algorithmic_bytes(wl)
+    gbs = ab["total"] / (ms * 1e-3) / 1e9
+    return {"ms": ms, "tokens_per_s": wl.B * wl.N / (ms * 1e-3), "algorithmic_bytes": ab["total"], "gbs": gbs,
+            "frac_of_peak": gbs / peak, "steps": steps,
+            "l2": (f"{copies} rotating input copies ({in_bytes / 2**20:.0f} MiB of K and V each)" if copies > 1
+                   else f"inputs larger than L2 ({in_bytes / 2**20:.0f} MiB of K and V)")}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -249,6 +335,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--pivot-steps", type=int, default=5,
                     help="calls timed for the pivot metrics (entropy pass, row statistics); 0 skips")
+    ap.add_argument("--config-steps", type=int, default=20,
+                    help="timed steps of each other configuration (32K, StructKV 8 layers, FastKV TSP); 0 skips")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--flags", type=int, default=0, help="kvc_params.flags (1 = CUDA-core scoring)")
     ap.add_argument("--no-clocks", action="store_true",
@@ -430,13 +518,36 @@ def main():
                           "gbs": dbytes / (t_dec * 1e-3) / 1e9, "algorithmic_bytes": dbytes,
                           "frac_of_peak": dbytes / (t_dec * 1e-3) / 1e9 / peak}
 
+    # sequence sharding's scoring, outside the timed region: the workload's keys cut into two
+    # blocks, both blocks' kvc_shard_stats and kvc_shard_scores on this GPU one after the
+    # other (what two ranks would run, without the exchanges), against kvc_score of the
+    # whole; the blocks are copied out of the inputs first
+    sharded = None
+    if args.pivot_steps > 0 and wl.n_layers == 1 and wl.scope == kvc.KVC_SCOPE_PER_KV_HEAD:
+        sharded = time_sharded_scoring(wl, p, dev, args.pivot_steps, stream)
+        if kvc.kvc_poll_error() != kvc.KVC_OK:
+            raise RuntimeError("device-side error in the sharded scoring")
+
+    # the other configurations at their full sizes (outside the timed region above): the
+    # whole compress step, inputs resident in HBM; when a configuration's inputs fit in L2,
+    # the steps rotate over enough input copies that every step reads its inputs from HBM
+    configs = None
+    if args.config_steps > 0:
+        configs = {}
+        for name in OTHER_CONFIGS:
+            wl2 = synth.WORKLOADS[name]
+            configs[name] = time_config(wl2, rank, args.config_steps, peak)
+        if kvc.kvc_poll_error() != kvc.KVC_OK:
+            raise RuntimeError("device-side error in the configuration runs")
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        threads = min(wl.Hkv, os.cpu_count() or 1)
-        dt, tok = oracle_sample(wl, inputs, wl.Hkv, threads)
-        cpu = {"value": tok / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-               "sample": f"sequence 0 of {wl.B}, all {wl.Hkv} KV heads ({wl.N} tokens), fp64 oracle, "
-                         f"one thread per KV head", "seconds": dt}
+        n_seq, heads = oracle_units(wl)
+        dt, tok = oracle_sample(wl, inputs, n_seq, heads)
+        cpu = {"value": tok / dt, "unit": "tokens/s", "cores": n_seq * heads, "host_cores": os.cpu_count(),
+               "kind": "oracle",
+               "sample": f"sequences 0-{n_seq - 1} of {wl.B}, KV heads 0-{heads - 1} of {wl.Hkv} ({wl.N} tokens "
+                         f"each), fp64 oracle, one thread per (sequence, KV head)", "seconds": dt}
 
     if rank == 0:
         line = {
@@ -450,6 +561,8 @@ def main():
                          "peak_source": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": traffic, "algorithmic_bytes_per_launch": ab["score"]},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
+            "configs": configs,
+            "sharded_scoring": sharded,
             "pivot_metrics": pivot,
             "csm_round": csm_round,
             "decode_attention": decode_att,

@@ -129,6 +129,8 @@ typedef struct kvc_params {
 /*
  * kvc_workspace_size -- bytes of device workspace that kvc_score / kvc_compress need for
  * these parameters.  Host only; enqueues nothing.
+ * Source: none on the pages (they describe no interface); the call exists because the
+ * library allocates no device memory of its own.
  */
 KVC_API kvc_status kvc_workspace_size(const kvc_params *p, size_t *bytes);
 
@@ -160,12 +162,17 @@ KVC_API kvc_status kvc_accumulate(float *acc, const float *src, int32_t B, int32
  *   out[r, j] = max{ in[r, t] : lo <= t < hi, |t - j| <= (kernel-1)/2 }  for lo <= j < hi,
  *   out[r, j] = in[r, j]                                                  otherwise.
  *   in, out  device [B, H, N] fp32 (distinct buffers).  0 <= lo <= hi <= N.
+ * Source: no page describes pooling; the step (max-pool of the summed scores before the
+ * top-k, clipped at the candidate range) is the target statement's, and it fixes no
+ * more than that.
  */
 KVC_API kvc_status kvc_pool(const float *in, float *out, int32_t B, int32_t H, int32_t N, int32_t lo,
                     int32_t hi, int32_t kernel, kvc_stream_t stream);
 
 /*
- * kvc_topk_workspace_size -- device workspace of kvc_topk for B*H rows of length N.
+ * kvc_topk_workspace_size -- device workspace of kvc_topk for B*H rows of length N
+ * (currently always 0 bytes: the selection keeps its state in shared memory).
+ * Source: none on the pages; the call keeps the workspace convention uniform.
  */
 KVC_API kvc_status kvc_topk_workspace_size(int32_t B, int32_t H, int32_t N, size_t *bytes);
 
@@ -367,9 +374,13 @@ KVC_API kvc_status kvc_shard_workspace_size(const kvc_params *p, int32_t n_local
  * kvc_shard_stats -- this block's part of each window row's softmax normaliser.
  *   q        device, [B, Hq, window, D] (all window queries; every shard holds them).
  *   k_local  device, [B, Hkv, n_local, D]: keys key_offset .. key_offset + n_local - 1.
- *   ml       device, [B * Hkv][G * window][2] fp32, written: (m, l) = (max y, sum 2^(y - m))
- *            over the block's keys that the row sees (y = q.k log2(e) / sqrt(D); window row
- *            i sits at position N - window + i); (-inf, 0) when it sees none.
+ *   ml       device, [B * Hkv][G * window][2] fp32, written: a pair (m, l) with l * 2^m =
+ *            the sum of 2^y over the block's keys that the row sees (y = q.k log2(e) /
+ *            sqrt(D); window row i sits at position N - window + i); (-inf, 0) when it
+ *            sees none.  The tensor-core path (bf16, G * window <= 128) writes 1 <= l < 2,
+ *            the CUDA-core path m = the largest such y; both merge the same way.
+ * Runs on the tensor cores when q and K are bf16 and G * window <= 128 (phase 1 of the
+ * score kernel alone), otherwise (or with KVC_FLAG_SIMT_SCORE) on the CUDA cores.
  */
 KVC_API kvc_status kvc_shard_stats(const kvc_params *p, const void *q, const void *k_local, int32_t n_local,
                                    int32_t key_offset, float *ml, void *workspace, size_t workspace_bytes,
@@ -411,6 +422,49 @@ KVC_API kvc_status kvc_select_emit(const float *pooled, int32_t rows, int32_t n,
                                    int32_t cap, int32_t *count, kvc_stream_t stream);
 
 /*
+ * kvc_select_pick -- one digit of the distributed radix select, after the shards'
+ * histograms of the digit have been summed: for each row, the bucket b (scanned from the
+ * top) that holds the need[row]-th largest key; need[row] becomes the number of keys still
+ * needed inside b, prefix[row] gets b in its next digit_bits bits below the top
+ * prefix_bits, and eq_local[row] = hist_local[row][b] (this shard's keys in b).
+ *   hist, hist_local  device uint32 [rows][1 << digit_bits]: summed over shards / this shard's
+ *   need (int32), prefix (uint32), eq_local (int32): device [rows]; need and prefix read and
+ *   written.  1 <= digit_bits <= 12, prefix_bits + digit_bits <= 32.
+ * Source: none on the pages; the sequence-sharded variant's selection step (one radix digit
+ * per exchange), the same ordering as kvc_topk (ties go to the lower positions).
+ */
+KVC_API kvc_status kvc_select_pick(const uint32_t *hist, const uint32_t *hist_local, int32_t rows,
+                                   int32_t digit_bits, int32_t prefix_bits, int32_t *need, uint32_t *prefix,
+                                   int32_t *eq_local, kvc_stream_t stream);
+
+/*
+ * kvc_select_ties -- this shard's share of the keys equal to the threshold: take[row] =
+ * clamp(need[row] - sum over shards s < rank of eq_all[s][row], 0, eq_all[rank][row])
+ * (the lower shards, i.e. the lower positions, take theirs first).
+ *   eq_all  device int32 [n_shards][rows] (every shard's eq_local after the last digit);
+ *   need, take  device int32 [rows].
+ * Source: none on the pages; the tie rule of kvc_topk spread over shards.
+ */
+KVC_API kvc_status kvc_select_ties(const int32_t *eq_all, int32_t n_shards, int32_t rank, int32_t rows,
+                                   const int32_t *need, int32_t *take, kvc_stream_t stream);
+
+/*
+ * kvc_select_kept -- the rows a shard keeps, in position order: the sinks [0, n_sink) that
+ * lie in the shard, the shard's selected positions (kvc_select_emit's sel [rows][cap_sel]
+ * and count_sel [rows]), the window keys [N - window, N) that lie in it.  Writes pos
+ * [rows][cap] (global positions, -1 past the count), local_idx [rows][cap] (pos -
+ * key_offset, 0 past the count; ready for kvc_gather) and count [rows] (all device int32).
+ * More than cap rows sets KVC_ERR_INDEX in kvc_poll_error (cap = min(n_local, budget) is
+ * always enough).
+ * Source: CentroidKV "Inferentie Pipeline" and FastKV sec. 2A (sinks and recent tokens kept
+ * beside the selection), spread over shards.
+ */
+KVC_API kvc_status kvc_select_kept(const int32_t *sel, const int32_t *count_sel, int32_t rows, int32_t cap_sel,
+                                   int32_t N, int32_t n_sink, int32_t window, int32_t key_offset, int32_t n_local,
+                                   int32_t cap, int32_t *pos, int32_t *local_idx, int32_t *count,
+                                   kvc_stream_t stream);
+
+/*
  * kvc_score_noalloc -- kvc_score for callers that cannot allocate device memory.  The
  * pages have no counterpart: it exists for engines that have already given all device
  * memory to their own pool, or plugin interfaces that forbid cudaMalloc/cudaFree during a
@@ -418,11 +472,16 @@ KVC_API kvc_status kvc_select_emit(const float *pooled, int32_t rows, int32_t n,
  * ws/ws_bytes; it always scores with the CUDA-core kernels and keeps their scratch in a
  * 4 MiB array compiled into the library, which every GPU that loads the library holds
  * until the process exits.
- *   Returns KVC_ERR_WORKSPACE when the scratch these parameters need exceeds 4 MiB (about
- *   n_layers * B * Hkv * ceil(N / 2048) * G * window * 8 bytes, plus n_layers * B * Hkv * N
- *   * 4 bytes when several layers or all heads are summed).
+ *   Returns KVC_ERR_WORKSPACE when the scratch these parameters need exceeds 4 MiB; that
+ *   check comes before the pointer checks.  With U = n_layers * B * Hkv, nq = (Hq / Hkv) *
+ *   window, chunk = min(2048, max(32, 32 * ceil(ceil(N * U / 296) / 32))) and n_chunks =
+ *   ceil(N / chunk), the scratch is r(U * n_chunks * nq * 8) + r(U * nq * 4) bytes, plus
+ *   U * N * 4 bytes when several layers or all heads are summed (r() rounds up to a
+ *   multiple of 256).
  *   The first call on each device looks up the array's address (with that device
- *   current); make it before any stream capture begins.  All calls on a device share the
+ *   current); make it before any stream capture begins.  The address is kept for the life
+ *   of the device's context: do not keep using the library across cudaDeviceReset or a
+ *   reset of the primary context.  All calls on a device share the
  *   array: calls whose kernels may overlap on the GPU race and must be ordered by the
  *   caller.  It allocates nothing and clears nothing between calls (every scratch byte it
  *   reads is written earlier in the same call).

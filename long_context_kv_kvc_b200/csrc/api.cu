@@ -337,14 +337,23 @@ kvc_status check_shard(const kvc_params* p, int32_t n_local, int32_t key_offset)
     return KVC_OK;
 }
 
+// The block's scoring runs on the tensor cores (bf16, G * window <= 128, unless the caller
+// asks for the CUDA-core path) or on the CUDA cores; the workspace is that path's.
 struct ShardPlan {
+    bool use_tc;
     int n_chunks, chunk;
     size_t off_partial, off_lse, total;
 };
 
 ShardPlan shard_plan(const kvc_params* p, int n_local) {
     ShardPlan P{};
-    const ScoreJob job = make_job(p, nullptr, nullptr);
+    ScoreJob job = make_job(p, nullptr, nullptr);
+    job.N = n_local;
+    P.use_tc = !(p->flags & KVC_FLAG_SIMT_SCORE) && tc_score_supported(job);
+    if (P.use_tc) {
+        P.total = align_up(tc_score_workspace(job.U, n_local, job.nq));
+        return P;
+    }
     const size_t pb = simt_score_workspace(job.U, n_local, job.nq, &P.n_chunks, &P.chunk);
     P.off_partial = 0;
     P.off_lse = align_up(pb);
@@ -358,6 +367,12 @@ ScoreJob shard_job(const kvc_params* p, const ShardPlan& P, const void* q, const
     job.N = n_local;
     job.key_off = key_offset;
     job.n_total = p->N;
+    if (P.use_tc) {
+        job.tc_ws = ws;
+        job.tc_ws_bytes = P.total;
+        job.err = device_error_word();
+        return job;
+    }
     job.partial = (float2*)(ws + P.off_partial);
     job.lse = (float*)(ws + P.off_lse);
     job.n_chunks = P.n_chunks;
@@ -382,7 +397,12 @@ kvc_status kvc_shard_stats(const kvc_params* p, const void* q, const void* k_loc
     const ShardPlan P = shard_plan(p, n_local);
     if (ws_bytes < P.total) return KVC_ERR_WORKSPACE;
     const ScoreJob job = shard_job(p, P, q, k_local, n_local, key_offset, (char*)ws);
-    KVC_CUDA(kvc::simt_shard_stats(job, (float2*)ml, (cudaStream_t)stream));
+    if (P.use_tc) {
+        if (!job.err) return KVC_ERR_CUDA;
+        KVC_CUDA(kvc::tc_shard_stats(job, (float2*)ml, (cudaStream_t)stream));
+    } else {
+        KVC_CUDA(kvc::simt_shard_stats(job, (float2*)ml, (cudaStream_t)stream));
+    }
     return KVC_OK;
 }
 
@@ -398,7 +418,12 @@ kvc_status kvc_shard_scores(const kvc_params* p, const void* q, const void* k_lo
     if (ws_bytes < P.total) return KVC_ERR_WORKSPACE;
     ScoreJob job = shard_job(p, P, q, k_local, n_local, key_offset, (char*)ws);
     job.unit_scores = scores;
-    KVC_CUDA(kvc::simt_shard_scores(job, (const float2*)ml_all, n_shards, (cudaStream_t)stream));
+    if (P.use_tc) {
+        if (!job.err) return KVC_ERR_CUDA;
+        KVC_CUDA(kvc::tc_shard_scores(job, (const float2*)ml_all, n_shards, (cudaStream_t)stream));
+    } else {
+        KVC_CUDA(kvc::simt_shard_scores(job, (const float2*)ml_all, n_shards, (cudaStream_t)stream));
+    }
     return KVC_OK;
 }
 
@@ -421,6 +446,36 @@ kvc_status kvc_select_emit(const float* pooled, int32_t rows, int32_t n, int32_t
         (hi > lo && (long long)pos_offset + lo < 0))
         return KVC_ERR_ARG;
     KVC_CUDA(kvc::select_emit(pooled, rows, n, lo, hi, thr, ties, pos_offset, out, cap, count, (cudaStream_t)stream));
+    return KVC_OK;
+}
+
+kvc_status kvc_select_pick(const uint32_t* hist, const uint32_t* hist_local, int32_t rows, int32_t digit_bits,
+                           int32_t prefix_bits, int32_t* need, uint32_t* prefix, int32_t* eq_local,
+                           kvc_stream_t stream) {
+    if (!hist || !hist_local || !need || !prefix || !eq_local || rows < 1) return KVC_ERR_ARG;
+    if (digit_bits < 1 || digit_bits > 12 || prefix_bits < 0 || prefix_bits + digit_bits > 32) return KVC_ERR_ARG;
+    KVC_CUDA(kvc::select_pick(hist, hist_local, rows, digit_bits, prefix_bits, need, prefix, eq_local,
+                              (cudaStream_t)stream));
+    return KVC_OK;
+}
+
+kvc_status kvc_select_ties(const int32_t* eq_all, int32_t n_shards, int32_t rank, int32_t rows, const int32_t* need,
+                           int32_t* take, kvc_stream_t stream) {
+    if (!eq_all || !need || !take || rows < 1 || n_shards < 1 || rank < 0 || rank >= n_shards) return KVC_ERR_ARG;
+    KVC_CUDA(kvc::select_ties(eq_all, n_shards, rank, rows, need, take, (cudaStream_t)stream));
+    return KVC_OK;
+}
+
+kvc_status kvc_select_kept(const int32_t* sel, const int32_t* count_sel, int32_t rows, int32_t cap_sel, int32_t N,
+                           int32_t n_sink, int32_t window, int32_t key_offset, int32_t n_local, int32_t cap,
+                           int32_t* pos, int32_t* local_idx, int32_t* count, kvc_stream_t stream) {
+    if (!sel || !count_sel || !pos || !local_idx || !count || rows < 1 || cap_sel < 1 || cap < 1) return KVC_ERR_ARG;
+    if (N < 1 || n_sink < 0 || window < 0 || key_offset < 0 || n_local < 1 || (long long)key_offset + n_local > N)
+        return KVC_ERR_ARG;
+    unsigned* err = device_error_word();
+    if (!err) return KVC_ERR_CUDA;
+    KVC_CUDA(kvc::select_kept(sel, count_sel, rows, cap_sel, N, n_sink, window, key_offset, n_local, cap, pos,
+                              local_idx, count, err, (cudaStream_t)stream));
     return KVC_OK;
 }
 

@@ -66,6 +66,10 @@ cudaError_t simt_shard_scores(const ScoreJob& job, const float2* ml_all, int W, 
 bool tc_score_supported(const ScoreJob& job);
 size_t tc_score_workspace(int U, int N, int nq);
 cudaError_t tc_score(const ScoreJob& job, cudaStream_t s);
+// sequence sharding on the tensor cores: this block's (m, l) per (unit, row) (phase 1 only),
+// then the block's scores given every shard's (m, l) [W][U * nq] (phase 2 only)
+cudaError_t tc_shard_stats(const ScoreJob& job, float2* ml, cudaStream_t s);
+cudaError_t tc_shard_scores(const ScoreJob& job, const float2* ml_all, int W, cudaStream_t s);
 
 // the tensor-core kernel's software exp2, element-wise (diagnostics)
 
@@ -85,6 +89,13 @@ cudaError_t select_hist(const float* pooled, int rows, int n, int lo, int hi, co
                         int digit_bits, uint32_t* hist, cudaStream_t s);
 cudaError_t select_emit(const float* pooled, int rows, int n, int lo, int hi, const uint32_t* thr, const int32_t* ties,
                         int pos_offset, int32_t* out, int cap, int32_t* count, cudaStream_t s);
+cudaError_t select_pick(const uint32_t* hist, const uint32_t* hist_local, int rows, int digit_bits, int prefix_bits,
+                        int32_t* need, uint32_t* prefix, int32_t* eq_local, cudaStream_t s);
+cudaError_t select_ties(const int32_t* eq_all, int W, int rank, int rows, const int32_t* need, int32_t* take,
+                        cudaStream_t s);
+cudaError_t select_kept(const int32_t* sel, const int32_t* cnt, int rows, int cap_sel, int N, int S, int w,
+                        int key_off, int n_local, int cap, int32_t* pos, int32_t* local, int32_t* count,
+                        unsigned* err, cudaStream_t s);
 cudaError_t topk_fused(const float* scores, int rows, int N, int n_sink, int window, int budget, int kernel,
                        int32_t* idx, cudaStream_t s);
 // two gathers of the same shape in one launch (src1/dst1 may be null)

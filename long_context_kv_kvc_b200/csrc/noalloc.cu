@@ -13,7 +13,9 @@
 // which the library is loaded holds that much memory until the process exits.  Host code
 // cannot use the array's name as a device address, so the first call on each device (with
 // that device current) looks the address up with cudaGetSymbolAddress and caches it; make
-// that first call before any stream capture starts.  All calls on a device share the one
+// that first call before any stream capture starts.  The cached address stays valid for the
+// life of the device's context: do not keep using the library across cudaDeviceReset or a
+// reset of the primary context.  All calls on a device share the one
 // array: two calls whose kernels overlap on the GPU (different streams, no ordering
 // between them) overwrite each other's scratch and give wrong results, so callers must
 // order them.  Every byte the kernels read from the array is written earlier in the same
@@ -52,8 +54,6 @@ extern "C" kvc_status kvc_score_noalloc(const kvc_params* p, const void* q, cons
     size_t ws_unused = 0;
     const kvc_status st = kvc_workspace_size(p, &ws_unused);
     if (st != KVC_OK) return st;
-    if (!q || !k || !scores) return KVC_ERR_ARG;
-    if (((uintptr_t)q | (uintptr_t)k | (uintptr_t)scores) & 15u) return KVC_ERR_ALIGN;
 
     kvc::ScoreJob job{};
     job.q = q;
@@ -70,7 +70,11 @@ extern "C" kvc_status kvc_score_noalloc(const kvc_params* p, const void* q, cons
     const size_t lse_off = round256(partial_bytes);
     const size_t units_off = round256(lse_off + (size_t)job.U * job.nq * sizeof(float));
     const size_t need = units ? units_off + (size_t)job.U * job.N * sizeof(float) : units_off;
+    // the size check comes before the pointer checks, so that a parameter set that does not
+    // fit is rejected whatever buffers come with it
     if (need > kStaticScratchBytes) return KVC_ERR_WORKSPACE;  // larger than the fixed array
+    if (!q || !k || !scores) return KVC_ERR_ARG;
+    if (((uintptr_t)q | (uintptr_t)k | (uintptr_t)scores) & 15u) return KVC_ERR_ALIGN;
 
     char* scratch = (char*)static_scratch();
     if (!scratch) return KVC_ERR_CUDA;

@@ -103,7 +103,16 @@ struct TcArgs {
     unsigned* err;
     long long spin_limit;
     int U, N, w, nq, T_u, total_tiles, P, max_lead, inject;
+    // sequence sharding: the N keys are positions key_off .. key_off + N - 1 of a sequence of
+    // n_total (0 and N when not sharded); window row i sits at position n_total - w + i
+    int key_off, n_total;
+    float2* ml_out;       // kStats: per (unit, row) (m, l) with l 2^m = the row's sum of 2^y over the block
+    const float* lse_in;  // kScores: [U][128] each row's log-sum-exp (base 2) over the whole sequence
 };
+
+// What a launch computes: the whole two-phase scoring, only the per-row normalisers of this
+// block of keys (phase 1), or only the scores given the normalisers (phase 2).
+enum TcMode { kFull = 0, kStats = 1, kScores = 2 };
 
 struct __align__(1024) Smem {
     uint8_t ringA[kStagesA][kBoxBytes];
@@ -309,7 +318,7 @@ struct TileSeq {
     }
 };
 
-template <bool ENT>
+template <bool ENT, int MODE>
 __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_constant__ TcArgs a) {
     extern __shared__ uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -368,8 +377,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
         // Warp 0 streams the phase-1 tiles from HBM, one 32 KiB op per tile (both 64-column
         // halves); warps 2 and 6 issue the phase-2 re-reads, half 0 and half 1 of every tile.
         // A single issuing thread completes TMA ops at a roughly fixed rate, so the phase-1
-        // stream uses large ops and the phase-2 stream two threads.
-        if (lane == 0) {
+        // stream uses large ops and the phase-2 stream two threads.  kScores: warp 0 loads only
+        // the Q of each unit; kStats: no phase-2 re-reads.
+        if (lane == 0 && !(MODE == kStats && warp != 0)) {
             const int ph = warp == 0 ? 0 : 1, hh = warp == 6 ? 1 : 0;
             const CUtensorMap* mk = ph == 0 ? &a.tmap_k4 : &a.tmap_k;
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(mk)) : "memory");
@@ -380,7 +390,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                 const int u = seq.unit(i), ti = seq.tile(i);
                 // phase 1 stays at most max_lead tiles ahead of phase 2 (L2 footprint);
                 // phase 2 never loads a tile before phase 1 has (so its read hits L2)
-                if (ph == 0 ? (i - *other >= a.max_lead) : (i >= *other)) {
+                const bool lead_rule = ph == 1 || MODE == kFull;
+                if (lead_rule && (ph == 0 ? (i - *other >= a.max_lead) : (i >= *other))) {
                     const long long t0 = globaltimer();
                     while (ph == 0 ? (i - *other >= a.max_lead) : (i >= *other)) {
                         if (*abort) break;
@@ -404,10 +415,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                     tma_load_2d(sm.q[slot] + kBoxBytes, &a.tmap_q, &sm.qfull[slot], 64, u * kQRows);
                 }
                 if (ph == 0) {
-                    const int st = i % kTilesA;
-                    mbar_spin(&sm.emptyA[st], ((i / kTilesA) & 1) ^ 1, abort, a.err);
-                    mbar_expect_tx(&sm.fullA[st], 2 * kBoxBytes);
-                    tma_load_4d(sm.ringA[2 * st], mk, &sm.fullA[st], 0, ti * kTileKeys, 0, u);
+                    if (MODE != kScores) {
+                        const int st = i % kTilesA;
+                        mbar_spin(&sm.emptyA[st], ((i / kTilesA) & 1) ^ 1, abort, a.err);
+                        mbar_expect_tx(&sm.fullA[st], 2 * kBoxBytes);
+                        tma_load_4d(sm.ringA[2 * st], mk, &sm.fullA[st], 0, ti * kTileKeys, 0, u);
+                    }
                     *reinterpret_cast<volatile int*>(&sm.p1_issued) = i + 1;
                 } else {
                     const int k = 2 * i + hh, st = k % kStagesB;
@@ -420,8 +433,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             if (*abort) {
                 // copies still in flight land before the CTA exits
                 if (ph == 0) {
-                    for (int n = std::max(0, i - kTilesA); n < i; ++n)
-                        drain_wait(&sm.fullA[n % kTilesA], (n / kTilesA) & 1, a.err);
+                    if (MODE != kScores)
+                        for (int n = std::max(0, i - kTilesA); n < i; ++n)
+                            drain_wait(&sm.fullA[n % kTilesA], (n / kTilesA) & 1, a.err);
                     for (int o = std::max(0, ord - kQSlots + 1); o <= ord; ++o)
                         drain_wait(&sm.qfull[o % kQSlots], (o / kQSlots) & 1, a.err);
                 } else {
@@ -437,9 +451,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
         // Warp 1 issues the phase-1 jobs, warp 3 the phase-2 jobs (a phase-2 tile once its
         // unit's lse is in shared memory).  Each claims the next job number n when its job is
         // ready and fills accumulator n % kAcc, so the consumers see one stream of jobs.  Two
-        // issuers keep the tensor pipe busy while either does its bookkeeping.
-        if (lane == 0) {
-            const int ph = warp == 1 ? 0 : 1;
+        // issuers keep the tensor pipe busy while either does its bookkeeping.  kStats has only
+        // phase-1 jobs, kScores only phase-2 jobs.
+        const int ph = warp == 1 ? 0 : 1;
+        if (lane == 0 && !(MODE == kStats && ph == 1) && !(MODE == kScores && ph == 0)) {
             const uint64_t dK0 = sw128_desc(smem_u32(ph == 0 ? sm.ringA[0] : sm.ringB[0]));
             const uint64_t dQ0 = sw128_desc(smem_u32(sm.q[0]));
             constexpr uint64_t kBoxStep = kBoxBytes >> 4, kQStep = (2 * kBoxBytes) >> 4;
@@ -503,7 +518,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                     ++nu;
                 }
                 if (nu != u) {
-                    if (ph == 1 && i + 1 < n_local) umma_commit(&sm.qempty[qslot]);
+                    // the last phase that reads the unit's Q releases its slot
+                    if ((ph == 1 || MODE == kStats) && i + 1 < n_local) umma_commit(&sm.qempty[qslot]);
                     u = nu;
                     ++ord;
                     if (++qslot == kQSlots) qslot = 0;
@@ -525,7 +541,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             ++ord;
             const int slot = ord & 1;
             // every phase-2 job of the unit that used this slot before has read it
-            if (lane == 0 && *reinterpret_cast<volatile unsigned*>(&sm.lse_done[slot]) < target[slot]) {
+            if (MODE != kStats && lane == 0 &&
+                *reinterpret_cast<volatile unsigned*>(&sm.lse_done[slot]) < target[slot]) {
                 const long long t0 = globaltimer();
                 while (*reinterpret_cast<volatile unsigned*>(&sm.lse_done[slot]) < target[slot]) {
                     if (*abort) break;
@@ -537,6 +554,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                 }
             }
             target[slot] += 4u * (unsigned)seq.count(u);
+            if (MODE == kScores) {
+                // the normalisers come from the caller (every shard's, merged)
+#pragma unroll
+                for (int rr = 0; rr < 4; ++rr) {
+                    const int r = lane + 32 * rr;
+                    const float lse = r < a.nq ? __ldg(a.lse_in + (size_t)u * kQRows + r) : INFINITY;
+                    sm.nlse[slot][r] = -lse;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.lsefull[slot]);
+                continue;
+            }
             // unit u is complete once every CTA holding tiles of it has added its part
             int ok = 0;
             if (lane == 0) {
@@ -575,6 +604,24 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                             (float)(0.69314718055994531 * ((double)log2_pos(tot[rr]) - tott[rr] / tot[rr]));
                 }
             }
+            if (MODE == kStats) {
+                // this block's part of each row's normaliser as (m, l) with l in [1, 2):
+                // total 2^ref = l 2^m; every CTA of the unit writes the same values
+#pragma unroll
+                for (int rr = 0; rr < 4; ++rr) {
+                    const int r = lane + 32 * rr;
+                    if (r >= a.nq) continue;
+                    float2 ml = make_float2(-INFINITY, 0.f);
+                    if (ok && tot[rr] > 0.0) {
+                        const long long b = __double_as_longlong(tot[rr]);
+                        const int e = (int)((b >> 52) & 0x7FF) - 1023;
+                        const double f = __longlong_as_double((b & ~(0x7FFLL << 52)) | (1023LL << 52));
+                        ml = make_float2(__ldg(a.ref + (size_t)u * kQRows + r) + (float)e, (float)f);
+                    }
+                    a.ml_out[(size_t)u * a.nq + r] = ml;
+                }
+                continue;
+            }
 #pragma unroll
             for (int rr = 0; rr < 4; ++rr) {
                 const int r = lane + 32 * rr;
@@ -598,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             T[k] = 0.f;
         }
         int u = cta / a.T_u, t = cta - (cta / a.T_u) * a.T_u;
-        for (int i = 0; i < n_local; ++i) {
+        for (int i = 0; i < (MODE == kScores ? 0 : n_local); ++i) {
             const int s = i % kRec;
             mbar_wait(&sm.recfull[s], (i / kRec) & 1, abort, a.err);
             if (*abort) break;
@@ -660,7 +707,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
         const int g = (warp - kConsumer0) >> 2;
         const int r = threadIdx.x - 32 * kConsumer0 - 128 * g;
         const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + g * 128;
-        const int n_jobs = 2 * n_local;
+        const int n_jobs = MODE == kFull ? 2 * n_local : n_local;
+        // the last local key index row q sees is min(N - 1, hz0 + q % w) (sharding: a key's
+        // position is key_off + its local index; row q sits at n_total - w + q % w)
+        const int hz0 = a.n_total - a.w - a.key_off;
         for (int n = g; n < n_jobs; n += kAcc) {
             mbar_wait(&sm.accfull[g], (n / kAcc) & 1, abort, a.err);
             if (*abort) break;
@@ -671,13 +721,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                          : "r"(smem_u32(&sm.job[g]))
                          : "memory");
             const int u = jb.y, ti = jb.z;
-            const bool full_tile = (ti + 1) * kTileKeys <= a.N - a.w + 1;
+            const bool full_tile = (ti + 1) * kTileKeys <= min(a.N, a.n_total - a.w - a.key_off + 1);
             if (jb.x == 0) {
                 // phase 1: this row's (m, sum of 2^(y - m)) over the tile's visible keys.  m is
                 // the row's reference logit (its own-position key), so no running max is
                 // needed; a chunk whose sum is not below 2^100 (a logit ~100 above the
                 // reference) is redone with its exact max.
-                const int t_r = a.N - a.w + (r % a.w);  // last key this row sees
+                const int t_r = min(a.N - 1, hz0 + r % a.w);  // last key this row sees
                 float m = __ldg(a.ref + (size_t)u * kQRows + r), l = 0.f, t = 0.f;
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
@@ -741,7 +791,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                         // query row q (position N - w + q % w) sees this key iff j <= that
 #pragma unroll
                         for (int e = 0; e < 32; ++e)
-                            if (j > a.N - a.w + (c * 32 + e) % a.w) x[e] = __float_as_uint(-INFINITY);
+                            if (j > min(a.N - 1, hz0 + (c * 32 + e) % a.w)) x[e] = __float_as_uint(-INFINITY);
                     }
                     sc += prob_sum(x, nlse + c * 32);
                 }
@@ -766,7 +816,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
 // clears the per-unit sums and counters of this call.
 __global__ void tc_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                                __nv_bfloat16* __restrict__ qpad, float* __restrict__ ref, double* __restrict__ sum,
-                               unsigned* __restrict__ flags, int n_flags, int U, int N, int w, int nq) {
+                               unsigned* __restrict__ flags, int n_flags, int U, int N, int w, int nq, int mode,
+                               int key_off, int n_total) {
     const long long total = (long long)U * kQRows * (kHeadDim / 8);  // 16-byte pieces
     for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
          e += (long long)gridDim.x * blockDim.x) {
@@ -786,10 +837,15 @@ __global__ void tc_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_b
          e += n_warps) {
         const int r = (int)(e % kQRows);
         const long long u = e / kQRows;
+        // the reference key: the row's own position (whole sequence), or the block's first key
+        // when the row sees it (kStats: the block may not hold the row's own position); rows
+        // without one keep 0 (they see no key of the block, and their sums stay 0)
+        const int kj = mode == kFull ? N - w + r % w : 0;
+        const bool has_ref = r < nq && (mode == kFull || (mode == kStats && key_off <= n_total - w + r % w));
         float x = 0.f;
-        if (r < nq) {
+        if (has_ref) {
             const uint2 qv = *reinterpret_cast<const uint2*>(q + (u * nq + r) * kHeadDim + 4 * lane);
-            const uint2 kv = *reinterpret_cast<const uint2*>(k + (u * N + (N - w + r % w)) * kHeadDim + 4 * lane);
+            const uint2 kv = *reinterpret_cast<const uint2*>(k + (u * N + kj) * kHeadDim + 4 * lane);
             const __nv_bfloat162* qh = reinterpret_cast<const __nv_bfloat162*>(&qv);
             const __nv_bfloat162* kh = reinterpret_cast<const __nv_bfloat162*>(&kv);
 #pragma unroll
@@ -811,12 +867,34 @@ __global__ void tc_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_b
         flags[e] = 0u;
 }
 
+// Each row's log-sum-exp (base 2) from every shard's (m, l) (l 2^m = the shard's sum of 2^y
+// over its keys), merged in shard order so that every shard computes the same value:
+// ml_all [W][U][nq] -> lse [U][128] (rows >= nq: +inf).
+__global__ void tc_shard_lse_kernel(const float2* __restrict__ ml_all, int W, int U, int nq, float* __restrict__ lse) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < U * kQRows; i += gridDim.x * blockDim.x) {
+        const int u = i / kQRows, r = i % kQRows;
+        if (r >= nq) {
+            lse[i] = INFINITY;
+            continue;
+        }
+        const size_t rows = (size_t)U * nq, at = (size_t)u * nq + r;
+        float M = -INFINITY;
+        for (int s = 0; s < W; ++s) M = fmaxf(M, ml_all[s * rows + at].x);
+        float S = 0.f;
+        for (int s = 0; s < W; ++s) {
+            const float2 v = ml_all[s * rows + at];
+            if (v.x != -INFINITY) S += v.y * exp2f(v.x - M);
+        }
+        lse[i] = M + log2f(S);
+    }
+}
+
 // ------------------------------------------------------------------------ host side
 
 size_t a256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct TcLayout {
-    size_t qpad, ref, sum, flags, n_flags, total;
+    size_t qpad, ref, sum, lse, flags, n_flags, total;
 };
 
 TcLayout tc_layout(int U) {
@@ -828,6 +906,8 @@ TcLayout tc_layout(int U) {
     off = a256(off + (size_t)U * kQRows * sizeof(float));
     L.sum = off;  // the totals, then the entropy's totals
     off = a256(off + 2 * (size_t)U * kSumCopies * kQRows * sizeof(double));
+    L.lse = off;  // kScores: the merged log-sum-exp per (unit, padded row)
+    off = a256(off + (size_t)U * kQRows * sizeof(float));
     L.flags = off;  // count[U], never
     L.n_flags = (size_t)U + 1;
     off = a256(off + L.n_flags * sizeof(unsigned));
@@ -868,7 +948,39 @@ bool tc_score_supported(const ScoreJob& j) {
 
 size_t tc_score_workspace(int U, int /*N*/, int /*nq*/) { return tc_layout(U).total; }
 
-cudaError_t tc_score(const ScoreJob& j, cudaStream_t s) {
+namespace {
+
+template <int MODE>
+cudaError_t launch_kernel(const TcArgs& a, bool ent, size_t smem, cudaStream_t s) {
+    static std::atomic<bool> attr_set[2][64];
+    int dev = 0;
+    cudaError_t e;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if (dev >= 64 || !attr_set[ent][dev].load()) {
+        e = ent ? cudaFuncSetAttribute(tc_score_kernel<true, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
+                : cudaFuncSetAttribute(tc_score_kernel<false, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+        if (e != cudaSuccess) return e;
+        if (dev < 64) attr_set[ent][dev].store(true);
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.P);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = ent ? cudaLaunchKernelEx(&cfg, tc_score_kernel<true, MODE>, a)
+            : cudaLaunchKernelEx(&cfg, tc_score_kernel<false, MODE>, a);
+    count_launches(1);
+    return e;
+}
+
+// The prep kernel and one launch of the score kernel in the given mode.
+cudaError_t tc_launch(const ScoreJob& j, int mode, float2* ml_out, cudaStream_t s) {
     const TcLayout L = tc_layout(j.U);
     char* ws = (char*)j.tc_ws;
     if (j.tc_ws_bytes < L.total) return cudaErrorInvalidValue;
@@ -898,6 +1010,11 @@ cudaError_t tc_score(const ScoreJob& j, cudaStream_t s) {
     // merge, while keeping the tiles between the two reads (max_lead x P x 32 KiB) in L2
     a.max_lead = (a.T_u + a.P - 1) / a.P + kLeadSlack;
     a.inject = j.inject_timeout;
+    a.key_off = j.key_off;
+    a.n_total = j.n_total > 0 ? j.n_total : j.N;
+    a.ml_out = ml_out;
+    a.lse_in = (const float*)(ws + L.lse);
+    if (mode != kFull && j.entropy) return cudaErrorInvalidValue;
 
     auto encode = encode_fn();
     if (!encode) return cudaErrorNotSupported;
@@ -936,35 +1053,34 @@ cudaError_t tc_score(const ScoreJob& j, cudaStream_t s) {
     const int prep_grid = (int)std::min<long long>((pieces + 255) / 256, 148LL * 8);
     tc_prep_kernel<<<prep_grid, 256, 0, s>>>((const __nv_bfloat16*)j.q, (const __nv_bfloat16*)j.k, qpad,
                                              (float*)(ws + L.ref), (double*)(ws + L.sum), flags, (int)L.n_flags,
-                                             j.U, j.N, j.window, j.nq);
+                                             j.U, j.N, j.window, j.nq, mode, a.key_off, a.n_total);
     count_launches(1);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
     const size_t smem = sizeof(Smem) + 1024;
     const bool ent = j.entropy != nullptr;
-    static std::atomic<bool> attr_set[2][64];
-    int dev = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if (dev >= 64 || !attr_set[ent][dev].load()) {
-        e = ent ? cudaFuncSetAttribute(tc_score_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
-                : cudaFuncSetAttribute(tc_score_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        if (dev < 64) attr_set[ent][dev].store(true);
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(a.P);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = ent ? cudaLaunchKernelEx(&cfg, tc_score_kernel<true>, a) : cudaLaunchKernelEx(&cfg, tc_score_kernel<false>, a);
+    if (mode == kStats) return launch_kernel<kStats>(a, false, smem, s);
+    if (mode == kScores) return launch_kernel<kScores>(a, false, smem, s);
+    return launch_kernel<kFull>(a, ent, smem, s);
+}
+
+}  // namespace
+
+cudaError_t tc_score(const ScoreJob& j, cudaStream_t s) { return tc_launch(j, kFull, nullptr, s); }
+
+cudaError_t tc_shard_stats(const ScoreJob& j, float2* ml, cudaStream_t s) { return tc_launch(j, kStats, ml, s); }
+
+cudaError_t tc_shard_scores(const ScoreJob& j, const float2* ml_all, int W, cudaStream_t s) {
+    const TcLayout L = tc_layout(j.U);
+    if (j.tc_ws_bytes < L.total) return cudaErrorInvalidValue;
+    const long long n = (long long)j.U * kQRows;
+    tc_shard_lse_kernel<<<(int)std::min<long long>((n + 255) / 256, 148LL * 8), 256, 0, s>>>(
+        ml_all, W, j.U, j.nq, (float*)((char*)j.tc_ws + L.lse));
     count_launches(1);
-    return e;
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return tc_launch(j, kScores, nullptr, s);
 }
 
 }  // namespace kvc

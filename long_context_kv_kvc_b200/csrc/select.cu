@@ -1,14 +1,20 @@
 // select.cu -- score sums, 1-D max-pool and top-k selection of kept positions.
 //
-// Top-k is a radix select on order-preserving 32-bit keys of the pooled fp32 scores
-// (four 8-bit digits, most significant first), followed by a stable compaction that
-// writes the kept candidate positions in ascending order: every candidate above the
-// threshold value T, and the lowest-indexed candidates equal to T up to the budget.
-// Sinks [0, S) and the recent window [N - w, N) are written around them (CentroidKV page,
-// "Inferentie Pipeline": sinks and recent tokens are preserved; FastKV page, sec. 2A: the
-// selected tokens plus a window of the newest tokens).  One CTA of 1024 threads owns a
-// row; each warp owns a contiguous segment of it, so all loads are coalesced and the only
-// block-wide steps are the digit search and one scan of per-warp counts.
+// Top-k is a radix select on order-preserving 32-bit keys of the pooled fp32 scores,
+// followed by a stable compaction that writes the kept candidate positions in ascending
+// order: every candidate above the threshold value T, and the lowest-indexed candidates
+// equal to T up to the budget.  Sinks [0, S) and the recent window [N - w, N) are written
+// around them (CentroidKV page, "Inferentie Pipeline": sinks and recent tokens are
+// preserved; FastKV page, sec. 2A: the selected tokens plus a window of the newest tokens).
+// Two kernels:
+//   * topk_cluster_kernel (the compress path's default): one 8-CTA cluster per row; each
+//     CTA max-pools its slice of the candidates into shared memory (counting the first
+//     digit's histogram as it forms the keys), and the cluster runs an 11/11/10-bit radix
+//     select whose per-CTA histograms are combined through distributed shared memory;
+//   * topk_kernel (rows too long for the clusters' shared memory): one CTA of 1024 threads
+//     per row, four 8-bit digits; each warp owns a contiguous segment of the row, so all
+//     loads are coalesced and the only block-wide steps are the digit search and one scan
+//     of per-warp counts.
 #include <cooperative_groups.h>
 
 #include <atomic>
@@ -626,6 +632,117 @@ cudaError_t row_stats(const float* scores, int rows, int N, int S, int w, const 
                       float* kept_mass, float* cand_var, unsigned* err, cudaStream_t s) {
     row_stats_kernel<<<rows, kRsThreads, 0, s>>>(scores, N, S, w, idx, budget, kept_mass, cand_var, err);
     count_launches(1);
+    return cudaGetLastError();
+}
+
+namespace {
+
+// One warp per row: the bucket (scanned from the top) that holds the need-th largest key of
+// the row's histogram summed over shards, the keys still needed inside it, the prefix
+// extended by the bucket, and this shard's count in that bucket.
+__global__ void select_pick_kernel(const uint32_t* __restrict__ hist, const uint32_t* __restrict__ hist_local,
+                                   int rows, int digit_bits, int prefix_bits, int32_t* __restrict__ need,
+                                   uint32_t* __restrict__ prefix, int32_t* __restrict__ eq_local) {
+    const int lane = threadIdx.x & 31;
+    const int row = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+    if (row >= rows) return;
+    const int nb = 1 << digit_bits;
+    const int per = (nb + 31) / 32;  // buckets per lane, lane 0 holding the top ones
+    const uint32_t* h = hist + (size_t)row * nb;
+    const long long want = need[row];
+    // this lane's buckets, from the top: nb - 1 - lane*per down to nb - (lane+1)*per
+    long long seg = 0;
+    for (int t = 0; t < per; ++t) {
+        const int b = nb - 1 - (lane * per + t);
+        if (b >= 0) seg += h[b];
+    }
+    long long incl = seg;  // inclusive prefix over lanes (from the top)
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const long long v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    const long long excl = incl - seg;
+    const unsigned hit = __ballot_sync(0xffffffffu, incl >= want);
+    const int owner = hit ? __ffs(hit) - 1 : 31;
+    if (lane == owner) {
+        long long above = excl;
+        int b = 0;
+        long long inside = want - above;
+        for (int t = 0; t < per; ++t) {
+            const int bb = nb - 1 - (lane * per + t);
+            if (bb < 0) break;
+            b = bb;
+            if (above + (long long)h[bb] >= want) break;
+            above += h[bb];
+        }
+        inside = want - above;
+        need[row] = (int32_t)inside;
+        prefix[row] |= (uint32_t)b << (32 - prefix_bits - digit_bits);
+        eq_local[row] = (int32_t)hist_local[(size_t)row * nb + b];
+    }
+}
+
+// take[row] = min(max(need[row] - sum of eq_all[s][row] over shards s < rank, 0), eq_all[rank][row])
+__global__ void select_ties_kernel(const int32_t* __restrict__ eq_all, int W, int rank, int rows,
+                                   const int32_t* __restrict__ need, int32_t* __restrict__ take) {
+    for (int r = blockIdx.x * blockDim.x + threadIdx.x; r < rows; r += gridDim.x * blockDim.x) {
+        long long before = 0;
+        for (int s = 0; s < rank; ++s) before += eq_all[(size_t)s * rows + r];
+        const long long t = (long long)need[r] - before;
+        const long long mine = eq_all[(size_t)rank * rows + r];
+        take[r] = (int32_t)(t < 0 ? 0 : (t > mine ? mine : t));
+    }
+}
+
+// The block's kept rows in position order: its sinks, its selected positions, its window
+// keys; global positions (-1 past the count) and local indices (0 past the count).
+__global__ void select_kept_kernel(const int32_t* __restrict__ sel, const int32_t* __restrict__ cnt, int rows,
+                                   int cap_sel, int N, int S, int w, int key_off, int n_local, int cap,
+                                   int32_t* __restrict__ pos, int32_t* __restrict__ local, int32_t* __restrict__ count,
+                                   unsigned* __restrict__ err) {
+    const int row = blockIdx.x;
+    const int s_lo = max(0, key_off), s_hi = min(S, key_off + n_local);            // sinks in the block
+    const int w_lo = max(N - w, key_off), w_hi = min(N, key_off + n_local);        // window keys in the block
+    const int n_s = max(0, s_hi - s_lo), n_w = max(0, w_hi - w_lo), n_sel = cnt[row];
+    const int total = n_s + n_sel + n_w;
+    if (threadIdx.x == 0) {
+        count[row] = total;
+        if (total > cap) atomicOr(err, kErrIndex);
+    }
+    for (int e = threadIdx.x; e < cap; e += blockDim.x) {
+        int gp = -1;
+        if (e < n_s) gp = s_lo + e;
+        else if (e < n_s + n_sel) gp = sel[(size_t)row * cap_sel + (e - n_s)];
+        else if (e < total) gp = w_lo + (e - n_s - n_sel);
+        pos[(size_t)row * cap + e] = gp;
+        local[(size_t)row * cap + e] = gp >= 0 ? gp - key_off : 0;
+    }
+}
+
+}  // namespace
+
+cudaError_t select_pick(const uint32_t* hist, const uint32_t* hist_local, int rows, int digit_bits, int prefix_bits,
+                        int32_t* need, uint32_t* prefix, int32_t* eq_local, cudaStream_t s) {
+    count_launches(1);
+    select_pick_kernel<<<(rows + 7) / 8, 256, 0, s>>>(hist, hist_local, rows, digit_bits, prefix_bits, need, prefix,
+                                                      eq_local);
+    return cudaGetLastError();
+}
+
+cudaError_t select_ties(const int32_t* eq_all, int W, int rank, int rows, const int32_t* need, int32_t* take,
+                        cudaStream_t s) {
+    count_launches(1);
+    select_ties_kernel<<<(rows + 255) / 256, 256, 0, s>>>(eq_all, W, rank, rows, need, take);
+    return cudaGetLastError();
+}
+
+cudaError_t select_kept(const int32_t* sel, const int32_t* cnt, int rows, int cap_sel, int N, int S, int w,
+                        int key_off, int n_local, int cap, int32_t* pos, int32_t* local, int32_t* count,
+                        unsigned* err, cudaStream_t s) {
+    count_launches(1);
+    select_kept_kernel<<<rows, 256, 0, s>>>(sel, cnt, rows, cap_sel, N, S, w, key_off, n_local, cap, pos, local,
+                                            count, err);
     return cudaGetLastError();
 }
 

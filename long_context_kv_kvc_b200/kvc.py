@@ -27,7 +27,8 @@ EXPORTED = ("kvc_workspace_size", "kvc_score", "kvc_accumulate", "kvc_pool", "kv
             "kvc_status_string", "kvc_version", "kvc_launch_count", "kvc_score_noalloc", "kvc_score_entropy",
             "kvc_row_stats", "kvc_csm_merges", "kvc_csm_ratio", "kvc_csm_workspace_size", "kvc_csm", "kvc_append",
             "kvc_decode_attention_workspace_size", "kvc_decode_attention", "kvc_shard_workspace_size",
-            "kvc_shard_stats", "kvc_shard_scores", "kvc_select_hist", "kvc_select_emit")
+            "kvc_shard_stats", "kvc_shard_scores", "kvc_select_hist", "kvc_select_emit", "kvc_select_pick",
+            "kvc_select_ties", "kvc_select_kept")
 
 
 class KvcError(RuntimeError):
@@ -82,6 +83,9 @@ def _load():
         "kvc_shard_scores": (st, [P, vp, vp, i32, i32, vp, i32, vp, vp, sz, vp]),
         "kvc_select_hist": (st, [vp, i32, i32, i32, i32, vp, i32, i32, vp, vp]),
         "kvc_select_emit": (st, [vp, i32, i32, i32, i32, vp, vp, i32, vp, i32, vp, vp]),
+        "kvc_select_pick": (st, [vp, vp, i32, i32, i32, vp, vp, vp, vp]),
+        "kvc_select_ties": (st, [vp, i32, i32, i32, vp, vp, vp]),
+        "kvc_select_kept": (st, [vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -300,6 +304,26 @@ def kvc_select_emit(pooled, lo, hi, thr, ties, pos_offset, out, count, stream=No
     rows, n = pooled.shape[0] * pooled.shape[1], pooled.shape[-1]
     _check(lib.kvc_select_emit(_ptr(pooled), rows, n, lo, hi, _ptr(thr), _ptr(ties), pos_offset, _ptr(out),
                                out.shape[-1], _ptr(count), _stream(stream)), "kvc_select_emit")
+
+
+def kvc_select_pick(hist, hist_local, prefix_bits, need, prefix, eq_local, stream=None):
+    rows, nb = hist.shape
+    digit_bits = nb.bit_length() - 1
+    _check(lib.kvc_select_pick(_ptr(hist), _ptr(hist_local), rows, digit_bits, prefix_bits, _ptr(need), _ptr(prefix),
+                               _ptr(eq_local), _stream(stream)), "kvc_select_pick")
+
+
+def kvc_select_ties(eq_all, rank, need, take, stream=None):
+    n_shards, rows = eq_all.shape
+    _check(lib.kvc_select_ties(_ptr(eq_all), n_shards, rank, rows, _ptr(need), _ptr(take), _stream(stream)),
+           "kvc_select_ties")
+
+
+def kvc_select_kept(sel, count_sel, N, n_sink, window, key_offset, n_local, pos, local_idx, count, stream=None):
+    rows, cap_sel = sel.shape
+    _check(lib.kvc_select_kept(_ptr(sel), _ptr(count_sel), rows, cap_sel, N, n_sink, window, key_offset, n_local,
+                               pos.shape[-1], _ptr(pos), _ptr(local_idx), _ptr(count), _stream(stream)),
+           "kvc_select_kept")
 
 
 def kvc_accumulate(acc, src, stream=None):

@@ -15,13 +15,13 @@ small exchange per step, all of a few KiB:
      the ties left after the lower ranks' (ties go to the lower positions);
   5. each rank gathers its kept rows; the compact cache is the ranks' parts in rank order.
 
-Every step on the data runs in the library's kernels (`Ops`); this module holds the order
-of the steps and the exchanges (`Comm`), both replaceable so that the host logic can be
-exercised with CPU ranks.
+Every step on the data runs in the library's kernels (`Ops`), the radix bucket picks, the
+split of ties and the kept positions included, so the data stays on the device and the host
+does not wait for it; this module holds the order of the steps and the exchanges (`Comm`),
+both replaceable so that the host logic can be exercised with CPU ranks.
 """
 from __future__ import annotations
 
-import numpy as np
 import torch
 
 DIGITS = (11, 11, 10)
@@ -87,6 +87,27 @@ class GpuOps:
         self.kvc.kvc_select_hist(pooled, lo, hi, prefix.to(pooled.device), prefix_bits, digit_bits, hist)
         return hist
 
+    def pick(self, hist, hist_local, prefix_bits, need, prefix):
+        """One digit: the bucket of every row's need-th largest key (device); returns the
+        updated need and prefix and this rank's count in the bucket."""
+        need, prefix = need.clone(), prefix.clone()
+        eq_local = torch.empty_like(need)
+        self.kvc.kvc_select_pick(hist, hist_local, prefix_bits, need, prefix, eq_local)
+        return need, prefix, eq_local
+
+    def ties(self, eq_all, rank, need):
+        take = torch.empty_like(need)
+        self.kvc.kvc_select_ties(eq_all.contiguous(), rank, need, take)
+        return take
+
+    def kept(self, sel, cnt, p, key_offset, n_local, cap):
+        rows = sel.shape[0]
+        pos = torch.empty((rows, cap), dtype=torch.int32, device=sel.device)
+        local = torch.empty_like(pos)
+        count = torch.empty((rows,), dtype=torch.int32, device=sel.device)
+        self.kvc.kvc_select_kept(sel, cnt, p.N, p.n_sink, p.window, key_offset, n_local, pos, local, count)
+        return pos, local, count
+
     def emit(self, pooled, lo, hi, thr, ties, pos_offset, cap):
         rows = pooled.shape[0] * pooled.shape[1]
         out = torch.empty((rows, max(cap, 1)), dtype=torch.int32, device=pooled.device)
@@ -101,27 +122,16 @@ class GpuOps:
         return dst
 
 
-def _pick_buckets(hist: np.ndarray, need: np.ndarray):
-    """Per row, the bucket b holding the need-th largest key (buckets scanned from the top)
-    and the number of keys still needed inside it."""
-    nb = hist.shape[1]
-    from_top = np.cumsum(hist[:, ::-1], axis=1)               # keys in buckets >= nb - 1 - i
-    i = np.argmax(from_top >= need[:, None], axis=1)
-    b = nb - 1 - i
-    rows = np.arange(hist.shape[0])
-    above = from_top[rows, i] - hist[rows, b]                  # keys in buckets above b
-    return b.astype(np.int64), need - above
-
-
 def sharded_compress(comm, ops, p, q, k_local, v_local, key_offset: int):
     """One rank's part of the sharded compaction.
 
     p         kvc Params of the whole sequence (N = all keys; n_layers 1, per-KV-head scope)
     q         [B, Hq, window, D] window queries (the same on every rank)
     k_local, v_local  [B, Hkv, n_local, D]: keys key_offset .. key_offset + n_local - 1
-    Returns {"pos": [B, Hkv, cap] global positions this rank keeps (ascending, padded with
-    -1), "count": [B, Hkv] kept per row, "k", "v": the kept rows [B, Hkv, cap, D] (rows past
-    count are padding), "scores": this rank's scores [B, Hkv, n_local]}.
+    Returns {"pos": [B, Hkv, cap] int32 global positions this rank keeps (ascending, padded
+    with -1), "count": [B, Hkv] int32 kept per row, "k", "v": the kept rows [B, Hkv, cap, D]
+    (rows past count are padding), "scores": this rank's scores [B, Hkv, n_local]}, all on the
+    ranks' device; cap = min(n_local, kv_budget).
     """
     B, H, n_local, D = k_local.shape
     N, S, w, P = p.N, p.n_sink, p.window, p.pool_kernel
@@ -156,41 +166,27 @@ def sharded_compress(comm, ops, p, q, k_local, v_local, key_offset: int):
     own_lo, own_hi = max(S, key_offset) - base, min(N - w, key_offset + n_local) - base
     own_hi = max(own_hi, own_lo)
 
-    # 3. radix select over every rank's candidates
-    need = np.full(rows, k_sel, dtype=np.int64)
-    prefix = np.zeros(rows, dtype=np.uint32)
+    # 3. radix select over every rank's candidates: per digit, the histograms summed over
+    #    ranks, then every rank picks the same bucket (on the device)
+    need = torch.full((rows,), k_sel, dtype=torch.int32, device=dev)
+    prefix = torch.zeros((rows,), dtype=torch.int32, device=dev)
     bits = 0
-    local_last = None
+    eq_local = None
     for d in DIGITS:
-        hist_local = ops.hist(pooled, own_lo, own_hi, torch.from_numpy(prefix.view(np.int32).copy()), bits, d)
-        hist = comm.all_reduce_sum(hist_local).cpu().numpy().astype(np.int64)
-        b, need = _pick_buckets(hist, need)
-        prefix = prefix | (b.astype(np.uint32) << np.uint32(32 - bits - d))
+        hist_local = ops.hist(pooled, own_lo, own_hi, prefix, bits, d)
+        hist = comm.all_reduce_sum(hist_local)
+        need, prefix, eq_local = ops.pick(hist, hist_local, bits, need, prefix)
         bits += d
-        local_last = (hist_local.cpu().numpy().astype(np.int64), b)
 
     # 4. ties: the lower ranks take theirs first
-    hl, b = local_last
-    mine_eq = hl[np.arange(rows), b]
-    eq_all = comm.all_gather(torch.from_numpy(mine_eq).to(dev)).cpu().numpy()
-    before = eq_all[:comm.rank].sum(axis=0) if comm.rank > 0 else np.zeros(rows, dtype=np.int64)
-    take = np.clip(need - before, 0, mine_eq).astype(np.int32)
+    eq_all = comm.all_gather(eq_local)
+    take = ops.ties(eq_all, comm.rank, need)
     cap_sel = max(own_hi - own_lo, 1)
-    sel, cnt = ops.emit(pooled, own_lo, own_hi, torch.from_numpy(prefix.view(np.int32).copy()),
-                        torch.from_numpy(take), base, cap_sel)
-    sel, cnt = sel.cpu().numpy(), cnt.cpu().numpy()
+    sel, cnt = ops.emit(pooled, own_lo, own_hi, prefix, take, base, cap_sel)
 
     # 5. kept positions of this block: sinks, the selection, the window; then the rows
-    sinks = [t for t in range(S) if key_offset <= t < key_offset + n_local]
-    window = [t for t in range(N - w, N) if key_offset <= t < key_offset + n_local]
-    counts = len(sinks) + cnt + len(window)
-    cap = int(counts.max()) if rows else 0
-    pos = np.full((rows, max(cap, 1)), -1, dtype=np.int64)
-    for r in range(rows):
-        kept = sinks + list(sel[r, :cnt[r]]) + window
-        pos[r, :len(kept)] = kept
-    pos = pos.reshape(B, H, -1)
-    local = np.where(pos >= 0, pos - key_offset, 0).astype(np.int32)
-    idx = torch.from_numpy(local).to(dev)
-    return {"pos": pos, "count": counts.reshape(B, H), "k": ops.gather(k_local, idx), "v": ops.gather(v_local, idx),
-            "scores": scores}
+    cap = max(1, min(n_local, p.kv_budget))
+    pos, local, count = ops.kept(sel, cnt, p, key_offset, n_local, cap)
+    idx = local.reshape(B, H, cap)
+    return {"pos": pos.reshape(B, H, cap), "count": count.reshape(B, H), "k": ops.gather(k_local, idx),
+            "v": ops.gather(v_local, idx), "scores": scores}

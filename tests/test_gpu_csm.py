@@ -3,10 +3,12 @@
 Cosine similarities are fp32 on the GPU and fp64 in the oracle, so the decisions they take
 follow the band rule used for the top-k: a match whose oracle similarity is clearly above
 (below) the m-th best must (must not) merge; only matches within 1e-5 of it may differ.
-Given the GPU's merge set, every kept row must equal the oracle's degree-weighted mean of
-the same tokens up to fp32 summation error (2e-6 of the summands' magnitude) plus, for bf16
-outputs, one unit in the last place; every unmerged row must be a bit-exact copy, and
-degrees and positions must be exact.
+Given the GPU's merge set, every kept row must equal the exact degree-weighted mean of the
+same tokens up to fp32 summation error (2e-6 of the summands' magnitude) plus, for bf16
+outputs, half a unit in the last place; every unmerged row must be a bit-exact copy, and
+degrees and positions must be exact.  When the GPU's merge set is the oracle's (the common
+case), the kept rows are also compared with the oracle's own rounded outputs (one unit in
+the last place for bf16) and the bit-identical fraction is reported.
 """
 import numpy as np
 import pytest
@@ -66,11 +68,19 @@ def test_csm_matches_oracle(K, case):
     out = K.kvc_csm(k.cuda(), v.cuda(), c["S"], c["w"], c["chunk"], c["ratio"],
                     deg=deg.cuda() if c["deg"] else None)
     assert K.kvc_poll_error() == K.KVC_OK
+    same = []
     for b in range(B):
         for h in range(H):
-            check_row(k[b, h], v[b, h], deg[b, h].numpy(), out["k_out"][b, h].cpu(), out["v_out"][b, h].cpu(),
-                      out["deg_out"][b, h].cpu().numpy(), out["pos_out"][b, h].cpu().numpy(), c["S"], c["w"],
-                      c["chunk"], c["ratio"], c["dtype"])
+            same.append(check_row(k[b, h], v[b, h], deg[b, h].numpy(), out["k_out"][b, h].cpu(),
+                                  out["v_out"][b, h].cpu(), out["deg_out"][b, h].cpu().numpy(),
+                                  out["pos_out"][b, h].cpu().numpy(), c["S"], c["w"], c["chunk"], c["ratio"],
+                                  c["dtype"]))
+    compared = [f for f in same if f is not None]
+    print(f"case {case}: {len(compared)}/{len(same)} rows with the oracle's merge set, bit-identical elements "
+          f"{(sum(compared) / len(compared)) if compared else float('nan'):.4f}")
+    if not c["zero"]:
+        # (zero keys tie at cosine 0 with every token, which leaves their rows ambiguous)
+        assert compared, "no row merged exactly the oracle's tokens"
 
 
 EDGE_CASES = [

@@ -9,7 +9,7 @@ import torch
 
 from long_context_kv_kvc_b200 import synth
 from oracle import oracle as O
-from parity_util import check_gather, check_index_sets, check_scores, error_band
+from parity_util import check_gather, check_index_sets, check_scores, error_band, run_case
 
 pytestmark = pytest.mark.gpu
 
@@ -27,36 +27,6 @@ def K():
 
 def _dev(inp):
     return {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
-
-
-def run_case(K, wl, flags=0):
-    inp = synth.make_inputs(wl)
-    dev = _dev(inp)
-    p = K.params_for(wl, flags=flags)
-    comp = K.Compressor(p)
-    out = comp(dev["q"], dev["k"], dev["v"], dev.get("hidden"))
-    Hs = wl.Hkv if wl.scope == K.KVC_SCOPE_PER_KV_HEAD else 1
-    scores = torch.empty((wl.B, Hs, wl.N), dtype=torch.float32, device="cuda")
-    K.kvc_score(p, dev["q"], dev["k"], scores, comp.ws)
-    assert K.kvc_poll_error() == K.KVC_OK
-    ref = O.compress(inp["q"], inp["k"], inp["v"], window=wl.window, n_sink=wl.n_sink,
-                     pool_kernel=wl.pool_kernel, kv_budget=wl.kv_budget, scope=wl.scope,
-                     tsp_rate=float(np.float32(wl.tsp_rate)), hidden=inp["hidden"])
-    worst = check_scores(scores.cpu().numpy(), ref["scores"])
-    band = error_band(worst)
-    exact = check_index_sets(out["idx_out"].cpu().numpy(), ref["pooled"], wl.N, wl.n_sink, wl.window,
-                             wl.kv_budget, rtol=band)
-    print(f"{wl.name}: worst score error {worst:.2e}, index band {band:.1e}, exact index sets {exact:.3f}")
-    check_gather(out["k_out"], dev["k"][-1], out["idx_out"].cpu().numpy())
-    check_gather(out["v_out"], dev["v"], out["idx_out"].cpu().numpy())
-    if wl.tsp_rate > 0:
-        n_tsp = K.kvc_tsp_count(wl.N, wl.window, wl.n_sink, wl.tsp_rate)
-        tsp_exact = check_index_sets(out["tsp_idx_out"].cpu().numpy(), ref["tsp_pooled"], wl.N, wl.n_sink,
-                                     wl.window, n_tsp, rtol=band)
-        print(f"{wl.name}: exact TSP index sets {tsp_exact:.3f}")
-        check_gather(out["hidden_out"].unsqueeze(1), dev["hidden"].unsqueeze(1),
-                     out["tsp_idx_out"].cpu().numpy())
-    return out, ref, scores
 
 
 def test_tiny_f32(K):

@@ -2,9 +2,11 @@
 share cuda:0 and exchange through an in-process collective (they wait for each other on
 the host only; no kernel waits on another).
 
-* kvc_shard_stats / kvc_shard_scores over blocks equal kvc_score of the whole sequence
-  (CUDA-core path) within 1e-5 relative (the log-sum-exp is merged in another order);
-* kvc_select_hist / kvc_select_emit equal their numpy contract bit for bit (ties, -0.0);
+* kvc_shard_stats / kvc_shard_scores over blocks equal kvc_score of the whole sequence on
+  the same path (tensor cores, and CUDA cores) within 1e-5 relative (the log-sum-exp is
+  merged in another order), and the oracle within 1e-3;
+* kvc_select_hist / kvc_select_emit / kvc_select_pick / kvc_select_ties / kvc_select_kept
+  equal their numpy contract bit for bit (ties, -0.0);
 * the sharded compaction's union of kept positions passes the band rule against the fp64
   oracle, and every rank's kept rows are its source rows.
 """
@@ -75,12 +77,13 @@ def order_key(x32):
     return np.where(neg, ~b, b | np.uint32(0x80000000)).astype(np.uint32)
 
 
-def test_shard_scores_match_whole_sequence(K):
+@pytest.mark.parametrize("flags", [0, 1], ids=["tensor-cores", "cuda-cores"])
+def test_shard_scores_match_whole_sequence(K, flags):
     from long_context_kv_kvc_b200 import synth
     wl = synth.scaled(synth.LLAMA8B_32K, B=2, Hq=8, Hkv=2, N=3001, kv_budget=300, n_hubs=16)
     inp = synth.make_inputs(wl, with_v=False, with_hidden=False)
     q, k = inp["q"][0].cuda(), inp["k"][0].cuda()
-    p = K.params_for(wl, flags=K.KVC_FLAG_SIMT_SCORE)
+    p = K.params_for(wl, flags=flags)
     whole = torch.empty((wl.B, wl.Hkv, wl.N), device="cuda")
     ws = torch.empty(K.kvc_workspace_size(p), dtype=torch.uint8, device="cuda")
     K.kvc_score(p, q, k, whole, ws)
@@ -144,6 +147,66 @@ def test_select_hist_and_emit_contract(K):
         assert np.array_equal(out[r, :want.size].cpu().numpy(), want)
 
 
+def test_select_pick_ties_kept_contract(K):
+    g = np.random.default_rng(5)
+    rows = 6
+    for digit_bits, prefix_bits in [(11, 0), (11, 11), (10, 22), (12, 3)]:
+        nb = 1 << digit_bits
+        hist_local = g.integers(0, 4, (rows, nb)).astype(np.int32)
+        hist_local[:, ::7] = 0
+        hist = hist_local + g.integers(0, 3, (rows, nb)).astype(np.int32)
+        need = np.array([1, 5, 100, int(hist[3].sum()), 2, 33], dtype=np.int32)
+        prefix = g.integers(0, 1 << 16, rows).astype(np.uint32) << np.uint32(32 - max(prefix_bits, 1)) \
+            if prefix_bits else np.zeros(rows, np.uint32)
+        d_need = torch.from_numpy(need.copy()).cuda()
+        d_pre = torch.from_numpy(prefix.view(np.int32).copy()).cuda()
+        d_eq = torch.empty(rows, dtype=torch.int32, device="cuda")
+        K.kvc_select_pick(torch.from_numpy(hist).cuda(), torch.from_numpy(hist_local).cuda(), prefix_bits, d_need,
+                          d_pre, d_eq)
+        from_top = np.cumsum(hist[:, ::-1].astype(np.int64), axis=1)
+        i = np.argmax(from_top >= need[:, None], axis=1)
+        b = nb - 1 - i
+        r = np.arange(rows)
+        want_need = need - (from_top[r, i] - hist[r, b])
+        want_pre = prefix | (b.astype(np.uint32) << np.uint32(32 - prefix_bits - digit_bits))
+        assert np.array_equal(d_need.cpu().numpy(), want_need)
+        assert np.array_equal(d_pre.cpu().numpy().view(np.uint32), want_pre)
+        assert np.array_equal(d_eq.cpu().numpy(), hist_local[r, b])
+    eq_all = g.integers(0, 5, (3, rows)).astype(np.int32)
+    need = np.array([0, 1, 4, 7, 20, 3], dtype=np.int32)
+    for rank in range(3):
+        take = torch.empty(rows, dtype=torch.int32, device="cuda")
+        K.kvc_select_ties(torch.from_numpy(eq_all).cuda(), rank, torch.from_numpy(need).cuda(), take)
+        want = np.clip(need - eq_all[:rank].sum(axis=0), 0, eq_all[rank])
+        assert np.array_equal(take.cpu().numpy(), want)
+    # kept rows: sinks, selection, window of a block of the sequence
+    N, S, w = 1000, 3, 16
+    for key_off, n_local in [(0, 400), (400, 590), (990, 10), (2, 5)]:
+        cap_sel = max(n_local, 1)
+        sel = np.full((rows, cap_sel), -7, dtype=np.int32)
+        cnt = g.integers(0, min(n_local, 40), rows).astype(np.int32)
+        for r_ in range(rows):
+            sel[r_, :cnt[r_]] = np.sort(g.choice(np.arange(key_off, key_off + n_local), cnt[r_], replace=False))
+        cap = min(n_local, 64)
+        pos = torch.empty((rows, cap), dtype=torch.int32, device="cuda")
+        local = torch.empty_like(pos)
+        count = torch.empty(rows, dtype=torch.int32, device="cuda")
+        K.kvc_select_kept(torch.from_numpy(sel).cuda(), torch.from_numpy(cnt).cuda(), N, S, w, key_off, n_local,
+                          pos, local, count)
+        sinks = [t for t in range(S) if key_off <= t < key_off + n_local]
+        window = [t for t in range(N - w, N) if key_off <= t < key_off + n_local]
+        over = False
+        for r_ in range(rows):
+            kept = sinks + sel[r_, :cnt[r_]].tolist() + window
+            over |= len(kept) > cap
+            assert count[r_].item() == len(kept)
+            k_ = kept[:cap]
+            assert pos[r_, :len(k_)].cpu().tolist() == k_
+            assert np.all(pos[r_, len(k_):].cpu().numpy() == -1)
+            assert local[r_, :len(k_)].cpu().tolist() == [t - key_off for t in k_]
+        assert K.kvc_poll_error() == (K.KVC_ERR_INDEX if over else K.KVC_OK)
+
+
 @pytest.mark.parametrize("cuts", [[0, 1000, 2001], [0, 3, 900, 1990, 2001]], ids=["2", "4-window-split"])
 def test_sharded_compress_on_threads(K, cuts):
     from long_context_kv_kvc_b200 import synth
@@ -164,12 +227,12 @@ def test_sharded_compress_on_threads(K, cuts):
     rows = wl.B * wl.Hkv
     kept = [[] for _ in range(rows)]
     for r, out in enumerate(res):
-        pos = out["pos"].reshape(rows, -1)
-        cnt = out["count"].reshape(-1)
+        pos = out["pos"].cpu().numpy().reshape(rows, -1)
+        cnt = out["count"].cpu().numpy().reshape(-1)
         for i in range(rows):
             b, h = divmod(i, wl.Hkv)
             kept[i].extend(pos[i, :cnt[i]].tolist())
-            src = torch.from_numpy(pos[i, :cnt[i]]).cuda()
+            src = torch.from_numpy(pos[i, :cnt[i]]).long().cuda()
             assert torch.equal(out["k"][b, h, :cnt[i]], k[b, h, src])
             assert torch.equal(out["v"][b, h, :cnt[i]], v[b, h, src])
     idx = np.array(kept, dtype=np.int64).reshape(wl.B, wl.Hkv, -1)

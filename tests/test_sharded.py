@@ -91,6 +91,41 @@ class NumpyOps:
             out[r] = np.bincount(d.astype(np.int64), minlength=nb)
         return torch.from_numpy(out)
 
+    def pick(self, hist, hist_local, prefix_bits, need, prefix):
+        """Per row, the bucket b (scanned from the top) holding the need-th largest key, the
+        keys still needed inside it, the prefix extended by b, this rank's count in b."""
+        h = hist.numpy().astype(np.int64)
+        nb = h.shape[1]
+        digit_bits = nb.bit_length() - 1
+        need_in = need.numpy().astype(np.int64)
+        from_top = np.cumsum(h[:, ::-1], axis=1)
+        i = np.argmax(from_top >= need_in[:, None], axis=1)
+        b = nb - 1 - i
+        r = np.arange(h.shape[0])
+        above = from_top[r, i] - h[r, b]
+        pre = prefix.numpy().view(np.uint32) | (b.astype(np.uint32) << np.uint32(32 - prefix_bits - digit_bits))
+        eq = hist_local.numpy()[r, b]
+        return (torch.from_numpy((need_in - above).astype(np.int32)), torch.from_numpy(pre.view(np.int32).copy()),
+                torch.from_numpy(eq.astype(np.int32)))
+
+    def ties(self, eq_all, rank, need):
+        e = eq_all.numpy().astype(np.int64)
+        before = e[:rank].sum(axis=0) if rank > 0 else np.zeros(e.shape[1], dtype=np.int64)
+        return torch.from_numpy(np.clip(need.numpy() - before, 0, e[rank]).astype(np.int32))
+
+    def kept(self, sel, cnt, p, key_offset, n_local, cap):
+        rows = sel.shape[0]
+        pos = np.full((rows, cap), -1, dtype=np.int32)
+        count = np.zeros(rows, dtype=np.int32)
+        sinks = [t for t in range(p.n_sink) if key_offset <= t < key_offset + n_local]
+        window = [t for t in range(p.N - p.window, p.N) if key_offset <= t < key_offset + n_local]
+        for r in range(rows):
+            kept = sinks + list(sel.numpy()[r, :int(cnt[r])]) + window
+            pos[r, :len(kept)] = kept
+            count[r] = len(kept)
+        local = np.where(pos >= 0, pos - key_offset, 0).astype(np.int32)
+        return torch.from_numpy(pos), torch.from_numpy(local), torch.from_numpy(count)
+
     def emit(self, pooled, lo, hi, thr, ties, pos_offset, cap):
         x = pooled.numpy().reshape(-1, pooled.shape[-1])
         T = thr.numpy().view(np.uint32)
@@ -130,8 +165,8 @@ def _worker(rank, world, port, cuts, out_dir):
     k, v = inp["k"][0], inp["v"]
     lo, hi = cuts[rank], cuts[rank + 1]
     res = sharded_compress(TorchComm(), NumpyOps(), p, q, k[:, :, lo:hi].contiguous(), v[:, :, lo:hi].contiguous(), lo)
-    np.save(os.path.join(out_dir, f"pos{rank}.npy"), res["pos"])
-    np.save(os.path.join(out_dir, f"count{rank}.npy"), res["count"])
+    np.save(os.path.join(out_dir, f"pos{rank}.npy"), res["pos"].numpy())
+    np.save(os.path.join(out_dir, f"count{rank}.npy"), res["count"].numpy())
     torch.save({"k": res["k"], "v": res["v"]}, os.path.join(out_dir, f"rows{rank}.pt"))
     dist.barrier()
     dist.destroy_process_group()

@@ -5,13 +5,14 @@ already handed all of device memory to its own pool, or a plugin interface that 
 cudaMalloc/cudaFree during a step).  This entry point keeps its scratch in a fixed array
 inside the library instead.  The test calls it through the C ABI twice in a row, on
 different inputs, and checks each result against kvc_score (which uses a caller
-workspace) within the score tolerance of the other parity tests.  It lives in its own
-file, named so that pytest collects it last.
+workspace) within the score tolerance of the other parity tests, and against the fp64
+oracle.  It lives in its own file, named so that pytest collects it last.
 """
 import pytest
 import torch
 
 from long_context_kv_kvc_b200 import synth
+from oracle import oracle as O
 from parity_util import SCORE_RTOL, check_scores
 
 pytestmark = pytest.mark.gpu
@@ -39,7 +40,8 @@ def _scores_both_ways(K, wl):
     no_ws = torch.full((wl.B, Hs, wl.N), float("nan"), dtype=torch.float32, device="cuda")
     K.kvc_score_noalloc(p, q, k, no_ws)
     assert K.kvc_poll_error() == K.KVC_OK
-    return no_ws.double().cpu().numpy(), with_ws.double().cpu().numpy()
+    ref = O.score(inp["q"], inp["k"], window=wl.window, scope=wl.scope)
+    return no_ws.double().cpu().numpy(), with_ws.double().cpu().numpy(), ref
 
 
 def test_noalloc_matches_workspace_entry_point_twice(K):
@@ -47,14 +49,15 @@ def test_noalloc_matches_workspace_entry_point_twice(K):
     second = synth.scaled(synth.STRUCTKV_8L_32K, N=3001, n_layers=2, kv_budget=300, n_hubs=16,
                           seeds=(7,))
     for wl in (first, second):
-        got, want = _scores_both_ways(K, wl)
+        got, want, ref = _scores_both_ways(K, wl)
         check_scores(got, want, rtol=SCORE_RTOL)
+        check_scores(got, ref, rtol=SCORE_RTOL)
 
 
 def test_noalloc_rejects_what_does_not_fit(K):
+    # no buffers at all: the size check must reject the call before anything is touched
     wl = synth.LLAMA8B_128K_B4.replace(n_layers=2)
     p = K.params_for(wl)
-    dummy = torch.empty(16, dtype=torch.uint8, device="cuda")
     with pytest.raises(K.KvcError) as e:
-        K.kvc_score_noalloc(p, dummy, dummy, dummy)
+        K.kvc_score_noalloc(p, None, None, None)
     assert e.value.status == K.KVC_ERR_WORKSPACE
