@@ -377,9 +377,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
         // Warp 0 streams the phase-1 tiles from HBM, one 32 KiB op per tile (both 64-column
         // halves); warps 2 and 6 issue the phase-2 re-reads, half 0 and half 1 of every tile.
         // A single issuing thread completes TMA ops at a roughly fixed rate, so the phase-1
-        // stream uses large ops and the phase-2 stream two threads.  kScores: warp 0 loads only
-        // the Q of each unit; kStats: no phase-2 re-reads.
-        if (lane == 0 && !(MODE == kStats && warp != 0)) {
+        // stream uses large ops and the phase-2 stream two threads.  kStats: no phase-2
+        // re-reads; kScores: no phase 1, so warp 0 streams the tiles (from HBM, one 32 KiB op
+        // each) straight to the phase-2 jobs.
+        if (lane == 0 && !(MODE != kFull && warp != 0)) {
             const int ph = warp == 0 ? 0 : 1, hh = warp == 6 ? 1 : 0;
             const CUtensorMap* mk = ph == 0 ? &a.tmap_k4 : &a.tmap_k;
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(mk)) : "memory");
@@ -415,12 +416,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                     tma_load_2d(sm.q[slot] + kBoxBytes, &a.tmap_q, &sm.qfull[slot], 64, u * kQRows);
                 }
                 if (ph == 0) {
-                    if (MODE != kScores) {
-                        const int st = i % kTilesA;
-                        mbar_spin(&sm.emptyA[st], ((i / kTilesA) & 1) ^ 1, abort, a.err);
-                        mbar_expect_tx(&sm.fullA[st], 2 * kBoxBytes);
-                        tma_load_4d(sm.ringA[2 * st], mk, &sm.fullA[st], 0, ti * kTileKeys, 0, u);
-                    }
+                    const int st = i % kTilesA;
+                    mbar_spin(&sm.emptyA[st], ((i / kTilesA) & 1) ^ 1, abort, a.err);
+                    mbar_expect_tx(&sm.fullA[st], 2 * kBoxBytes);
+                    tma_load_4d(sm.ringA[2 * st], mk, &sm.fullA[st], 0, ti * kTileKeys, 0, u);
                     *reinterpret_cast<volatile int*>(&sm.p1_issued) = i + 1;
                 } else {
                     const int k = 2 * i + hh, st = k % kStagesB;
@@ -433,9 +432,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             if (*abort) {
                 // copies still in flight land before the CTA exits
                 if (ph == 0) {
-                    if (MODE != kScores)
-                        for (int n = std::max(0, i - kTilesA); n < i; ++n)
-                            drain_wait(&sm.fullA[n % kTilesA], (n / kTilesA) & 1, a.err);
+                    for (int n = std::max(0, i - kTilesA); n < i; ++n)
+                        drain_wait(&sm.fullA[n % kTilesA], (n / kTilesA) & 1, a.err);
                     for (int o = std::max(0, ord - kQSlots + 1); o <= ord; ++o)
                         drain_wait(&sm.qfull[o % kQSlots], (o / kQSlots) & 1, a.err);
                 } else {
@@ -471,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                 }
                 // phase 2 of a tile waits until its unit's lse is in shared memory
                 if (ph == 1) mbar_spin(&sm.lsefull[ord & 1], (ord >> 1) & 1, abort, a.err);
-                if (ph == 0)
+                if (ph == 0 || MODE == kScores)
                     mbar_spin(&sm.fullA[i % kTilesA], (i / kTilesA) & 1, abort, a.err);
                 else
                     mbar_spin(&sm.fullB[s], sph, abort, a.err);
@@ -494,6 +492,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                     const uint64_t dk = dK0 + (uint64_t)(2 * st) * kBoxStep;
                     umma_half(d, dq, dk, 0);
                     umma_half(d, dq + kBoxStep, dk + kBoxStep, 1);
+                    umma_commit(&sm.emptyA[st]);
+                } else if (MODE == kScores) {
+                    // phase 2 alone: the tile came through the phase-1 ring
+                    const int st = i % kTilesA;
+                    const uint64_t dk = sw128_desc(smem_u32(sm.ringA[0])) + (uint64_t)(2 * st) * kBoxStep;
+                    tc_fence_after();
+                    umma_half(d, dk, dq, 0);
+                    umma_half(d, dk + kBoxStep, dq + kBoxStep, 1);
                     umma_commit(&sm.emptyA[st]);
                 } else {
 #pragma unroll

@@ -306,7 +306,14 @@ def kvc_select_emit(pooled, lo, hi, thr, ties, pos_offset, out, count, stream=No
                                out.shape[-1], _ptr(count), _stream(stream)), "kvc_select_emit")
 
 
+def _int32(*ts):
+    for t in ts:
+        if t.dtype != torch.int32:
+            raise TypeError(f"expected int32 tensors, got {t.dtype}")
+
+
 def kvc_select_pick(hist, hist_local, prefix_bits, need, prefix, eq_local, stream=None):
+    _int32(hist, hist_local, need, prefix, eq_local)
     rows, nb = hist.shape
     digit_bits = nb.bit_length() - 1
     _check(lib.kvc_select_pick(_ptr(hist), _ptr(hist_local), rows, digit_bits, prefix_bits, _ptr(need), _ptr(prefix),
@@ -314,12 +321,14 @@ def kvc_select_pick(hist, hist_local, prefix_bits, need, prefix, eq_local, strea
 
 
 def kvc_select_ties(eq_all, rank, need, take, stream=None):
+    _int32(eq_all, need, take)
     n_shards, rows = eq_all.shape
     _check(lib.kvc_select_ties(_ptr(eq_all), n_shards, rank, rows, _ptr(need), _ptr(take), _stream(stream)),
            "kvc_select_ties")
 
 
 def kvc_select_kept(sel, count_sel, N, n_sink, window, key_offset, n_local, pos, local_idx, count, stream=None):
+    _int32(sel, count_sel, pos, local_idx, count)
     rows, cap_sel = sel.shape
     _check(lib.kvc_select_kept(_ptr(sel), _ptr(count_sel), rows, cap_sel, N, n_sink, window, key_offset, n_local,
                                pos.shape[-1], _ptr(pos), _ptr(local_idx), _ptr(count), _stream(stream)),

@@ -92,12 +92,13 @@ class GpuOps:
         updated need and prefix and this rank's count in the bucket."""
         need, prefix = need.clone(), prefix.clone()
         eq_local = torch.empty_like(need)
-        self.kvc.kvc_select_pick(hist, hist_local, prefix_bits, need, prefix, eq_local)
+        # a collective may hand back the summed counts widened to int64
+        self.kvc.kvc_select_pick(hist.to(torch.int32).contiguous(), hist_local, prefix_bits, need, prefix, eq_local)
         return need, prefix, eq_local
 
     def ties(self, eq_all, rank, need):
         take = torch.empty_like(need)
-        self.kvc.kvc_select_ties(eq_all.contiguous(), rank, need, take)
+        self.kvc.kvc_select_ties(eq_all.to(torch.int32).contiguous(), rank, need, take)
         return take
 
     def kept(self, sel, cnt, p, key_offset, n_local, cap):
