@@ -46,6 +46,13 @@
  *              (a CUDA launch failed part way).  Device-side problems (a bounded wait that
  *              gave up, an index out of range in kvc_gather) never fault or hang the GPU:
  *              the kernel skips the work, records a flag, and kvc_poll_error reports it.
+ *   Checks     The same sources also build as libkvc_checks.so (compile flag KVC_CHECKS=1):
+ *              every kernel then tests the indices and coordinates it forms (score and
+ *              index writes, gather rows, TMA tile coordinates, CSM owners and output
+ *              slots, decode partial slots) against the extents of the buffers they
+ *              address, plus the counts the selection must reach; a failed test skips the
+ *              access and kvc_poll_error returns KVC_ERR_CHECK.  kvc_checks_enabled tells
+ *              the two builds apart.  The regular build compiles the tests away.
  *   Threading  Calls are thread-safe; concurrent calls need distinct workspaces.
  *   Alignment  q, k, v, hidden and all outputs must be 16-byte aligned; ws 256-byte.
  */
@@ -76,7 +83,8 @@ typedef enum kvc_status {
     KVC_ERR_WORKSPACE = 5,   /* ws_bytes smaller than kvc_workspace_size                  */
     KVC_ERR_CUDA = 6,        /* a CUDA runtime call failed                                */
     KVC_ERR_TIMEOUT = 7,     /* a device-side bounded wait gave up (reported by poll)      */
-    KVC_ERR_INDEX = 8        /* kvc_gather met an index outside [0, N) (reported by poll)  */
+    KVC_ERR_INDEX = 8,       /* kvc_gather met an index outside [0, N) (reported by poll)  */
+    KVC_ERR_CHECK = 9        /* a device-side range check failed: checks build only (poll)  */
 } kvc_status;
 
 enum { KVC_F32 = 0, KVC_BF16 = 1 };
@@ -497,11 +505,18 @@ KVC_API kvc_status kvc_score_noalloc(const kvc_params *p, const void *q, const v
 KVC_API int32_t kvc_tsp_count(int32_t N, int32_t window, int32_t n_sink, float tsp_rate);
 
 /*
- * kvc_poll_error -- synchronises `stream`, then returns (and clears) the first device-side
- * problem recorded since the last poll on this device: KVC_ERR_TIMEOUT, KVC_ERR_INDEX, or
- * KVC_OK.  KVC_ERR_CUDA if the synchronisation itself failed.
+ * kvc_poll_error -- synchronises `stream`, then returns (and clears) the device-side
+ * problems recorded since the last poll on this device, reporting the first of
+ * KVC_ERR_TIMEOUT, KVC_ERR_INDEX, KVC_ERR_CHECK (checks build only) that is set, else KVC_OK.
+ * KVC_ERR_CUDA if the synchronisation itself failed.
  */
 KVC_API kvc_status kvc_poll_error(kvc_stream_t stream);
+
+/*
+ * kvc_checks_enabled -- 1 for the range-checking build (libkvc_checks.so, compiled with
+ * KVC_CHECKS=1), 0 for the regular one.  Host only.
+ */
+KVC_API int32_t kvc_checks_enabled(void);
 
 /*
  * kvc_launch_count -- number of CUDA kernels this library has launched in this process

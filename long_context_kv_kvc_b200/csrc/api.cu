@@ -367,10 +367,10 @@ ScoreJob shard_job(const kvc_params* p, const ShardPlan& P, const void* q, const
     job.N = n_local;
     job.key_off = key_offset;
     job.n_total = p->N;
+    job.err = device_error_word();
     if (P.use_tc) {
         job.tc_ws = ws;
         job.tc_ws_bytes = P.total;
-        job.err = device_error_word();
         return job;
     }
     job.partial = (float2*)(ws + P.off_partial);
@@ -397,8 +397,8 @@ kvc_status kvc_shard_stats(const kvc_params* p, const void* q, const void* k_loc
     const ShardPlan P = shard_plan(p, n_local);
     if (ws_bytes < P.total) return KVC_ERR_WORKSPACE;
     const ScoreJob job = shard_job(p, P, q, k_local, n_local, key_offset, (char*)ws);
+    if (!job.err) return KVC_ERR_CUDA;
     if (P.use_tc) {
-        if (!job.err) return KVC_ERR_CUDA;
         KVC_CUDA(kvc::tc_shard_stats(job, (float2*)ml, (cudaStream_t)stream));
     } else {
         KVC_CUDA(kvc::simt_shard_stats(job, (float2*)ml, (cudaStream_t)stream));
@@ -418,8 +418,8 @@ kvc_status kvc_shard_scores(const kvc_params* p, const void* q, const void* k_lo
     if (ws_bytes < P.total) return KVC_ERR_WORKSPACE;
     ScoreJob job = shard_job(p, P, q, k_local, n_local, key_offset, (char*)ws);
     job.unit_scores = scores;
+    if (!job.err) return KVC_ERR_CUDA;
     if (P.use_tc) {
-        if (!job.err) return KVC_ERR_CUDA;
         KVC_CUDA(kvc::tc_shard_scores(job, (const float2*)ml_all, n_shards, (cudaStream_t)stream));
     } else {
         KVC_CUDA(kvc::simt_shard_scores(job, (const float2*)ml_all, n_shards, (cudaStream_t)stream));
@@ -618,8 +618,11 @@ kvc_status kvc_poll_error(kvc_stream_t stream) {
     }
     if (h & kErrTimeout) return KVC_ERR_TIMEOUT;
     if (h & kErrIndex) return KVC_ERR_INDEX;
+    if (h & kErrCheck) return KVC_ERR_CHECK;
     return KVC_OK;
 }
+
+int32_t kvc_checks_enabled(void) { return kChecks ? 1 : 0; }
 
 const char* kvc_status_string(kvc_status st) {
     switch (st) {
@@ -632,6 +635,7 @@ const char* kvc_status_string(kvc_status st) {
         case KVC_ERR_CUDA: return "CUDA runtime error";
         case KVC_ERR_TIMEOUT: return "a device-side bounded wait gave up";
         case KVC_ERR_INDEX: return "gather index out of range";
+        case KVC_ERR_CHECK: return "a device-side range check failed (checks build)";
     }
     return "unknown status";
 }

@@ -102,7 +102,7 @@ __device__ __forceinline__ void from_f8(const float (&x)[8], uint4 (&r)[2]) {
 // forms a 2 x 2 block of A-B dot products.
 __global__ void __launch_bounds__(kMatchThreads)
 csm_match_f32_kernel(const float* __restrict__ k, int N, long long ld, int S, int w, int chunk, int n_chunks,
-                     int n_a_row, float* __restrict__ score, int32_t* __restrict__ best) {
+                     int n_a_row, float* __restrict__ score, int32_t* __restrict__ best, unsigned* err) {
     extern __shared__ __align__(16) float ks[];  // [chunk][kKS]
     __shared__ float inv_norm[128];
     __shared__ float sim[64][65];                // [A index][B index]
@@ -115,6 +115,9 @@ csm_match_f32_kernel(const float* __restrict__ k, int N, long long ld, int S, in
     int32_t* br = best + (size_t)row * N;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int kW = kMatchThreads / 32;
+    // a non-empty chunk of at most 128 tokens (64 A x 64 B similarities) whose A tokens fit the
+    // row's score entries
+    if (!dcheck(err, len >= 1 && len <= chunk && chunk <= 128 && (c0 - S) / 2 + (len + 1) / 2 <= n_a_row)) return;
 
     for (int e = threadIdx.x; e < len * (D / 4); e += kMatchThreads) {
         const int t = e / (D / 4), d = (e - t * (D / 4)) * 4;
@@ -262,6 +265,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) csm_match_tc_kernel(const __gri
                 const int g = cta + i * P;
                 const int u = g / a.tiles_per_row, tau = g - u * a.tiles_per_row;
                 const int s = i % kTcStages;
+                // the tile starts inside the row's candidates and holds whole chunks
+                if (!dcheck(a.err, tau >= 0 && a.S + tau * a.tt < a.N - a.w && a.tt <= kTileTok &&
+                                       a.tt % a.chunk == 0)) {
+                    *abort = 1;
+                    break;
+                }
                 mbar_wait(&sm.empty[s], ((i / kTcStages) & 1) ^ 1, abort, a.err);
                 if (*abort) break;
                 mbar_expect_tx(&sm.full[s], 2 * kHalfBytes);
@@ -375,7 +384,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) csm_match_tc_kernel(const __gri
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.accempty[grp]);
-            if (is_a) {  // A token (t0 + r - S) / 2 of the row (tiles start at even offsets)
+            if (is_a && dcheck(a.err, (t0 + r - a.S) / 2 < a.n_a_row && t0 + r < a.N - a.w)) {
+                // A token (t0 + r - S) / 2 of the row (tiles start at even offsets)
                 a.score[(size_t)u * a.n_a_row + (t0 + r - a.S) / 2] = bb >= 0 ? bs : -INFINITY;
                 a.best[(size_t)u * a.N + t0 + r] = bb >= 0 ? t0 + bb : -1;
             }
@@ -407,6 +417,7 @@ __global__ void csm_mark_kernel(const int32_t* __restrict__ sel, int rows, int N
             atomicOr(err, kErrIndex);
             continue;
         }
+        if (!dcheck(err, (p - S) / chunk < n_chunks)) continue;  // the owner chunk of token p
         merged[row * N + p] = 1;
         atomicAdd(&cb[row * (n_chunks + 1) + (p - S) / chunk], 1);
     }
@@ -416,7 +427,7 @@ __global__ void csm_mark_kernel(const int32_t* __restrict__ sel, int rows, int N
 // chunk c (sinks included); cb[n_chunks] becomes the number before the window.  Each thread
 // owns a contiguous run of chunks.
 __global__ void __launch_bounds__(kScanThreads)
-csm_base_kernel(int N, int S, int w, int chunk, int n_chunks, int32_t* __restrict__ cb) {
+csm_base_kernel(int N, int S, int w, int chunk, int n_chunks, int m, int32_t* __restrict__ cb, unsigned* err) {
     __shared__ int warp_tot[kScanThreads / 32];
     int32_t* c = cb + (size_t)blockIdx.x * (n_chunks + 1);
     const int per = (n_chunks + kScanThreads - 1) / kScanThreads;
@@ -440,7 +451,10 @@ csm_base_kernel(int N, int S, int w, int chunk, int n_chunks, int32_t* __restric
         c[q] = o;
         o += kept;
     }
-    if (threadIdx.x == kScanThreads - 1) c[n_chunks] = o;  // the last thread ends at the total
+    if (threadIdx.x == kScanThreads - 1) {
+        c[n_chunks] = o;  // the last thread ends at the total
+        dcheck(err, o == N - w - m);  // exactly m tokens of the row were marked merged
+    }
 }
 
 // ------------------------------------------------------------------------ write
@@ -505,6 +519,9 @@ csm_write_kernel(const T* __restrict__ k, const T* __restrict__ v, const int32_t
     T* sk = reinterpret_cast<T*>(wsm);
     T* sv = sk + (size_t)n * D;
 
+    // the block is a non-empty slice of the row that fits the shared arrays, and its first
+    // output slot lies inside the output row (the slots it writes are checked one by one)
+    if (!dcheck(err, n >= 1 && n <= 128 && p0 >= 0 && p0 + n <= N && o0 >= 0 && o0 < n_out)) return;
     if (tid == 0) {
         failed = 0;
         mbar_init(&bar, 1);
@@ -546,9 +563,10 @@ csm_write_kernel(const T* __restrict__ k, const T* __restrict__ v, const int32_t
                 for (uint32_t mm = amask[tid >> 1][wd]; mm; mm &= mm - 1u) nsum += dg[2 * (32 * wd + __ffs(mm) - 1)];
         }
         ns[tid] = nsum;
-        const size_t o = (size_t)row * ld_out + slot_of(tid);
-        deg_out[o] = nsum;
-        pos_out[o] = pos ? pos[rI + p0 + tid] : p0 + tid;
+        const int so = slot_of(tid);
+        const size_t o = (size_t)row * ld_out + so;
+        if (dcheck(err, so >= o0 && so < n_out)) deg_out[o] = nsum;
+        if (dcheck(err, so >= o0 && so < n_out)) pos_out[o] = pos ? pos[rI + p0 + tid] : p0 + tid;
     }
     // the rows have landed (bounded wait; a copy that never lands is reported, not used)
     if (!mbar_try_wait(&bar, 0)) {
@@ -608,13 +626,17 @@ csm_write_kernel(const T* __restrict__ k, const T* __restrict__ v, const int32_t
                 break;
             }
         }
-        const size_t o = (size_t)row * ld_out + slot_of(tid);
+        const int so = slot_of(tid);
+        const size_t o = (size_t)row * ld_out + so;
         const uint32_t bytes = (uint32_t)(e - tid) * D * sizeof(T);
-        bulk_store(k_out + o * D, sk + (size_t)tid * D, bytes);
-        bulk_store(v_out + o * D, sv + (size_t)tid * D, bytes);
-        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-        // shared memory stays valid until the stores have read it
-        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+        // the run's rows land inside the output row
+        if (dcheck(err, so >= o0 && so + (e - tid) <= n_out)) {
+            bulk_store(k_out + o * D, sk + (size_t)tid * D, bytes);
+            bulk_store(v_out + o * D, sv + (size_t)tid * D, bytes);
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            // shared memory stays valid until the stores have read it
+            asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+        }
     }
 }
 
@@ -701,7 +723,7 @@ cudaError_t match_f32(const float* k, int rows, int N, long long ld, int S, int 
     const long long grid = (long long)rows * n_chunks;
     if (grid > (1LL << 31) - 1) return cudaErrorInvalidValue;
     csm_match_f32_kernel<<<(unsigned)grid, kMatchThreads, (size_t)chunk * kKS * sizeof(float), s>>>(
-        k, N, ld, S, w, chunk, n_chunks, n_a_row, score, best);
+        k, N, ld, S, w, chunk, n_chunks, n_a_row, score, best, device_error_word());
     count_launches(1);
     return cudaGetLastError();
 }
@@ -746,7 +768,7 @@ cudaError_t csm(const void* k, const void* v, int dtype, const int32_t* deg, con
         count_launches(1);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    csm_base_kernel<<<rows, kScanThreads, 0, s>>>(N, S, w, chunk, n_chunks, cb);
+    csm_base_kernel<<<rows, kScanThreads, 0, s>>>(N, S, w, chunk, n_chunks, m, cb, err);
     count_launches(1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int n_blk = n_chunks + (S + kSeg - 1) / kSeg + (w + kSeg - 1) / kSeg;

@@ -94,6 +94,8 @@ decode_attn_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
     if (gw >= (long long)U * splits) return;
     const int u = (int)(gw / splits), sp = (int)(gw - (long long)u * splits);
     const int t_beg = sp * span, t_end = min(n, t_beg + span);
+    // the split's rows lie inside the unit's cache rows
+    if (!dcheck(err, t_beg >= 0 && n <= ld)) return;
     const T* k_row0 = k + (size_t)u * ld * D;
     const T* v_row0 = v + (size_t)u * ld * D;
     const T* kr = k_row0 + 4 * lane;
@@ -342,6 +344,11 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
                 const long long g = g0 + i;
                 const int u = (int)(g / a.T_u), tau = (int)(g - (long long)u * a.T_u);
                 const int s = i % kDtStages;
+                // the tile starts inside the unit's cached rows
+                if (!dcheck(a.err, u >= 0 && u < a.U && tau >= 0 && (long long)tau * kDtTile < a.n && a.n <= a.ld)) {
+                    *abort = 1;
+                    break;
+                }
                 mbar_wait(&sm.empty[s], ((i / kDtStages) & 1) ^ 1, abort, a.err);
                 if (*abort) break;
                 mbar_expect_tx(&sm.full[s], 4 * kDtHalf + 2 * kDtQHalf);
@@ -401,6 +408,8 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
             }
         };
         auto flush = [&](int u) {
+            // partial slots: (P + U) * kDtEpiWarps, CTA c's k-th unit boundary at c + k
+            if (!dcheck(a.err, u >= 0 && c + u < P + a.U)) return;
             const size_t slot = ((size_t)(c + u)) * kDtEpiWarps + wi;
             float mm = -INFINITY, ll = 0.f;
 #pragma unroll
@@ -656,12 +665,13 @@ template <typename T>
 __global__ void __launch_bounds__(256)
 append_kernel(T* __restrict__ k_cache, T* __restrict__ v_cache, int32_t* __restrict__ deg_cache,
               int32_t* __restrict__ pos_cache, int U, long long ld, int n, const T* __restrict__ k_new,
-              const T* __restrict__ v_new, int t_new, int pos0) {
+              const T* __restrict__ v_new, int t_new, int pos0, unsigned* err) {
     constexpr int kPieces = D * (int)sizeof(T) / 16;  // 16-byte pieces per row
     const int lane = threadIdx.x & 31;
     const long long gw = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
     if (gw >= (long long)U * t_new) return;
     const int u = (int)(gw / t_new), i = (int)(gw - (long long)u * t_new);
+    if (!dcheck(err, n + i < ld)) return;  // the new row fits the unit's cache rows
     const size_t src = ((size_t)u * t_new + i) * D, dst = ((size_t)u * ld + n + i) * D;
     for (int c = lane; c < 2 * kPieces; c += 32) {
         const bool isv = c >= kPieces;
@@ -794,11 +804,11 @@ cudaError_t append_rows(void* k_cache, void* v_cache, int32_t* deg_cache, int32_
     if (dtype == KVC_BF16)
         append_kernel<__nv_bfloat16><<<(unsigned)grid, 256, 0, s>>>(
             (__nv_bfloat16*)k_cache, (__nv_bfloat16*)v_cache, deg_cache, pos_cache, U, ld, n,
-            (const __nv_bfloat16*)k_new, (const __nv_bfloat16*)v_new, t_new, pos0);
+            (const __nv_bfloat16*)k_new, (const __nv_bfloat16*)v_new, t_new, pos0, device_error_word());
     else
         append_kernel<float><<<(unsigned)grid, 256, 0, s>>>((float*)k_cache, (float*)v_cache, deg_cache, pos_cache, U,
                                                             ld, n, (const float*)k_new, (const float*)v_new, t_new,
-                                                            pos0);
+                                                            pos0, device_error_word());
     count_launches(1);
     return cudaGetLastError();
 }

@@ -29,6 +29,7 @@ gather_kernel(const uint4* __restrict__ src0, uint4* __restrict__ dst0,
         uint4 a = make_uint4(0, 0, 0, 0), c = make_uint4(0, 0, 0, 0);
         if ((unsigned)j < (unsigned)N) {
             const long long s = (bh * N + j) * cpr + piece;
+            if (!dcheck_idx(err, s, total / K * N)) continue;  // B * Hsrc * N rows of cpr pieces
             a = __ldcs(src0 + s);
             if (src1) c = __ldcs(src1 + s);
         } else if (piece == 0) {

@@ -14,6 +14,32 @@ constexpr int kHeadDim = 128;  // D: the only head dimension the kernels are bui
 // bits of the per-device error word (see kvc_poll_error)
 constexpr unsigned kErrTimeout = 1u;
 constexpr unsigned kErrIndex = 2u;
+constexpr unsigned kErrCheck = 4u;  // a device-side range check failed (checks build only)
+
+// Device-side range checks.  Built with -DKVC_CHECKS=1 (libkvc_checks.so), every kernel tests
+// the indices and coordinates it forms against the extents of the buffers they address; a
+// failed test sets kErrCheck in the error word and the access is skipped.  In the regular
+// build dcheck is the constant true and the tests compile away.
+#if defined(KVC_CHECKS) && KVC_CHECKS
+constexpr bool kChecks = true;
+#else
+constexpr bool kChecks = false;
+#endif
+
+__device__ __forceinline__ bool dcheck(unsigned* err, bool ok) {
+    if constexpr (kChecks) {
+        if (!ok) {
+            if (err) atomicOr(err, kErrCheck);
+            return false;
+        }
+    }
+    return true;
+}
+
+// index i in [0, n)
+__device__ __forceinline__ bool dcheck_idx(unsigned* err, long long i, long long n) {
+    return dcheck(err, i >= 0 && i < n);
+}
 
 // counts kernel launches issued by the library (kvc_launch_count)
 void count_launches(int n);

@@ -69,11 +69,13 @@ __device__ __forceinline__ void merge_stats3(float& m, float& l, float& t, float
 template <typename T, bool ENT>
 __global__ void __launch_bounds__(kThreads)
 stats_kernel(const T* __restrict__ q, const T* __restrict__ k, int N, int key_off, int n_total, int w, int nq,
-             int chunk, int n_chunks, float2* __restrict__ partial, float* __restrict__ partial_t) {
+             int chunk, int n_chunks, float2* __restrict__ partial, float* __restrict__ partial_t, unsigned* err) {
     __shared__ float Qs[kQB][D + 1];
     __shared__ float Ks[kKT][D + 1];
     const int u = blockIdx.y, c = blockIdx.x;
     const int j0 = c * chunk, j1 = min(N, j0 + chunk);
+    // the chunk is a non-empty slice of the unit's keys and a column of the partials
+    if (!dcheck(err, j0 < j1 && c < n_chunks)) return;
     const T* qu = q + (size_t)u * nq * D;
     const T* ku = k + (size_t)u * N * D;
     const int tid = threadIdx.x, qi = tid >> 3, kj = tid & 7;
@@ -200,7 +202,7 @@ __global__ void shard_lse_kernel(const float2* __restrict__ ml_all, int W, int r
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 scores_kernel(const T* __restrict__ q, const T* __restrict__ k, int N, int key_off, int n_total, int w, int nq,
-              int chunk, const float* __restrict__ lse, float* __restrict__ out) {
+              int chunk, const float* __restrict__ lse, float* __restrict__ out, unsigned* err) {
     __shared__ float Qs[kQB][D + 1];
     __shared__ float Ks[kKT][D + 1];
     __shared__ float Ls[kQB];
@@ -211,6 +213,8 @@ scores_kernel(const T* __restrict__ q, const T* __restrict__ k, int N, int key_o
     const T* qu = q + (size_t)u * nq * D;
     const T* ku = k + (size_t)u * N * D;
     const int tid = threadIdx.x, qi = tid >> 3, kj = tid & 7, warp = tid >> 5, lane = tid & 31;
+    // the chunk's sums fit the shared accumulator
+    if (!dcheck(err, j0 < j1 && j1 - j0 <= kChunkMax)) return;
 
     for (int j = tid; j < j1 - j0; j += kThreads) sacc[j] = 0.f;
     for (int qb = 0; qb < nq; qb += kQB) {
@@ -287,20 +291,20 @@ cudaError_t launch_stats(const ScoreJob& j, cudaStream_t s) {
         if (ent)
             stats_kernel<float, true><<<grid, kThreads, 0, s>>>((const float*)j.q, (const float*)j.k, j.N, j.key_off,
                                                                  n_total, j.window, j.nq, j.chunk, j.n_chunks,
-                                                                 j.partial, partial_t);
+                                                                 j.partial, partial_t, j.err);
         else
             stats_kernel<float, false><<<grid, kThreads, 0, s>>>((const float*)j.q, (const float*)j.k, j.N,
                                                                   j.key_off, n_total, j.window, j.nq, j.chunk,
-                                                                  j.n_chunks, j.partial, partial_t);
+                                                                  j.n_chunks, j.partial, partial_t, j.err);
     } else {
         if (ent)
             stats_kernel<__nv_bfloat16, true><<<grid, kThreads, 0, s>>>(
                 (const __nv_bfloat16*)j.q, (const __nv_bfloat16*)j.k, j.N, j.key_off, n_total, j.window, j.nq,
-                j.chunk, j.n_chunks, j.partial, partial_t);
+                j.chunk, j.n_chunks, j.partial, partial_t, j.err);
         else
             stats_kernel<__nv_bfloat16, false><<<grid, kThreads, 0, s>>>(
                 (const __nv_bfloat16*)j.q, (const __nv_bfloat16*)j.k, j.N, j.key_off, n_total, j.window, j.nq,
-                j.chunk, j.n_chunks, j.partial, partial_t);
+                j.chunk, j.n_chunks, j.partial, partial_t, j.err);
     }
     return cudaGetLastError();
 }
@@ -310,11 +314,11 @@ cudaError_t launch_scores(const ScoreJob& j, cudaStream_t s) {
     const int n_total = j.n_total > 0 ? j.n_total : j.N;
     if (j.dtype == KVC_F32) {
         scores_kernel<float><<<grid, kThreads, 0, s>>>((const float*)j.q, (const float*)j.k, j.N, j.key_off, n_total,
-                                                        j.window, j.nq, j.chunk, j.lse, j.unit_scores);
+                                                        j.window, j.nq, j.chunk, j.lse, j.unit_scores, j.err);
     } else {
         scores_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(
             (const __nv_bfloat16*)j.q, (const __nv_bfloat16*)j.k, j.N, j.key_off, n_total, j.window, j.nq, j.chunk,
-            j.lse, j.unit_scores);
+            j.lse, j.unit_scores, j.err);
     }
     return cudaGetLastError();
 }

@@ -389,6 +389,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             int qunit = -1, ord = -1, i = 0;
             for (; i < n_local && !*abort; ++i) {
                 const int u = seq.unit(i), ti = seq.tile(i);
+                // the tile's coordinates address the unit's keys (and its Q block)
+                if (!dcheck(a.err, u >= 0 && u < a.U && ti >= 0 && (long long)ti * kTileKeys < a.N)) {
+                    *abort = 1;
+                    break;
+                }
                 // phase 1 stays at most max_lead tiles ahead of phase 2 (L2 footprint);
                 // phase 2 never loads a tile before phase 1 has (so its read hits L2)
                 const bool lead_rule = ph == 1 || MODE == kFull;
@@ -565,7 +570,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
 #pragma unroll
                 for (int rr = 0; rr < 4; ++rr) {
                     const int r = lane + 32 * rr;
-                    const float lse = r < a.nq ? __ldg(a.lse_in + (size_t)u * kQRows + r) : INFINITY;
+                    const float lse = r < a.nq && dcheck_idx(a.err, u, a.U)
+                                          ? __ldg(a.lse_in + (size_t)u * kQRows + r) : INFINITY;
                     sm.nlse[slot][r] = -lse;
                 }
                 __syncwarp();
@@ -605,7 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
 #pragma unroll
                 for (int rr = 0; rr < 4; ++rr) {
                     const int r = lane + 32 * rr;
-                    if (r < a.nq && tot[rr] > 0.0)
+                    if (r < a.nq && tot[rr] > 0.0 && dcheck_idx(a.err, u, a.U))
                         a.entropy[(size_t)u * a.nq + r] =
                             (float)(0.69314718055994531 * ((double)log2_pos(tot[rr]) - tott[rr] / tot[rr]));
                 }
@@ -624,7 +630,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                         const double f = __longlong_as_double((b & ~(0x7FFLL << 52)) | (1023LL << 52));
                         ml = make_float2(__ldg(a.ref + (size_t)u * kQRows + r) + (float)e, (float)f);
                     }
-                    a.ml_out[(size_t)u * a.nq + r] = ml;
+                    if (dcheck_idx(a.err, u, a.U)) a.ml_out[(size_t)u * a.nq + r] = ml;
                 }
                 continue;
             }
@@ -801,7 +807,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                     }
                     sc += prob_sum(x, nlse + c * 32);
                 }
-                if (j < a.N) a.unit_scores[(size_t)u * a.N + j] = sc;
+                if (j < a.N && dcheck_idx(a.err, u, a.U)) a.unit_scores[(size_t)u * a.N + j] = sc;
                 __syncwarp();
                 if (lane == 0) atomicAdd(&sm.lse_done[jb.w], 1u);
             }
@@ -823,7 +829,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
 __global__ void tc_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                                __nv_bfloat16* __restrict__ qpad, float* __restrict__ ref, double* __restrict__ sum,
                                unsigned* __restrict__ flags, int n_flags, int U, int N, int w, int nq, int mode,
-                               int key_off, int n_total) {
+                               int key_off, int n_total, unsigned* err) {
     const long long total = (long long)U * kQRows * (kHeadDim / 8);  // 16-byte pieces
     for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
          e += (long long)gridDim.x * blockDim.x) {
@@ -849,7 +855,7 @@ __global__ void tc_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_b
         const int kj = mode == kFull ? N - w + r % w : 0;
         const bool has_ref = r < nq && (mode == kFull || (mode == kStats && key_off <= n_total - w + r % w));
         float x = 0.f;
-        if (has_ref) {
+        if (has_ref && dcheck(err, kj >= 0 && kj < N)) {
             const uint2 qv = *reinterpret_cast<const uint2*>(q + (u * nq + r) * kHeadDim + 4 * lane);
             const uint2 kv = *reinterpret_cast<const uint2*>(k + (u * N + kj) * kHeadDim + 4 * lane);
             const __nv_bfloat162* qh = reinterpret_cast<const __nv_bfloat162*>(&qv);
@@ -1059,7 +1065,7 @@ cudaError_t tc_launch(const ScoreJob& j, int mode, float2* ml_out, cudaStream_t 
     const int prep_grid = (int)std::min<long long>((pieces + 255) / 256, 148LL * 8);
     tc_prep_kernel<<<prep_grid, 256, 0, s>>>((const __nv_bfloat16*)j.q, (const __nv_bfloat16*)j.k, qpad,
                                              (float*)(ws + L.ref), (double*)(ws + L.sum), flags, (int)L.n_flags,
-                                             j.U, j.N, j.window, j.nq, mode, a.key_off, a.n_total);
+                                             j.U, j.N, j.window, j.nq, mode, a.key_off, a.n_total, j.err);
     count_launches(1);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -29,7 +29,8 @@ namespace {
 // ------------------------------------------------------------------------------- sums
 
 __global__ void reduce_units_kernel(const float* __restrict__ units, int L, int B, int Hkv, int N,
-                                    int all_heads, float* __restrict__ out) {
+                                    int all_heads, float* __restrict__ out, unsigned* err) {
+    const long long n_units = (long long)L * B * Hkv * N;
     const int Hs = all_heads ? 1 : Hkv;
     const long long total = (long long)B * Hs * N;
     for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
@@ -41,14 +42,18 @@ __global__ void reduce_units_kernel(const float* __restrict__ units, int L, int 
         const int h0 = all_heads ? 0 : hs, h1 = all_heads ? Hkv : hs + 1;
         float s = 0.f;
         for (int l = 0; l < L; ++l)
-            for (int h = h0; h < h1; ++h) s += units[(((size_t)l * B + b) * Hkv + h) * N + j];
+            for (int h = h0; h < h1; ++h) {
+                const long long i = (((long long)l * B + b) * Hkv + h) * N + j;
+                if (dcheck_idx(err, i, n_units)) s += units[i];
+            }
         out[e] = s;
     }
 }
 
 __global__ void accumulate_kernel(float* __restrict__ acc, const float* __restrict__ src, int B,
-                                  int Hi, int Ho, int N) {
+                                  int Hi, int Ho, int N, unsigned* err) {
     const int R = Hi / Ho;
+    const long long n_src = (long long)B * Hi * N;
     const long long total = (long long)B * Ho * N;
     for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
          e += (long long)gridDim.x * blockDim.x) {
@@ -57,7 +62,10 @@ __global__ void accumulate_kernel(float* __restrict__ acc, const float* __restri
         const int o = (int)(bo % Ho);
         const int b = (int)(bo / Ho);
         float s = acc[e];
-        for (int r = 0; r < R; ++r) s += src[((size_t)b * Hi + o * R + r) * N + j];
+        for (int r = 0; r < R; ++r) {
+            const long long i = ((long long)b * Hi + o * R + r) * N + j;
+            if (dcheck_idx(err, i, n_src)) s += src[i];
+        }
         acc[e] = s;
     }
 }
@@ -65,7 +73,7 @@ __global__ void accumulate_kernel(float* __restrict__ acc, const float* __restri
 // ------------------------------------------------------------------------------- pool
 
 __global__ void pool_kernel(const float* __restrict__ in, float* __restrict__ out, int rows, int N,
-                            int lo, int hi, int radius) {
+                            int lo, int hi, int radius, unsigned* err) {
     const long long total = (long long)rows * N;
     for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
          e += (long long)gridDim.x * blockDim.x) {
@@ -76,6 +84,8 @@ __global__ void pool_kernel(const float* __restrict__ in, float* __restrict__ ou
             m = r[j];
         } else {
             const int t0 = max(lo, j - radius), t1 = min(hi - 1, j + radius);
+            // the clipped window stays inside the row's candidates
+            if (!dcheck(err, t0 >= 0 && t0 <= j && j <= t1 && t1 < N)) continue;
             m = r[t0];
             for (int t = t0 + 1; t <= t1; ++t) m = fmaxf(m, r[t]);
         }
@@ -103,7 +113,7 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 
 __global__ void __launch_bounds__(kTopkThreads)
 topk_kernel(const float* __restrict__ pooled, int N, int S, int w, int budget,
-            int32_t* __restrict__ idx) {
+            int32_t* __restrict__ idx, unsigned* err) {
     __shared__ unsigned hist[kWarps][256];
     __shared__ unsigned wsum[8];
     __shared__ uint32_t s_prefix;
@@ -120,8 +130,11 @@ topk_kernel(const float* __restrict__ pooled, int N, int S, int w, int budget,
     const int seg = (n_c + kWarps - 1) / kWarps;
     const int seg0 = lo + min(n_c, warp * seg), seg1 = lo + min(n_c, (warp + 1) * seg);
 
-    for (int i = tid; i < S; i += kTopkThreads) out[i] = i;
-    for (int i = tid; i < w; i += kTopkThreads) out[budget - w + i] = N - w + i;
+    // sinks fill [0, S), the window [budget - w, budget); the selected go between them
+    for (int i = tid; i < S; i += kTopkThreads)
+        if (dcheck(err, i < budget - w)) out[i] = i;
+    for (int i = tid; i < w; i += kTopkThreads)
+        if (dcheck(err, budget - w + i >= S)) out[budget - w + i] = N - w + i;
 
     if (tid == 0) {
         s_prefix = 0u;
@@ -204,10 +217,12 @@ topk_kernel(const float* __restrict__ pooled, int N, int S, int w, int budget,
         const bool take = gt || (eq && eq_seen + __popc(eq_mask & lanemask_lt()) < krem);
         const unsigned take_mask = __ballot_sync(0xffffffffu, take);
         const int pos = taken + __popc(take_mask & lanemask_lt());
-        if (take && pos < k_sel) out[S + pos] = j;  // pos < k_sel always holds; kept as a guard
+        if (take && dcheck(err, pos < k_sel && j >= lo && j < hi)) out[S + pos] = j;
         taken += __popc(take_mask);
         eq_seen += __popc(eq_mask);
     }
+    // the last warp's running count is the row's: exactly k_sel were written
+    if (warp == kWarps - 1 && lane == 0) dcheck(err, taken == k_sel);
 }
 
 // --------------------------------------------------------------- cluster top-k (fused pool)
@@ -237,7 +252,7 @@ struct TopkSmem {
 
 __global__ void __launch_bounds__(kCtThreads, 2) __cluster_dims__(kClusterCtas, 1, 1)
 topk_cluster_kernel(const float* __restrict__ scores, int N, int S, int w, int budget, int radius, int seg,
-                    int32_t* __restrict__ idx) {
+                    int32_t* __restrict__ idx, unsigned* err) {
     extern __shared__ uint8_t smem_raw[];
     TopkSmem& sm = *reinterpret_cast<TopkSmem*>(smem_raw);
     cg::cluster_group cluster = cg::this_cluster();
@@ -251,9 +266,13 @@ topk_cluster_kernel(const float* __restrict__ scores, int N, int S, int w, int b
     const int n_mine = s1 - s0;
 
     if (rank == 0) {
-        for (int i = tid; i < S; i += kCtThreads) out[i] = i;
-        for (int i = tid; i < w; i += kCtThreads) out[budget - w + i] = N - w + i;
+        for (int i = tid; i < S; i += kCtThreads)
+            if (dcheck(err, i < budget - w)) out[i] = i;
+        for (int i = tid; i < w; i += kCtThreads)
+            if (dcheck(err, budget - w + i >= S)) out[budget - w + i] = N - w + i;
     }
+    // this CTA's keys fit its shared memory
+    if (tid == 0) dcheck(err, n_mine <= seg && seg <= kSegMax);
     // pooled keys of this CTA's candidates (max over the clipped window of raw scores); the
     // first digit's histogram (the top 11 bits of every key) is counted as they are formed
     for (int i = tid; i < kBins; i += kCtThreads) sm.hist[i] = 0u;
@@ -261,10 +280,13 @@ topk_cluster_kernel(const float* __restrict__ scores, int N, int S, int w, int b
     for (int e = tid; e < n_mine; e += kCtThreads) {
         const int j = s0 + e;
         const int t0 = max(lo, j - radius), t1 = min(hi - 1, j + radius);
-        float m = __ldg(v + t0);
-        for (int t = t0 + 1; t <= t1; ++t) m = fmaxf(m, __ldg(v + t));
+        float m = 0.f;
+        if (dcheck(err, t0 >= 0 && t0 <= j && j <= t1 && t1 < N)) {
+            m = __ldg(v + t0);
+            for (int t = t0 + 1; t <= t1; ++t) m = fmaxf(m, __ldg(v + t));
+        }
         const uint32_t key = order_key(m);
-        sm.keys[e] = key;
+        if (dcheck(err, e < kSegMax)) sm.keys[e] = key;
         const unsigned digit = key >> 21;
         const unsigned peers = __match_any_sync(__activemask(), digit);
         if (lane == __ffs(peers) - 1) atomicAdd(&sm.hist[digit], (unsigned)__popc(peers));
@@ -404,10 +426,12 @@ topk_cluster_kernel(const float* __restrict__ scores, int N, int S, int w, int b
         const bool take = gt || (eq && eq_seen + __popc(eq_mask & lanemask_lt()) < krem);
         const unsigned take_mask = __ballot_sync(0xffffffffu, take);
         const int pos = taken + __popc(take_mask & lanemask_lt());
-        if (take && pos < k_sel) out[S + pos] = s0 + e;  // pos < k_sel always holds; kept as a guard
+        if (take && dcheck(err, pos < k_sel && s0 + e >= lo && s0 + e < hi)) out[S + pos] = s0 + e;
         taken += __popc(take_mask);
         eq_seen += __popc(eq_mask);
     }
+    // the last CTA's last warp ends at the row's count: exactly k_sel were written
+    if (rank == kClusterCtas - 1 && warp == kCtWarps - 1 && lane == 0) dcheck(err, taken == k_sel);
     cluster.sync();  // siblings may still read this CTA's counts until here
 }
 
@@ -491,7 +515,7 @@ constexpr int kHistBlocksPerRow = 16;
 // prefix[row]'s and whose next digit_bits are d.
 __global__ void __launch_bounds__(kHistThreads)
 select_hist_kernel(const float* __restrict__ v, int n, int lo, int hi, const uint32_t* __restrict__ prefix,
-                   int prefix_bits, int digit_bits, uint32_t* __restrict__ hist) {
+                   int prefix_bits, int digit_bits, uint32_t* __restrict__ hist, unsigned* err) {
     extern __shared__ uint32_t h[];
     const int row = blockIdx.y, nb = 1 << digit_bits;
     for (int i = threadIdx.x; i < nb; i += kHistThreads) h[i] = 0u;
@@ -502,9 +526,10 @@ select_hist_kernel(const float* __restrict__ v, int n, int lo, int hi, const uin
     const int span = (hi - lo + gridDim.x - 1) / gridDim.x;
     const int j0 = lo + blockIdx.x * span, j1 = min(hi, j0 + span);
     for (int j = j0 + threadIdx.x; j < j1; j += kHistThreads) {
+        if (!dcheck(err, j >= 0 && j < n)) continue;
         const uint32_t key = order_key(vr[j]);
         const bool match = prefix_bits == 0 || (key >> (32 - prefix_bits)) == (want >> (32 - prefix_bits));
-        if (match) atomicAdd(&h[(key >> shift) & (nb - 1)], 1u);
+        if (match && dcheck(err, shift >= 0 && shift + digit_bits <= 32)) atomicAdd(&h[(key >> shift) & (nb - 1)], 1u);
     }
     __syncthreads();
     for (int i = threadIdx.x; i < nb; i += kHistThreads)
@@ -532,8 +557,9 @@ select_emit_kernel(const float* __restrict__ v, int n, int lo, int hi, const uin
     __syncthreads();
     for (int j0 = lo; j0 < hi; j0 += kTopkThreads) {
         const int j = j0 + tid;
-        const uint32_t key = j < hi ? order_key(vr[j]) : 0u;
-        const bool gt = j < hi && key > T, eq = j < hi && key == T;
+        const bool in = j < hi && dcheck(err, j >= 0 && j < n);
+        const uint32_t key = in ? order_key(vr[j]) : 0u;
+        const bool gt = in && key > T, eq = in && key == T;
         const unsigned beq = __ballot_sync(0xffffffffu, eq);
         if (lane == 0) weq[warp] = __popc(beq);
         __syncthreads();
@@ -571,7 +597,8 @@ select_emit_kernel(const float* __restrict__ v, int n, int lo, int hi, const uin
 cudaError_t reduce_units(const float* units, int L, int B, int Hkv, int N, int all_heads, float* out,
                          cudaStream_t s) {
     const long long total = (long long)B * (all_heads ? 1 : Hkv) * N;
-    reduce_units_kernel<<<grid_for(total, 256), 256, 0, s>>>(units, L, B, Hkv, N, all_heads, out);
+    reduce_units_kernel<<<grid_for(total, 256), 256, 0, s>>>(units, L, B, Hkv, N, all_heads, out,
+                                                             device_error_word());
     count_launches(1);
     return cudaGetLastError();
 }
@@ -579,7 +606,7 @@ cudaError_t reduce_units(const float* units, int L, int B, int Hkv, int N, int a
 cudaError_t accumulate(float* acc, const float* src, int B, int Hi, int Ho, int N, cudaStream_t s) {
     const long long total = (long long)B * Ho * N;
     if (total == 0) return cudaSuccess;
-    accumulate_kernel<<<grid_for(total, 256), 256, 0, s>>>(acc, src, B, Hi, Ho, N);
+    accumulate_kernel<<<grid_for(total, 256), 256, 0, s>>>(acc, src, B, Hi, Ho, N, device_error_word());
     count_launches(1);
     return cudaGetLastError();
 }
@@ -588,7 +615,8 @@ cudaError_t pool(const float* in, float* out, int rows, int N, int lo, int hi, i
                  cudaStream_t s) {
     const long long total = (long long)rows * N;
     if (total == 0) return cudaSuccess;
-    pool_kernel<<<grid_for(total, 256), 256, 0, s>>>(in, out, rows, N, lo, hi, (kernel - 1) / 2);
+    pool_kernel<<<grid_for(total, 256), 256, 0, s>>>(in, out, rows, N, lo, hi, (kernel - 1) / 2,
+                                                     device_error_word());
     count_launches(1);
     return cudaGetLastError();
 }
@@ -615,7 +643,8 @@ cudaError_t topk_fused(const float* scores, int rows, int N, int n_sink, int win
         if (dev < 64) attr_done[dev].store(true);
     }
     topk_cluster_kernel<<<rows * kClusterCtas, kCtThreads, smem, s>>>(scores, N, n_sink, window, budget,
-                                                                     (kernel - 1) / 2, seg, idx);
+                                                                     (kernel - 1) / 2, seg, idx,
+                                                                     device_error_word());
     count_launches(1);
     return cudaGetLastError();
 }
@@ -623,7 +652,7 @@ cudaError_t topk_fused(const float* scores, int rows, int N, int n_sink, int win
 cudaError_t topk(const float* pooled, int rows, int N, int n_sink, int window, int budget,
                  int32_t* idx, cudaStream_t s) {
     if (rows == 0) return cudaSuccess;
-    topk_kernel<<<rows, kTopkThreads, 0, s>>>(pooled, N, n_sink, window, budget, idx);
+    topk_kernel<<<rows, kTopkThreads, 0, s>>>(pooled, N, n_sink, window, budget, idx, device_error_word());
     count_launches(1);
     return cudaGetLastError();
 }
@@ -642,7 +671,7 @@ namespace {
 // extended by the bucket, and this shard's count in that bucket.
 __global__ void select_pick_kernel(const uint32_t* __restrict__ hist, const uint32_t* __restrict__ hist_local,
                                    int rows, int digit_bits, int prefix_bits, int32_t* __restrict__ need,
-                                   uint32_t* __restrict__ prefix, int32_t* __restrict__ eq_local) {
+                                   uint32_t* __restrict__ prefix, int32_t* __restrict__ eq_local, unsigned* err) {
     const int lane = threadIdx.x & 31;
     const int row = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
     if (row >= rows) return;
@@ -677,6 +706,8 @@ __global__ void select_pick_kernel(const uint32_t* __restrict__ hist, const uint
             above += h[bb];
         }
         inside = want - above;
+        // the bucket holds the need-th largest: 1 <= inside <= its count
+        dcheck(err, hit != 0 && inside >= 1 && inside <= (long long)h[b]);
         need[row] = (int32_t)inside;
         prefix[row] |= (uint32_t)b << (32 - prefix_bits - digit_bits);
         eq_local[row] = (int32_t)hist_local[(size_t)row * nb + b];
@@ -713,7 +744,10 @@ __global__ void select_kept_kernel(const int32_t* __restrict__ sel, const int32_
     for (int e = threadIdx.x; e < cap; e += blockDim.x) {
         int gp = -1;
         if (e < n_s) gp = s_lo + e;
-        else if (e < n_s + n_sel) gp = sel[(size_t)row * cap_sel + (e - n_s)];
+        else if (e < n_s + n_sel) {
+            if (dcheck(err, e - n_s < cap_sel)) gp = sel[(size_t)row * cap_sel + (e - n_s)];
+            dcheck(err, gp >= max(S, key_off) && gp < min(N - w, key_off + n_local));
+        }
         else if (e < total) gp = w_lo + (e - n_s - n_sel);
         pos[(size_t)row * cap + e] = gp;
         local[(size_t)row * cap + e] = gp >= 0 ? gp - key_off : 0;
@@ -726,7 +760,7 @@ cudaError_t select_pick(const uint32_t* hist, const uint32_t* hist_local, int ro
                         int32_t* need, uint32_t* prefix, int32_t* eq_local, cudaStream_t s) {
     count_launches(1);
     select_pick_kernel<<<(rows + 7) / 8, 256, 0, s>>>(hist, hist_local, rows, digit_bits, prefix_bits, need, prefix,
-                                                      eq_local);
+                                                      eq_local, device_error_word());
     return cudaGetLastError();
 }
 
@@ -753,7 +787,7 @@ cudaError_t select_hist(const float* pooled, int rows, int n, int lo, int hi, co
     if (e != cudaSuccess || hi <= lo) return e;
     dim3 grid(kHistBlocksPerRow, rows);
     select_hist_kernel<<<grid, kHistThreads, nb * sizeof(uint32_t), s>>>(pooled, n, lo, hi, prefix, prefix_bits,
-                                                                          digit_bits, hist);
+                                                                          digit_bits, hist, device_error_word());
     count_launches(1);
     return cudaGetLastError();
 }

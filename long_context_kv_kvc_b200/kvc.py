@@ -2,7 +2,8 @@
 
 Argument marshalling only: every step of the compaction runs in the library's CUDA
 kernels.  PyTorch supplies device memory and the current stream.  Importing this module
-loads the in-tree libkvc.so and raises if it is missing; there is no fallback.
+loads the in-tree libkvc.so (with KVC_CHECKS=1 in the environment: the range-checking build
+libkvc_checks.so) and raises if it is missing; there is no fallback.
 """
 from __future__ import annotations
 
@@ -12,10 +13,11 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libkvc.so")
+CHECKS = os.environ.get("KVC_CHECKS", "0") == "1"
+LIB_PATH = os.path.join(_PKG, "libkvc_checks.so" if CHECKS else "libkvc.so")
 
 KVC_OK, KVC_ERR_ARG, KVC_ERR_UNSUPPORTED, KVC_ERR_BUDGET, KVC_ERR_ALIGN = 0, 1, 2, 3, 4
-KVC_ERR_WORKSPACE, KVC_ERR_CUDA, KVC_ERR_TIMEOUT, KVC_ERR_INDEX = 5, 6, 7, 8
+KVC_ERR_WORKSPACE, KVC_ERR_CUDA, KVC_ERR_TIMEOUT, KVC_ERR_INDEX, KVC_ERR_CHECK = 5, 6, 7, 8, 9
 KVC_F32, KVC_BF16 = 0, 1
 KVC_SCOPE_PER_KV_HEAD, KVC_SCOPE_ALL_HEADS = 0, 1
 KVC_FLAG_SIMT_SCORE = 1
@@ -28,7 +30,7 @@ EXPORTED = ("kvc_workspace_size", "kvc_score", "kvc_accumulate", "kvc_pool", "kv
             "kvc_row_stats", "kvc_csm_merges", "kvc_csm_ratio", "kvc_csm_workspace_size", "kvc_csm", "kvc_append",
             "kvc_decode_attention_workspace_size", "kvc_decode_attention", "kvc_shard_workspace_size",
             "kvc_shard_stats", "kvc_shard_scores", "kvc_select_hist", "kvc_select_emit", "kvc_select_pick",
-            "kvc_select_ties", "kvc_select_kept")
+            "kvc_select_ties", "kvc_select_kept", "kvc_checks_enabled")
 
 
 class KvcError(RuntimeError):
@@ -50,7 +52,8 @@ class Params(ctypes.Structure):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is not built; run `python -m long_context_kv_kvc_b200.build`")
+        raise ImportError(f"{LIB_PATH} is not built; run `python -m long_context_kv_kvc_b200.build"
+                          f"{' --checks' if CHECKS else ''}`")
     L = ctypes.CDLL(LIB_PATH)
     P, vp, i32, sz, st = ctypes.POINTER(Params), ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.c_int
     sig = {
@@ -86,6 +89,7 @@ def _load():
         "kvc_select_pick": (st, [vp, vp, i32, i32, i32, vp, vp, vp, vp]),
         "kvc_select_ties": (st, [vp, i32, i32, i32, vp, vp, vp]),
         "kvc_select_kept": (st, [vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp]),
+        "kvc_checks_enabled": (i32, []),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -381,6 +385,10 @@ def kvc_tsp_count(N, window, n_sink, rate) -> int:
 
 def kvc_poll_error(stream=None) -> int:
     return int(lib.kvc_poll_error(_stream(stream)))
+
+
+def kvc_checks_enabled() -> bool:
+    return bool(lib.kvc_checks_enabled())
 
 
 def kvc_status_string(st: int) -> str:

@@ -36,6 +36,23 @@ def test_exports_every_declared_symbol(K):
     assert set(names) == set(K.EXPORTED)
 
 
+def test_checks_build_exports_the_same_symbols_and_says_so(K):
+    """libkvc_checks.so (KVC_CHECKS=1) is the same ABI; kvc_checks_enabled tells the builds apart."""
+    from long_context_kv_kvc_b200 import build
+    path = build.build(checks=True)
+    out = subprocess.check_output(["nm", "-D", "--defined-only", path], text=True)
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert set(declared_symbols()) <= exported
+    for lib_path, want in ((path, 1), (build.LIB, 0)):
+        L = ctypes.CDLL(lib_path)
+        L.kvc_checks_enabled.restype = ctypes.c_int32
+        assert L.kvc_checks_enabled() == want
+    L = ctypes.CDLL(path)
+    L.kvc_status_string.restype = ctypes.c_char_p
+    L.kvc_status_string.argtypes = [ctypes.c_int]
+    assert b"range check" in L.kvc_status_string(K.KVC_ERR_CHECK)
+
+
 def test_params_layout_matches_c(K, tmp_path):
     fields = [f[0] for f in K.Params._fields_]
     src = tmp_path / "layout.c"
