@@ -118,10 +118,11 @@ def test_csm_odd_shapes(K, shape):
 @pytest.mark.parametrize("cuts", [(0, 129, 300, 513), (0, 1, 512, 513), (0, 256, 257, 513)],
                          ids=["ragged", "one_key_block", "one_key_middle"])
 def test_sharded_compress_odd_cuts(K, cuts):
-    """Sequence sharding over blocks of 1 to 512 keys (the ranks are host threads on one GPU)."""
+    """Sequence sharding over blocks of 1 to 512 keys (the ranks are host threads on one GPU);
+    a block must hold the pool's half-width (pool_kernel - 1) / 2 of keys, here 1."""
     from long_context_kv_kvc_b200.sharded import GpuOps, sharded_compress
     from test_gpu_sharded import run_ranks
-    wl = synth.scaled(synth.LLAMA8B_32K, B=1, Hq=8, Hkv=2, N=513, window=9, n_sink=2, pool_kernel=5, kv_budget=40,
+    wl = synth.scaled(synth.LLAMA8B_32K, B=1, Hq=8, Hkv=2, N=513, window=9, n_sink=2, pool_kernel=3, kv_budget=40,
                       n_hubs=8)
     inp = synth.make_inputs(wl, with_hidden=False)
     q, k, v = inp["q"][0].cuda(), inp["k"][0].cuda(), inp["v"].cuda()
