@@ -315,6 +315,26 @@ __device__ __forceinline__ void wait_pos(const int* pos, int want, volatile int*
     }
 }
 
+// The lead rule of the phase-1 producer for local tile i of unit u: wait while i is max_lead
+// or more tiles ahead of the phase-2 loads, unless u is the unit the phase-2 issuer is at (its
+// lse cannot be known before this tile's phase 1 is done).
+__device__ __forceinline__ void lead_wait(Smem& sm, int i, int u, int max_lead, int T_u, volatile int* abort,
+                                          unsigned* err) {
+    if (i - vload(sm.p2_issued) < max_lead) return;
+    const long long t0 = globaltimer();
+    while (i - vload(sm.p2_issued) >= max_lead) {
+        const int p = vload(sm.p2_pos);  // < i: its entry is published and still in the ring
+        if (*reinterpret_cast<const volatile int*>(&sm.seq[p % kSeqRing]) / T_u == u) return;
+        if (*abort) return;
+        if (globaltimer() - t0 > kBarrierTimeoutNs) {
+            atomicOr(err, kErrTimeout);
+            *abort = 1;
+            return;
+        }
+        __nanosleep(32);
+    }
+}
+
 // Largest of 32 logits.
 __device__ __forceinline__ float chunk_max(const uint32_t (&x)[32]) {
     float mx[8];
@@ -473,31 +493,21 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             const uint64_t evict_first = policy_evict_first();
             int qunit = -1, ord = -1, i = 0;
             // Warp 0 claims the CTA's tiles from the global counter (unit-major order), kClaim
-            // at a time, so that CTAs which run ahead take more tiles of a unit and all CTAs
-            // finish its phase 1 together.  A claim is made only when the lead rule below
-            // already admits all of its tiles (a CTA never holds an unprocessed tile while it
-            // waits for phase 2); the next claim is issued while the current one loads.  The
-            // other roles read the CTA's tiles from the ring it publishes.
-            int claim_base = 0, claim_used = kClaim, claim_next = -1;
+            // at a time with the next claim always in flight, so that CTAs which run ahead take
+            // more tiles of a unit and all CTAs finish its phase 1 together.  The other roles
+            // read the CTA's tiles from the ring it publishes.
+            int claim_base = 0, claim_used = kClaim, claim_next = 0;
+            if (ph == 0) claim_next = (int)atomicAdd(a.claim, (unsigned)kClaim);
             for (;; ++i) {
                 int u, ti;
                 if (ph == 0) {
                     if (claim_used == kClaim) {
-                        if (claim_next < 0) {
-                            // phase 1 stays less than max_lead tiles ahead of phase 2 (L2 footprint)
-                            if (MODE == kFull) wait_pos(&sm.p2_issued, i + kClaim - a.max_lead, abort, a.err);
-                            if (*abort) break;
-                            claim_next = (int)atomicAdd(a.claim, (unsigned)kClaim);
-                        }
                         claim_base = claim_next;
-                        claim_next = -1;
                         claim_used = 0;
+                        if (claim_base < a.total_tiles) claim_next = (int)atomicAdd(a.claim, (unsigned)kClaim);
                     }
                     const int g = claim_base + claim_used++;
                     if (g >= a.total_tiles || *abort) break;
-                    if (claim_used == 1 && claim_base + kClaim < a.total_tiles &&
-                        (MODE != kFull || i + 2 * kClaim - 1 - vload(sm.p2_issued) < a.max_lead))
-                        claim_next = (int)atomicAdd(a.claim, (unsigned)kClaim);
                     u = g / a.T_u;
                     ti = g - u * a.T_u;
                     // ring entry i is free once every reader has passed entry i - kSeqRing
@@ -508,6 +518,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                     sm.seq[i % kSeqRing] = g;
                     __threadfence_block();
                     *reinterpret_cast<volatile int*>(&sm.seq_pub) = i + 1;
+                    // Phase 1 stays less than max_lead tiles ahead of phase 2 (L2 footprint),
+                    // except for tiles of the unit whose lse the phase-2 issuer waits for: a
+                    // claimed tile of that unit must never wait on its own unit's completion.
+                    if (MODE == kFull) lead_wait(sm, i, u, a.max_lead, a.T_u, abort, a.err);
                 } else {
                     int2 e;
                     if (!seq_get(sm, i, a.T_u, e, abort, a.err)) break;
