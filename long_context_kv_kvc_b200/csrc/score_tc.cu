@@ -15,11 +15,8 @@
 // second read is scheduled to hit L2.  With 128 query rows per unit the work is two
 // exponentials per byte of K, which makes the special-function unit, not HBM, the
 // tightest resource; the kernel is therefore organised to keep every consumer warp fed:
-//   * one persistent CTA per SM (cooperative launch: all CTAs resident); the 128-key tiles,
-//     in global (unit-major) order, are claimed two at a time from a global counter, so a
-//     CTA that runs ahead takes more of a unit and all CTAs finish its phase 1 within about
-//     a tile of each other (a fixed deal left them up to a unit's time apart, and the whole
-//     GPU waited on the slowest for each unit's lse);
+//   * one persistent CTA per SM (cooperative launch: all CTAs resident), 128-key tiles
+//     dealt round-robin over the CTAs in global (unit-major) order;
 //   * phase 1 streams K from HBM: D[128 q x 128 keys] = Q K^T (tcgen05.mma kind::f16,
 //     M = N = 128, fp32 accumulator in TMEM); phase 2 re-reads each tile a bounded number
 //     of tiles later (so it comes from L2, loaded evict-first): D[128 keys x 128 q] = K Q^T;
@@ -30,19 +27,14 @@
 //     phase-1 work exists.  Accumulators are taken in job order and the phase-1 record ring
 //     is released through a monotonic counter: a parity wait on an mbarrier that may lag two
 //     phases behind its waiter would pass early;
-//   * a phase-1 job yields per query row the tile's sum of 2^(y - ref) relative to a fixed
-//     per-row reference ref (the row's logit with the key at its own position, computed
-//     before the kernel; a tile with a much larger logit reports its own max instead); a
-//     publisher warp turns each tile's sum into fp64, adds the CTA's run of tiles of a unit
-//     to the unit's fp64 total with fire-and-forget atomics and adds the run's length to
-//     the unit's tile count (a tile's part does not depend on which CTA took it; fp64
-//     addition order moves the total by ~1e-16, far below fp32);
-//   * an lse warp waits until a unit's count reaches its tile count, turns the totals into
-//     lse = ref + log2(total) in shared memory and releases the unit's phase-2 jobs; a
-//     phase-2 job gives each key of the tile its sum over the query rows of 2^(y - lse).
-//   * warp 0 publishes the CTA's claimed tiles in a shared ring (and each new unit with its
-//     first local tile), which the other roles follow; after the last job the issuers post
-//     an end job to every accumulator.
+//   * a phase-1 job yields per query row the tile's (max, sum of 2^(y - max)); a publisher
+//     warp merges them in tile order, rescales the CTA's sum to a fixed per-row reference
+//     (the row's logit with the key at its own position, computed before the kernel), adds
+//     it to the unit's fp64 total with a fire-and-forget atomic and bumps the unit's arrival
+//     count (fp64 addition order moves the total by ~1e-16, far below fp32);
+//   * an lse warp waits for each unit's count, turns the totals into lse = ref + log2(total)
+//     in shared memory and releases the unit's phase-2 jobs; a phase-2 job gives each key
+//     of the tile its sum over the query rows of 2^(y - lse).
 // Phase 1 streams each 128-key tile from HBM as one 32 KiB TMA op (both 64-column halves, the
 // 128-byte swizzle atom) into a 2-tile ring; phase 2 re-reads each tile as two 16 KiB halves,
 // issued by two threads, into a 3-stage ring (a single issuing thread completes TMA ops at a
@@ -93,14 +85,6 @@ constexpr int kConsumer0 = 8;          // first consumer warp
 #endif
 constexpr int kSumCopies = KVC_TC_SUM_COPIES;  // copies of each unit's totals (CTA c adds to copy c % kSumCopies)
 constexpr int kMaxCtas = 160;                          // upper bound on the persistent grid
-constexpr int kClaim = 2;        // tiles a CTA claims from the global counter at a time
-constexpr int kSeqRing = 256;    // the CTA's claimed tiles (unit, tile) between claim and last use
-constexpr int kOrdRing = 16;     // the CTA's units in claim order: (unit, first local tile)
-constexpr int kJobEnd = 2;       // job kind after the last job: the consumers stop
-// Phase 1 runs at most max_lead = ceil(T_u / P) + kLeadSlack tiles ahead of phase 2; the
-// rings above hold that many tiles with room to spare (units longer than about
-// kMaxLead * 148 tiles take the CUDA-core path).
-constexpr int kMaxLead = 192;
 constexpr uint32_t kTmemCols = 512;
 
 struct TcArgs {
@@ -116,7 +100,6 @@ struct TcArgs {
     float* entropy;      // [U][nq] attention entropy (nats) per window row, or null
     unsigned* count;     // [U] CTAs that have added their part of unit u
     unsigned* never;     // a counter nothing increments (wait-timeout injection)
-    unsigned* claim;     // tiles claimed so far (global order: unit-major), kClaim at a time
     unsigned* err;
     long long spin_limit;
     int U, N, w, nq, T_u, total_tiles, P, max_lead, inject;
@@ -148,19 +131,10 @@ struct __align__(1024) Smem {
     int next_job;          // job numbers claimed by the two MMA issuers
     int jobs_started;      // jobs that own their accumulator (taken in job order)
     int rec_consumed;      // phase-1 records the publisher has read (monotonic)
-    int seq[kSeqRing];     // local tile i: its global tile index in slot i % kSeqRing
-    int2 ord_info[kOrdRing];  // the CTA's o-th unit: (unit, first local tile) in slot o % kOrdRing
-    int seq_pub, ord_pub;  // entries published (monotonic)
-    int seq_fin;           // 1 once the CTA has claimed its last tile
-    int p2_pos;            // local tiles the phase-2 issuer is done with
-    int lse_ord;           // units the lse warp is done with
-    int issuers_done;
     uint32_t tmem_base;
     int abort;
     int p1_issued, p2_issued;  // tiles whose loads each producer has issued (L2 lead control)
 };
-
-static_assert(sizeof(Smem) + 1024 <= 227 * 1024, "shared memory of the score kernel");
 
 // Spinning bounded wait (no suspension) for the single-thread roles, which must react fast.
 __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
@@ -240,99 +214,6 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
     unsigned v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
-}
-
-__device__ __forceinline__ int vload(const int& x) { return *reinterpret_cast<const volatile int*>(&x); }
-
-// The CTA's claimed tiles.  Local tile i's (unit, tile within the unit of T_u tiles) once
-// warp 0 has published it; false once the sequence has ended before i (or on abort).
-__device__ __forceinline__ bool seq_get(Smem& sm, int i, int T_u, int2& e, volatile int* abort, unsigned* err) {
-    const long long t0 = globaltimer();
-    for (;;) {
-        if (vload(sm.seq_pub) > i) break;
-        if (vload(sm.seq_fin)) {
-            if (vload(sm.seq_pub) > i) break;
-            return false;
-        }
-        if (*abort) return false;
-        if (globaltimer() - t0 > kBarrierTimeoutNs) {
-            atomicOr(err, kErrTimeout);
-            *abort = 1;
-            return false;
-        }
-    }
-    const int g = *reinterpret_cast<const volatile int*>(&sm.seq[i % kSeqRing]);
-    e = make_int2(g / T_u, g % T_u);
-    return true;
-}
-
-// Local tile i's entry only if it is already published (no wait): 1 = published, 0 = the
-// sequence ended before i, -1 = not yet known.
-__device__ __forceinline__ int seq_peek(Smem& sm, int i, int T_u, int2& e) {
-    const int fin = vload(sm.seq_fin);  // read before the count: a set flag means the count is final
-    if (vload(sm.seq_pub) > i) {
-        const int g = *reinterpret_cast<const volatile int*>(&sm.seq[i % kSeqRing]);
-        e = make_int2(g / T_u, g % T_u);
-        return 1;
-    }
-    return fin ? 0 : -1;
-}
-
-// The CTA's o-th unit: (unit, first local tile); false once the sequence has ended without it.
-__device__ __forceinline__ bool ord_get(Smem& sm, int o, int2& e, volatile int* abort, unsigned* err) {
-    const long long t0 = globaltimer();
-    for (;;) {
-        if (vload(sm.ord_pub) > o) break;
-        if (vload(sm.seq_fin)) {
-            if (vload(sm.ord_pub) > o) break;
-            return false;
-        }
-        if (*abort) return false;
-        if (globaltimer() - t0 > kBarrierTimeoutNs) {
-            atomicOr(err, kErrTimeout);
-            *abort = 1;
-            return false;
-        }
-        __nanosleep(64);
-    }
-    const volatile int2* p = &sm.ord_info[o % kOrdRing];
-    e = make_int2(p->x, p->y);
-    return true;
-}
-
-// Bounded wait until `*pos >= want` (a reader's progress counter) or abort.
-__device__ __forceinline__ void wait_pos(const int* pos, int want, volatile int* abort, unsigned* err) {
-    if (vload(*pos) >= want) return;
-    const long long t0 = globaltimer();
-    while (vload(*pos) < want) {
-        if (*abort) return;
-        if (globaltimer() - t0 > kBarrierTimeoutNs) {
-            atomicOr(err, kErrTimeout);
-            *abort = 1;
-            return;
-        }
-        __nanosleep(32);
-    }
-}
-
-// The lead rule of the phase-1 producer for local tile i of unit u: wait while i is max_lead
-// or more tiles ahead of the phase-2 loads, unless u is the unit the phase-2 issuer is at (its
-// lse cannot be known before this tile's phase 1 is done).
-__device__ __forceinline__ void lead_wait(Smem& sm, int i, int u, int max_lead, int T_u, volatile int* abort,
-                                          unsigned* err) {
-    if (i - vload(sm.p2_issued) < max_lead) return;
-    const long long t0 = globaltimer();
-    while (i - vload(sm.p2_issued) >= max_lead) {
-        const int p = vload(sm.p2_pos);  // < i: its entry is published and still in the ring
-        if (*reinterpret_cast<const volatile int*>(&sm.seq[p % kSeqRing]) / T_u == u) return;
-        if (*abort) return;
-        if (globaltimer() - t0 > kBarrierTimeoutNs) {
-            atomicOr(err, kErrTimeout);
-            *abort = 1;
-            return;
-        }
-        __nanosleep(32);
-    }
 }
 
 // Largest of 32 logits.
@@ -420,12 +301,31 @@ __device__ __forceinline__ float prob_sum(const uint32_t (&x)[32], const float* 
 
 // ------------------------------------------------------------------------ the kernel
 
+// The CTA's local tiles i = 0, 1, ... are the global tiles cta + i * P; these helpers give
+// their unit and the local range of each unit.
+struct TileSeq {
+    int cta, P, T_u, n_local;
+    __device__ __forceinline__ int unit(int i) const { return (cta + i * P) / T_u; }
+    __device__ __forceinline__ int tile(int i) const { return cta + i * P - unit(i) * T_u; }
+    // first local tile whose global index is >= g
+    __device__ __forceinline__ int first_at(long long g) const {
+        const long long d = g - cta;
+        const long long i = d <= 0 ? 0 : (d + P - 1) / P;
+        return (int)(i < n_local ? i : n_local);
+    }
+    __device__ __forceinline__ int count(int u) const {
+        return first_at((long long)(u + 1) * T_u) - first_at((long long)u * T_u);
+    }
+};
+
 template <bool ENT, int MODE>
 __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_constant__ TcArgs a) {
     extern __shared__ uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int cta = blockIdx.x;
+    const int cta = blockIdx.x, P = a.P;
+    const int n_local = cta < a.total_tiles ? (a.total_tiles - cta + P - 1) / P : 0;
+    const TileSeq seq{cta, P, a.T_u, n_local};
     volatile int* abort = &sm.abort;
 
     if (threadIdx.x == 0) {
@@ -456,12 +356,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
         sm.next_job = 0;
         sm.jobs_started = 0;
         sm.rec_consumed = 0;
-        sm.seq_pub = 0;
-        sm.ord_pub = 0;
-        sm.seq_fin = 0;
-        sm.p2_pos = 0;
-        sm.lse_ord = 0;
-        sm.issuers_done = 0;
         sm.p1_issued = 0;
         sm.p2_issued = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -491,60 +385,35 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             const CUtensorMap* mk = ph == 0 ? &a.tmap_k4 : &a.tmap_k;
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(mk)) : "memory");
             const uint64_t evict_first = policy_evict_first();
+            volatile int* other = ph == 0 ? &sm.p2_issued : &sm.p1_issued;
             int qunit = -1, ord = -1, i = 0;
-            // Warp 0 claims the CTA's tiles from the global counter (unit-major order), kClaim
-            // at a time with the next claim always in flight, so that CTAs which run ahead take
-            // more tiles of a unit and all CTAs finish its phase 1 together.  The other roles
-            // read the CTA's tiles from the ring it publishes.
-            int claim_base = 0, claim_used = kClaim, claim_next = 0;
-            if (ph == 0) claim_next = (int)atomicAdd(a.claim, (unsigned)kClaim);
-            for (;; ++i) {
-                int u, ti;
-                if (ph == 0) {
-                    if (claim_used == kClaim) {
-                        claim_base = claim_next;
-                        claim_used = 0;
-                        if (claim_base < a.total_tiles) claim_next = (int)atomicAdd(a.claim, (unsigned)kClaim);
-                    }
-                    const int g = claim_base + claim_used++;
-                    if (g >= a.total_tiles || *abort) break;
-                    u = g / a.T_u;
-                    ti = g - u * a.T_u;
-                    // ring entry i is free once every reader has passed entry i - kSeqRing
-                    if (i >= kSeqRing) {
-                        if (MODE != kScores) wait_pos(&sm.rec_consumed, i - kSeqRing + 2, abort, a.err);
-                        if (MODE != kStats) wait_pos(&sm.p2_pos, i - kSeqRing + 2, abort, a.err);
-                    }
-                    sm.seq[i % kSeqRing] = g;
-                    __threadfence_block();
-                    *reinterpret_cast<volatile int*>(&sm.seq_pub) = i + 1;
-                    // Phase 1 stays less than max_lead tiles ahead of phase 2 (L2 footprint),
-                    // except for tiles of the unit whose lse the phase-2 issuer waits for: a
-                    // claimed tile of that unit must never wait on its own unit's completion.
-                    if (MODE == kFull) lead_wait(sm, i, u, a.max_lead, a.T_u, abort, a.err);
-                } else {
-                    int2 e;
-                    if (!seq_get(sm, i, a.T_u, e, abort, a.err)) break;
-                    u = e.x;
-                    ti = e.y;
-                    // phase 2 never loads a tile before phase 1 has (so its read hits L2)
-                    if (MODE == kFull) wait_pos(&sm.p1_issued, i + 1, abort, a.err);
-                }
+            for (; i < n_local && !*abort; ++i) {
+                const int u = seq.unit(i), ti = seq.tile(i);
                 // the tile's coordinates address the unit's keys (and its Q block)
                 if (!dcheck(a.err, u >= 0 && u < a.U && ti >= 0 && (long long)ti * kTileKeys < a.N)) {
                     *abort = 1;
                     break;
                 }
+                // phase 1 stays at most max_lead tiles ahead of phase 2 (L2 footprint);
+                // phase 2 never loads a tile before phase 1 has (so its read hits L2)
+                const bool lead_rule = ph == 1 || MODE == kFull;
+                if (lead_rule && (ph == 0 ? (i - *other >= a.max_lead) : (i >= *other))) {
+                    const long long t0 = globaltimer();
+                    while (ph == 0 ? (i - *other >= a.max_lead) : (i >= *other)) {
+                        if (*abort) break;
+                        if (globaltimer() - t0 > kBarrierTimeoutNs) {
+                            atomicOr(a.err, kErrTimeout);
+                            *abort = 1;
+                            break;
+                        }
+                        __nanosleep(32);
+                    }
+                }
                 if (ph == 0 && u != qunit) {
-                    // the CTA's ord-th unit: publish it for the lse warp, then load its Q into
-                    // slot ord % kQSlots once phase 2 is done with the unit that used the slot
-                    // kQSlots units ago
+                    // the CTA's ord-th unit: load its Q into slot ord % kQSlots once phase 2
+                    // is done with the unit that used the slot kQSlots units ago
                     qunit = u;
                     ++ord;
-                    if (ord >= kOrdRing) wait_pos(&sm.lse_ord, ord - kOrdRing + 1, abort, a.err);
-                    sm.ord_info[ord % kOrdRing] = make_int2(u, i);
-                    __threadfence_block();
-                    *reinterpret_cast<volatile int*>(&sm.ord_pub) = ord + 1;
                     const int slot = ord % kQSlots;
                     if (ord >= kQSlots) mbar_spin(&sm.qempty[slot], ((ord / kQSlots) - 1) & 1, abort, a.err);
                     mbar_expect_tx(&sm.qfull[slot], 2 * kBoxBytes);
@@ -564,11 +433,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                     tma_load_3d_hint(sm.ringB[st], mk, &sm.fullB[st], 64 * hh, ti * kTileKeys, u, evict_first);
                     if (hh == 0) *reinterpret_cast<volatile int*>(&sm.p2_issued) = i + 1;
                 }
-            }
-            if (ph == 0) {
-                // no more tiles for this CTA: the sequence ends at i
-                __threadfence_block();
-                *reinterpret_cast<volatile int*>(&sm.seq_fin) = 1;
             }
             if (*abort) {
                 // copies still in flight land before the CTA exits
@@ -597,22 +461,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             const uint64_t dK0 = sw128_desc(smem_u32(ph == 0 ? sm.ringA[0] : sm.ringB[0]));
             const uint64_t dQ0 = sw128_desc(smem_u32(sm.q[0]));
             constexpr uint64_t kBoxStep = kBoxBytes >> 4, kQStep = (2 * kBoxBytes) >> 4;
-            int u = -1, ord = -1, qslot = 0;  // the current unit, its ordinal and Q slot
+            int u = cta / a.T_u, t = cta - (cta / a.T_u) * a.T_u;  // unit and tile of local tile i
+            int ord = 0, qslot = 0;                                 // unit ordinal, its Q slot
             int s = 0;
             uint32_t sph = 0;  // phase-2 ring stage and phase
-            for (int i = 0; !*abort; ++i) {
-                int2 e;
-                if (!seq_get(sm, i, a.T_u, e, abort, a.err)) break;
-                if (e.x != u) {
-                    // a new unit: the last phase that reads the previous unit's Q releases its
-                    // slot (not refilled before then), and the new unit's Q must have landed
-                    if (u >= 0 && (ph == 1 || MODE == kStats)) umma_commit(&sm.qempty[qslot]);
-                    u = e.x;
-                    ++ord;
-                    qslot = ord % kQSlots;
+            bool have_q = false;
+            for (int i = 0; i < n_local && !*abort; ++i) {
+                if (!have_q) {
+                    // the unit's Q (its slot is not refilled before phase 2 releases it)
                     mbar_spin(&sm.qfull[qslot], (ord / kQSlots) & 1, abort, a.err);
+                    have_q = true;
                 }
-                const int t = e.y;
                 // phase 2 of a tile waits until its unit's lse is in shared memory
                 if (ph == 1) mbar_spin(&sm.lsefull[ord & 1], (ord >> 1) & 1, abort, a.err);
                 if (ph == 0 || MODE == kScores)
@@ -662,41 +521,35 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                     }
                 }
                 umma_commit(&sm.accfull[slot]);
-                if (ph == 1) *reinterpret_cast<volatile int*>(&sm.p2_pos) = i + 1;
-            }
-            // The issuer that finishes last posts an end job to every accumulator (job numbers
-            // n .. n + kAcc - 1 after the last real job, one per consumer warpgroup).
-            if (atomicAdd(&sm.issuers_done, 1) + 1 == (MODE == kFull ? 2 : 1)) {
-                for (int k = 0; k < kAcc; ++k) {
-                    const int n = atomicAdd(&sm.next_job, 1);
-                    const int slot = n % kAcc;
-                    spin_until_at_least(&sm.jobs_started, n, abort, a.err);
-                    mbar_spin(&sm.accempty[slot], ((n / kAcc) & 1) ^ 1, abort, a.err);
-                    *reinterpret_cast<volatile int*>(&sm.jobs_started) = n + 1;
-                    sm.job[slot] = make_int4(kJobEnd, 0, 0, 0);
-                    mbar_arrive(&sm.accfull[slot]);  // no MMA: both arrivals from here
-                    mbar_arrive(&sm.accfull[slot]);
+                // next tile; a new unit moves to the next Q slot (phase 2 releases the old one)
+                t += P;
+                int nu = u;
+                while (t >= a.T_u) {
+                    t -= a.T_u;
+                    ++nu;
+                }
+                if (nu != u) {
+                    // the last phase that reads the unit's Q releases its slot
+                    if ((ph == 1 || MODE == kStats) && i + 1 < n_local) umma_commit(&sm.qempty[qslot]);
+                    u = nu;
+                    ++ord;
+                    if (++qslot == kQSlots) qslot = 0;
+                    have_q = false;
                 }
             }
         }
     } else if (warp == 4) {
         // ------------------------------------------------------------ lse of each unit
         // lane l handles query rows l, l + 32, l + 64, l + 96
+        int cur = -1, ord = -1;
         unsigned target[2] = {0u, 0u};
         bool gave_up = false;
-        const unsigned n_contrib = (unsigned)a.T_u;  // a unit is complete once all its tiles are added
-        int first_prev = 0;
-        for (int ord = 0; !*abort; ++ord) {
-            // the CTA's ord-th unit and its first local tile (published by warp 0 with its claim)
-            int2 info;
-            if (!ord_get(sm, ord, info, abort, a.err)) break;
-            __syncwarp();
-            if (lane == 0) *reinterpret_cast<volatile int*>(&sm.lse_ord) = ord + 1;
-            const int u = info.x;
-            // the previous unit's tile count is now known: its phase-2 jobs, one arrival per
-            // consumer warp each, release its lse slot
-            if (ord > 0) target[(ord - 1) & 1] += 4u * (unsigned)(info.y - first_prev);
-            first_prev = info.y;
+        const unsigned n_contrib = (unsigned)min(a.T_u, a.P);
+        for (int i = 0; i < n_local && !*abort; ++i) {
+            const int u = seq.unit(i);
+            if (u == cur) continue;
+            cur = u;
+            ++ord;
             const int slot = ord & 1;
             // every phase-2 job of the unit that used this slot before has read it
             if (MODE != kStats && lane == 0 &&
@@ -711,6 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                     }
                 }
             }
+            target[slot] += 4u * (unsigned)seq.count(u);
             if (MODE == kScores) {
                 // the normalisers come from the caller (every shard's, merged)
 #pragma unroll
@@ -724,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                 if (lane == 0) mbar_arrive(&sm.lsefull[slot]);
                 continue;
             }
-            // unit u is complete once the parts of all its T_u tiles have been added
+            // unit u is complete once every CTA holding tiles of it has added its part
             int ok = 0;
             if (lane == 0) {
                 const unsigned* cnt = a.inject ? a.never : a.count + u;
@@ -793,19 +647,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
         }
     } else if (warp == 5) {
         // ------------------------------------------------------------ publisher
-        // lane l holds query rows l + 32 k.  Each phase-1 tile record (m, l) becomes the tile's
-        // part of the row's total relative to the row's reference logit, l 2^(m - ref), in
-        // fp64 (m is the reference itself unless the tile holds a much larger logit, so the
-        // part is exactly l): what a tile adds does not depend on which CTA took it or on the
-        // order of addition beyond fp64 rounding.  The CTA's parts of a unit are added to the
-        // unit's total when its next local tile belongs to another unit or is not claimed
-        // yet, together with the number of tiles they cover.
-        double L[4] = {0.0, 0.0, 0.0, 0.0}, T[4] = {0.0, 0.0, 0.0, 0.0};
-        int n_merged = 0;
-        for (int i = 0; MODE != kScores && !*abort; ++i) {
-            int2 e;
-            if (!seq_get(sm, i, a.T_u, e, abort, a.err)) break;
-            const int u = e.x;
+        // lane l holds query rows l + 32 k; merges the phase-1 tile records in tile order and
+        // adds the CTA's part of each unit to the unit's total
+        float M[4], L[4], T[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            M[k] = -INFINITY;
+            L[k] = 0.f;
+            T[k] = 0.f;
+        }
+        int u = cta / a.T_u, t = cta - (cta / a.T_u) * a.T_u;
+        for (int i = 0; i < (MODE == kScores ? 0 : n_local); ++i) {
             const int s = i % kRec;
             mbar_wait(&sm.recfull[s], (i / kRec) & 1, abort, a.err);
             if (*abort) break;
@@ -824,30 +676,41 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 if (v[k].x != -INFINITY) {
-                    const float d = v[k].x - __ldg(a.ref + (size_t)u * kQRows + lane + 32 * k);
-                    L[k] += scale_exp2(v[k].y, d);
-                    // sum of 2^(y - ref) (y - ref) = 2^d (t + d l)
-                    if (ENT) T[k] += scale_exp2(fmaf(d, v[k].y, vt[k]), d);
+                    const float mn = fmaxf(M[k], v[k].x);
+                    const float fa = M[k] == -INFINITY ? 0.f : ex2(M[k] - mn), fb = ex2(v[k].x - mn);
+                    if (ENT)
+                        T[k] = (M[k] == -INFINITY ? 0.f : fa * (T[k] + (M[k] - mn) * L[k])) +
+                               fb * (vt[k] + (v[k].x - mn) * v[k].y);
+                    L[k] = (M[k] == -INFINITY ? 0.f : L[k] * fa) + v[k].y * fb;
+                    M[k] = mn;
                 }
             }
-            ++n_merged;
-            int2 nx = make_int2(-1, -1);
-            int known = lane == 0 ? seq_peek(sm, i + 1, a.T_u, nx) : 0;
-            known = __shfl_sync(0xffffffffu, known, 0);
-            const int nu = __shfl_sync(0xffffffffu, known == 1 ? nx.x : -1, 0);
-            if (known == 1 && nu == u) continue;
+            t += P;
+            int nu = u;
+            while (t >= a.T_u) {
+                t -= a.T_u;
+                ++nu;
+            }
+            if (nu == u && i + 1 < n_local) continue;
+            // last tile of unit u on this CTA
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                const size_t at = ((size_t)u * kSumCopies + cta % kSumCopies) * kQRows + lane + 32 * k;
-                if (L[k] != 0.0) atomicAdd(a.sum + at, L[k]);
-                if (ENT && T[k] != 0.0) atomicAdd(a.sum_t + at, T[k]);
-                L[k] = 0.0;
-                T[k] = 0.0;
+                const int r = lane + 32 * k;
+                if (M[k] != -INFINITY) {
+                    const size_t at = ((size_t)u * kSumCopies + cta % kSumCopies) * kQRows + r;
+                    const float d = M[k] - __ldg(a.ref + (size_t)u * kQRows + r);
+                    atomicAdd(a.sum + at, scale_exp2(L[k], d));
+                    // sum of 2^(y - ref) (y - ref) = 2^d (T + d L)
+                    if (ENT) atomicAdd(a.sum_t + at, scale_exp2(fmaf(d, L[k], T[k]), d));
+                }
+                M[k] = -INFINITY;
+                L[k] = 0.f;
+                T[k] = 0.f;
             }
             __threadfence();
             __syncwarp();
-            if (lane == 0) atomicAdd(a.count + u, (unsigned)n_merged);
-            n_merged = 0;
+            if (lane == 0) atomicAdd(a.count + u, 1u);
+            u = nu;
         }
     } else if (warp >= kConsumer0) {
         // ------------------------------------------------------------ consumers
@@ -856,10 +719,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
         const int g = (warp - kConsumer0) >> 2;
         const int r = threadIdx.x - 32 * kConsumer0 - 128 * g;
         const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + g * 128;
+        const int n_jobs = MODE == kFull ? 2 * n_local : n_local;
         // the last local key index row q sees is min(N - 1, hz0 + q % w) (sharding: a key's
         // position is key_off + its local index; row q sits at n_total - w + q % w)
         const int hz0 = a.n_total - a.w - a.key_off;
-        for (int n = g;; n += kAcc) {
+        for (int n = g; n < n_jobs; n += kAcc) {
             mbar_wait(&sm.accfull[g], (n / kAcc) & 1, abort, a.err);
             if (*abort) break;
             tc_fence_after();
@@ -868,7 +732,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                          : "=r"(jb.x), "=r"(jb.y), "=r"(jb.z), "=r"(jb.w)
                          : "r"(smem_u32(&sm.job[g]))
                          : "memory");
-            if (jb.x == kJobEnd) break;
             const int u = jb.y, ti = jb.z;
             const bool full_tile = (ti + 1) * kTileKeys <= min(a.N, a.n_total - a.w - a.key_off + 1);
             if (jb.x == 0) {
@@ -1057,8 +920,8 @@ TcLayout tc_layout(int U) {
     off = a256(off + 2 * (size_t)U * kSumCopies * kQRows * sizeof(double));
     L.lse = off;  // kScores: the merged log-sum-exp per (unit, padded row)
     off = a256(off + (size_t)U * kQRows * sizeof(float));
-    L.flags = off;  // count[U], never, claim
-    L.n_flags = (size_t)U + 2;
+    L.flags = off;  // count[U], never
+    L.n_flags = (size_t)U + 1;
     off = a256(off + L.n_flags * sizeof(unsigned));
     L.total = off;
     return L;
@@ -1091,13 +954,8 @@ int sm_count() {
 }
 
 bool tc_score_supported(const ScoreJob& j) {
-    if (!(j.dtype == KVC_BF16 && j.nq >= 1 && j.nq <= kQRows && j.N >= 1 && j.U >= 1 &&
-          (long long)j.U * kQRows < (1LL << 31)))
-        return false;
-    // the lead of phase 1 over phase 2 must cover a unit's share of tiles per CTA
-    const long long T_u = (j.N + kTileKeys - 1) / kTileKeys;
-    const long long P = std::min<long long>(std::min(sm_count(), kMaxCtas), T_u * j.U);
-    return P > 0 && (T_u + P - 1) / P + kLeadSlack <= kMaxLead && T_u * j.U < (1LL << 30);
+    return j.dtype == KVC_BF16 && j.nq >= 1 && j.nq <= kQRows && j.N >= 1 && j.U >= 1 &&
+           (long long)j.U * kQRows < (1LL << 31);
 }
 
 size_t tc_score_workspace(int U, int /*N*/, int /*nq*/) { return tc_layout(U).total; }
@@ -1149,7 +1007,6 @@ cudaError_t tc_launch(const ScoreJob& j, int mode, float2* ml_out, cudaStream_t 
     a.entropy = j.entropy;
     a.count = flags;
     a.never = flags + j.U;
-    a.claim = flags + j.U + 1;
     a.err = j.err;
     a.spin_limit = j.spin_limit;
     a.U = j.U;
@@ -1164,7 +1021,6 @@ cudaError_t tc_launch(const ScoreJob& j, int mode, float2* ml_out, cudaStream_t 
     // phase 1 may run this many tiles ahead of phase 2: a unit's worth plus slack for the
     // merge, while keeping the tiles between the two reads (max_lead x P x 32 KiB) in L2
     a.max_lead = (a.T_u + a.P - 1) / a.P + kLeadSlack;
-    if (a.max_lead > kMaxLead) return cudaErrorInvalidValue;  // tc_score_supported rules this out
     a.inject = j.inject_timeout;
     a.key_off = j.key_off;
     a.n_total = j.n_total > 0 ? j.n_total : j.N;
