@@ -73,6 +73,10 @@ constexpr int kBoxBytes = kTileKeys * 64 * 2;          // a 128-row x 64-column 
 constexpr int kStagesA = KVC_TC_STAGES_A;              // phase-1 ring, in 16 KiB halves (HBM stream)
 constexpr int kTilesA = kStagesA / 2;                  // the same ring in whole tiles (one op each)
 constexpr int kStagesB = KVC_TC_STAGES_B;              // phase-2 ring (L2 re-read)
+// A single-phase launch (kStats, kScores) has no phase-2 ring: its tiles stream through the
+// phase-1 ring extended over the phase-2 ring's memory (which follows it), one more tile in
+// flight per SM.
+constexpr int kTiles1 = (kStagesA + kStagesB) / 2;
 constexpr int kQSlots = KVC_TC_Q_SLOTS;                // Q of the CTA's last units, by unit ordinal
 constexpr int kLeadSlack = KVC_TC_LEAD_SLACK;          // phase-1 lead beyond one unit, in tiles
 constexpr int kAcc = 4;                // TMEM accumulators (128 columns each) = consumer warpgroups
@@ -135,6 +139,10 @@ struct __align__(1024) Smem {
     int abort;
     int p1_issued, p2_issued;  // tiles whose loads each producer has issued (L2 lead control)
 };
+
+static_assert(offsetof(Smem, ringB) == offsetof(Smem, ringA) + sizeof(Smem::ringA) && kTiles1 <= kStagesA &&
+                  2 * kTiles1 <= kStagesA + kStagesB,
+              "the single-phase ring spans the phase-1 and phase-2 rings");
 
 // Spinning bounded wait (no suspension) for the single-thread roles, which must react fast.
 __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
@@ -323,6 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
     extern __shared__ uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int kRing = MODE == kFull ? kTilesA : kTiles1;  // tiles of the HBM ring
     const int cta = blockIdx.x, P = a.P;
     const int n_local = cta < a.total_tiles ? (a.total_tiles - cta + P - 1) / P : 0;
     const TileSeq seq{cta, P, a.T_u, n_local};
@@ -379,7 +388,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
         // A single issuing thread completes TMA ops at a roughly fixed rate, so the phase-1
         // stream uses large ops and the phase-2 stream two threads.  kStats: no phase-2
         // re-reads; kScores: no phase 1, so warp 0 streams the tiles (from HBM, one 32 KiB op
-        // each) straight to the phase-2 jobs.
+        // each) straight to the phase-2 jobs.  Both single-phase modes stream through a ring of
+        // kTiles1 tiles (the phase-2 ring's memory added), which keeps more of HBM's latency
+        // covered than the two tiles of the two-phase launch.
         if (lane == 0 && !(MODE != kFull && warp != 0)) {
             const int ph = warp == 0 ? 0 : 1, hh = warp == 6 ? 1 : 0;
             const CUtensorMap* mk = ph == 0 ? &a.tmap_k4 : &a.tmap_k;
@@ -421,10 +432,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                     tma_load_2d(sm.q[slot] + kBoxBytes, &a.tmap_q, &sm.qfull[slot], 64, u * kQRows);
                 }
                 if (ph == 0) {
-                    const int st = i % kTilesA;
-                    mbar_spin(&sm.emptyA[st], ((i / kTilesA) & 1) ^ 1, abort, a.err);
+                    const int st = i % kRing;
+                    mbar_spin(&sm.emptyA[st], ((i / kRing) & 1) ^ 1, abort, a.err);
                     mbar_expect_tx(&sm.fullA[st], 2 * kBoxBytes);
-                    tma_load_4d(sm.ringA[2 * st], mk, &sm.fullA[st], 0, ti * kTileKeys, 0, u);
+                    tma_load_4d(&sm.ringA[0][0] + (size_t)2 * st * kBoxBytes, mk, &sm.fullA[st], 0, ti * kTileKeys, 0, u);
                     *reinterpret_cast<volatile int*>(&sm.p1_issued) = i + 1;
                 } else {
                     const int k = 2 * i + hh, st = k % kStagesB;
@@ -437,8 +448,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             if (*abort) {
                 // copies still in flight land before the CTA exits
                 if (ph == 0) {
-                    for (int n = std::max(0, i - kTilesA); n < i; ++n)
-                        drain_wait(&sm.fullA[n % kTilesA], (n / kTilesA) & 1, a.err);
+                    for (int n = std::max(0, i - kRing); n < i; ++n)
+                        drain_wait(&sm.fullA[n % kRing], (n / kRing) & 1, a.err);
                     for (int o = std::max(0, ord - kQSlots + 1); o <= ord; ++o)
                         drain_wait(&sm.qfull[o % kQSlots], (o / kQSlots) & 1, a.err);
                 } else {
@@ -475,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                 // phase 2 of a tile waits until its unit's lse is in shared memory
                 if (ph == 1) mbar_spin(&sm.lsefull[ord & 1], (ord >> 1) & 1, abort, a.err);
                 if (ph == 0 || MODE == kScores)
-                    mbar_spin(&sm.fullA[i % kTilesA], (i / kTilesA) & 1, abort, a.err);
+                    mbar_spin(&sm.fullA[i % kRing], (i / kRing) & 1, abort, a.err);
                 else
                     mbar_spin(&sm.fullB[s], sph, abort, a.err);
                 const int n = atomicAdd(&sm.next_job, 1);
@@ -493,14 +504,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                 const uint64_t dq = dQ0 + (uint64_t)qslot * kQStep;
                 if (ph == 0) {
                     // both halves of the tile arrived with one op
-                    const int st = i % kTilesA;
+                    const int st = i % kRing;
                     const uint64_t dk = dK0 + (uint64_t)(2 * st) * kBoxStep;
                     umma_half(d, dq, dk, 0);
                     umma_half(d, dq + kBoxStep, dk + kBoxStep, 1);
                     umma_commit(&sm.emptyA[st]);
                 } else if (MODE == kScores) {
                     // phase 2 alone: the tile came through the phase-1 ring
-                    const int st = i % kTilesA;
+                    const int st = i % kRing;
                     const uint64_t dk = sw128_desc(smem_u32(sm.ringA[0])) + (uint64_t)(2 * st) * kBoxStep;
                     tc_fence_after();
                     umma_half(d, dk, dq, 0);

@@ -184,9 +184,11 @@ def test_select_pick_ties_kept_contract(K):
     for key_off, n_local in [(0, 400), (400, 590), (990, 10), (2, 5)]:
         cap_sel = max(n_local, 1)
         sel = np.full((rows, cap_sel), -7, dtype=np.int32)
-        cnt = g.integers(0, min(n_local, 40), rows).astype(np.int32)
+        # a block's selected positions are candidates: past the sinks, before the window
+        cand = np.arange(max(S, key_off), min(N - w, key_off + n_local))
+        cnt = g.integers(0, min(cand.size, 40) + 1, rows).astype(np.int32)
         for r_ in range(rows):
-            sel[r_, :cnt[r_]] = np.sort(g.choice(np.arange(key_off, key_off + n_local), cnt[r_], replace=False))
+            sel[r_, :cnt[r_]] = np.sort(g.choice(cand, cnt[r_], replace=False))
         cap = min(n_local, 64)
         pos = torch.empty((rows, cap), dtype=torch.int32, device="cuda")
         local = torch.empty_like(pos)
