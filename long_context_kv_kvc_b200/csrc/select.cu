@@ -241,19 +241,53 @@ constexpr int kCtWarps = kCtThreads / 32;
 constexpr int kBins = 2048;
 constexpr int kSegMax = 24576;  // keys per CTA: 96 KiB of shared memory (two CTAs per SM)
 
+// Adds `n` keys of histogram bin `d` for each thread of the warp that holds a run (has):
+// threads with the same bin combine their counts, one shared-memory atomic per bin.
+__device__ __forceinline__ void hist_add_runs(uint32_t* hist, bool has, unsigned d, unsigned n, int lane) {
+    if (!has) return;
+    const unsigned peers = __match_any_sync(__activemask(), d);
+    const unsigned sum = __reduce_add_sync(peers, n);
+    if (lane == __ffs(peers) - 1) atomicAdd(&hist[d], sum);
+}
+
+// Counts digit (key >> shift) & dmask of the keys among k[0..7] that are valid and match
+// the prefix, as runs of equal digits (neighbouring positions mostly share the leading
+// digits): a run that ends is added directly, the last goes through hist_add_runs.
+__device__ __forceinline__ void hist_count8(uint32_t* hist, const uint32_t (&k)[8], unsigned valid, uint32_t mask,
+                                            uint32_t prefix, int shift, uint32_t dmask, int lane) {
+    unsigned run_d = 0xffffffffu, run_n = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        if (!((valid >> i) & 1u) || (k[i] & mask) != prefix) continue;
+        const unsigned d = (k[i] >> shift) & dmask;
+        if (d != run_d) {
+            if (run_n) atomicAdd(&hist[run_d], run_n);
+            run_d = d;
+            run_n = 0;
+        }
+        ++run_n;
+    }
+    hist_add_runs(hist, run_n > 0, run_d, run_n, lane);
+}
+
 struct TopkSmem {
     uint32_t hist[kBins];
     uint32_t slice_tot[kBins / kClusterCtas];  // this CTA's slice of the cluster-wide totals
     uint32_t slice_sum;
     int gt, eq;
     int wcnt_gt[kCtWarps], wcnt_eq[kCtWarps];
-    uint32_t keys[kSegMax];
+    alignas(16) uint32_t keys[kSegMax];  // slot x: the key of row position (s0 & ~3) + x (16-byte accesses)
 };
+constexpr int kSlotPad = 16;  // slots beyond a CTA's candidates: alignment to 4 and whole groups of 8
+static_assert(offsetof(TopkSmem, keys) % 16 == 0, "16-byte key accesses");
 
+// R >= 0: the pool radius, scores rows 16-byte aligned (vector loads); R = -1: any radius
+// (scalar loads, runtime radius).
+template <int R>
 __global__ void __launch_bounds__(kCtThreads, 2) __cluster_dims__(kClusterCtas, 1, 1)
 topk_cluster_kernel(const float* __restrict__ scores, int N, int S, int w, int budget, int radius, int seg,
                     int32_t* __restrict__ idx, unsigned* err) {
-    extern __shared__ uint8_t smem_raw[];
+    extern __shared__ __align__(16) uint8_t smem_raw[];
     TopkSmem& sm = *reinterpret_cast<TopkSmem*>(smem_raw);
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
@@ -271,25 +305,65 @@ topk_cluster_kernel(const float* __restrict__ scores, int N, int S, int w, int b
         for (int i = tid; i < w; i += kCtThreads)
             if (dcheck(err, budget - w + i >= S)) out[budget - w + i] = N - w + i;
     }
+    // Slot x of keys[] holds row position A0 + x, A0 = s0 rounded down to 4 (16-byte aligned
+    // when the vector loads are used); this CTA's candidates are slots [off, off + n_mine).
+    const int A0 = R >= 0 ? (s0 & ~3) : s0, off = s0 - A0, n_slots = off + n_mine;
     // this CTA's keys fit its shared memory
-    if (tid == 0) dcheck(err, n_mine <= seg && seg <= kSegMax);
+    if (tid == 0) dcheck(err, n_mine <= seg && seg + kSlotPad <= kSegMax);
     // pooled keys of this CTA's candidates (max over the clipped window of raw scores); the
-    // first digit's histogram (the top 11 bits of every key) is counted as they are formed
+    // first digit's histogram (the top 11 bits of every key) is counted as they are formed.
+    // A thread forms 8 neighbouring keys at a time from 16 raw scores (positions p - 4 ..
+    // p + 11, four 16-byte loads; outside [lo, hi) they count as -inf).
     for (int i = tid; i < kBins; i += kCtThreads) sm.hist[i] = 0u;
     __syncthreads();
-    for (int e = tid; e < n_mine; e += kCtThreads) {
-        const int j = s0 + e;
-        const int t0 = max(lo, j - radius), t1 = min(hi - 1, j + radius);
-        float m = 0.f;
-        if (dcheck(err, t0 >= 0 && t0 <= j && j <= t1 && t1 < N)) {
-            m = __ldg(v + t0);
-            for (int t = t0 + 1; t <= t1; ++t) m = fmaxf(m, __ldg(v + t));
+    for (int x = 8 * tid; x < n_slots; x += 8 * kCtThreads) {
+        const int p = A0 + x;
+        uint32_t kk[8];
+        if constexpr (R >= 0) {
+            float r16[16];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const int q = p - 4 + 4 * q4;
+                if (q >= lo && q + 3 < hi) {
+                    const float4 f = __ldg(reinterpret_cast<const float4*>(v + q));
+                    r16[4 * q4] = f.x;
+                    r16[4 * q4 + 1] = f.y;
+                    r16[4 * q4 + 2] = f.z;
+                    r16[4 * q4 + 3] = f.w;
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        r16[4 * q4 + c] = (q + c >= lo && q + c < hi) ? __ldg(v + q + c) : -INFINITY;
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                float m = r16[4 + k];
+#pragma unroll
+                for (int d = 1; d <= R; ++d) m = fmaxf(m, fmaxf(r16[4 + k - d], r16[4 + k + d]));
+                kk[k] = order_key(m);
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int j = min(max(p + k, lo), hi - 1);  // slots outside the candidates are never read
+                const int t0 = max(lo, j - radius), t1 = min(hi - 1, j + radius);
+                float m = 0.f;
+                if (dcheck(err, t0 >= 0 && t0 <= j && j <= t1 && t1 < N)) {
+                    m = __ldg(v + t0);
+                    for (int t = t0 + 1; t <= t1; ++t) m = fmaxf(m, __ldg(v + t));
+                }
+                kk[k] = order_key(m);
+            }
         }
-        const uint32_t key = order_key(m);
-        if (dcheck(err, e < kSegMax)) sm.keys[e] = key;
-        const unsigned digit = key >> 21;
-        const unsigned peers = __match_any_sync(__activemask(), digit);
-        if (lane == __ffs(peers) - 1) atomicAdd(&sm.hist[digit], (unsigned)__popc(peers));
+        if (dcheck(err, x + 8 <= kSegMax)) {
+            *reinterpret_cast<uint4*>(&sm.keys[x]) = make_uint4(kk[0], kk[1], kk[2], kk[3]);
+            *reinterpret_cast<uint4*>(&sm.keys[x + 4]) = make_uint4(kk[4], kk[5], kk[6], kk[7]);
+        }
+        unsigned valid = 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) valid |= (x + k >= off && x + k < n_slots) ? 1u << k : 0u;
+        hist_count8(sm.hist, kk, valid, 0u, 0u, 21, 0x7ffu, lane);
     }
 
     uint32_t prefix = 0, mask = 0;
@@ -302,13 +376,14 @@ topk_cluster_kernel(const float* __restrict__ scores, int N, int S, int w, int b
         if (pass > 0) {  // the first pass's histogram was built with the keys
             for (int i = tid; i < kBins; i += kCtThreads) sm.hist[i] = 0u;
             __syncthreads();
-            for (int e = tid; e < n_mine; e += kCtThreads) {
-                const uint32_t key = sm.keys[e];
-                if ((key & mask) == prefix) {
-                    const unsigned digit = (key >> shift) & dmask;
-                    const unsigned peers = __match_any_sync(__activemask(), digit);
-                    if (lane == __ffs(peers) - 1) atomicAdd(&sm.hist[digit], (unsigned)__popc(peers));
-                }
+            for (int x = 8 * tid; x < n_slots; x += 8 * kCtThreads) {
+                const uint4 a4 = *reinterpret_cast<const uint4*>(&sm.keys[x]);
+                const uint4 b4 = *reinterpret_cast<const uint4*>(&sm.keys[x + 4]);
+                const uint32_t kk[8] = {a4.x, a4.y, a4.z, a4.w, b4.x, b4.y, b4.z, b4.w};
+                unsigned valid = 0;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) valid |= (x + k >= off && x + k < n_slots) ? 1u << k : 0u;
+                hist_count8(sm.hist, kk, valid, mask, prefix, shift, dmask, lane);
             }
         }
         cluster.sync();  // every CTA's histogram is complete
@@ -382,7 +457,7 @@ topk_cluster_kernel(const float* __restrict__ scores, int N, int S, int w, int b
     const int w0 = min(n_mine, warp * wseg), w1 = min(n_mine, (warp + 1) * wseg);
     int n_gt = 0, n_eq = 0;
     for (int e = w0 + lane; e < w1; e += 32) {
-        const uint32_t key = sm.keys[e];
+        const uint32_t key = sm.keys[e + off];
         n_gt += key > T;
         n_eq += key == T;
     }
@@ -419,7 +494,7 @@ topk_cluster_kernel(const float* __restrict__ scores, int N, int S, int w, int b
     int eq_seen = eq_before;
     for (int base = w0; base < w1; base += 32) {
         const int e = base + lane;
-        const uint32_t key = e < w1 ? sm.keys[e] : 0u;
+        const uint32_t key = e < w1 ? sm.keys[e + off] : 0u;
         const bool gt = e < w1 && key > T;
         const bool eq = e < w1 && key == T;
         const unsigned eq_mask = __ballot_sync(0xffffffffu, eq);
@@ -623,30 +698,51 @@ cudaError_t pool(const float* in, float* out, int rows, int N, int lo, int hi, i
 
 bool topk_fused_fits(int N, int n_sink, int window) {
     const int n_c = N - n_sink - window;
-    return (n_c + kClusterCtas - 1) / kClusterCtas <= kSegMax;
+    return (n_c + kClusterCtas - 1) / kClusterCtas + kSlotPad <= kSegMax;
 }
+
+namespace {
+
+template <int R>
+cudaError_t launch_topk_cluster(const float* scores, int rows, int N, int n_sink, int window, int budget, int radius,
+                                int seg, int32_t* idx, size_t smem, cudaStream_t s) {
+    static std::atomic<bool> attr_done[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 64 || !attr_done[dev].load()) {
+        e = cudaFuncSetAttribute(topk_cluster_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sizeof(TopkSmem));
+        if (e != cudaSuccess) return e;
+        if (dev < 64) attr_done[dev].store(true);
+    }
+    topk_cluster_kernel<R><<<rows * kClusterCtas, kCtThreads, smem, s>>>(scores, N, n_sink, window, budget, radius, seg,
+                                                                        idx, device_error_word());
+    return cudaGetLastError();
+}
+
+}  // namespace
 
 cudaError_t topk_fused(const float* scores, int rows, int N, int n_sink, int window, int budget, int kernel,
                        int32_t* idx, cudaStream_t s) {
     if (rows == 0) return cudaSuccess;
     const int n_c = N - n_sink - window;
     const int seg = (n_c + kClusterCtas - 1) / kClusterCtas;
-    if (seg > kSegMax) return cudaErrorInvalidValue;
-    const size_t smem = sizeof(TopkSmem) - sizeof(uint32_t) * (size_t)(kSegMax - seg);
-    static std::atomic<bool> attr_done[64];
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev >= 64 || !attr_done[dev].load()) {
-        e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(TopkSmem));
-        if (e != cudaSuccess) return e;
-        if (dev < 64) attr_done[dev].store(true);
-    }
-    topk_cluster_kernel<<<rows * kClusterCtas, kCtThreads, smem, s>>>(scores, N, n_sink, window, budget,
-                                                                     (kernel - 1) / 2, seg, idx,
-                                                                     device_error_word());
+    if (seg + kSlotPad > kSegMax) return cudaErrorInvalidValue;
+    const size_t smem = sizeof(TopkSmem) - sizeof(uint32_t) * (size_t)(kSegMax - seg - kSlotPad);
+    const int radius = (kernel - 1) / 2;
+    // 16-byte loads need every row 16-byte aligned
+    const bool vec = N % 4 == 0 && reinterpret_cast<uintptr_t>(scores) % 16 == 0;
     count_launches(1);
-    return cudaGetLastError();
+    if (vec) switch (radius) {
+            case 0: return launch_topk_cluster<0>(scores, rows, N, n_sink, window, budget, radius, seg, idx, smem, s);
+            case 1: return launch_topk_cluster<1>(scores, rows, N, n_sink, window, budget, radius, seg, idx, smem, s);
+            case 2: return launch_topk_cluster<2>(scores, rows, N, n_sink, window, budget, radius, seg, idx, smem, s);
+            case 3: return launch_topk_cluster<3>(scores, rows, N, n_sink, window, budget, radius, seg, idx, smem, s);
+            case 4: return launch_topk_cluster<4>(scores, rows, N, n_sink, window, budget, radius, seg, idx, smem, s);
+            default: break;
+        }
+    return launch_topk_cluster<-1>(scores, rows, N, n_sink, window, budget, radius, seg, idx, smem, s);
 }
 
 cudaError_t topk(const float* pooled, int rows, int N, int n_sink, int window, int budget,
