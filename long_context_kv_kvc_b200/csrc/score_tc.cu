@@ -27,11 +27,13 @@
 //     phase-1 work exists.  Accumulators are taken in job order and the phase-1 record ring
 //     is released through a monotonic counter: a parity wait on an mbarrier that may lag two
 //     phases behind its waiter would pass early;
-//   * a phase-1 job yields per query row the tile's (max, sum of 2^(y - max)); a publisher
-//     warp merges them in tile order, rescales the CTA's sum to a fixed per-row reference
-//     (the row's logit with the key at its own position, computed before the kernel), adds
-//     it to the unit's fp64 total with a fire-and-forget atomic and bumps the unit's arrival
-//     count (fp64 addition order moves the total by ~1e-16, far below fp32);
+//   * a phase-1 job yields per query row the tile's sum of 2^(y - ref) relative to a fixed
+//     per-row reference ref (the row's logit with the key at its own position, computed
+//     before the kernel; a tile with a much larger logit records its own shift of the
+//     reference); a publisher warp adds the records in fp64 -- without an exponential
+//     unless the reference moved -- and adds the CTA's part of a unit to the unit's fp64
+//     total with fire-and-forget atomics, then bumps the unit's arrival count (fp64 addition
+//     order moves the total by ~1e-16, far below fp32);
 //   * an lse warp waits for each unit's count, turns the totals into lse = ref + log2(total)
 //     in shared memory and releases the unit's phase-2 jobs; a phase-2 job gives each key
 //     of the tile its sum over the query rows of 2^(y - lse).
@@ -89,6 +91,7 @@ constexpr int kConsumer0 = 8;          // first consumer warp
 #endif
 constexpr int kSumCopies = KVC_TC_SUM_COPIES;  // copies of each unit's totals (CTA c adds to copy c % kSumCopies)
 constexpr int kMaxCtas = 160;                          // upper bound on the persistent grid
+constexpr int kRefSamples = 8;         // kStats: keys whose largest logit is a row's reference
 constexpr uint32_t kTmemCols = 512;
 
 struct TcArgs {
@@ -122,7 +125,7 @@ struct __align__(1024) Smem {
     uint8_t ringA[kStagesA][kBoxBytes];
     uint8_t ringB[kStagesB][kBoxBytes];
     uint8_t q[kQSlots][2 * kBoxBytes];  // Q of the CTA's k-th unit in slot k % kQSlots (two boxes)
-    float2 rec[kRec][kQRows];           // phase-1 tile i: per row (m, sum of 2^(y - m))
+    float2 rec[kRec][kQRows];           // phase-1 tile i: per row (m - ref, sum of 2^(y - m))
     float rec_t[kRec][kQRows];          // with the entropy: sum of 2^(y - m) (y - m)
     float nlse[2][kQRows];              // -lse of the CTA's k-th unit in slot k % 2
     int4 job[kAcc];                     // {kind, unit, tile within unit, record or lse slot}
@@ -658,15 +661,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
         }
     } else if (warp == 5) {
         // ------------------------------------------------------------ publisher
-        // lane l holds query rows l + 32 k; merges the phase-1 tile records in tile order and
-        // adds the CTA's part of each unit to the unit's total
-        float M[4], L[4], T[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            M[k] = -INFINITY;
-            L[k] = 0.f;
-            T[k] = 0.f;
-        }
+        // lane l holds query rows l + 32 k; adds the phase-1 tile records to the CTA's part of
+        // each unit's total relative to the row's reference logit, in fp64: a record (d, l)
+        // with d = m - ref adds l 2^d, which is l itself unless the tile moved the reference
+        // (so the common case needs no exponential), and the part goes to the unit's total
+        // after the CTA's last tile of the unit
+        double L[4] = {0.0, 0.0, 0.0, 0.0}, T[4] = {0.0, 0.0, 0.0, 0.0};
         int u = cta / a.T_u, t = cta - (cta / a.T_u) * a.T_u;
         for (int i = 0; i < (MODE == kScores ? 0 : n_local); ++i) {
             const int s = i % kRec;
@@ -686,15 +686,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             }
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                if (v[k].x != -INFINITY) {
-                    const float mn = fmaxf(M[k], v[k].x);
-                    const float fa = M[k] == -INFINITY ? 0.f : ex2(M[k] - mn), fb = ex2(v[k].x - mn);
-                    if (ENT)
-                        T[k] = (M[k] == -INFINITY ? 0.f : fa * (T[k] + (M[k] - mn) * L[k])) +
-                               fb * (vt[k] + (v[k].x - mn) * v[k].y);
-                    L[k] = (M[k] == -INFINITY ? 0.f : L[k] * fa) + v[k].y * fb;
-                    M[k] = mn;
-                }
+                const float d = v[k].x;
+                L[k] += d == 0.f ? (double)v[k].y : scale_exp2(v[k].y, d);
+                // sum of 2^(y - ref) (y - ref) = 2^d (t + d l)
+                if (ENT) T[k] += d == 0.f ? (double)vt[k] : scale_exp2(fmaf(d, v[k].y, vt[k]), d);
             }
             t += P;
             int nu = u;
@@ -706,17 +701,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             // last tile of unit u on this CTA
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                const int r = lane + 32 * k;
-                if (M[k] != -INFINITY) {
-                    const size_t at = ((size_t)u * kSumCopies + cta % kSumCopies) * kQRows + r;
-                    const float d = M[k] - __ldg(a.ref + (size_t)u * kQRows + r);
-                    atomicAdd(a.sum + at, scale_exp2(L[k], d));
-                    // sum of 2^(y - ref) (y - ref) = 2^d (T + d L)
-                    if (ENT) atomicAdd(a.sum_t + at, scale_exp2(fmaf(d, L[k], T[k]), d));
-                }
-                M[k] = -INFINITY;
-                L[k] = 0.f;
-                T[k] = 0.f;
+                const size_t at = ((size_t)u * kSumCopies + cta % kSumCopies) * kQRows + lane + 32 * k;
+                if (L[k] != 0.0) atomicAdd(a.sum + at, L[k]);
+                if (ENT && T[k] != 0.0) atomicAdd(a.sum_t + at, T[k]);
+                L[k] = 0.0;
+                T[k] = 0.0;
             }
             __threadfence();
             __syncwarp();
@@ -751,7 +740,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                 // needed; a chunk whose sum is not below 2^100 (a logit ~100 above the
                 // reference) is redone with its exact max.
                 const int t_r = min(a.N - 1, hz0 + r % a.w);  // last key this row sees
-                float m = __ldg(a.ref + (size_t)u * kQRows + r), l = 0.f, t = 0.f;
+                const float ref = __ldg(a.ref + (size_t)u * kQRows + r);
+                float m = ref, l = 0.f, t = 0.f;
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     uint32_t x[32];
@@ -790,7 +780,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                 const int i = jb.w, s = i % kRec;
                 if (lane == 0) spin_until_at_least(&sm.rec_consumed, i - kRec + 1, abort, a.err);
                 __syncwarp();
-                sm.rec[s][r] = make_float2(m, l);
+                sm.rec[s][r] = make_float2(m - ref, l);  // 0 unless a chunk moved the reference
                 if (ENT) sm.rec_t[s][r] = t;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.recfull[s]);
@@ -860,27 +850,35 @@ __global__ void tc_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_b
          e += n_warps) {
         const int r = (int)(e % kQRows);
         const long long u = e / kQRows;
-        // the reference key: the row's own position (whole sequence), or the block's first key
-        // when the row sees it (kStats: the block may not hold the row's own position); rows
-        // without one keep 0 (they see no key of the block, and their sums stay 0)
-        const int kj = mode == kFull ? N - w + r % w : 0;
-        const bool has_ref = r < nq && (mode == kFull || (mode == kStats && key_off <= n_total - w + r % w));
-        float x = 0.f;
-        if (has_ref && dcheck(err, kj >= 0 && kj < N)) {
+        // The reference logit.  kFull: the key at the row's own position.  kStats (the block
+        // may not hold the row's own position): the largest logit over kRefSamples keys spread
+        // evenly over the ones the row sees, so that the phase-1 sums rarely have to move
+        // their reference.  Rows that see no key of the block keep 0 (their sums stay 0).
+        const int t_r = mode == kFull ? N - w + r % w : min(N - 1, n_total - w + r % w - key_off);
+        const bool has_ref = r < nq && (mode == kFull || (mode == kStats && t_r >= 0));
+        const int n_s = mode == kFull ? 1 : kRefSamples;
+        float best = -INFINITY;
+        if (has_ref) {
             const uint2 qv = *reinterpret_cast<const uint2*>(q + (u * nq + r) * kHeadDim + 4 * lane);
-            const uint2 kv = *reinterpret_cast<const uint2*>(k + (u * N + kj) * kHeadDim + 4 * lane);
             const __nv_bfloat162* qh = reinterpret_cast<const __nv_bfloat162*>(&qv);
-            const __nv_bfloat162* kh = reinterpret_cast<const __nv_bfloat162*>(&kv);
+            for (int si = 0; si < n_s; ++si) {
+                const int kj = mode == kFull ? t_r : (int)((long long)si * t_r / (n_s - 1));
+                if (!dcheck(err, kj >= 0 && kj < N)) continue;
+                const uint2 kv = *reinterpret_cast<const uint2*>(k + (u * N + kj) * kHeadDim + 4 * lane);
+                const __nv_bfloat162* kh = reinterpret_cast<const __nv_bfloat162*>(&kv);
+                float x = 0.f;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const float2 qf = __bfloat1622float2(qh[h]), kf = __bfloat1622float2(kh[h]);
-                x = fmaf(qf.x, kf.x, x);
-                x = fmaf(qf.y, kf.y, x);
+                for (int h = 0; h < 2; ++h) {
+                    const float2 qf = __bfloat1622float2(qh[h]), kf = __bfloat1622float2(kh[h]);
+                    x = fmaf(qf.x, kf.x, x);
+                    x = fmaf(qf.y, kf.y, x);
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+                best = fmaxf(best, x);
             }
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-        if (lane == 0) ref[e] = x * kLog2eOverSqrtD;
+        if (lane == 0) ref[e] = has_ref ? best * kLog2eOverSqrtD : 0.f;
     }
     for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < 2LL * U * kSumCopies * kQRows;
          e += (long long)gridDim.x * blockDim.x)
