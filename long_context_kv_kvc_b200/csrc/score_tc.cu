@@ -131,6 +131,7 @@ struct __align__(1024) Smem {
     int4 job[kAcc];                     // {kind, unit, tile within unit, record or lse slot}
     uint64_t fullA[kStagesA], emptyA[kStagesA], fullB[kStagesB], emptyB[kStagesB];
     uint64_t qfull[kQSlots], qempty[kQSlots];
+    uint64_t qempty2[kQSlots];  // single-phase launches: the second issuer's release of a Q slot
     uint64_t accfull[kAcc], accempty[kAcc];
     uint64_t recfull[kRec];
     uint64_t lsefull[2];
@@ -352,6 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
         for (int b = 0; b < kQSlots; ++b) {
             mbar_init(&sm.qfull[b], 1);
             mbar_init(&sm.qempty[b], 1);
+            mbar_init(&sm.qempty2[b], 1);
         }
         for (int b = 0; b < kAcc; ++b) {
             mbar_init(&sm.accfull[b], 2);   // the issuer's arrive (job record) + the MMA commit
@@ -429,7 +431,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                     qunit = u;
                     ++ord;
                     const int slot = ord % kQSlots;
-                    if (ord >= kQSlots) mbar_spin(&sm.qempty[slot], ((ord / kQSlots) - 1) & 1, abort, a.err);
+                    if (ord >= kQSlots) {
+                        mbar_spin(&sm.qempty[slot], ((ord / kQSlots) - 1) & 1, abort, a.err);
+                        if (MODE != kFull) mbar_spin(&sm.qempty2[slot], ((ord / kQSlots) - 1) & 1, abort, a.err);
+                    }
                     mbar_expect_tx(&sm.qfull[slot], 2 * kBoxBytes);
                     tma_load_2d(sm.q[slot], &a.tmap_q, &sm.qfull[slot], 0, u * kQRows);
                     tma_load_2d(sm.q[slot] + kBoxBytes, &a.tmap_q, &sm.qfull[slot], 64, u * kQRows);
@@ -469,9 +474,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
         // unit's lse is in shared memory).  Each claims the next job number n when its job is
         // ready and fills accumulator n % kAcc, so the consumers see one stream of jobs.  Two
         // issuers keep the tensor pipe busy while either does its bookkeeping.  kStats has only
-        // phase-1 jobs, kScores only phase-2 jobs.
-        const int ph = warp == 1 ? 0 : 1;
-        if (lane == 0 && !(MODE == kStats && ph == 1) && !(MODE == kScores && ph == 0)) {
+        // phase-1 jobs, kScores only phase-2 jobs: there both warps issue the one phase,
+        // warp 1 the even and warp 3 the odd local tiles (a single issuer was the slower side
+        // of those launches), and each releases the Q slots through its own barriers.
+        const int ph = MODE == kFull ? (warp == 1 ? 0 : 1) : (MODE == kStats ? 0 : 1);
+        const int parity = warp == 1 ? 0 : 1;  // single-phase launches: the local tiles this warp issues
+        uint64_t* qrelease = MODE != kFull && warp == 3 ? sm.qempty2 : sm.qempty;
+        if (lane == 0) {
             const uint64_t dK0 = sw128_desc(smem_u32(ph == 0 ? sm.ringA[0] : sm.ringB[0]));
             const uint64_t dQ0 = sw128_desc(smem_u32(sm.q[0]));
             constexpr uint64_t kBoxStep = kBoxBytes >> 4, kQStep = (2 * kBoxBytes) >> 4;
@@ -481,60 +490,62 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
             uint32_t sph = 0;  // phase-2 ring stage and phase
             bool have_q = false;
             for (int i = 0; i < n_local && !*abort; ++i) {
-                if (!have_q) {
-                    // the unit's Q (its slot is not refilled before phase 2 releases it)
-                    mbar_spin(&sm.qfull[qslot], (ord / kQSlots) & 1, abort, a.err);
-                    have_q = true;
-                }
-                // phase 2 of a tile waits until its unit's lse is in shared memory
-                if (ph == 1) mbar_spin(&sm.lsefull[ord & 1], (ord >> 1) & 1, abort, a.err);
-                if (ph == 0 || MODE == kScores)
-                    mbar_spin(&sm.fullA[i % kRing], (i / kRing) & 1, abort, a.err);
-                else
-                    mbar_spin(&sm.fullB[s], sph, abort, a.err);
-                const int n = atomicAdd(&sm.next_job, 1);
-                const int slot = n % kAcc;
-                // Accumulators are taken in job order: job n waits for the release of job
-                // n - kAcc only after job n - 1 has taken its own, so that the accumulator's
-                // barrier is never two phases behind this wait (a parity wait would pass).
-                spin_until_at_least(&sm.jobs_started, n, abort, a.err);
-                mbar_spin(&sm.accempty[slot], ((n / kAcc) & 1) ^ 1, abort, a.err);
-                tc_fence_after();
-                *reinterpret_cast<volatile int*>(&sm.jobs_started) = n + 1;
-                sm.job[slot] = make_int4(ph, u, t, ph == 0 ? i : (ord & 1));
-                mbar_arrive(&sm.accfull[slot]);
-                const uint32_t d = tmem + slot * 128;
-                const uint64_t dq = dQ0 + (uint64_t)qslot * kQStep;
-                if (ph == 0) {
-                    // both halves of the tile arrived with one op
-                    const int st = i % kRing;
-                    const uint64_t dk = dK0 + (uint64_t)(2 * st) * kBoxStep;
-                    umma_half(d, dq, dk, 0);
-                    umma_half(d, dq + kBoxStep, dk + kBoxStep, 1);
-                    umma_commit(&sm.emptyA[st]);
-                } else if (MODE == kScores) {
-                    // phase 2 alone: the tile came through the phase-1 ring
-                    const int st = i % kRing;
-                    const uint64_t dk = sw128_desc(smem_u32(sm.ringA[0])) + (uint64_t)(2 * st) * kBoxStep;
+                if (MODE == kFull || (i & 1) == parity) {
+                    if (!have_q) {
+                        // the unit's Q (its slot is not refilled before phase 2 releases it)
+                        mbar_spin(&sm.qfull[qslot], (ord / kQSlots) & 1, abort, a.err);
+                        have_q = true;
+                    }
+                    // phase 2 of a tile waits until its unit's lse is in shared memory
+                    if (ph == 1) mbar_spin(&sm.lsefull[ord & 1], (ord >> 1) & 1, abort, a.err);
+                    if (ph == 0 || MODE == kScores)
+                        mbar_spin(&sm.fullA[i % kRing], (i / kRing) & 1, abort, a.err);
+                    else
+                        mbar_spin(&sm.fullB[s], sph, abort, a.err);
+                    const int n = atomicAdd(&sm.next_job, 1);
+                    const int slot = n % kAcc;
+                    // Accumulators are taken in job order: job n waits for the release of job
+                    // n - kAcc only after job n - 1 has taken its own, so that the accumulator's
+                    // barrier is never two phases behind this wait (a parity wait would pass).
+                    spin_until_at_least(&sm.jobs_started, n, abort, a.err);
+                    mbar_spin(&sm.accempty[slot], ((n / kAcc) & 1) ^ 1, abort, a.err);
                     tc_fence_after();
-                    umma_half(d, dk, dq, 0);
-                    umma_half(d, dk + kBoxStep, dq + kBoxStep, 1);
-                    umma_commit(&sm.emptyA[st]);
-                } else {
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        if (h == 1) mbar_spin(&sm.fullB[s], sph, abort, a.err);
+                    *reinterpret_cast<volatile int*>(&sm.jobs_started) = n + 1;
+                    sm.job[slot] = make_int4(ph, u, t, ph == 0 ? i : (ord & 1));
+                    mbar_arrive(&sm.accfull[slot]);
+                    const uint32_t d = tmem + slot * 128;
+                    const uint64_t dq = dQ0 + (uint64_t)qslot * kQStep;
+                    if (ph == 0) {
+                        // both halves of the tile arrived with one op
+                        const int st = i % kRing;
+                        const uint64_t dk = dK0 + (uint64_t)(2 * st) * kBoxStep;
+                        umma_half(d, dq, dk, 0);
+                        umma_half(d, dq + kBoxStep, dk + kBoxStep, 1);
+                        umma_commit(&sm.emptyA[st]);
+                    } else if (MODE == kScores) {
+                        // phase 2 alone: the tile came through the phase-1 ring
+                        const int st = i % kRing;
+                        const uint64_t dk = sw128_desc(smem_u32(sm.ringA[0])) + (uint64_t)(2 * st) * kBoxStep;
                         tc_fence_after();
-                        const uint64_t dk = dK0 + (uint64_t)s * kBoxStep;
-                        umma_half(d, dk, dq + h * kBoxStep, h);
-                        umma_commit(&sm.emptyB[s]);
-                        if (++s == kStagesB) {
-                            s = 0;
-                            sph ^= 1u;
+                        umma_half(d, dk, dq, 0);
+                        umma_half(d, dk + kBoxStep, dq + kBoxStep, 1);
+                        umma_commit(&sm.emptyA[st]);
+                    } else {
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            if (h == 1) mbar_spin(&sm.fullB[s], sph, abort, a.err);
+                            tc_fence_after();
+                            const uint64_t dk = dK0 + (uint64_t)s * kBoxStep;
+                            umma_half(d, dk, dq + h * kBoxStep, h);
+                            umma_commit(&sm.emptyB[s]);
+                            if (++s == kStagesB) {
+                                s = 0;
+                                sph ^= 1u;
+                            }
                         }
                     }
+                    umma_commit(&sm.accfull[slot]);
                 }
-                umma_commit(&sm.accfull[slot]);
                 // next tile; a new unit moves to the next Q slot (phase 2 releases the old one)
                 t += P;
                 int nu = u;
@@ -544,7 +555,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_score_kernel(const __grid_cons
                 }
                 if (nu != u) {
                     // the last phase that reads the unit's Q releases its slot
-                    if ((ph == 1 || MODE == kStats) && i + 1 < n_local) umma_commit(&sm.qempty[qslot]);
+                    if ((ph == 1 || MODE == kStats) && i + 1 < n_local) umma_commit(&qrelease[qslot]);
                     u = nu;
                     ++ord;
                     if (++qslot == kQSlots) qslot = 0;
