@@ -448,7 +448,9 @@ topk_cluster_kernel(const float* __restrict__ scores, int N, int S, int w, int b
         prefix |= (uint32_t)sm.gt << shift;
         mask |= dmask << shift;
         krem = sm.eq;
-        cluster.sync();  // nobody reads this pass's histograms any more
+        // (no cluster barrier here: every remote read of this pass -- the histograms before
+        // the second barrier, the slice totals in the digit search -- ends before the readers
+        // reach the next pass's first barrier, and only then are they overwritten)
     }
     const uint32_t T = prefix;  // the k_sel-th largest key; keep krem of the keys equal to T
 
