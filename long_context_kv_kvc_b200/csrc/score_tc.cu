@@ -70,7 +70,7 @@ constexpr int kBoxBytes = kTileKeys * 64 * 2;          // a 128-row x 64-column 
 #define KVC_TC_Q_SLOTS 3
 #endif
 #ifndef KVC_TC_LEAD_SLACK
-#define KVC_TC_LEAD_SLACK 6
+#define KVC_TC_LEAD_SLACK 5
 #endif
 constexpr int kStagesA = KVC_TC_STAGES_A;              // phase-1 ring, in 16 KiB halves (HBM stream)
 constexpr int kTilesA = kStagesA / 2;                  // the same ring in whole tiles (one op each)
