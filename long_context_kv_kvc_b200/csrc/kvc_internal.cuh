@@ -97,8 +97,6 @@ cudaError_t tc_score(const ScoreJob& job, cudaStream_t s);
 cudaError_t tc_shard_stats(const ScoreJob& job, float2* ml, cudaStream_t s);
 cudaError_t tc_shard_scores(const ScoreJob& job, const float2* ml_all, int W, cudaStream_t s);
 
-// the tensor-core kernel's software exp2, element-wise (diagnostics)
-
 // sums of unit scores over layers (and KV heads for the all-heads scope)
 cudaError_t reduce_units(const float* unit_scores, int L, int B, int Hkv, int N, int all_heads,
                          float* out, cudaStream_t s);
