@@ -870,13 +870,21 @@ __global__ void tc_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_b
         const int n_s = mode == kFull ? 1 : kRefSamples;
         float best = -INFINITY;
         if (has_ref) {
+            // all the samples' loads first, then the dot products (one round of load latency)
             const uint2 qv = *reinterpret_cast<const uint2*>(q + (u * nq + r) * kHeadDim + 4 * lane);
             const __nv_bfloat162* qh = reinterpret_cast<const __nv_bfloat162*>(&qv);
-            for (int si = 0; si < n_s; ++si) {
-                const int kj = mode == kFull ? t_r : (int)((long long)si * t_r / (n_s - 1));
-                if (!dcheck(err, kj >= 0 && kj < N)) continue;
-                const uint2 kv = *reinterpret_cast<const uint2*>(k + (u * N + kj) * kHeadDim + 4 * lane);
-                const __nv_bfloat162* kh = reinterpret_cast<const __nv_bfloat162*>(&kv);
+            uint2 kv[kRefSamples];
+#pragma unroll
+            for (int si = 0; si < kRefSamples; ++si) {
+                const int kj = mode == kFull ? t_r : (int)((long long)si * t_r / (kRefSamples - 1));
+                const bool use = si < n_s && dcheck(err, kj >= 0 && kj < N);
+                kv[si] = use ? *reinterpret_cast<const uint2*>(k + (u * N + kj) * kHeadDim + 4 * lane)
+                             : make_uint2(0u, 0u);
+            }
+#pragma unroll
+            for (int si = 0; si < kRefSamples; ++si) {
+                if (si >= n_s) break;
+                const __nv_bfloat162* kh = reinterpret_cast<const __nv_bfloat162*>(&kv[si]);
                 float x = 0.f;
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
